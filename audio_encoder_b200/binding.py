@@ -1,0 +1,248 @@
+"""Thin ctypes binding of the moss_enc C ABI (``include/moss_enc.h``).
+
+Argument marshalling only: every step of the encoder runs in the CUDA
+library.  PyTorch provides device memory and the stream.  Loading fails
+loudly if ``libmoss_enc.so`` has not been built; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoss_enc.so")
+
+OK = 0
+STATUS = {0: "ok", 1: "invalid argument", 2: "capacity", 3: "out of memory", 4: "cuda error",
+          5: "device timeout"}
+OUT_F32, OUT_BF16 = 0, 1
+STAGE_STEM, STAGE_LAYERS, STAGE_HEAD, STAGE_ADAPTER = 0, 1, 2, 3
+D_MODEL, D_OUT = 1280, 2048
+
+EXPORTED = [
+    "moss_enc_weight_count", "moss_enc_num_frames", "moss_enc_num_tokens", "moss_enc_range_tokens",
+    "moss_enc_create", "moss_enc_set_stream", "moss_enc_synchronize", "moss_enc_destroy",
+    "moss_enc_status_string", "moss_enc_last_error", "moss_enc_logmel", "moss_enc_log_max",
+    "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
+]
+
+
+class MossEncError(RuntimeError):
+    def __init__(self, status: int, msg: str = ""):
+        super().__init__(f"moss_enc status {status} ({STATUS.get(status, '?')}): {msg}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int), ("max_samples", ctypes.c_int64),
+                ("max_clips", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+class Clip(ctypes.Structure):
+    _fields_ = [("pcm", ctypes.c_void_p), ("n_samples", ctypes.c_int64), ("begin", ctypes.c_int64),
+                ("end", ctypes.c_int64), ("log_max", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run `python -m audio_encoder_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, i32, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+        L.moss_enc_weight_count.restype = i64
+        L.moss_enc_weight_count.argtypes = [i32]
+        L.moss_enc_num_frames.restype = i64
+        L.moss_enc_num_frames.argtypes = [i64]
+        L.moss_enc_num_tokens.restype = i64
+        L.moss_enc_num_tokens.argtypes = [i64]
+        L.moss_enc_range_tokens.restype = i64
+        L.moss_enc_range_tokens.argtypes = [i64, i64, i64]
+        L.moss_enc_create.restype = i32
+        L.moss_enc_create.argtypes = [ctypes.POINTER(Config), vp, ctypes.c_size_t, i32, vp, ctypes.POINTER(vp)]
+        L.moss_enc_set_stream.restype = i32
+        L.moss_enc_set_stream.argtypes = [vp, vp]
+        L.moss_enc_synchronize.restype = i32
+        L.moss_enc_synchronize.argtypes = [vp]
+        L.moss_enc_destroy.restype = None
+        L.moss_enc_destroy.argtypes = [vp]
+        L.moss_enc_status_string.restype = ctypes.c_char_p
+        L.moss_enc_status_string.argtypes = [i32]
+        L.moss_enc_last_error.restype = ctypes.c_char_p
+        L.moss_enc_last_error.argtypes = [vp]
+        L.moss_enc_logmel.restype = i32
+        L.moss_enc_logmel.argtypes = [vp, ctypes.POINTER(Clip), vp, ctypes.POINTER(i64), vp]
+        L.moss_enc_log_max.restype = i32
+        L.moss_enc_log_max.argtypes = [vp, vp, i64, vp]
+        L.moss_enc_forward.restype = i32
+        L.moss_enc_forward.argtypes = [vp, ctypes.POINTER(Clip), i32, vp, ctypes.POINTER(i64)]
+        L.moss_enc_forward_stage.restype = i32
+        L.moss_enc_forward_stage.argtypes = [vp, ctypes.POINTER(Clip), i32, i32, vp, ctypes.POINTER(i64)]
+        L.moss_enc_forward_host.restype = i32
+        L.moss_enc_forward_host.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(i64), i32, vp,
+                                            ctypes.POINTER(i64)]
+        _lib = L
+    return _lib
+
+
+def weight_count(n_layers: int) -> int:
+    return int(lib().moss_enc_weight_count(n_layers))
+
+
+def num_frames(n: int) -> int:
+    return int(lib().moss_enc_num_frames(n))
+
+
+def num_tokens(n: int) -> int:
+    return int(lib().moss_enc_num_tokens(n))
+
+
+def range_tokens(n: int, begin: int, end: int) -> int:
+    return int(lib().moss_enc_range_tokens(n, begin, end))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+class Encoder:
+    """One moss_enc handle on the current CUDA device.
+
+    blob: uint16 numpy array of bf16 bits (host) or a torch uint16/int16 CUDA
+    tensor.  Work is enqueued on ``stream`` (default: torch's current stream).
+    """
+
+    def __init__(self, blob, n_layers: int, max_samples: int, max_clips: int = 1,
+                 out_dtype: int = OUT_F32, stream=None):
+        import torch
+        self.torch = torch
+        self.n_layers = n_layers
+        self.out_dtype = out_dtype
+        cfg = Config(n_layers, int(max_samples), int(max_clips), int(out_dtype))
+        if stream is None:
+            stream = torch.cuda.current_stream()
+        self.stream = stream
+        h = ctypes.c_void_p()
+        if isinstance(blob, np.ndarray):
+            blob = np.ascontiguousarray(blob, dtype=np.uint16)
+            st = lib().moss_enc_create(ctypes.byref(cfg), blob.ctypes.data_as(ctypes.c_void_p),
+                                       blob.nbytes, 0, ctypes.c_void_p(stream.cuda_stream), ctypes.byref(h))
+        else:
+            st = lib().moss_enc_create(ctypes.byref(cfg), ctypes.c_void_p(blob.data_ptr()),
+                                       blob.numel() * 2, 1, ctypes.c_void_p(stream.cuda_stream),
+                                       ctypes.byref(h))
+        if st != OK:
+            raise MossEncError(st, "create failed")
+        self.h = h
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib().moss_enc_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, st):
+        if st != OK:
+            msg = lib().moss_enc_last_error(self.h) or b""
+            raise MossEncError(st, msg.decode())
+
+    def set_stream(self, stream):
+        self.stream = stream
+        self._check(lib().moss_enc_set_stream(self.h, ctypes.c_void_p(stream.cuda_stream)))
+
+    def synchronize(self):
+        self._check(lib().moss_enc_synchronize(self.h))
+
+    @staticmethod
+    def _clip(pcm, begin=0, end=None, log_max=None):
+        n = pcm.numel()
+        return Clip(pcm.data_ptr(), n, int(begin), int(n if end is None else end),
+                    log_max.data_ptr() if log_max is not None else None)
+
+    def log_max(self, pcm):
+        out = self.torch.empty(1, dtype=self.torch.float32, device=pcm.device)
+        self._check(lib().moss_enc_log_max(self.h, _ptr(pcm), pcm.numel(), _ptr(out)))
+        return out
+
+    def logmel(self, pcm, begin=0, end=None, log_max=None):
+        """Normalised log-mel [frames][128] fp32 and the log-mel maximum (device)."""
+        n = pcm.numel()
+        end = n if end is None else end
+        fb = begin // 160
+        fe = num_frames(n) if end == n else end // 160
+        mel = self.torch.empty((max(fe - fb, 0), 128), dtype=self.torch.float32, device=pcm.device)
+        mx = self.torch.empty(1, dtype=self.torch.float32, device=pcm.device)
+        c = self._clip(pcm, begin, end, log_max)
+        nf = ctypes.c_int64()
+        self._check(lib().moss_enc_logmel(self.h, ctypes.byref(c), _ptr(mel) if mel.numel() else None,
+                                          ctypes.byref(nf), _ptr(mx)))
+        assert nf.value == mel.shape[0]
+        return mel, mx
+
+    def _clips(self, clips):
+        arr = (Clip * max(len(clips), 1))()
+        total = 0
+        for i, c in enumerate(clips):
+            if isinstance(c, tuple):
+                pcm, begin, end, lm = (list(c) + [None, None, None])[:4]
+                n = pcm.numel()
+                arr[i] = self._clip(pcm, begin or 0, n if end is None else end, lm)
+                total += range_tokens(n, begin or 0, n if end is None else end)
+            else:
+                arr[i] = self._clip(c)
+                total += num_tokens(c.numel())
+        return arr, total
+
+    def forward(self, clips, out=None, stage: int = STAGE_ADAPTER):
+        """Encode clips (device fp32 tensors, or (pcm, begin, end, log_max) tuples).
+
+        Returns (rows, row_offsets): rows [T][2048] (or [T][1280] for the stem
+        and layer stages), row_offsets a Python list of n_clips + 1 ints.
+        """
+        torch = self.torch
+        arr, T = self._clips(clips)
+        width = D_MODEL if stage in (STAGE_STEM, STAGE_LAYERS) else D_OUT
+        if stage == STAGE_ADAPTER:
+            dt = torch.float32 if self.out_dtype == OUT_F32 else torch.bfloat16
+        else:
+            dt = torch.float32
+        dev = clips[0][0].device if isinstance(clips[0], tuple) else clips[0].device
+        if out is None:
+            out = torch.empty((T, width), dtype=dt, device=dev)
+        offs = (ctypes.c_int64 * (len(clips) + 1))()
+        if stage == STAGE_ADAPTER:
+            st = lib().moss_enc_forward(self.h, arr, len(clips), _ptr(out) if T else None, offs)
+        else:
+            st = lib().moss_enc_forward_stage(self.h, arr, len(clips), stage, _ptr(out) if T else None, offs)
+        self._check(st)
+        return out, list(offs)
+
+    def forward_host(self, clips_host, rows_host=None):
+        """End-to-end from host fp32 arrays to host rows (synchronises)."""
+        n = len(clips_host)
+        ptrs = (ctypes.c_void_p * max(n, 1))()
+        lens = (ctypes.c_int64 * max(n, 1))()
+        T = 0
+        for i, c in enumerate(clips_host):
+            ptrs[i] = c.data_ptr() if hasattr(c, "data_ptr") else c.ctypes.data
+            lens[i] = c.numel() if hasattr(c, "numel") else c.size
+            T += num_tokens(lens[i])
+        if rows_host is None:
+            dt = np.float32 if self.out_dtype == OUT_F32 else np.uint16
+            rows_host = np.empty((T, D_OUT), dtype=dt)
+        rp = rows_host.data_ptr() if hasattr(rows_host, "data_ptr") else rows_host.ctypes.data
+        offs = (ctypes.c_int64 * (n + 1))()
+        self._check(lib().moss_enc_forward_host(self.h, ptrs, lens, n, ctypes.c_void_p(rp), offs))
+        return rows_host, list(offs)

@@ -1,0 +1,935 @@
+// C ABI of the B200 audio encoder (declared in include/moss_enc.h): weight
+// repacking, the device workspace, per-call chunk planning on the host, and
+// the launch sequence of one forward.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/moss_enc.h"
+#include "attn.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "mel.cuh"
+#include "norm.cuh"
+#include "stem.cuh"
+
+using namespace moss;
+
+namespace {
+
+constexpr int D = 1280, DQKV = 3840, DFF = 5120, CST = 480, DOUT = 2048, DADP = 8192;
+constexpr int CHUNK_FRAMES = 800, CHUNK_TOKENS = 100, CHUNK_SAMPLES = 128000, HOP = 160;
+constexpr int CONV_K = 9 * 512;  // conv2/conv3 patch width: 9 taps x 480 channels padded to 512
+constexpr int STEM_GROUP_DEFAULT = 16;
+
+struct LayerDev {
+    float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+    bf16 *wqkv, *wo, *w1, *w2;
+    float *bqkv, *bo, *b1, *b2;
+};
+
+struct ClipPlan {
+    int64_t n, F, f_begin, f_end, c_first, c_last, tok0, ntok;
+};
+
+}  // namespace
+
+struct moss_enc {
+    moss_enc_config cfg{};
+    int device = 0, num_sms = 148;
+    cudaStream_t stream = nullptr;
+    std::string last_error;
+
+    // weights (one allocation)
+    void *wmem = nullptr;
+    float *conv1_w = nullptr, *conv1_b = nullptr, *conv2_b = nullptr, *conv3_b = nullptr;
+    bf16 *conv2_w = nullptr, *conv3_w = nullptr, *conv_out_w = nullptr;
+    std::vector<LayerDev> layers;
+    float *lnp_g = nullptr, *lnp_b = nullptr, *bp1 = nullptr, *bp2 = nullptr, *bgu = nullptr, *bd = nullptr;
+    bf16 *wp1 = nullptr, *wp2 = nullptr, *wgu = nullptr, *wd = nullptr;
+    float *pos = nullptr;
+    MelTables *mel_tab = nullptr;
+
+    // capacity
+    int64_t max_tokens = 0, max_chunks = 0;
+    int stem_group = STEM_GROUP_DEFAULT;
+
+    // workspace (one allocation)
+    void *ws = nullptr;
+    float *mel_raw = nullptr;
+    bf16 *c1out = nullptr, *a2 = nullptr, *c2out = nullptr, *a3 = nullptr, *c3out = nullptr;
+    float *X = nullptr;
+    bf16 *xn = nullptr, *qkv = nullptr, *attn = nullptr, *ffn = nullptr, *hb = nullptr, *h2 = nullptr, *gu = nullptr;
+    int *gmax_ord = nullptr;
+    int *err = nullptr;
+    float *pcm_stage = nullptr;
+    void *out_stage = nullptr;
+
+    // per-call tables: device copies and one pinned host staging area
+    size_t tab_bytes = 0;
+    void *d_tab = nullptr, *h_tab = nullptr;
+    cudaEvent_t tab_event = nullptr;
+};
+
+// ------------------------------------------------------------ small helpers
+
+static moss_enc_status fail(moss_enc *h, moss_enc_status s, const std::string &msg)
+{
+    if (h) h->last_error = msg;
+    return s;
+}
+
+#define CUDA_TRY(h, call)                                                                       \
+    do {                                                                                        \
+        cudaError_t e_ = (call);                                                                \
+        if (e_ != cudaSuccess)                                                                  \
+            return fail(h, MOSS_ENC_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+    } while (0)
+
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                      const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                      const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled_t encode_fn()
+{
+    static PFN_encodeTiled_t fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled_t>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map: rows of `inner` elements, `row_bytes` apart; box of
+// box_inner x box_rows with 128-byte swizzle (box_inner = 64).
+static bool tmap_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_rows)
+{
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI>
+static moss_enc_status gemm(moss_enc *h, const bf16 *A, int64_t M, int K, const bf16 *B, int N, GemmArgs a)
+{
+    if (M <= 0) return MOSS_ENC_OK;
+    if (K % 64 != 0 || N % BN != 0 || M > INT32_MAX)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "gemm shape not supported");
+    CUtensorMap ta, tb;
+    if (!tmap_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128) ||
+        !tmap_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, 64, BN))
+        return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    a.M = (int)M;
+    a.N = N;
+    a.K = K;
+    a.m_tiles = (int)((M + 127) / 128);
+    a.n_tiles = N / BN;
+    a.err = h->err;
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int grid = std::min(tiles, h->num_sms);
+    gemm_tc_kernel<BN, EPI><<<grid, 192, GemmCfg<BN>::SMEM, h->stream>>>(ta, tb, a);
+    CUDA_TRY(h, cudaGetLastError());
+    return MOSS_ENC_OK;
+}
+
+#define TRY(x)                                  \
+    do {                                        \
+        moss_enc_status s_ = (x);               \
+        if (s_ != MOSS_ENC_OK) return s_;       \
+    } while (0)
+
+template <int BN, int EPI>
+static cudaError_t gemm_attr()
+{
+    return cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)GemmCfg<BN>::SMEM);
+}
+
+static float bf16_bits_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+}
+
+// ------------------------------------------------------ host-side constants
+
+// Slaney mel scale (linear below 1 kHz at 200/3 Hz per mel, logarithmic above
+// with a step of ln(6.4)/27 per mel).
+static double slaney_mel(double hz)
+{
+    return hz < 1000.0 ? hz * 3.0 / 200.0 : 15.0 + std::log(hz / 1000.0) * 27.0 / std::log(6.4);
+}
+
+static double slaney_hz(double mel)
+{
+    return mel < 15.0 ? mel * 200.0 / 3.0 : 1000.0 * std::exp((mel - 15.0) * std::log(6.4) / 27.0);
+}
+
+// Twiddles, periodic Hann and the banded 128 x 201 Slaney filterbank
+// (triangles between mel-spaced edges over 0..8 kHz, area-normalised).
+static bool build_mel_tables(MelTables *t)
+{
+    for (int k = 0; k < 400; k++) {
+        const double a = -2.0 * M_PI * k / 400.0;
+        t->tw400[k] = make_float2((float)std::cos(a), (float)std::sin(a));
+        t->hann[k] = (float)(0.5 - 0.5 * std::cos(2.0 * M_PI * k / 400.0));
+    }
+    double edge[130];
+    const double top = slaney_mel(8000.0);
+    for (int i = 0; i < 130; i++) edge[i] = slaney_hz(top * i / 129.0);
+    for (int m = 0; m < 128; m++) {
+        double w[201];
+        int lo = -1, hi = -1;
+        for (int k = 0; k <= 200; k++) {
+            const double f = 40.0 * k;
+            const double rise = (f - edge[m]) / (edge[m + 1] - edge[m]);
+            const double fall = (edge[m + 2] - f) / (edge[m + 2] - edge[m + 1]);
+            double v = std::min(rise, fall);
+            v = v > 0.0 ? v * 2.0 / (edge[m + 2] - edge[m]) : 0.0;
+            w[k] = v;
+            if (v > 0.0) {
+                if (lo < 0) lo = k;
+                hi = k;
+            }
+        }
+        if (lo < 0) lo = hi = 0;
+        if (hi - lo + 1 > MEL_BAND) return false;
+        t->band_lo[m] = lo;
+        for (int b = 0; b < MEL_BAND; b++) t->band_w[m][b] = (lo + b <= 200) ? (float)w[lo + b] : 0.0f;
+    }
+    return true;
+}
+
+// ----------------------------------------------------------------- sizes
+
+extern "C" int64_t moss_enc_weight_count(int n_layers)
+{
+    if (n_layers < 0) return -1;
+    int64_t n = (int64_t)CST * 9 + CST + 2 * ((int64_t)CST * CST * 9 + CST) + (int64_t)D * CST * 16;
+    const int64_t per_layer = 4 * (int64_t)D + 4 * ((int64_t)D * D + D) + ((int64_t)DFF * D + DFF) +
+                              ((int64_t)D * DFF + D);
+    n += per_layer * n_layers;
+    n += 2 * (int64_t)D + ((int64_t)D * D + D) + ((int64_t)DOUT * D + DOUT);
+    n += 2 * ((int64_t)DADP * DOUT + DADP) + ((int64_t)DOUT * DADP + DOUT);
+    return n;
+}
+
+extern "C" int64_t moss_enc_num_frames(int64_t n_samples) { return n_samples <= 0 ? 0 : n_samples / HOP; }
+
+static int64_t chunk_tokens(int64_t frames) { return (frames + 7) / 8; }
+
+static bool plan_clip(int64_t n, int64_t begin, int64_t end, ClipPlan *p)
+{
+    if (n < 0 || begin < 0 || end > n || begin > end) return false;
+    if (begin % CHUNK_SAMPLES != 0) return false;
+    if (end != n && end % CHUNK_SAMPLES != 0) return false;
+    p->n = n;
+    p->F = moss_enc_num_frames(n);
+    p->f_begin = begin / HOP;
+    p->f_end = end == n ? p->F : end / HOP;
+    if (p->f_begin > p->f_end) p->f_begin = p->f_end;
+    p->c_first = p->f_begin / CHUNK_FRAMES;
+    p->c_last = (p->f_end + CHUNK_FRAMES - 1) / CHUNK_FRAMES;
+    if (p->f_end <= p->f_begin) p->c_last = p->c_first;
+    p->ntok = 0;
+    for (int64_t c = p->c_first; c < p->c_last; c++)
+        p->ntok += chunk_tokens(std::min<int64_t>(CHUNK_FRAMES, p->F - c * CHUNK_FRAMES));
+    return true;
+}
+
+extern "C" int64_t moss_enc_num_tokens(int64_t n_samples)
+{
+    ClipPlan p;
+    if (!plan_clip(n_samples < 0 ? 0 : n_samples, 0, n_samples < 0 ? 0 : n_samples, &p)) return -1;
+    return p.ntok;
+}
+
+extern "C" int64_t moss_enc_range_tokens(int64_t n_samples, int64_t begin, int64_t end)
+{
+    ClipPlan p;
+    if (!plan_clip(n_samples, begin, end, &p)) return -1;
+    return p.ntok;
+}
+
+extern "C" const char *moss_enc_status_string(moss_enc_status s)
+{
+    switch (s) {
+    case MOSS_ENC_OK: return "ok";
+    case MOSS_ENC_ERR_INVALID_ARG: return "invalid argument";
+    case MOSS_ENC_ERR_CAPACITY: return "request exceeds capacity";
+    case MOSS_ENC_ERR_OOM: return "out of device memory";
+    case MOSS_ENC_ERR_CUDA: return "CUDA error";
+    case MOSS_ENC_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+extern "C" const char *moss_enc_last_error(const moss_enc *h) { return h ? h->last_error.c_str() : ""; }
+
+// ------------------------------------------------------------ create/destroy
+
+// Table layout inside the per-call staging area.
+struct TabLayout {
+    size_t clips_main, clips_max, chunks, chunk_tok, logmax_src, total;
+};
+
+static TabLayout tab_layout(int64_t max_clips, int64_t max_chunks)
+{
+    TabLayout t;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t r = o;
+        o += (bytes + 255) & ~size_t(255);
+        return r;
+    };
+    t.clips_main = take(sizeof(MelClip) * max_clips);
+    t.clips_max = take(sizeof(MelClip) * max_clips);
+    t.chunks = take(sizeof(StemChunk) * max_chunks);
+    t.chunk_tok = take(sizeof(int2) * max_chunks);
+    t.logmax_src = take(sizeof(float *) * max_clips);
+    t.total = o;
+    return t;
+}
+
+extern "C" void moss_enc_destroy(moss_enc *h)
+{
+    if (!h) return;
+    cudaSetDevice(h->device);
+    if (h->stream) cudaStreamSynchronize(h->stream);
+    else cudaDeviceSynchronize();
+    if (h->wmem) cudaFree(h->wmem);
+    if (h->ws) cudaFree(h->ws);
+    if (h->d_tab) cudaFree(h->d_tab);
+    if (h->h_tab) cudaFreeHost(h->h_tab);
+    if (h->tab_event) cudaEventDestroy(h->tab_event);
+    delete h;
+}
+
+static moss_enc_status set_kernel_attrs(moss_enc *h)
+{
+    CUDA_TRY(h, (gemm_attr<160, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm_attr<128, EPI_CONVOUT_F32>()));
+    CUDA_TRY(h, (gemm_attr<256, EPI_BF16>()));
+    CUDA_TRY(h, (gemm_attr<256, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm_attr<128, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm_attr<128, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm_attr<256, EPI_F32>()));
+    CUDA_TRY(h, (gemm_attr<256, EPI_SWIGLU_BF16>()));
+    CUDA_TRY(h, (gemm_attr<128, EPI_F32>()));
+    CUDA_TRY(h, (gemm_attr<128, EPI_BF16>()));
+    CUDA_TRY(h, cudaFuncSetAttribute(window_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATTN_SMEM));
+    CUDA_TRY(h, cudaFuncSetAttribute(logmel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(MelSmem)));
+    return MOSS_ENC_OK;
+}
+
+extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const void *weights, size_t bytes,
+                                           int weights_on_device, void *stream, moss_enc **out)
+{
+    if (!out) return MOSS_ENC_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!cfg || !weights || cfg->n_layers < 1 || cfg->n_layers > 32 || cfg->max_samples < 1 ||
+        cfg->max_clips < 1 || (cfg->out_dtype != MOSS_ENC_OUT_F32 && cfg->out_dtype != MOSS_ENC_OUT_BF16))
+        return MOSS_ENC_ERR_INVALID_ARG;
+    const int64_t count = moss_enc_weight_count(cfg->n_layers);
+    if ((int64_t)bytes != count * 2) return MOSS_ENC_ERR_INVALID_ARG;
+
+    moss_enc *h = new (std::nothrow) moss_enc();
+    if (!h) return MOSS_ENC_ERR_OOM;
+    h->cfg = *cfg;
+    h->stream = (cudaStream_t)stream;
+    moss_enc_status st = MOSS_ENC_OK;
+    auto bail = [&](moss_enc_status s) {
+        moss_enc_destroy(h);
+        return s;
+    };
+    if (cudaGetDevice(&h->device) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, h->device) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+    if (prop.major != 10) return bail(MOSS_ENC_ERR_CUDA);  // built for sm_100a only
+    h->num_sms = prop.multiProcessorCount;
+    if (!encode_fn()) return bail(MOSS_ENC_ERR_CUDA);
+    if ((st = set_kernel_attrs(h)) != MOSS_ENC_OK) return bail(st);
+
+    // ---- host copy of the blob
+    std::vector<uint16_t> host;
+    const uint16_t *src = static_cast<const uint16_t *>(weights);
+    if (weights_on_device) {
+        host.resize(count);
+        if (cudaMemcpy(host.data(), weights, bytes, cudaMemcpyDeviceToHost) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+        src = host.data();
+    }
+
+    // ---- sizes of the packed weights
+    const int L = cfg->n_layers;
+    size_t off = 0;
+    auto take = [&](size_t b) {
+        size_t r = off;
+        off += (b + 255) & ~size_t(255);
+        return r;
+    };
+    const size_t o_c1w = take(4 * CST * 9), o_c1b = take(4 * CST);
+    const size_t o_c2w = take(2 * (size_t)CST * CONV_K), o_c2b = take(4 * CST);
+    const size_t o_c3w = take(2 * (size_t)CST * CONV_K), o_c3b = take(4 * CST);
+    const size_t o_cow = take(2 * (size_t)D * CST * 16);
+    std::vector<size_t> o_layer(L);
+    const size_t layer_bytes = 4 * 4 * D + 2 * ((size_t)DQKV * D + (size_t)D * D + (size_t)DFF * D + (size_t)D * DFF) +
+                               4 * (DQKV + D + DFF + D) + 8 * 256;
+    for (int l = 0; l < L; l++) o_layer[l] = take(layer_bytes);
+    const size_t o_lnp = take(4 * 2 * D), o_p1 = take(2 * (size_t)D * D), o_bp1 = take(4 * D);
+    const size_t o_p2 = take(2 * (size_t)DOUT * D), o_bp2 = take(4 * DOUT);
+    const size_t o_gu = take(2 * (size_t)2 * DADP * DOUT), o_bgu = take(4 * 2 * DADP);
+    const size_t o_wd = take(2 * (size_t)DOUT * DADP), o_bd = take(4 * DOUT);
+    const size_t o_pos = take(4 * (size_t)CHUNK_TOKENS * D), o_mel = take(sizeof(MelTables));
+    const size_t wtotal = off;
+
+    std::vector<uint8_t> pk(wtotal, 0);
+    auto F32 = [&](size_t o) { return reinterpret_cast<float *>(pk.data() + o); };
+    auto U16 = [&](size_t o) { return reinterpret_cast<uint16_t *>(pk.data() + o); };
+    const uint16_t *p = src;
+    // conv1 [480][1][3][3] -> fp32 [480][9]
+    for (int i = 0; i < CST * 9; i++) F32(o_c1w)[i] = bf16_bits_to_float(p[i]);
+    p += CST * 9;
+    for (int i = 0; i < CST; i++) F32(o_c1b)[i] = bf16_bits_to_float(p[i]);
+    p += CST;
+    // conv2/conv3 [o][c][kf][kt] -> [o][(kf*3+kt)*512 + c]
+    for (int which = 0; which < 2; which++) {
+        uint16_t *dst = U16(which == 0 ? o_c2w : o_c3w);
+        for (int o = 0; o < CST; o++)
+            for (int c = 0; c < CST; c++)
+                for (int tap = 0; tap < 9; tap++) dst[(size_t)o * CONV_K + tap * 512 + c] = p[((size_t)o * CST + c) * 9 + tap];
+        p += (size_t)CST * CST * 9;
+        float *b = F32(which == 0 ? o_c2b : o_c3b);
+        for (int i = 0; i < CST; i++) b[i] = bf16_bits_to_float(p[i]);
+        p += CST;
+    }
+    // conv_out [1280][c*16+f] -> [1280][f*480+c] (NHWC conv3 output rows)
+    {
+        uint16_t *dst = U16(o_cow);
+        for (int o = 0; o < D; o++)
+            for (int c = 0; c < CST; c++)
+                for (int f = 0; f < 16; f++) dst[(size_t)o * 7680 + f * CST + c] = p[(size_t)o * 7680 + c * 16 + f];
+        p += (size_t)D * 7680;
+    }
+    h->layers.resize(L);
+    std::vector<size_t> lo(L * 12);
+    for (int l = 0; l < L; l++) {
+        size_t b = o_layer[l];
+        size_t q = b;
+        auto sub = [&](size_t n) {
+            size_t r = q;
+            q += (n + 255) & ~size_t(255);
+            return r;
+        };
+        const size_t ln1g = sub(4 * D), ln1b = sub(4 * D), ln2g = sub(4 * D), ln2b = sub(4 * D);
+        const size_t wqkv = sub(2 * (size_t)DQKV * D), bqkv = sub(4 * DQKV);
+        const size_t wo = sub(2 * (size_t)D * D), bo = sub(4 * D);
+        const size_t w1 = sub(2 * (size_t)DFF * D), b1 = sub(4 * DFF);
+        const size_t w2 = sub(2 * (size_t)D * DFF), b2 = sub(4 * D);
+        size_t *L12 = &lo[l * 12];
+        L12[0] = ln1g; L12[1] = ln1b; L12[2] = ln2g; L12[3] = ln2b; L12[4] = wqkv; L12[5] = bqkv;
+        L12[6] = wo; L12[7] = bo; L12[8] = w1; L12[9] = b1; L12[10] = w2; L12[11] = b2;
+        for (int i = 0; i < D; i++) F32(ln1g)[i] = bf16_bits_to_float(p[i]);
+        p += D;
+        for (int i = 0; i < D; i++) F32(ln1b)[i] = bf16_bits_to_float(p[i]);
+        p += D;
+        for (int part = 0; part < 3; part++) {  // q, k, v -> rows part*1280 .. of wqkv
+            std::memcpy(U16(wqkv) + (size_t)part * D * D, p, 2 * (size_t)D * D);
+            p += (size_t)D * D;
+            for (int i = 0; i < D; i++) F32(bqkv)[part * D + i] = bf16_bits_to_float(p[i]);
+            p += D;
+        }
+        std::memcpy(U16(wo), p, 2 * (size_t)D * D);
+        p += (size_t)D * D;
+        for (int i = 0; i < D; i++) F32(bo)[i] = bf16_bits_to_float(p[i]);
+        p += D;
+        for (int i = 0; i < D; i++) F32(ln2g)[i] = bf16_bits_to_float(p[i]);
+        p += D;
+        for (int i = 0; i < D; i++) F32(ln2b)[i] = bf16_bits_to_float(p[i]);
+        p += D;
+        std::memcpy(U16(w1), p, 2 * (size_t)DFF * D);
+        p += (size_t)DFF * D;
+        for (int i = 0; i < DFF; i++) F32(b1)[i] = bf16_bits_to_float(p[i]);
+        p += DFF;
+        std::memcpy(U16(w2), p, 2 * (size_t)D * DFF);
+        p += (size_t)D * DFF;
+        for (int i = 0; i < D; i++) F32(b2)[i] = bf16_bits_to_float(p[i]);
+        p += D;
+    }
+    for (int i = 0; i < D; i++) F32(o_lnp)[i] = bf16_bits_to_float(p[i]);
+    p += D;
+    for (int i = 0; i < D; i++) F32(o_lnp)[D + i] = bf16_bits_to_float(p[i]);
+    p += D;
+    std::memcpy(U16(o_p1), p, 2 * (size_t)D * D);
+    p += (size_t)D * D;
+    for (int i = 0; i < D; i++) F32(o_bp1)[i] = bf16_bits_to_float(p[i]);
+    p += D;
+    std::memcpy(U16(o_p2), p, 2 * (size_t)DOUT * D);
+    p += (size_t)DOUT * D;
+    for (int i = 0; i < DOUT; i++) F32(o_bp2)[i] = bf16_bits_to_float(p[i]);
+    p += DOUT;
+    // gate and up interleaved in blocks of 32 output rows: g[0:32], u[0:32], g[32:64], ...
+    {
+        const uint16_t *gw = p;
+        const uint16_t *gb = gw + (size_t)DADP * DOUT;
+        const uint16_t *uw = gb + DADP;
+        const uint16_t *ub = uw + (size_t)DADP * DOUT;
+        uint16_t *dst = U16(o_gu);
+        float *bdst = F32(o_bgu);
+        for (int j = 0; j < DADP / 32; j++)
+            for (int r = 0; r < 32; r++) {
+                std::memcpy(dst + ((size_t)(64 * j + r)) * DOUT, gw + (size_t)(32 * j + r) * DOUT, 2 * DOUT);
+                std::memcpy(dst + ((size_t)(64 * j + 32 + r)) * DOUT, uw + (size_t)(32 * j + r) * DOUT, 2 * DOUT);
+                bdst[64 * j + r] = bf16_bits_to_float(gb[32 * j + r]);
+                bdst[64 * j + 32 + r] = bf16_bits_to_float(ub[32 * j + r]);
+            }
+        p = ub + DADP;
+    }
+    std::memcpy(U16(o_wd), p, 2 * (size_t)DOUT * DADP);
+    p += (size_t)DOUT * DADP;
+    for (int i = 0; i < DOUT; i++) F32(o_bd)[i] = bf16_bits_to_float(p[i]);
+    p += DOUT;
+    if (p - src != count) return bail(MOSS_ENC_ERR_INVALID_ARG);
+    // sinusoidal positions 0..99: 640 sin channels then 640 cos channels,
+    // inv_timescale_i = exp(-i ln(10000) / 639)
+    for (int t = 0; t < CHUNK_TOKENS; t++)
+        for (int i = 0; i < D / 2; i++) {
+            const double inv = std::exp(-(double)i * std::log(10000.0) / (D / 2 - 1));
+            F32(o_pos)[t * D + i] = (float)std::sin(t * inv);
+            F32(o_pos)[t * D + D / 2 + i] = (float)std::cos(t * inv);
+        }
+    if (!build_mel_tables(reinterpret_cast<MelTables *>(pk.data() + o_mel))) return bail(MOSS_ENC_ERR_INVALID_ARG);
+
+    if (cudaMalloc(&h->wmem, wtotal) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
+    if (cudaMemcpy(h->wmem, pk.data(), wtotal, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+    uint8_t *W = static_cast<uint8_t *>(h->wmem);
+    h->conv1_w = (float *)(W + o_c1w);
+    h->conv1_b = (float *)(W + o_c1b);
+    h->conv2_w = (bf16 *)(W + o_c2w);
+    h->conv2_b = (float *)(W + o_c2b);
+    h->conv3_w = (bf16 *)(W + o_c3w);
+    h->conv3_b = (float *)(W + o_c3b);
+    h->conv_out_w = (bf16 *)(W + o_cow);
+    for (int l = 0; l < L; l++) {
+        size_t *L12 = &lo[l * 12];
+        LayerDev &d = h->layers[l];
+        d.ln1_g = (float *)(W + L12[0]);
+        d.ln1_b = (float *)(W + L12[1]);
+        d.ln2_g = (float *)(W + L12[2]);
+        d.ln2_b = (float *)(W + L12[3]);
+        d.wqkv = (bf16 *)(W + L12[4]);
+        d.bqkv = (float *)(W + L12[5]);
+        d.wo = (bf16 *)(W + L12[6]);
+        d.bo = (float *)(W + L12[7]);
+        d.w1 = (bf16 *)(W + L12[8]);
+        d.b1 = (float *)(W + L12[9]);
+        d.w2 = (bf16 *)(W + L12[10]);
+        d.b2 = (float *)(W + L12[11]);
+    }
+    h->lnp_g = (float *)(W + o_lnp);
+    h->lnp_b = h->lnp_g + D;
+    h->wp1 = (bf16 *)(W + o_p1);
+    h->bp1 = (float *)(W + o_bp1);
+    h->wp2 = (bf16 *)(W + o_p2);
+    h->bp2 = (float *)(W + o_bp2);
+    h->wgu = (bf16 *)(W + o_gu);
+    h->bgu = (float *)(W + o_bgu);
+    h->wd = (bf16 *)(W + o_wd);
+    h->bd = (float *)(W + o_bd);
+    h->pos = (float *)(W + o_pos);
+    h->mel_tab = (MelTables *)(W + o_mel);
+
+    // ---- workspace
+    h->max_tokens = cfg->max_samples / 1280 + cfg->max_clips + 1;
+    h->max_chunks = cfg->max_samples / CHUNK_SAMPLES + cfg->max_clips + 1;
+    h->stem_group = (int)std::min<int64_t>(STEM_GROUP_DEFAULT, h->max_chunks);
+    const int64_t T = h->max_tokens, G = h->stem_group;
+    off = 0;
+    const size_t w_mel = take(4 * (size_t)h->max_chunks * CHUNK_FRAMES * 128);
+    const size_t w_c1 = take(2 * (size_t)G * 400 * 64 * CST);
+    const size_t w_a2 = take(2 * (size_t)G * 6400 * CONV_K);
+    const size_t w_c2 = take(2 * (size_t)G * 6400 * CST);
+    const size_t w_a3 = take(2 * (size_t)G * 1600 * CONV_K);
+    const size_t w_c3 = take(2 * (size_t)G * 1600 * CST);
+    const size_t w_X = take(4 * (size_t)T * D);
+    const size_t w_xn = take(2 * (size_t)T * D);
+    const size_t w_qkv = take(2 * (size_t)T * DQKV);
+    const size_t w_at = take(2 * (size_t)T * D);
+    const size_t w_ffn = take(2 * (size_t)T * DFF);
+    const size_t w_hb = take(2 * (size_t)T * D);
+    const size_t w_h2 = take(2 * (size_t)T * DOUT);
+    const size_t w_gu = take(2 * (size_t)T * DADP);
+    const size_t w_gm = take(4 * (size_t)cfg->max_clips);
+    const size_t w_err = take(256);
+    const size_t w_pcm = take(4 * (size_t)cfg->max_samples);
+    const size_t w_out = take(4 * (size_t)T * DOUT);
+    if (cudaMalloc(&h->ws, off) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
+    uint8_t *S = static_cast<uint8_t *>(h->ws);
+    h->mel_raw = (float *)(S + w_mel);
+    h->c1out = (bf16 *)(S + w_c1);
+    h->a2 = (bf16 *)(S + w_a2);
+    h->c2out = (bf16 *)(S + w_c2);
+    h->a3 = (bf16 *)(S + w_a3);
+    h->c3out = (bf16 *)(S + w_c3);
+    h->X = (float *)(S + w_X);
+    h->xn = (bf16 *)(S + w_xn);
+    h->qkv = (bf16 *)(S + w_qkv);
+    h->attn = (bf16 *)(S + w_at);
+    h->ffn = (bf16 *)(S + w_ffn);
+    h->hb = (bf16 *)(S + w_hb);
+    h->h2 = (bf16 *)(S + w_h2);
+    h->gu = (bf16 *)(S + w_gu);
+    h->gmax_ord = (int *)(S + w_gm);
+    h->err = (int *)(S + w_err);
+    h->pcm_stage = (float *)(S + w_pcm);
+    h->out_stage = (void *)(S + w_out);
+    if (cudaMemset(h->err, 0, 256) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+
+    const TabLayout tl = tab_layout(cfg->max_clips, h->max_chunks);
+    h->tab_bytes = tl.total;
+    if (cudaMalloc(&h->d_tab, tl.total) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
+    if (cudaMallocHost(&h->h_tab, tl.total) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
+    if (cudaEventCreateWithFlags(&h->tab_event, cudaEventDisableTiming) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+    if (cudaDeviceSynchronize() != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+    *out = h;
+    return MOSS_ENC_OK;
+}
+
+extern "C" moss_enc_status moss_enc_set_stream(moss_enc *h, void *stream)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    h->stream = (cudaStream_t)stream;
+    return MOSS_ENC_OK;
+}
+
+extern "C" moss_enc_status moss_enc_synchronize(moss_enc *h)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+    int e = 0;
+    CUDA_TRY(h, cudaMemcpy(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+    if (e != 0) {
+        CUDA_TRY(h, cudaMemset(h->err, 0, sizeof(int)));
+        return fail(h, MOSS_ENC_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait timed out");
+    }
+    return MOSS_ENC_OK;
+}
+
+// --------------------------------------------------------- per-call tables
+
+// The host staging area is reused by every call; wait until the copy that
+// last read it has run (not while a stream is being captured).
+static moss_enc_status tab_begin(moss_enc *h)
+{
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    CUDA_TRY(h, cudaStreamIsCapturing(h->stream, &cs));
+    if (cs == cudaStreamCaptureStatusNone) CUDA_TRY(h, cudaEventSynchronize(h->tab_event));
+    return MOSS_ENC_OK;
+}
+
+static moss_enc_status tab_upload(moss_enc *h)
+{
+    CUDA_TRY(h, cudaMemcpyAsync(h->d_tab, h->h_tab, h->tab_bytes, cudaMemcpyHostToDevice, h->stream));
+    CUDA_TRY(h, cudaEventRecord(h->tab_event, h->stream));
+    return MOSS_ENC_OK;
+}
+
+static int mel_grid_x(int64_t max_frames) { return (int)std::max<int64_t>(1, (max_frames + MEL_FRAMES_PER_BLOCK - 1) / MEL_FRAMES_PER_BLOCK); }
+
+static moss_enc_status launch_logmel(moss_enc *h, const MelClip *d_clips, int n_clips, int64_t max_frames,
+                                     float *out, int write_out)
+{
+    if (n_clips <= 0 || max_frames <= 0) return MOSS_ENC_OK;
+    dim3 grid(mel_grid_x(max_frames), n_clips);
+    logmel_kernel<<<grid, 256, sizeof(MelSmem), h->stream>>>(d_clips, h->mel_tab, out, h->gmax_ord, write_out);
+    CUDA_TRY(h, cudaGetLastError());
+    return MOSS_ENC_OK;
+}
+
+// ------------------------------------------------------------------ logmel
+
+extern "C" moss_enc_status moss_enc_log_max(moss_enc *h, const float *pcm, int64_t n_samples, float *out)
+{
+    if (!h || !pcm || !out || n_samples < 0) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad argument");
+    if (n_samples / HOP > INT32_MAX) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "clip too long");
+    TRY(tab_begin(h));
+    const TabLayout tl = tab_layout(h->cfg.max_clips, h->max_chunks);
+    uint8_t *H = static_cast<uint8_t *>(h->h_tab);
+    const float **src = reinterpret_cast<const float **>(H + tl.logmax_src);
+    src[0] = nullptr;
+    MelClip *mc = reinterpret_cast<MelClip *>(H + tl.clips_max);
+    mc[0] = MelClip{pcm, (long long)n_samples, 0, 0, (int)(n_samples / HOP), 0, 0};
+    TRY(tab_upload(h));
+    uint8_t *Dt = static_cast<uint8_t *>(h->d_tab);
+    gmax_init_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), 1);
+    CUDA_TRY(h, cudaGetLastError());
+    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), 1, n_samples / HOP, nullptr, 0));
+    gmax_export_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, out);
+    CUDA_TRY(h, cudaGetLastError());
+    return MOSS_ENC_OK;
+}
+
+extern "C" moss_enc_status moss_enc_logmel(moss_enc *h, const moss_enc_clip *clip, float *mel_out,
+                                           int64_t *n_frames, float *log_max_out)
+{
+    if (!h || !clip || !clip->pcm) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad argument");
+    ClipPlan pl;
+    if (!plan_clip(clip->n_samples, clip->begin, clip->end, &pl)) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad range");
+    if (pl.F > INT32_MAX) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "clip too long");
+    if (clip->end - clip->begin > h->cfg.max_samples) return fail(h, MOSS_ENC_ERR_CAPACITY, "range exceeds max_samples");
+    const int64_t nf = pl.f_end - pl.f_begin;
+    if (n_frames) *n_frames = nf;
+    if (nf > 0 && !mel_out) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "mel_out is null");
+    const bool whole = pl.f_begin == 0 && pl.f_end == pl.F;
+    TRY(tab_begin(h));
+    const TabLayout tl = tab_layout(h->cfg.max_clips, h->max_chunks);
+    uint8_t *H = static_cast<uint8_t *>(h->h_tab);
+    reinterpret_cast<const float **>(H + tl.logmax_src)[0] = clip->log_max;
+    MelClip *mm = reinterpret_cast<MelClip *>(H + tl.clips_main);
+    MelClip *mx = reinterpret_cast<MelClip *>(H + tl.clips_max);
+    const bool own_max = clip->log_max == nullptr;
+    mm[0] = MelClip{clip->pcm, (long long)pl.n, 0, (int)pl.f_begin, (int)pl.f_end, own_max && whole ? 0 : -1, 0};
+    mx[0] = MelClip{clip->pcm, (long long)pl.n, 0, 0, (int)pl.F, 0, 0};
+    TRY(tab_upload(h));
+    uint8_t *Dt = static_cast<uint8_t *>(h->d_tab);
+    gmax_init_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), 1);
+    CUDA_TRY(h, cudaGetLastError());
+    if (own_max && !whole)
+        TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), 1, pl.F, nullptr, 0));
+    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_main), 1, nf, mel_out, 1));
+    if (nf > 0) {
+        mel_normalize_kernel<<<std::min<int64_t>(4096, (nf * 128 + 255) / 256), 256, 0, h->stream>>>(mel_out, nf * 128, h->gmax_ord);
+        CUDA_TRY(h, cudaGetLastError());
+    }
+    if (log_max_out) {
+        gmax_export_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, log_max_out);
+        CUDA_TRY(h, cudaGetLastError());
+    }
+    return MOSS_ENC_OK;
+}
+
+// ----------------------------------------------------------------- forward
+
+static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int n_clips, int stage,
+                                    void *out, int64_t *row_offsets)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (n_clips < 0 || (n_clips > 0 && !clips) || !row_offsets) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad argument");
+    if (n_clips > h->cfg.max_clips) return fail(h, MOSS_ENC_ERR_CAPACITY, "too many clips");
+    if (stage < MOSS_ENC_STAGE_STEM || stage > MOSS_ENC_STAGE_ADAPTER) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad stage");
+
+    std::vector<ClipPlan> plans(n_clips);
+    int64_t samples = 0, T = 0, n_chunks = 0, max_range_frames = 0, max_clip_frames = 0;
+    row_offsets[0] = 0;
+    for (int i = 0; i < n_clips; i++) {
+        const moss_enc_clip &c = clips[i];
+        if (!plan_clip(c.n_samples, c.begin, c.end, &plans[i])) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad clip range");
+        if (plans[i].ntok > 0 && !c.pcm) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null pcm");
+        if (plans[i].F > INT32_MAX / 2) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "clip too long");
+        plans[i].tok0 = T;
+        T += plans[i].ntok;
+        row_offsets[i + 1] = T;
+        samples += c.end - c.begin;
+        n_chunks += plans[i].c_last - plans[i].c_first;
+        max_range_frames = std::max(max_range_frames, plans[i].f_end - plans[i].f_begin);
+        max_clip_frames = std::max(max_clip_frames, plans[i].F);
+    }
+    if (samples > h->cfg.max_samples || T > h->max_tokens || n_chunks > h->max_chunks)
+        return fail(h, MOSS_ENC_ERR_CAPACITY, "request exceeds the capacity set at create");
+    if (T > 0 && !out) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null output");
+    if (T == 0) return MOSS_ENC_OK;
+
+    // ---- tables
+    TRY(tab_begin(h));
+    const TabLayout tl = tab_layout(h->cfg.max_clips, h->max_chunks);
+    uint8_t *H = static_cast<uint8_t *>(h->h_tab);
+    const float **lsrc = reinterpret_cast<const float **>(H + tl.logmax_src);
+    MelClip *mm = reinterpret_cast<MelClip *>(H + tl.clips_main);
+    MelClip *mx = reinterpret_cast<MelClip *>(H + tl.clips_max);
+    StemChunk *sc = reinterpret_cast<StemChunk *>(H + tl.chunks);
+    int2 *ct = reinterpret_cast<int2 *>(H + tl.chunk_tok);
+    int n_max_pass = 0;
+    int64_t chunk = 0;
+    for (int i = 0; i < n_clips; i++) {
+        const ClipPlan &pl = plans[i];
+        const bool whole = pl.f_begin == 0 && pl.f_end == pl.F;
+        const bool own = clips[i].log_max == nullptr;
+        lsrc[i] = clips[i].log_max;
+        // main pass: frames [800 c_first, f_end) into rows of this clip's chunks
+        const int64_t fb = pl.c_first * CHUNK_FRAMES;
+        mm[i] = MelClip{clips[i].pcm, (long long)pl.n, (long long)chunk * CHUNK_FRAMES, (int)fb, (int)pl.f_end,
+                        own && whole ? i : -1, 0};
+        if (own && !whole) mx[n_max_pass++] = MelClip{clips[i].pcm, (long long)pl.n, 0, 0, (int)pl.F, i, 0};
+        int64_t tok = pl.tok0;
+        for (int64_t c = pl.c_first; c < pl.c_last; c++, chunk++) {
+            const int nf = (int)std::min<int64_t>(CHUNK_FRAMES, pl.F - c * CHUNK_FRAMES);
+            sc[chunk] = StemChunk{i, (int)(chunk * CHUNK_FRAMES), nf, 0};
+            const int nt = (int)chunk_tokens(nf);
+            ct[chunk] = make_int2((int)tok, nt);
+            tok += nt;
+        }
+    }
+    TRY(tab_upload(h));
+    uint8_t *Dt = static_cast<uint8_t *>(h->d_tab);
+    const StemChunk *d_chunks = reinterpret_cast<const StemChunk *>(Dt + tl.chunks);
+    const int2 *d_ct = reinterpret_cast<const int2 *>(Dt + tl.chunk_tok);
+
+    // ---- log-mel (raw) and per-clip maxima
+    gmax_init_kernel<<<(n_clips + 127) / 128, 128, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), n_clips);
+    CUDA_TRY(h, cudaGetLastError());
+    if (n_max_pass > 0)
+        TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), n_max_pass, max_clip_frames, nullptr, 0));
+    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_main), n_clips, max_range_frames, h->mel_raw, 1));
+
+    // ---- conv stem, in groups of chunks
+    for (int64_t g0 = 0; g0 < n_chunks; g0 += h->stem_group) {
+        const int gc = (int)std::min<int64_t>(h->stem_group, n_chunks - g0);
+        conv1_kernel<<<dim3(400, gc), 240, 0, h->stream>>>(h->mel_raw, d_chunks + g0, h->gmax_ord, h->conv1_w, h->conv1_b, h->c1out);
+        CUDA_TRY(h, cudaGetLastError());
+        const int64_t r2 = (int64_t)gc * 6400, r3 = (int64_t)gc * 1600;
+        im2col_s2_kernel<<<(int)std::min<int64_t>(65535, (r2 * 576 + 255) / 256), 256, 0, h->stream>>>(h->c1out, 400, 64, r2, h->a2);
+        CUDA_TRY(h, cudaGetLastError());
+        GemmArgs a{};
+        a.bias = h->conv2_b;
+        a.out = h->c2out;
+        a.ldo = CST;
+        TRY((gemm<160, EPI_GELU_BF16>(h, h->a2, r2, CONV_K, h->conv2_w, CST, a)));
+        im2col_s2_kernel<<<(int)std::min<int64_t>(65535, (r3 * 576 + 255) / 256), 256, 0, h->stream>>>(h->c2out, 200, 32, r3, h->a3);
+        CUDA_TRY(h, cudaGetLastError());
+        a.bias = h->conv3_b;
+        a.out = h->c3out;
+        TRY((gemm<160, EPI_GELU_BF16>(h, h->a3, r3, CONV_K, h->conv3_w, CST, a)));
+        GemmArgs co{};
+        co.out = h->X;
+        co.ldo = D;
+        co.pos = h->pos;
+        co.chunk_tok = d_ct + g0;
+        TRY((gemm<128, EPI_CONVOUT_F32>(h, h->c3out, (int64_t)gc * 100, 7680, h->conv_out_w, D, co)));
+    }
+    if (stage == MOSS_ENC_STAGE_STEM) {
+        CUDA_TRY(h, cudaMemcpyAsync(out, h->X, sizeof(float) * T * D, cudaMemcpyDeviceToDevice, h->stream));
+        return MOSS_ENC_OK;
+    }
+
+    // ---- Transformer layers
+    const int ln_grid = (int)((T + 7) / 8);
+    for (size_t l = 0; l < h->layers.size(); l++) {
+        const LayerDev &L = h->layers[l];
+        layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln1_g, L.ln1_b, h->xn, (int)T);
+        CUDA_TRY(h, cudaGetLastError());
+        GemmArgs a{};
+        a.bias = L.bqkv;
+        a.out = h->qkv;
+        a.ldo = DQKV;
+        TRY((gemm<256, EPI_BF16>(h, h->xn, T, D, L.wqkv, DQKV, a)));
+        window_attn_kernel<<<dim3((unsigned)n_chunks, 20), 256, ATTN_SMEM, h->stream>>>(h->qkv, d_ct, h->attn);
+        CUDA_TRY(h, cudaGetLastError());
+        a.bias = L.bo;
+        a.out = h->X;
+        a.ldo = D;
+        TRY((gemm<128, EPI_RESID_F32>(h, h->attn, T, D, L.wo, D, a)));
+        layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln2_g, L.ln2_b, h->xn, (int)T);
+        CUDA_TRY(h, cudaGetLastError());
+        a.bias = L.b1;
+        a.out = h->ffn;
+        a.ldo = DFF;
+        TRY((gemm<256, EPI_GELU_BF16>(h, h->xn, T, D, L.w1, DFF, a)));
+        a.bias = L.b2;
+        a.out = h->X;
+        a.ldo = D;
+        TRY((gemm<128, EPI_RESID_F32>(h, h->ffn, T, DFF, L.w2, D, a)));
+    }
+    if (stage == MOSS_ENC_STAGE_LAYERS) {
+        CUDA_TRY(h, cudaMemcpyAsync(out, h->X, sizeof(float) * T * D, cudaMemcpyDeviceToDevice, h->stream));
+        return MOSS_ENC_OK;
+    }
+
+    // ---- head: ln_post -> proj1 -> GELU -> proj2
+    layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, h->lnp_g, h->lnp_b, h->xn, (int)T);
+    CUDA_TRY(h, cudaGetLastError());
+    GemmArgs a{};
+    a.bias = h->bp1;
+    a.out = h->hb;
+    a.ldo = D;
+    TRY((gemm<128, EPI_GELU_BF16>(h, h->xn, T, D, h->wp1, D, a)));
+    a.bias = h->bp2;
+    a.ldo = DOUT;
+    if (stage == MOSS_ENC_STAGE_HEAD) {
+        a.out = out;
+        return gemm<256, EPI_F32>(h, h->hb, T, D, h->wp2, DOUT, a);
+    }
+    a.out = h->h2;
+    TRY((gemm<256, EPI_BF16>(h, h->hb, T, D, h->wp2, DOUT, a)));
+    // ---- SwiGLU adapter
+    a.bias = h->bgu;
+    a.out = h->gu;
+    a.ldo = DADP;
+    TRY((gemm<256, EPI_SWIGLU_BF16>(h, h->h2, T, DOUT, h->wgu, 2 * DADP, a)));
+    a.bias = h->bd;
+    a.out = out;
+    a.ldo = DOUT;
+    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm<128, EPI_F32>(h, h->gu, T, DADP, h->wd, DOUT, a);
+    return gemm<128, EPI_BF16>(h, h->gu, T, DADP, h->wd, DOUT, a);
+}
+
+extern "C" moss_enc_status moss_enc_forward(moss_enc *h, const moss_enc_clip *clips, int n_clips, void *rows_out,
+                                            int64_t *row_offsets)
+{
+    return forward_impl(h, clips, n_clips, MOSS_ENC_STAGE_ADAPTER, rows_out, row_offsets);
+}
+
+extern "C" moss_enc_status moss_enc_forward_stage(moss_enc *h, const moss_enc_clip *clips, int n_clips, int stage,
+                                                  void *out, int64_t *row_offsets)
+{
+    return forward_impl(h, clips, n_clips, stage, out, row_offsets);
+}
+
+extern "C" moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host, const int64_t *n_samples,
+                                                 int n_clips, void *rows_host, int64_t *row_offsets)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (n_clips < 0 || n_clips > h->cfg.max_clips || (n_clips > 0 && (!pcm_host || !n_samples)) || !row_offsets)
+        return fail(h, n_clips > h->cfg.max_clips ? MOSS_ENC_ERR_CAPACITY : MOSS_ENC_ERR_INVALID_ARG, "bad argument");
+    int64_t total = 0;
+    for (int i = 0; i < n_clips; i++) {
+        if (n_samples[i] < 0 || (n_samples[i] > 0 && !pcm_host[i])) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad clip");
+        total += (n_samples[i] + 3) & ~int64_t(3);  // keep every clip 16-byte aligned
+    }
+    if (total > h->cfg.max_samples) return fail(h, MOSS_ENC_ERR_CAPACITY, "clips exceed max_samples");
+    std::vector<moss_enc_clip> cl(n_clips);
+    int64_t o = 0;
+    for (int i = 0; i < n_clips; i++) {
+        if (n_samples[i] > 0)
+            CUDA_TRY(h, cudaMemcpyAsync(h->pcm_stage + o, pcm_host[i], sizeof(float) * n_samples[i],
+                                        cudaMemcpyHostToDevice, h->stream));
+        cl[i] = moss_enc_clip{h->pcm_stage + o, n_samples[i], 0, n_samples[i], nullptr};
+        o += (n_samples[i] + 3) & ~int64_t(3);
+    }
+    TRY(forward_impl(h, cl.data(), n_clips, MOSS_ENC_STAGE_ADAPTER, h->out_stage, row_offsets));
+    const int64_t T = row_offsets[n_clips];
+    const size_t esz = h->cfg.out_dtype == MOSS_ENC_OUT_F32 ? 4 : 2;
+    if (T > 0) {
+        if (!rows_host) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null rows_host");
+        CUDA_TRY(h, cudaMemcpyAsync(rows_host, h->out_stage, esz * T * DOUT, cudaMemcpyDeviceToHost, h->stream));
+    }
+    return moss_enc_synchronize(h);
+}

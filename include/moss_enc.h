@@ -1,0 +1,191 @@
+/*
+ * moss_enc: audio-encoder forward of the MOSS-Audio / MOSS-Transcribe family
+ * (the Qwen3-Omni AuT tower) for NVIDIA B200 (sm_100a).
+ *
+ * The method (page "MOSS-Transcribe-preview-2B - GGUF", "Architecture" table):
+ * 16 kHz mono PCM -> Whisper-style 128-bin log-mel (n_fft 400, hop 160) ->
+ * 3 x Conv2D stride 2 (1->480->480->480) -> conv_out (480*16 = 7680 -> 1280,
+ * no bias) + sinusoidal positions -> 32 pre-LN Transformer layers (d 1280,
+ * 20 heads x 64, FFN 5120) with windowed (block-diagonal) attention ->
+ * ln_post -> proj1 (1280->1280) -> GELU -> proj2 (1280->2048) -> SwiGLU
+ * adapter (2048->8192->2048).  The caller gets 12.5 rows per second of audio
+ * (page "Ossicle-4B", "Model Overview").
+ *
+ * Conventions for every call:
+ *  - Pointers documented as "device" must be device memory of the handle's
+ *    device; "host" pointers are ordinary (preferably pinned) host memory.
+ *  - Calls that take a handle enqueue their work on the handle's stream and
+ *    return without waiting, except where a call says it synchronises.  The
+ *    caller keeps device inputs alive and unmodified until the work is done.
+ *  - No call allocates device memory after moss_enc_create; a request larger
+ *    than the capacity fixed at create time returns MOSS_ENC_ERR_CAPACITY.
+ *  - No C++ exception crosses this interface.  A handle is used by one host
+ *    thread at a time.
+ *  - Errors found on the device (a bounded wait that timed out) are reported
+ *    by moss_enc_synchronize.
+ */
+#ifndef MOSS_ENC_H
+#define MOSS_ENC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOSS_ENC_OK = 0,
+    MOSS_ENC_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad size or range */
+    MOSS_ENC_ERR_CAPACITY = 2,       /* request exceeds the capacity set at create */
+    MOSS_ENC_ERR_OOM = 3,            /* device allocation failed inside create */
+    MOSS_ENC_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
+    MOSS_ENC_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait gave up */
+} moss_enc_status;
+
+typedef struct moss_enc moss_enc; /* opaque; owned by the library */
+
+/* Output element type of the embedding rows. */
+enum { MOSS_ENC_OUT_F32 = 0, MOSS_ENC_OUT_BF16 = 1 };
+
+/* Forward stages, for moss_enc_forward_stage (boundary checks). */
+enum {
+    MOSS_ENC_STAGE_STEM = 0,    /* after conv_out + positions: fp32 [T][1280] */
+    MOSS_ENC_STAGE_LAYERS = 1,  /* after the last layer, before ln_post: fp32 [T][1280] */
+    MOSS_ENC_STAGE_HEAD = 2,    /* after proj2: fp32 [T][2048] */
+    MOSS_ENC_STAGE_ADAPTER = 3  /* final rows: out_dtype [T][2048] (same as moss_enc_forward) */
+};
+
+typedef struct {
+    int n_layers;          /* 1..32 encoder layers held by the weight blob */
+    int64_t max_samples;   /* capacity: sum over clips of encoded samples per call */
+    int max_clips;         /* capacity: clips per call */
+    int out_dtype;         /* MOSS_ENC_OUT_F32 or MOSS_ENC_OUT_BF16 */
+} moss_enc_config;
+
+/* One clip (or one piece of a clip) to encode.
+ *  pcm        device, 16 kHz mono fp32, the WHOLE clip [n_samples].
+ *  n_samples  whole-clip length; reflect padding is applied only at sample 0
+ *             and at n_samples, so a piece sees its true neighbours.
+ *  begin,end  sample range to encode.  begin must be a multiple of 128000
+ *             (one 800-frame chunk = 8 s); end must equal n_samples or be a
+ *             multiple of 128000.  {0, n_samples} encodes the whole clip.
+ *  log_max    device pointer to the clip's log-mel maximum (the Whisper
+ *             floor is log_max - 8), or NULL to compute it over the whole
+ *             clip [0, n_samples).  Pieces of one long clip pass the value of
+ *             moss_enc_log_max so that every piece uses the same floor
+ *             (page "Ossicle-4B", "Long Audio": piece log-mel is identical
+ *             to the whole clip's). */
+typedef struct {
+    const float *pcm;
+    int64_t n_samples;
+    int64_t begin;
+    int64_t end;
+    const float *log_max;
+} moss_enc_clip;
+
+/* ---------------------------------------------------------------- sizes */
+
+/* bf16 elements in the weight blob for n_layers layers.  Blob order
+ * (PyTorch layouts, linear [out][in], conv [out][in][k_freq][k_time]):
+ *   conv1.w [480][1][3][3], conv1.b [480], conv2.w [480][480][3][3],
+ *   conv2.b, conv3.w, conv3.b, conv_out.w [1280][7680] (input index c*16+f,
+ *   no bias); per layer: ln1.g, ln1.b [1280], q.w [1280][1280], q.b, k.w,
+ *   k.b, v.w, v.b, o.w, o.b, ln2.g, ln2.b, fc1.w [5120][1280], fc1.b [5120],
+ *   fc2.w [1280][5120], fc2.b [1280]; then ln_post.g, ln_post.b,
+ *   proj1.w [1280][1280], proj1.b, proj2.w [2048][1280], proj2.b [2048],
+ *   gate.w [8192][2048], gate.b [8192], up.w [8192][2048], up.b [8192],
+ *   down.w [2048][8192], down.b [2048]. */
+int64_t moss_enc_weight_count(int n_layers);
+
+/* Mel frames of a clip: n_samples / 160 (Whisper drops the trailing STFT
+ * frame; page "MOSS-Transcribe-preview-2B - GGUF", gotcha 2).  Pure. */
+int64_t moss_enc_num_frames(int64_t n_samples);
+
+/* Output rows of a whole clip: the sum over 800-frame chunks of
+ * ceil(frames_in_chunk / 8) (three stride-2 convs).  Pure. */
+int64_t moss_enc_num_tokens(int64_t n_samples);
+
+/* Output rows of the sample range [begin, end) of a clip of n_samples
+ * (same alignment rules as moss_enc_clip).  Returns -1 on a bad range. */
+int64_t moss_enc_range_tokens(int64_t n_samples, int64_t begin, int64_t end);
+
+/* ------------------------------------------------------------- lifetime */
+
+/* Create a handle on the current CUDA device.
+ *  weights        bf16 blob (uint16 bit patterns) of moss_enc_weight_count
+ *                 (cfg->n_layers) elements; host or device memory as
+ *                 weights_on_device says.  The library copies and repacks
+ *                 it; the caller may free it when create returns.
+ *  bytes          size of the blob in bytes (checked).
+ *  stream         cudaStream_t to enqueue on (NULL = legacy default stream).
+ *  out            receives the handle.
+ * Synchronises.  Allocates the weights and a workspace sized from cfg. */
+moss_enc_status moss_enc_create(const moss_enc_config *cfg, const void *weights, size_t bytes,
+                                int weights_on_device, void *stream, moss_enc **out);
+
+/* Change the stream later calls enqueue on. */
+moss_enc_status moss_enc_set_stream(moss_enc *h, void *stream);
+
+/* Wait for the handle's stream; return MOSS_ENC_ERR_DEVICE_TIMEOUT if a kernel
+ * reported a timed-out wait since the last call (and clear the flag). */
+moss_enc_status moss_enc_synchronize(moss_enc *h);
+
+void moss_enc_destroy(moss_enc *h);
+
+const char *moss_enc_status_string(moss_enc_status s);
+
+/* Text of the last error on this handle ("" if none). */
+const char *moss_enc_last_error(const moss_enc *h);
+
+/* ---------------------------------------------------------------- compute */
+
+/* Whisper log-mel of one clip's range (page "MOSS-Transcribe-preview-2B -
+ * GGUF", "Architecture" table, Audio row; gotcha 2): frames t in
+ * [begin/160, end/160) (end == n_samples: n_samples/160), each centred on
+ * sample 160 t with reflect padding at the clip ends, periodic Hann 400,
+ * |rFFT|^2 (201 bins), Slaney mel 128 x 201 over 0-8 kHz, log10(max(., 1e-10)),
+ * floor at log_max - 8, then (x + 4) / 4.
+ *  mel_out      device fp32 [n_frames][128], frame-major.
+ *  n_frames     host, receives the frame count (may be NULL).
+ *  log_max_out  device float receiving the clip's log-mel maximum (may be NULL).
+ * The range must hold at most cfg.max_samples samples. */
+moss_enc_status moss_enc_logmel(moss_enc *h, const moss_enc_clip *clip, float *mel_out,
+                                int64_t *n_frames, float *log_max_out);
+
+/* Whole-clip log-mel maximum only (one pass, nothing else written).
+ *  pcm device [n_samples]; out device float.  Any length is accepted. */
+moss_enc_status moss_enc_log_max(moss_enc *h, const float *pcm, int64_t n_samples, float *out);
+
+/* Encode n_clips clips (or pieces) into embedding rows.
+ *  clips        host array [n_clips].
+ *  rows_out     device [sum of tokens][2048] of cfg.out_dtype; the rows of
+ *               clip i are rows row_offsets[i] .. row_offsets[i+1]-1.
+ *  row_offsets  host int64 [n_clips + 1], written before the call returns
+ *               (computed on the host, no synchronisation).
+ * Each clip is encoded independently: its 800-frame chunks are the conv
+ * stem's chunks (zero-padded at the tail) and the attention windows. */
+moss_enc_status moss_enc_forward(moss_enc *h, const moss_enc_clip *clips, int n_clips,
+                                 void *rows_out, int64_t *row_offsets);
+
+/* Like moss_enc_forward but stops after `stage` (MOSS_ENC_STAGE_*) and writes
+ * that boundary's rows (fp32 except the final stage) to out. */
+moss_enc_status moss_enc_forward_stage(moss_enc *h, const moss_enc_clip *clips, int n_clips,
+                                       int stage, void *out, int64_t *row_offsets);
+
+/* End-to-end from host memory: copies each clip's samples host->device,
+ * encodes, copies the rows device->host and synchronises.
+ *  pcm_host     host array of n_clips pointers to fp32 [n_samples[i]].
+ *  n_samples    host [n_clips].
+ *  rows_host    host [sum of tokens][2048] of cfg.out_dtype.
+ *  row_offsets  host [n_clips + 1].
+ * Whole clips only; the sum of n_samples must fit cfg.max_samples. */
+moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host,
+                                      const int64_t *n_samples, int n_clips, void *rows_host,
+                                      int64_t *row_offsets);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOSS_ENC_H */

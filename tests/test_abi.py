@@ -1,0 +1,71 @@
+"""The C-ABI library loads and exports every symbol its header declares;
+the pure host functions agree with the oracle's counts.  No GPU needed."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from audio_encoder_b200 import binding, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "moss_enc.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moss_enc_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_calls():
+    syms = declared_symbols()
+    for s in ["moss_enc_create", "moss_enc_logmel", "moss_enc_forward", "moss_enc_destroy"]:
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol():
+    L = binding.lib()
+    for s in declared_symbols():
+        assert hasattr(L, s), s
+    assert set(declared_symbols()) <= set(binding.EXPORTED)
+
+
+def test_weight_count_matches_generator_and_oracle():
+    for n in [1, 4, 32]:
+        _, total = synth.weight_offsets(n)
+        assert binding.weight_count(n) == total == oracle.weight_count(n)
+
+
+@pytest.mark.parametrize("n", [0, 1, 159, 160, 161, 16000, 16159, 127999, 128000, 128160, 480000,
+                               9_600_000, 57_600_000, 1_024_000, 160 * 801])
+def test_counts_match_oracle(n):
+    assert binding.num_frames(n) == oracle.num_frames(n)
+    assert binding.num_tokens(n) == oracle.num_tokens(n)
+
+
+def test_range_tokens_add_up_over_pieces():
+    n = 57_600_000
+    piece = 1_024_000
+    total = sum(binding.range_tokens(n, b, min(b + piece, n)) for b in range(0, n, piece))
+    assert total == binding.num_tokens(n) == 45000
+    assert binding.range_tokens(n, 0, n) == 45000
+    assert binding.range_tokens(n, 1000, n) == -1          # begin not chunk-aligned
+    assert binding.range_tokens(n, 0, 1000) == -1          # end neither n nor aligned
+    assert binding.range_tokens(n, 128000, 128000) == 0
+
+
+def test_create_rejects_bad_arguments_before_touching_a_device():
+    import ctypes
+    L = binding.lib()
+    h = ctypes.c_void_p()
+    cfg = binding.Config(0, 1000, 1, 0)  # n_layers 0
+    blob = np.zeros(4, dtype=np.uint16)
+    st = L.moss_enc_create(ctypes.byref(cfg), blob.ctypes.data_as(ctypes.c_void_p), 8, 0, None, ctypes.byref(h))
+    assert st == 1 and not h.value
+    assert L.moss_enc_create(None, None, 0, 0, None, ctypes.byref(h)) == 1
+    cfg = binding.Config(4, 1000, 1, 0)
+    st = L.moss_enc_create(ctypes.byref(cfg), blob.ctypes.data_as(ctypes.c_void_p), 8, 0, None, ctypes.byref(h))
+    assert st == 1  # blob size does not match 4 layers
+    assert L.moss_enc_status_string(2) == b"request exceeds capacity"

@@ -1,0 +1,261 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Small cases are compared whole, element by element (mel) or row by row
+(embeddings).  The full-size workloads run on the GPU in the launch
+configuration the benchmark times and are compared on sampled windows the
+oracle computes one by one (every 800-frame chunk is independent given the
+clip's log-mel maximum)."""
+import numpy as np
+import pytest
+
+import oracle
+from audio_encoder_b200 import binding, synth
+from conftest import oracle_model, weights
+from metrics import MEL_ATOL, assert_rows_close
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+_ENC = {}
+
+
+def encoder(n_layers, max_samples, max_clips=1, out_dtype=binding.OUT_F32):
+    key = (n_layers, max_samples, max_clips, out_dtype)
+    if key not in _ENC:
+        for k in list(_ENC):
+            if k[0] != n_layers or k[1] * k[2] > 4 * 10**8:
+                _ENC.pop(k).close()
+        _ENC[key] = binding.Encoder(weights(n_layers), n_layers, max_samples, max_clips, out_dtype)
+    return _ENC[key]
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+
+
+# ------------------------------------------------------------------ log-mel
+
+@pytest.mark.parametrize("n", [170, 400, 16000, 16001, 16159, 48000 + 77, 480000])
+def test_logmel_matches_oracle(n):
+    enc = encoder(1, 600_000)
+    pcm = synth.pcm_30s(1, n) if n == 480000 else synth.pcm_tones(n % 97, n)
+    mel, mx = enc.logmel(dev(pcm))
+    ref, rmx = oracle.logmel(pcm)
+    torch.cuda.synchronize()
+    assert mel.shape == ref.shape == (n // 160, 128)
+    assert abs(float(mx.item()) - rmx) < 1e-4
+    np.testing.assert_allclose(mel.cpu().numpy(), ref, rtol=0, atol=MEL_ATOL)
+
+
+def test_logmel_silence_and_empty():
+    enc = encoder(1, 600_000)
+    mel, mx = enc.logmel(dev(np.zeros(3200, np.float32)))
+    np.testing.assert_array_equal(mel.cpu().numpy(), np.full((20, 128), -1.5, np.float32))
+    mel, _ = enc.logmel(dev(np.zeros(100, np.float32) + 0.1))
+    assert mel.shape == (0, 128)
+
+
+def test_logmel_range_uses_whole_clip_max():
+    enc = encoder(1, 600_000)
+    n = 128000 * 3 + 5000
+    pcm = synth.pcm_long(4, n)
+    whole, mx = enc.logmel(dev(pcm))
+    part, mx2 = enc.logmel(dev(pcm), 128000, 256000)
+    torch.cuda.synchronize()
+    assert float(mx.item()) == float(mx2.item())
+    np.testing.assert_array_equal(part.cpu().numpy(), whole.cpu().numpy()[800:1600])
+
+
+def test_logmel_10min_bandwidth_workload():
+    # the full 10-min clip in the benchmark's configuration, checked against
+    # oracle frames sampled across it (start, the 2 s tone changes, the end)
+    enc = encoder(1, 9_600_000)
+    pcm = synth.pcm_long(2, 9_600_000)
+    mel, mx = enc.logmel(dev(pcm))
+    gmax = oracle.clip_log_max(pcm)
+    assert abs(float(mx.item()) - gmax) < 1e-4
+    m = mel.cpu().numpy()
+    for f0 in [0, 199, 30000, 59968]:
+        ref = oracle.normalize(oracle.logmel_raw(pcm, f0, f0 + 32), gmax)
+        np.testing.assert_allclose(m[f0:f0 + 32], ref, rtol=0, atol=MEL_ATOL)
+
+
+# ---------------------------------------------------------- module boundaries
+
+@pytest.fixture(scope="module")
+def tiny_case():
+    pcm = synth.pcm_tones(0, 16000)
+    out, d = oracle_model(4).encode(pcm, dumps=True)
+    return pcm, out, d
+
+
+def test_tiny_stem_boundary(tiny_case):
+    pcm, _, d = tiny_case
+    enc = encoder(4, 600_000)
+    x, offs = enc.forward([dev(pcm)], stage=binding.STAGE_STEM)
+    assert offs == [0, 13]
+    assert_rows_close(x.cpu().numpy(), d["stem"], "post-stem")
+
+
+def test_tiny_layers_boundary(tiny_case):
+    pcm, _, d = tiny_case
+    enc = encoder(4, 600_000)
+    x, _ = enc.forward([dev(pcm)], stage=binding.STAGE_LAYERS)
+    assert_rows_close(x.cpu().numpy(), d["enc"], "after 4 layers")
+
+
+def test_tiny_head_boundary(tiny_case):
+    pcm, _, d = tiny_case
+    enc = encoder(4, 600_000)
+    x, _ = enc.forward([dev(pcm)], stage=binding.STAGE_HEAD)
+    assert_rows_close(x.cpu().numpy(), d["head"], "after proj2")
+
+
+def test_tiny_final_rows(tiny_case):
+    pcm, out, _ = tiny_case
+    enc = encoder(4, 600_000)
+    y, offs = enc.forward([dev(pcm)])
+    assert y.shape == (13, 2048) and offs == [0, 13]
+    assert_rows_close(y.cpu().numpy(), out, "tiny rows")
+
+
+def test_one_layer_from_oracle_stem():
+    # layer 0 alone (conv + windowed attention), three chunks with a ragged tail
+    n = 128000 * 2 + 40000
+    pcm = synth.pcm_tones(21, n)
+    om = oracle_model(1)
+    ref, d = om.encode(pcm, dumps=True)
+    enc = encoder(1, 600_000)
+    x, offs = enc.forward([dev(pcm)], stage=binding.STAGE_LAYERS)
+    assert offs == [0, oracle.num_tokens(n)]
+    assert_rows_close(x.cpu().numpy(), d["enc"], "after layer 0")
+    y, _ = enc.forward([dev(pcm)])
+    assert_rows_close(y.cpu().numpy(), ref, "1-layer rows")
+
+
+def test_bf16_output_matches_f32_output(tiny_case):
+    pcm, out, _ = tiny_case
+    enc = encoder(4, 600_000, out_dtype=binding.OUT_BF16)
+    y, _ = enc.forward([dev(pcm)])
+    assert y.dtype == torch.bfloat16
+    assert_rows_close(y.float().cpu().numpy(), out, "bf16 rows")
+
+
+# ------------------------------------------------------- full-size workloads
+
+def test_single_30s_clip_full():
+    pcm = synth.pcm_30s(1)
+    enc = encoder(32, 9_600_000, 16)
+    y, offs = enc.forward([dev(pcm)])
+    assert offs == [0, 375] and y.shape == (375, 2048)
+    ref = oracle_model(32).encode(pcm)
+    assert_rows_close(y.cpu().numpy(), ref, "30 s rows")
+
+
+def test_batch16_sampled_windows_and_invariance():
+    clips = synth.pcm_batch(16)
+    enc = encoder(32, 9_600_000, 16)
+    y, offs = enc.forward([dev(c) for c in clips])
+    assert offs[-1] == sum(oracle.num_tokens(c.size) for c in clips)
+    Y = y.cpu().numpy()
+    om = oracle_model(32)
+    for i, c in [(0, 0), (7, None), (15, 1)]:
+        pcm = clips[i]
+        nc = oracle.num_chunks(pcm.size)
+        c = nc - 1 if c is None else c
+        ref = om.encode_chunks(pcm, c, c + 1)
+        t0 = offs[i] + 100 * c
+        assert_rows_close(Y[t0:t0 + ref.shape[0]], ref, f"clip {i} chunk {c}")
+    # a clip encoded alone gives the same rows as inside the batch
+    for i in [3, 15]:
+        yi, _ = enc.forward([dev(clips[i])])
+        np.testing.assert_array_equal(yi.cpu().numpy(), Y[offs[i]:offs[i + 1]])
+
+
+def test_10min_clip_sampled_windows():
+    pcm = synth.pcm_long(2, 9_600_000)
+    enc = encoder(32, 9_600_000, 16)
+    y, offs = enc.forward([dev(pcm)])
+    assert offs == [0, 7500]
+    Y = y.cpu().numpy()
+    om = oracle_model(32)
+    gmax = oracle.clip_log_max(pcm)
+    for c in [0, 37, 74]:
+        ref = om.encode_chunks(pcm, c, c + 1, gmax=gmax)
+        assert_rows_close(Y[100 * c:100 * c + 100], ref, f"10-min window {c}")
+
+
+def test_60min_streamed_equals_whole_clip_and_oracle():
+    n = 57_600_000
+    pcm = synth.pcm_long(3, n)
+    enc = encoder(32, 57_600_000, 1)
+    x = dev(pcm)
+    whole, offs = enc.forward([x])
+    assert offs == [0, 45000]
+    lm = enc.log_max(x)
+    piece = 1_024_000
+    rows = []
+    for b in range(0, n, piece):
+        e = min(b + piece, n)
+        y, o = enc.forward([(x, b, e, lm)])
+        assert o[1] == (800 if e - b == piece else 200)
+        rows.append(y)
+    streamed = torch.cat(rows)
+    torch.cuda.synchronize()
+    W = whole.cpu().numpy()
+    assert_rows_close(streamed.cpu().numpy(), W, "streamed vs whole")
+    om = oracle_model(32)
+    gmax = oracle.clip_log_max(pcm)
+    assert abs(float(lm.item()) - gmax) < 1e-4
+    for c in [0, 79, 80, 449]:
+        ref = om.encode_chunks(pcm, c, c + 1, gmax=gmax)
+        assert_rows_close(W[100 * c:100 * c + ref.shape[0]], ref, f"60-min window {c}")
+
+
+# ---------------------------------------------------------------- edge cases
+
+def test_ragged_batch_with_empty_and_tiny_clips():
+    enc = encoder(4, 600_000, 8)
+    lens = [0, 170, 16000, 128000, 128160, 100]
+    clips = [synth.pcm_tones(30 + i, n) for i, n in enumerate(lens)]
+    y, offs = enc.forward([dev(c) if c.size else torch.empty(0, device="cuda") for c in clips])
+    assert offs == list(np.cumsum([0] + [oracle.num_tokens(n) for n in lens]))
+    om = oracle_model(4)
+    Y = y.cpu().numpy()
+    for i, c in enumerate(clips):
+        ref = om.encode(c)
+        assert_rows_close(Y[offs[i]:offs[i + 1]], ref, f"clip of {lens[i]} samples")
+
+
+def test_deterministic_and_prompt_independent(tiny_case):
+    pcm, _, _ = tiny_case
+    enc = encoder(4, 600_000)
+    a, _ = enc.forward([dev(pcm)])
+    b, _ = enc.forward([dev(pcm)])
+    assert torch.equal(a, b)
+
+
+def test_host_end_to_end_matches_device_path(tiny_case):
+    pcm, _, _ = tiny_case
+    enc = encoder(4, 600_000, 4)
+    clips = [pcm, synth.pcm_tones(5, 30000)]
+    yd, od = enc.forward([dev(c) for c in clips])
+    yh, oh = enc.forward_host(clips)
+    assert od == oh
+    np.testing.assert_array_equal(yh, yd.cpu().numpy())
+
+
+def test_capacity_and_range_errors():
+    enc = encoder(4, 600_000, 2)
+    x = dev(synth.pcm_tones(1, 700_000))
+    with pytest.raises(binding.MossEncError) as e:
+        enc.forward([x])
+    assert e.value.status == 2
+    with pytest.raises(binding.MossEncError) as e:
+        enc.forward([(x, 1000, 700_000, None)])
+    assert e.value.status == 1
+    with pytest.raises(binding.MossEncError) as e:
+        enc.forward([x[:1000]] * 3)
+    assert e.value.status == 2
+    enc.synchronize()
