@@ -7,7 +7,6 @@ loudly if ``libmoss_enc.so`` has not been built; there is no fallback.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 import numpy as np
@@ -27,6 +26,7 @@ EXPORTED = [
     "moss_enc_create", "moss_enc_set_stream", "moss_enc_synchronize", "moss_enc_destroy",
     "moss_enc_status_string", "moss_enc_last_error", "moss_enc_logmel", "moss_enc_log_max",
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
+    "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
 ]
 
 
@@ -39,6 +39,11 @@ class MossEncError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int), ("max_samples", ctypes.c_int64),
                 ("max_clips", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 class Clip(ctypes.Structure):
@@ -88,6 +93,12 @@ def lib():
         L.moss_enc_forward_host.restype = i32
         L.moss_enc_forward_host.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(i64), i32, vp,
                                             ctypes.POINTER(i64)]
+        L.moss_enc_profile_enable.restype = i32
+        L.moss_enc_profile_enable.argtypes = [vp, i32]
+        L.moss_enc_profile_read.restype = i32
+        L.moss_enc_profile_read.argtypes = [vp, ctypes.POINTER(KernelStat), i32]
+        L.moss_enc_launch_count.restype = i64
+        L.moss_enc_launch_count.argtypes = [vp]
         _lib = L
     return _lib
 
@@ -165,6 +176,21 @@ class Encoder:
     def synchronize(self):
         self._check(lib().moss_enc_synchronize(self.h))
 
+    def profile_enable(self, max_launches: int):
+        self._check(lib().moss_enc_profile_enable(self.h, int(max_launches)))
+
+    def profile_read(self):
+        """{category: dict(launches, ms, flops, bytes)} since the last read."""
+        arr = (KernelStat * 64)()
+        n = lib().moss_enc_profile_read(self.h, arr, 64)
+        if n < 0:
+            raise MossEncError(4, "profile_read failed")
+        return {arr[i].name.decode(): dict(launches=arr[i].launches, ms=arr[i].ms, flops=arr[i].flops,
+                                           bytes=arr[i].bytes) for i in range(n)}
+
+    def launch_count(self) -> int:
+        return int(lib().moss_enc_launch_count(self.h))
+
     @staticmethod
     def _clip(pcm, begin=0, end=None, log_max=None):
         n = pcm.numel()
@@ -199,7 +225,7 @@ class Encoder:
                 pcm, begin, end, lm = (list(c) + [None, None, None])[:4]
                 n = pcm.numel()
                 arr[i] = self._clip(pcm, begin or 0, n if end is None else end, lm)
-                total += range_tokens(n, begin or 0, n if end is None else end)
+                total += max(0, range_tokens(n, begin or 0, n if end is None else end))
             else:
                 arr[i] = self._clip(c)
                 total += num_tokens(c.numel())

@@ -75,7 +75,44 @@ struct moss_enc {
     size_t tab_bytes = 0;
     void *d_tab = nullptr, *h_tab = nullptr;
     cudaEvent_t tab_event = nullptr;
+
+    // measurement: launch counter and optional per-launch CUDA events
+    int64_t launches = 0;
+    bool profiling = false;
+    struct Rec {
+        const char *name;
+        int e0;
+        double flops, bytes;
+    };
+    std::vector<cudaEvent_t> prof_ev;
+    std::vector<Rec> prof_rec;
 };
+
+namespace {
+// Counts one kernel launch and, while profiling, brackets it with events.
+struct Launch {
+    moss_enc *h;
+    const char *name;
+    double flops, bytes;
+    int e0 = -1;
+    Launch(moss_enc *h_, const char *name_, double flops_, double bytes_)
+        : h(h_), name(name_), flops(flops_), bytes(bytes_)
+    {
+        h->launches++;
+        if (h->profiling && h->prof_rec.size() * 2 + 2 <= h->prof_ev.size()) {
+            e0 = (int)h->prof_rec.size() * 2;
+            cudaEventRecord(h->prof_ev[e0], h->stream);
+        }
+    }
+    ~Launch()
+    {
+        if (e0 >= 0) {
+            cudaEventRecord(h->prof_ev[e0 + 1], h->stream);
+            h->prof_rec.push_back(moss_enc::Rec{name, e0, flops, bytes});
+        }
+    }
+};
+}  // namespace
 
 // ------------------------------------------------------------ small helpers
 
@@ -127,8 +164,16 @@ static bool tmap_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t ro
     return r == CUDA_SUCCESS;
 }
 
+// Output bytes per element for the epilogue kinds (for the byte count).
+static double epi_out_bytes(int epi)
+{
+    return epi == EPI_RESID_F32 ? 8.0 : (epi == EPI_F32 || epi == EPI_CONVOUT_F32) ? 4.0 : epi == EPI_SWIGLU_BF16 ? 1.0 : 2.0;
+}
+
+// k_alg: the contraction length the method needs (padding excluded).
 template <int BN, int EPI>
-static moss_enc_status gemm(moss_enc *h, const bf16 *A, int64_t M, int K, const bf16 *B, int N, GemmArgs a)
+static moss_enc_status gemm(moss_enc *h, const char *name, const bf16 *A, int64_t M, int K, const bf16 *B, int N,
+                            GemmArgs a, int k_alg = 0)
 {
     if (M <= 0) return MOSS_ENC_OK;
     if (K % 64 != 0 || N % BN != 0 || M > INT32_MAX)
@@ -145,6 +190,8 @@ static moss_enc_status gemm(moss_enc *h, const bf16 *A, int64_t M, int K, const 
     a.err = h->err;
     const int tiles = a.m_tiles * a.n_tiles;
     const int grid = std::min(tiles, h->num_sms);
+    const double ka = k_alg > 0 ? k_alg : K;
+    Launch L(h, name, 2.0 * M * N * ka, 2.0 * M * ka + 2.0 * N * ka + epi_out_bytes(EPI) * M * N);
     gemm_tc_kernel<BN, EPI><<<grid, 192, GemmCfg<BN>::SMEM, h->stream>>>(ta, tb, a);
     CUDA_TRY(h, cudaGetLastError());
     return MOSS_ENC_OK;
@@ -322,6 +369,7 @@ extern "C" void moss_enc_destroy(moss_enc *h)
     if (h->d_tab) cudaFree(h->d_tab);
     if (h->h_tab) cudaFreeHost(h->h_tab);
     if (h->tab_event) cudaEventDestroy(h->tab_event);
+    for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
     delete h;
 }
 
@@ -656,10 +704,11 @@ static moss_enc_status tab_upload(moss_enc *h)
 static int mel_grid_x(int64_t max_frames) { return (int)std::max<int64_t>(1, (max_frames + MEL_FRAMES_PER_BLOCK - 1) / MEL_FRAMES_PER_BLOCK); }
 
 static moss_enc_status launch_logmel(moss_enc *h, const MelClip *d_clips, int n_clips, int64_t max_frames,
-                                     float *out, int write_out)
+                                     float *out, int write_out, int64_t total_frames)
 {
     if (n_clips <= 0 || max_frames <= 0) return MOSS_ENC_OK;
     dim3 grid(mel_grid_x(max_frames), n_clips);
+    Launch L(h, write_out ? "logmel" : "logmel_max", 0.0, 4.0 * 160 * (double)total_frames + (write_out ? 512.0 * total_frames : 0.0));
     logmel_kernel<<<grid, 256, sizeof(MelSmem), h->stream>>>(d_clips, h->mel_tab, out, h->gmax_ord, write_out);
     CUDA_TRY(h, cudaGetLastError());
     return MOSS_ENC_OK;
@@ -680,10 +729,16 @@ extern "C" moss_enc_status moss_enc_log_max(moss_enc *h, const float *pcm, int64
     mc[0] = MelClip{pcm, (long long)n_samples, 0, 0, (int)(n_samples / HOP), 0, 0};
     TRY(tab_upload(h));
     uint8_t *Dt = static_cast<uint8_t *>(h->d_tab);
-    gmax_init_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), 1);
+    {
+        Launch Lk(h, "gmax", 0.0, 0.0);
+        gmax_init_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), 1);
+    }
     CUDA_TRY(h, cudaGetLastError());
-    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), 1, n_samples / HOP, nullptr, 0));
-    gmax_export_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, out);
+    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), 1, n_samples / HOP, nullptr, 0, n_samples / HOP));
+    {
+        Launch Lk(h, "gmax", 0.0, 0.0);
+        gmax_export_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, out);
+    }
     CUDA_TRY(h, cudaGetLastError());
     return MOSS_ENC_OK;
 }
@@ -711,17 +766,26 @@ extern "C" moss_enc_status moss_enc_logmel(moss_enc *h, const moss_enc_clip *cli
     mx[0] = MelClip{clip->pcm, (long long)pl.n, 0, 0, (int)pl.F, 0, 0};
     TRY(tab_upload(h));
     uint8_t *Dt = static_cast<uint8_t *>(h->d_tab);
-    gmax_init_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), 1);
+    {
+        Launch Lk(h, "gmax", 0.0, 0.0);
+        gmax_init_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), 1);
+    }
     CUDA_TRY(h, cudaGetLastError());
     if (own_max && !whole)
-        TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), 1, pl.F, nullptr, 0));
-    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_main), 1, nf, mel_out, 1));
+        TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), 1, pl.F, nullptr, 0, pl.F));
+    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_main), 1, nf, mel_out, 1, nf));
     if (nf > 0) {
-        mel_normalize_kernel<<<std::min<int64_t>(4096, (nf * 128 + 255) / 256), 256, 0, h->stream>>>(mel_out, nf * 128, h->gmax_ord);
+        {
+            Launch Lk(h, "mel_normalize", 0.0, 8.0 * nf * 128);
+            mel_normalize_kernel<<<std::min<int64_t>(4096, (nf * 128 + 255) / 256), 256, 0, h->stream>>>(mel_out, nf * 128, h->gmax_ord);
+        }
         CUDA_TRY(h, cudaGetLastError());
     }
     if (log_max_out) {
-        gmax_export_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, log_max_out);
+        {
+            Launch Lk(h, "gmax", 0.0, 0.0);
+            gmax_export_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, log_max_out);
+        }
         CUDA_TRY(h, cudaGetLastError());
     }
     return MOSS_ENC_OK;
@@ -768,7 +832,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     StemChunk *sc = reinterpret_cast<StemChunk *>(H + tl.chunks);
     int2 *ct = reinterpret_cast<int2 *>(H + tl.chunk_tok);
     int n_max_pass = 0;
-    int64_t chunk = 0;
+    int64_t chunk = 0, max_pass_frames = 0, range_frames = 0;
     for (int i = 0; i < n_clips; i++) {
         const ClipPlan &pl = plans[i];
         const bool whole = pl.f_begin == 0 && pl.f_end == pl.F;
@@ -778,7 +842,11 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         const int64_t fb = pl.c_first * CHUNK_FRAMES;
         mm[i] = MelClip{clips[i].pcm, (long long)pl.n, (long long)chunk * CHUNK_FRAMES, (int)fb, (int)pl.f_end,
                         own && whole ? i : -1, 0};
-        if (own && !whole) mx[n_max_pass++] = MelClip{clips[i].pcm, (long long)pl.n, 0, 0, (int)pl.F, i, 0};
+        if (own && !whole) {
+            mx[n_max_pass++] = MelClip{clips[i].pcm, (long long)pl.n, 0, 0, (int)pl.F, i, 0};
+            max_pass_frames += pl.F;
+        }
+        range_frames += pl.f_end - fb;
         int64_t tok = pl.tok0;
         for (int64_t c = pl.c_first; c < pl.c_last; c++, chunk++) {
             const int nf = (int)std::min<int64_t>(CHUNK_FRAMES, pl.F - c * CHUNK_FRAMES);
@@ -794,36 +862,48 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     const int2 *d_ct = reinterpret_cast<const int2 *>(Dt + tl.chunk_tok);
 
     // ---- log-mel (raw) and per-clip maxima
-    gmax_init_kernel<<<(n_clips + 127) / 128, 128, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), n_clips);
+    {
+        Launch Lk(h, "gmax", 0.0, 0.0);
+        gmax_init_kernel<<<(n_clips + 127) / 128, 128, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), n_clips);
+    }
     CUDA_TRY(h, cudaGetLastError());
     if (n_max_pass > 0)
-        TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), n_max_pass, max_clip_frames, nullptr, 0));
-    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_main), n_clips, max_range_frames, h->mel_raw, 1));
+        TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), n_max_pass, max_clip_frames, nullptr, 0, max_pass_frames));
+    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_main), n_clips, max_range_frames, h->mel_raw, 1, range_frames));
 
     // ---- conv stem, in groups of chunks
     for (int64_t g0 = 0; g0 < n_chunks; g0 += h->stem_group) {
         const int gc = (int)std::min<int64_t>(h->stem_group, n_chunks - g0);
+        {
+        Launch L1(h, "conv1", 2.0 * 9 * CST * 400 * 64 * gc, 2.0 * CST * 400 * 64 * gc + 4.0 * 128 * 800 * gc);
         conv1_kernel<<<dim3(400, gc), 240, 0, h->stream>>>(h->mel_raw, d_chunks + g0, h->gmax_ord, h->conv1_w, h->conv1_b, h->c1out);
         CUDA_TRY(h, cudaGetLastError());
+        }
         const int64_t r2 = (int64_t)gc * 6400, r3 = (int64_t)gc * 1600;
+        {
+        Launch L2(h, "im2col", 0.0, 2.0 * r2 * CONV_K + 2.0 * CST * 400 * 64 * gc);
         im2col_s2_kernel<<<(int)std::min<int64_t>(65535, (r2 * 576 + 255) / 256), 256, 0, h->stream>>>(h->c1out, 400, 64, r2, h->a2);
         CUDA_TRY(h, cudaGetLastError());
+        }
         GemmArgs a{};
         a.bias = h->conv2_b;
         a.out = h->c2out;
         a.ldo = CST;
-        TRY((gemm<160, EPI_GELU_BF16>(h, h->a2, r2, CONV_K, h->conv2_w, CST, a)));
+        TRY((gemm<160, EPI_GELU_BF16>(h, "gemm_conv2", h->a2, r2, CONV_K, h->conv2_w, CST, a, 9 * CST)));
+        {
+        Launch L3(h, "im2col", 0.0, 2.0 * r3 * CONV_K + 2.0 * CST * 200 * 32 * gc);
         im2col_s2_kernel<<<(int)std::min<int64_t>(65535, (r3 * 576 + 255) / 256), 256, 0, h->stream>>>(h->c2out, 200, 32, r3, h->a3);
         CUDA_TRY(h, cudaGetLastError());
+        }
         a.bias = h->conv3_b;
         a.out = h->c3out;
-        TRY((gemm<160, EPI_GELU_BF16>(h, h->a3, r3, CONV_K, h->conv3_w, CST, a)));
+        TRY((gemm<160, EPI_GELU_BF16>(h, "gemm_conv3", h->a3, r3, CONV_K, h->conv3_w, CST, a, 9 * CST)));
         GemmArgs co{};
         co.out = h->X;
         co.ldo = D;
         co.pos = h->pos;
         co.chunk_tok = d_ct + g0;
-        TRY((gemm<128, EPI_CONVOUT_F32>(h, h->c3out, (int64_t)gc * 100, 7680, h->conv_out_w, D, co)));
+        TRY((gemm<128, EPI_CONVOUT_F32>(h, "gemm_conv_out", h->c3out, (int64_t)gc * 100, 7680, h->conv_out_w, D, co)));
     }
     if (stage == MOSS_ENC_STAGE_STEM) {
         CUDA_TRY(h, cudaMemcpyAsync(out, h->X, sizeof(float) * T * D, cudaMemcpyDeviceToDevice, h->stream));
@@ -832,31 +912,42 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
 
     // ---- Transformer layers
     const int ln_grid = (int)((T + 7) / 8);
+    double attn_pairs = 0.0;  // query-key pairs inside windows
+    for (int64_t c = 0; c < n_chunks; c++) attn_pairs += (double)ct[c].y * ct[c].y;
     for (size_t l = 0; l < h->layers.size(); l++) {
         const LayerDev &L = h->layers[l];
-        layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln1_g, L.ln1_b, h->xn, (int)T);
+        {
+            Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
+            layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln1_g, L.ln1_b, h->xn, (int)T);
+        }
         CUDA_TRY(h, cudaGetLastError());
         GemmArgs a{};
         a.bias = L.bqkv;
         a.out = h->qkv;
         a.ldo = DQKV;
-        TRY((gemm<256, EPI_BF16>(h, h->xn, T, D, L.wqkv, DQKV, a)));
-        window_attn_kernel<<<dim3((unsigned)n_chunks, 20), 256, ATTN_SMEM, h->stream>>>(h->qkv, d_ct, h->attn);
+        TRY((gemm<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
+        {
+            Launch Lk(h, "attention", 4.0 * 64 * 20 * attn_pairs, 2.0 * T * (DQKV + D));
+            window_attn_kernel<<<dim3((unsigned)n_chunks, 20), 256, ATTN_SMEM, h->stream>>>(h->qkv, d_ct, h->attn);
+        }
         CUDA_TRY(h, cudaGetLastError());
         a.bias = L.bo;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm<128, EPI_RESID_F32>(h, h->attn, T, D, L.wo, D, a)));
-        layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln2_g, L.ln2_b, h->xn, (int)T);
+        TRY((gemm<128, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a)));
+        {
+            Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
+            layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln2_g, L.ln2_b, h->xn, (int)T);
+        }
         CUDA_TRY(h, cudaGetLastError());
         a.bias = L.b1;
         a.out = h->ffn;
         a.ldo = DFF;
-        TRY((gemm<256, EPI_GELU_BF16>(h, h->xn, T, D, L.w1, DFF, a)));
+        TRY((gemm<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.w1, DFF, a)));
         a.bias = L.b2;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm<128, EPI_RESID_F32>(h, h->ffn, T, DFF, L.w2, D, a)));
+        TRY((gemm<128, EPI_RESID_F32>(h, "gemm_fc2", h->ffn, T, DFF, L.w2, D, a)));
     }
     if (stage == MOSS_ENC_STAGE_LAYERS) {
         CUDA_TRY(h, cudaMemcpyAsync(out, h->X, sizeof(float) * T * D, cudaMemcpyDeviceToDevice, h->stream));
@@ -864,31 +955,34 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     }
 
     // ---- head: ln_post -> proj1 -> GELU -> proj2
-    layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, h->lnp_g, h->lnp_b, h->xn, (int)T);
+    {
+        Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
+        layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, h->lnp_g, h->lnp_b, h->xn, (int)T);
+    }
     CUDA_TRY(h, cudaGetLastError());
     GemmArgs a{};
     a.bias = h->bp1;
     a.out = h->hb;
     a.ldo = D;
-    TRY((gemm<128, EPI_GELU_BF16>(h, h->xn, T, D, h->wp1, D, a)));
+    TRY((gemm<128, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, D, h->wp1, D, a)));
     a.bias = h->bp2;
     a.ldo = DOUT;
     if (stage == MOSS_ENC_STAGE_HEAD) {
         a.out = out;
-        return gemm<256, EPI_F32>(h, h->hb, T, D, h->wp2, DOUT, a);
+        return gemm<256, EPI_F32>(h, "gemm_proj2", h->hb, T, D, h->wp2, DOUT, a);
     }
     a.out = h->h2;
-    TRY((gemm<256, EPI_BF16>(h, h->hb, T, D, h->wp2, DOUT, a)));
+    TRY((gemm<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, D, h->wp2, DOUT, a)));
     // ---- SwiGLU adapter
     a.bias = h->bgu;
     a.out = h->gu;
     a.ldo = DADP;
-    TRY((gemm<256, EPI_SWIGLU_BF16>(h, h->h2, T, DOUT, h->wgu, 2 * DADP, a)));
+    TRY((gemm<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, h->wgu, 2 * DADP, a)));
     a.bias = h->bd;
     a.out = out;
     a.ldo = DOUT;
-    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm<128, EPI_F32>(h, h->gu, T, DADP, h->wd, DOUT, a);
-    return gemm<128, EPI_BF16>(h, h->gu, T, DADP, h->wd, DOUT, a);
+    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm<128, EPI_F32>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
+    return gemm<128, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
 }
 
 extern "C" moss_enc_status moss_enc_forward(moss_enc *h, const moss_enc_clip *clips, int n_clips, void *rows_out,
@@ -933,3 +1027,51 @@ extern "C" moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const
     }
     return moss_enc_synchronize(h);
 }
+
+// ------------------------------------------------------------- measurement
+
+extern "C" moss_enc_status moss_enc_profile_enable(moss_enc *h, int max_launches)
+{
+    if (!h || max_launches < 0) return MOSS_ENC_ERR_INVALID_ARG;
+    CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+    for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
+    h->prof_ev.clear();
+    h->prof_rec.clear();
+    h->profiling = max_launches > 0;
+    for (int i = 0; i < 2 * max_launches; i++) {
+        cudaEvent_t e;
+        CUDA_TRY(h, cudaEventCreate(&e));
+        h->prof_ev.push_back(e);
+    }
+    h->prof_rec.reserve(max_launches);
+    return MOSS_ENC_OK;
+}
+
+extern "C" int moss_enc_profile_read(moss_enc *h, moss_enc_kernel_stat *out, int max)
+{
+    if (!h || (max > 0 && !out)) return -1;
+    if (cudaStreamSynchronize(h->stream) != cudaSuccess) return -1;
+    std::vector<moss_enc_kernel_stat> agg;
+    for (const auto &r : h->prof_rec) {
+        float ms = 0.0f;
+        if (cudaEventElapsedTime(&ms, h->prof_ev[r.e0], h->prof_ev[r.e0 + 1]) != cudaSuccess) return -1;
+        moss_enc_kernel_stat *st = nullptr;
+        for (auto &a : agg)
+            if (std::strncmp(a.name, r.name, sizeof(a.name)) == 0) st = &a;
+        if (!st) {
+            agg.push_back(moss_enc_kernel_stat{});
+            st = &agg.back();
+            std::strncpy(st->name, r.name, sizeof(st->name) - 1);
+        }
+        st->launches++;
+        st->ms += ms;
+        st->flops += r.flops;
+        st->bytes += r.bytes;
+    }
+    h->prof_rec.clear();
+    const int n = (int)std::min<size_t>(agg.size(), (size_t)std::max(max, 0));
+    for (int i = 0; i < n; i++) out[i] = agg[i];
+    return n;
+}
+
+extern "C" int64_t moss_enc_launch_count(const moss_enc *h) { return h ? h->launches : -1; }

@@ -1,0 +1,363 @@
+"""Throughput of the B200 audio-encoder forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload batch16_10to30s|single_30s|clip_10min|tiny_1s]
+
+A step is one forward of the whole hot path (log-mel, conv stem, 32 layers,
+head, adapter) over one batch: by default the 16 clips of 10-30 s (seeds
+0-15), which is the batched 30 s throughput case.  Inputs are synthetic and
+seeded; weights are random-init bf16.  Timing: CUDA events on the encoder's
+stream around each step, with a 512 MB buffer written between steps (L2
+flush, outside the events); barrier + synchronize on both sides of the K
+steps; multi-GPU runs take the max over ranks, each rank encoding its own
+batch (clips are independent: weak scaling, no collective on the data path).
+
+The reference arm (--impl reference) times the CPU oracle on the host cores
+on one 800-frame window of the same batch per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from audio_encoder_b200 import synth  # noqa: E402
+
+MFLOP_PER_TOKEN = 1737.5e6   # algorithmic work per valid token (stem + 32 layers + head + adapter)
+L2_FLUSH_BYTES = 512 << 20
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
+                    src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def workload_clips(name):
+    desc, make, n_layers = synth.WORKLOADS[name]
+    return desc, make(), n_layers
+
+
+def model_flops(tokens, n_layers):
+    # stem 353.6 + 39.83 per layer + head/adapter 109.2 MFLOP per token
+    return tokens * (353.6e6 + 39.83e6 * n_layers + 109.2e6)
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.p = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.p:
+            self.p.terminate()
+            try:
+                out, _ = self.p.communicate(timeout=5)
+            except Exception:
+                self.p.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except Exception:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        load = [s for s in sm if s > 0.5 * (mx or 1)] or sm
+        return {"sm_mhz": float(np.median(load)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    if n_gpus <= 1 or "RANK" not in os.environ:
+        return 0, 1, None
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    world = int(os.environ["WORLD_SIZE"])
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, dist
+
+
+def oracle_sample(clips, n_layers, windows, blob=None):
+    import oracle
+    blob = synth.make_weights(n_layers) if blob is None else blob
+    m = oracle.Model(blob, n_layers)
+    pcm = clips[0]
+    gmax = oracle.clip_log_max(pcm)
+    t0 = time.perf_counter()
+    toks = 0
+    for c in range(windows):
+        toks += m.encode_chunks(pcm, c, c + 1, gmax=gmax).shape[0]
+    dt = time.perf_counter() - t0
+    m.close()
+    return dt, toks, oracle.max_threads()
+
+
+def gemm_source_hash():
+    h = hashlib.sha256()
+    for f in ["gemm.cuh", "common.cuh"]:
+        with open(os.path.join(ROOT, "audio_encoder_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the
+    GEMM sources are unchanged since the capture; else None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[kernel]
+        if e.get("source_hash") != gemm_source_hash():
+            return None
+        return e["bytes_per_launch_full_size"]
+    except Exception:
+        return None
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    desc, clips, n_layers = workload_clips(args.workload)
+    blob = synth.make_weights(n_layers)
+    import oracle
+    m = oracle.Model(blob, n_layers)
+    pcm = clips[0]
+    gmax = oracle.clip_log_max(pcm)
+    nc = oracle.num_chunks(pcm.size)
+
+    def step(i):
+        c = i % nc
+        return m.encode_chunks(pcm, c, c + 1, gmax=gmax).shape[0]
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    toks = 0
+    for i in range(args.steps):
+        toks += step(i)
+    dt = time.perf_counter() - t0
+    audio_s = toks / 12.5
+    v = audio_s / dt
+    line = {
+        "impl": "reference", "metric": "audio-sec encoded/sec", "value": v, "unit": "audio-s/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "tokens_per_s": toks / dt,
+        "config": {"workload": args.workload, "description": desc, "step": "one 800-frame window of clip 0",
+                   "layers": n_layers},
+        "cpu_baseline": {"value": v, "unit": "audio-s/s", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"{args.steps} windows of 100 tokens (8 s of audio each) of clip 0"},
+        "e2e": {"value": v, "unit": "audio-s/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+
+    from audio_encoder_b200 import binding
+
+    rank, world, dist = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    desc, clips, n_layers = workload_clips(args.workload)
+    blob = synth.make_weights(n_layers)
+    total_samples = sum(c.size for c in clips)
+    stream = torch.cuda.Stream()
+    enc = binding.Encoder(blob, n_layers, max_samples=total_samples + 4 * len(clips), max_clips=len(clips),
+                          out_dtype=binding.OUT_BF16, stream=stream)
+    with torch.cuda.stream(stream):
+        xs = [torch.from_numpy(c).to(dev) for c in clips]
+        tokens = sum(binding.num_tokens(c.size) for c in clips)
+        out = torch.empty((tokens, 2048), dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    audio_s = total_samples / 16000.0
+    torch.cuda.synchronize()
+
+    def step():
+        enc.forward(xs, out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    enc.synchronize()
+
+    # ---- timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = enc.launch_count()
+    enc.profile_enable(400 * (args.steps + 1))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(dev.index) as clk:
+        for i in range(args.steps):
+            with torch.cuda.stream(stream):
+                flush.fill_(float(i))
+                ev[i][0].record(stream)
+                step()
+                ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    launches = enc.launch_count() - launches0
+    stats = enc.profile_read()
+    enc.profile_enable(0)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    enc.synchronize()
+
+    # ---- end to end through the host API: pinned PCM in, rows out to host
+    pinned = [torch.from_numpy(c).pin_memory() for c in clips]
+    rows_host = torch.empty((tokens, 2048), dtype=torch.bfloat16).pin_memory()
+    enc.forward_host(pinned, rows_host)
+    e2e_ms = []
+    for i in range(max(2, min(args.steps, 10))):
+        flush.fill_(float(i))
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        enc.forward_host(pinned, rows_host)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_step = float(np.mean(e2e_ms))
+    if dist:
+        t = torch.tensor([e2e_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_step = float(t.item())
+
+    if rank != 0:
+        enc.close()
+        if dist:
+            dist.destroy_process_group()
+        return
+
+    pk = peaks()
+    ms_per_step = total_ms / args.steps
+    value = world * audio_s / (ms_per_step / 1e3)
+    flops_step = model_flops(tokens, n_layers)
+    tflops = flops_step / (ms_per_step / 1e3) / 1e12
+    # dominant kernel: the category with the most device time
+    dom_name, dom = max(stats.items(), key=lambda kv: kv[1]["ms"])
+    per_launch_ms = dom["ms"] / dom["launches"]
+    kernel_ms = sum(v["ms"] for v in stats.values())
+    if dom["flops"] > 0 and dom_name.startswith("gemm"):
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_sus"],
+                "peak_note": f"{pk['src']} sustained bf16 (kernel timed inside a long step)"}
+    else:
+        achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "peak_note": f"{pk['src']} HBM copy bandwidth"}
+    roof.update({"kernel": dom_name, "launches_per_step": dom["launches"] / args.steps,
+                 "ms_per_launch": per_launch_ms, "share_of_kernel_time": dom["ms"] / kernel_ms,
+                 "traffic": profiled_traffic(dom_name)})
+
+    kernels = {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps,
+                   "tflops": (v["flops"] / (v["ms"] / 1e3) / 1e12) if v["flops"] and v["ms"] else None,
+                   "gbs": (v["bytes"] / (v["ms"] / 1e3) / 1e9) if v["bytes"] and v["ms"] else None}
+               for k, v in sorted(stats.items(), key=lambda kv: -kv[1]["ms"])}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        dt, toks, cores = oracle_sample(clips, n_layers, windows=args.cpu_windows, blob=blob)
+        cpu = {"value": (toks / 12.5) / dt, "unit": "audio-s/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {args.cpu_windows} 800-frame windows of clip 0 ({toks} tokens, "
+                         f"{toks / 12.5:.0f} s of audio), all {n_layers} layers, {dt:.1f} s"}
+
+    line = {
+        "metric": "audio-sec encoded/sec", "value": value, "unit": "audio-s/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded PCM, random-init bf16 weights)",
+        "tokens_per_s": world * tokens / (ms_per_step / 1e3),
+        "model_tflops": tflops,
+        "tc_roofline_frac": tflops / pk["bf16"],
+        "tc_roofline_frac_sustained": tflops / pk["bf16_sus"],
+        "config": {"workload": args.workload, "description": desc, "clips_per_gpu": len(clips),
+                   "audio_s_per_gpu": audio_s, "tokens_per_gpu": tokens, "layers": n_layers,
+                   "out_dtype": "bf16", "l2": "512 MB buffer written between timed steps (outside the events)",
+                   "parallelism": f"dp{world}" if world > 1 else "single"},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "e2e": {"value": world * audio_s / (e2e_step / 1e3), "unit": "audio-s/s",
+                "h2d_bytes_per_step": 4 * total_samples, "d2h_bytes_per_step": 2 * tokens * 2048,
+                "ms_per_step": e2e_step},
+        "cpu_baseline": cpu,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    enc.close()
+    if dist:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="batch16_10to30s", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--cpu-windows", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

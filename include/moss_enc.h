@@ -184,6 +184,30 @@ moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host,
                                       const int64_t *n_samples, int n_clips, void *rows_host,
                                       int64_t *row_offsets);
 
+/* ------------------------------------------------------------ measurement */
+
+/* Per-kernel timing by kernel category, taken with CUDA events recorded on the
+ * handle's stream around every launch while profiling is enabled. */
+typedef struct {
+    char name[32];     /* kernel category, e.g. "gemm_fc1" */
+    int64_t launches;  /* launches since the last read */
+    double ms;         /* summed device time of those launches */
+    double flops;      /* summed algorithmic flops (padding not counted) */
+    double bytes;      /* summed algorithmic HBM bytes (compulsory reads + writes) */
+} moss_enc_kernel_stat;
+
+/* max_launches > 0 enables profiling with room for that many launches
+ * between reads (host-side events are created here); 0 disables it. */
+moss_enc_status moss_enc_profile_enable(moss_enc *h, int max_launches);
+
+/* Synchronises, aggregates the recorded launches by category into out
+ * (up to max entries), clears the record, and returns the number of
+ * categories written (negative on error). */
+int moss_enc_profile_read(moss_enc *h, moss_enc_kernel_stat *out, int max);
+
+/* Kernels this handle has launched since create (all calls). */
+int64_t moss_enc_launch_count(const moss_enc *h);
+
 #ifdef __cplusplus
 }
 #endif
