@@ -27,7 +27,9 @@ EXPORTED = [
     "moss_enc_status_string", "moss_enc_last_error", "moss_enc_logmel", "moss_enc_log_max",
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
+    "moss_enc_logmel_static",
 ]
+STATIC_MAX_CLIPS = 64
 
 
 class MossEncError(RuntimeError):
@@ -99,6 +101,8 @@ def lib():
         L.moss_enc_profile_read.argtypes = [vp, ctypes.POINTER(KernelStat), i32]
         L.moss_enc_launch_count.restype = i64
         L.moss_enc_launch_count.argtypes = [vp]
+        L.moss_enc_logmel_static.restype = i32
+        L.moss_enc_logmel_static.argtypes = [ctypes.POINTER(Clip), i32, ctypes.POINTER(vp), vp, vp]
         _lib = L
     return _lib
 
@@ -272,3 +276,35 @@ class Encoder:
         offs = (ctypes.c_int64 * (n + 1))()
         self._check(lib().moss_enc_forward_host(self.h, ptrs, lens, n, ctypes.c_void_p(rp), offs))
         return rows_host, list(offs)
+
+
+def logmel_static(clips, stream=None):
+    """Allocation-free log-mel of up to STATIC_MAX_CLIPS clips (no handle).
+
+    clips: device fp32 tensors or (pcm, begin, end, log_max) tuples.  The
+    output tensors are made here by PyTorch on the caller's behalf; the
+    library call itself allocates nothing.  Returns (list of [frames][128]
+    tensors, log_max tensor [n_clips]).
+    """
+    import torch
+    n = len(clips)
+    arr = (Clip * max(n, 1))()
+    outs = []
+    for i, c in enumerate(clips):
+        pcm, begin, end, lm = (list(c) + [None, None, None])[:4] if isinstance(c, tuple) else (c, 0, None, None)
+        ns = pcm.numel()
+        end = ns if end is None else end
+        arr[i] = Clip(pcm.data_ptr(), ns, int(begin or 0), int(end), lm.data_ptr() if lm is not None else None)
+        fb = (begin or 0) // 160
+        fe = num_frames(ns) if end == ns else end // 160
+        outs.append(torch.empty((max(fe - fb, 0), 128), dtype=torch.float32, device=pcm.device))
+    ptrs = (ctypes.c_void_p * max(n, 1))(*[o.data_ptr() if o.numel() else None for o in outs])
+    dev = clips[0][0].device if isinstance(clips[0], tuple) else clips[0].device
+    mx = torch.empty(max(n, 1), dtype=torch.float32, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    st = lib().moss_enc_logmel_static(arr, n, ptrs, ctypes.c_void_p(mx.data_ptr()),
+                                      ctypes.c_void_p(stream.cuda_stream))
+    if st != OK:
+        raise MossEncError(st, "logmel_static failed")
+    return outs, mx[:n]

@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -1075,3 +1076,114 @@ extern "C" int moss_enc_profile_read(moss_enc *h, moss_enc_kernel_stat *out, int
 }
 
 extern "C" int64_t moss_enc_launch_count(const moss_enc *h) { return h ? h->launches : -1; }
+
+// ------------------------------------------------- allocation-free log-mel
+//
+// Scratch for moss_enc_logmel_static: a fixed-size device array, laid out as
+// [MelTables | main-pass MelClip x 64 | max-pass MelClip x 64 | log_max
+// source pointers x 64 | ordered-int maxima x 64].  Nothing here allocates.
+
+namespace {
+constexpr int STATIC_MAX_CLIPS = MOSS_ENC_STATIC_MAX_CLIPS;
+constexpr size_t ST_TABLES = 0;
+constexpr size_t ST_MAIN = (sizeof(MelTables) + 255) & ~size_t(255);
+constexpr size_t ST_MAXP = ST_MAIN + ((sizeof(MelClip) * STATIC_MAX_CLIPS + 255) & ~size_t(255));
+constexpr size_t ST_SRC = ST_MAXP + ((sizeof(MelClip) * STATIC_MAX_CLIPS + 255) & ~size_t(255));
+constexpr size_t ST_GMAX = ST_SRC + ((sizeof(float *) * STATIC_MAX_CLIPS + 255) & ~size_t(255));
+constexpr size_t ST_USED = ST_GMAX + sizeof(int) * STATIC_MAX_CLIPS;
+constexpr size_t ST_BYTES = 20480;
+static_assert(ST_USED <= ST_BYTES, "static log-mel scratch too small");
+
+// Per-call descriptors staged on the host before one copy into the array.
+struct StaticStage {
+    MelClip main[STATIC_MAX_CLIPS];
+    MelClip maxp[STATIC_MAX_CLIPS];
+    const float *src[STATIC_MAX_CLIPS];
+};
+
+constexpr int STATIC_MAX_DEVICES = 64;
+std::mutex g_static_mu;
+uint8_t *g_static_ptr[STATIC_MAX_DEVICES] = {};
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_logmel_scratch[ST_BYTES];
+
+// Device address of the scratch on the current device; the first call per
+// device looks it up and writes the constant tables into it.
+static moss_enc_status static_scratch(uint8_t **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= STATIC_MAX_DEVICES) return MOSS_ENC_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_logmel_scratch) != cudaSuccess || !p) return MOSS_ENC_ERR_CUDA;
+        if (cudaFuncSetAttribute(logmel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(MelSmem)) !=
+            cudaSuccess)
+            return MOSS_ENC_ERR_CUDA;
+        MelTables tab;
+        if (!build_mel_tables(&tab)) return MOSS_ENC_ERR_INVALID_ARG;
+        if (cudaMemcpy(static_cast<uint8_t *>(p) + ST_TABLES, &tab, sizeof(tab), cudaMemcpyHostToDevice) != cudaSuccess)
+            return MOSS_ENC_ERR_CUDA;
+        g_static_ptr[dev] = static_cast<uint8_t *>(p);
+    }
+    *out = g_static_ptr[dev];
+    return MOSS_ENC_OK;
+}
+
+extern "C" moss_enc_status moss_enc_logmel_static(const moss_enc_clip *clips, int n_clips, float *const *mel_out,
+                                                  float *log_max_out, void *stream)
+{
+    if (n_clips < 0 || (n_clips > 0 && (!clips || !mel_out))) return MOSS_ENC_ERR_INVALID_ARG;
+    if (n_clips > STATIC_MAX_CLIPS) return MOSS_ENC_ERR_CAPACITY;
+    if (n_clips == 0) return MOSS_ENC_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    StaticStage stage;
+    std::memset(&stage, 0, sizeof(stage));
+    int n_max = 0;
+    int64_t max_range = 0, max_clip = 0;
+    for (int i = 0; i < n_clips; i++) {
+        const moss_enc_clip &c = clips[i];
+        ClipPlan pl;
+        if (!plan_clip(c.n_samples, c.begin, c.end, &pl) || pl.F > INT32_MAX) return MOSS_ENC_ERR_INVALID_ARG;
+        const int64_t nf = pl.f_end - pl.f_begin;
+        if (nf > 0 && (!c.pcm || !mel_out[i])) return MOSS_ENC_ERR_INVALID_ARG;
+        const bool whole = pl.f_begin == 0 && pl.f_end == pl.F;
+        const bool own = c.log_max == nullptr;
+        stage.src[i] = c.log_max;
+        // every clip has its own output buffer, so each clip gets its own
+        // launch below and writes from row 0 of that buffer
+        stage.main[i] = MelClip{c.pcm, (long long)pl.n, 0, (int)pl.f_begin, (int)pl.f_end, own && whole ? i : -1, 0};
+        if (own && !whole) stage.maxp[n_max++] = MelClip{c.pcm, (long long)pl.n, 0, 0, (int)pl.F, i, 0};
+        max_range = std::max(max_range, nf);
+        max_clip = std::max(max_clip, pl.F);
+    }
+    uint8_t *S = nullptr;
+    moss_enc_status s = static_scratch(&S);
+    if (s != MOSS_ENC_OK) return s;
+    MelClip *d_main = reinterpret_cast<MelClip *>(S + ST_MAIN);
+    MelClip *d_maxp = reinterpret_cast<MelClip *>(S + ST_MAXP);
+    const float *const *d_src = reinterpret_cast<const float *const *>(S + ST_SRC);
+    int *d_gmax = reinterpret_cast<int *>(S + ST_GMAX);
+    const MelTables *d_tab = reinterpret_cast<const MelTables *>(S + ST_TABLES);
+    if (cudaMemcpyAsync(S + ST_MAIN, stage.main, sizeof(stage.main), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(S + ST_MAXP, stage.maxp, sizeof(stage.maxp), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(S + ST_SRC, stage.src, sizeof(stage.src), cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MOSS_ENC_ERR_CUDA;
+    // the maxima start at -inf or at the caller's value
+    gmax_init_kernel<<<1, STATIC_MAX_CLIPS, 0, st>>>(d_gmax, d_src, n_clips);
+    if (n_max > 0)
+        logmel_kernel<<<dim3(mel_grid_x(max_clip), n_max), 256, sizeof(MelSmem), st>>>(d_maxp, d_tab, nullptr, d_gmax, 0);
+    for (int i = 0; i < n_clips; i++) {
+        const int nf = stage.main[i].f_end - stage.main[i].f_begin;
+        if (nf <= 0) continue;
+        logmel_kernel<<<dim3(mel_grid_x(nf), 1), 256, sizeof(MelSmem), st>>>(d_main + i, d_tab, mel_out[i], d_gmax, 1);
+    }
+    for (int i = 0; i < n_clips; i++) {
+        const int64_t nf = stage.main[i].f_end - stage.main[i].f_begin;
+        if (nf > 0)
+            mel_normalize_kernel<<<(int)std::min<int64_t>(4096, (nf * 128 + 255) / 256), 256, 0, st>>>(mel_out[i], nf * 128, d_gmax + i);
+        if (log_max_out) gmax_export_kernel<<<1, 32, 0, st>>>(d_gmax + i, log_max_out + i);
+    }
+    return cudaGetLastError() == cudaSuccess ? MOSS_ENC_OK : MOSS_ENC_ERR_CUDA;
+}

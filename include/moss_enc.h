@@ -184,6 +184,40 @@ moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host,
                                       const int64_t *n_samples, int n_clips, void *rows_host,
                                       int64_t *row_offsets);
 
+/* ------------------------------------------------- allocation-free log-mel */
+
+/* The source pages describe no such call; it exists for callers that cannot
+ * allocate device memory.  Examples: a process whose GPU memory is owned by
+ * another framework's pool (a raw cudaMalloc there can fail under pressure or
+ * force the pool to release its cache), or a real-time audio front end that
+ * must not allocate once it is running.  moss_enc_create allocates the
+ * weights and a workspace, so such callers use this call instead: it needs
+ * no handle and never allocates.
+ *
+ * It computes the same Whisper log-mel as moss_enc_logmel for up to
+ * MOSS_ENC_STATIC_MAX_CLIPS clips.  Its scratch (the filterbank and FFT
+ * tables, per-clip range descriptors and per-clip maxima; 20 KiB) is one
+ * statically sized device array inside the library, which every GPU that
+ * loads the library keeps until the process exits.
+ *  clips        host [n_clips]; same fields and range rules as moss_enc_clip.
+ *  mel_out      host array of n_clips device pointers, each fp32
+ *               [frames of that clip's range][128] (may be NULL for an empty
+ *               range).
+ *  log_max_out  device float [n_clips] receiving each clip's log-mel maximum,
+ *               or NULL.
+ *  stream       cudaStream_t to enqueue on.
+ * Returns MOSS_ENC_ERR_CAPACITY when n_clips exceeds MOSS_ENC_STATIC_MAX_CLIPS
+ * and MOSS_ENC_ERR_INVALID_ARG for a bad pointer or range.
+ * The first call on a device sets the scratch up (finds the array's device
+ * address and fills the tables, synchronously); make that first call before
+ * any stream capture.  All calls share the one array, and each call
+ * overwrites what the previous call left there: calls whose work overlaps on
+ * the GPU (different streams, or several host threads) race and must be
+ * serialised by the caller. */
+#define MOSS_ENC_STATIC_MAX_CLIPS 64
+moss_enc_status moss_enc_logmel_static(const moss_enc_clip *clips, int n_clips, float *const *mel_out,
+                                       float *log_max_out, void *stream);
+
 /* ------------------------------------------------------------ measurement */
 
 /* Per-kernel timing by kernel category, taken with CUDA events recorded on the
