@@ -27,7 +27,7 @@ EXPORTED = [
     "moss_enc_status_string", "moss_enc_last_error", "moss_enc_logmel", "moss_enc_log_max",
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
-    "moss_enc_logmel_static",
+    "moss_enc_logmel_static", "moss_enc_gemm",
 ]
 STATIC_MAX_CLIPS = 64
 
@@ -101,6 +101,8 @@ def lib():
         L.moss_enc_profile_read.argtypes = [vp, ctypes.POINTER(KernelStat), i32]
         L.moss_enc_launch_count.restype = i64
         L.moss_enc_launch_count.argtypes = [vp]
+        L.moss_enc_gemm.restype = i32
+        L.moss_enc_gemm.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32]
         L.moss_enc_logmel_static.restype = i32
         L.moss_enc_logmel_static.argtypes = [ctypes.POINTER(Clip), i32, ctypes.POINTER(vp), vp, vp]
         _lib = L
@@ -191,6 +193,14 @@ class Encoder:
             raise MossEncError(4, "profile_read failed")
         return {arr[i].name.decode(): dict(launches=arr[i].launches, ms=arr[i].ms, flops=arr[i].flops,
                                            bytes=arr[i].bytes) for i in range(n)}
+
+    def gemm(self, A, B, bias, out, epilogue: int, block_n: int):
+        """out = epi(A @ B.T + bias) on the tensor cores (A [M][K], B [N][K] bf16)."""
+        M, K = A.shape
+        N = B.shape[0]
+        self._check(lib().moss_enc_gemm(self.h, _ptr(A), _ptr(B), _ptr(bias), _ptr(out), M, N, K,
+                                        int(epilogue), int(block_n)))
+        return out
 
     def launch_count(self) -> int:
         return int(lib().moss_enc_launch_count(self.h))

@@ -2,162 +2,158 @@
 // GGUF", "Architecture" table, Audio encoder row): every token attends only
 // the tokens of its own window (one 800-frame chunk, at most 100 tokens).
 //
-// One CTA per (window, head).  The window's Q, K, V slices (<= 128 rows x 64)
-// are staged in shared memory; each of 8 warps owns 16 query rows, computes
-// S = Q K^T / 8 with bf16 tensor-core MMAs, an fp32 softmax in registers
-// (keys past the window length masked), and O = P V.  Nothing crosses
-// windows, so windows never exchange data.
+// Windows hold at most 128 tokens (here 100); nothing crosses windows, so
+// windows never exchange data.
 #pragma once
 
 #include "common.cuh"
 
 namespace moss {
 
-static constexpr int ATTN_MAX_WIN = 128;
-static constexpr int ATTN_PITCH = 72;  // bf16 per shared row (144 B: conflict-free ldmatrix)
-static constexpr size_t ATTN_SMEM = 3 * ATTN_MAX_WIN * ATTN_PITCH * sizeof(bf16);
+// One CTA of 128 threads per (window, head); thread i owns query row i, which
+// is TMEM lane i.  TMA brings the 128-row Q, K and V slices of the window
+// (rows past the window belong to the next window or lie past the end and are
+// masked / zero).  S = Q K^T (M = N = 128, K = 64) accumulates in TMEM; each
+// thread reads its row of S, masks keys past the window, and writes
+// P = exp(S/8 - max) as bf16 into shared memory in the swizzled K-major layout
+// (over the Q and K slots, which are free once S is done).  O = P V (M = 128,
+// N = 64, K = 128) takes V straight from its TMA layout as an MN-major
+// operand, lands in TMEM, and is scaled by 1 / rowsum on the way out.
+static constexpr size_t ATTN_TC_SMEM = 1024 + 3 * 16384 + 64;
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p)
+// Shared-memory descriptor of an MN-major operand with 128-byte swizzle:
+// rows of 64 bf16 along N (128 B) for consecutive K, 8-row K groups 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t smem_addr)
 {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_u32(p)));
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(1024 >> 4) << 32;  // stride between 8-row groups along K
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
 }
 
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void *p)
+__global__ void __launch_bounds__(128) window_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
+                                                             const int2 *__restrict__ windows,
+                                                             bf16 *__restrict__ out, int *err)
 {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_u32(p)));
-}
-
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// qkv [T][3840] bf16 = q | k | v (each 20 heads x 64); out [T][1280] bf16.
-// windows[w] = {first token, tokens} with 1 <= tokens <= 128.
-__global__ void __launch_bounds__(256) window_attn_kernel(const bf16 *__restrict__ qkv,
-                                                          const int2 *__restrict__ windows,
-                                                          bf16 *__restrict__ out)
-{
-    extern __shared__ __align__(16) uint8_t attn_smem[];
-    bf16 *Qs = reinterpret_cast<bf16 *>(attn_smem);
-    bf16 *Ks = Qs + ATTN_MAX_WIN * ATTN_PITCH;
-    bf16 *Vs = Ks + ATTN_MAX_WIN * ATTN_PITCH;
+    extern __shared__ uint8_t attn_tc_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(attn_tc_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = sm, *sK = sm + 16384, *sV = sm + 32768;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 49152);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
     const int h = blockIdx.y;
     const int2 win = windows[blockIdx.x];
     const int s = win.x, n = win.y;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5;
 
-    for (int i = tid; i < 3 * ATTN_MAX_WIN * 8; i += 256) {
-        const int mat = i / (ATTN_MAX_WIN * 8), r = (i / 8) % ATTN_MAX_WIN, c8 = i % 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < n) v = *reinterpret_cast<const uint4 *>(qkv + (size_t)(s + r) * 3840 + mat * 1280 + h * 64 + c8 * 8);
-        *reinterpret_cast<uint4 *>(Qs + (size_t)mat * ATTN_MAX_WIN * ATTN_PITCH + r * ATTN_PITCH + c8 * 8) = v;
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_qkv);
     }
+    if (warp == 0) {
+        tmem_alloc(tslot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tslot;
+    const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
 
-    const int warp = tid >> 5, lane = tid & 31;
-    const int r0 = warp * 16;
-    if (r0 >= n) return;
-    const int nkb = (n + 15) >> 4;  // key blocks of 16
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bars[0], 3 * 16384);
+        tma_load_2d(&tm_qkv, &bars[0], sQ, h * 64, s);
+        tma_load_2d(&tm_qkv, &bars[0], sK, 1280 + h * 64, s);
+        tma_load_2d(&tm_qkv, &bars[0], sV, 2560 + h * 64, s);
+        if (mbar_wait(&bars[0], 0, err)) {
+            tc_fence_after();
+            constexpr uint32_t idesc = idesc_bf16(128, 128);
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+                mma_bf16(tbase, sw128_desc(smem_u32(sQ) + 32 * k), sw128_desc(smem_u32(sK) + 32 * k), idesc, k > 0);
+            mma_commit(&bars[1]);
+        }
+    }
+    bool ok = mbar_wait(&bars[1], 0, err);
+    tc_fence_after();
 
-    uint32_t qf[4][4];
+    // softmax of this thread's row (keys >= n masked); P to shared memory
+    const float scale = 0.125f * 1.4426950408889634f;
+    float mx = -INFINITY;
 #pragma unroll
-    for (int kk = 0; kk < 4; kk++)
-        ldsm_x4(qf[kk], Qs + (r0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ATTN_PITCH + kk * 16 + 8 * (lane >> 4));
-
-    float sc[16][4];
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + c0, v);
+        tmem_ld_wait();
 #pragma unroll
-    for (int j = 0; j < 16; j++) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.0f;
+        for (int j = 0; j < 32; j++)
+            if (c0 + j < n) mx = fmaxf(mx, __uint_as_float(v[j]) * scale);
+    }
+    float sum = 0.0f;
+    const int r = tid, sw = r & 7;
 #pragma unroll
-    for (int jb = 0; jb < 8; jb++) {
-        if (jb < nkb) {
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + c0, v);
+        tmem_ld_wait();
+        uint8_t *blk = (c0 < 64 ? sQ : sK) + r * 128;
 #pragma unroll
-            for (int kk = 0; kk < 4; kk++) {
-                uint32_t b[4];
-                ldsm_x4(b, Ks + (jb * 16 + (lane & 7) + 8 * (lane >> 4)) * ATTN_PITCH + kk * 16 + 8 * ((lane >> 3) & 1));
-                mma16816(sc[2 * jb], qf[kk], b[0], b[1]);
-                mma16816(sc[2 * jb + 1], qf[kk], b[2], b[3]);
+        for (int q = 0; q < 4; q++) {
+            float p[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int key = c0 + 8 * q + j;
+                p[j] = key < n ? exp2f(__uint_as_float(v[8 * q + j]) * scale - mx) : 0.0f;
+                sum += p[j];
             }
+            const int chunk16 = ((c0 & 63) >> 3) + q;  // 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4 *>(blk + ((chunk16 ^ sw) << 4)) =
+                make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                           pack_bf16x2(p[6], p[7]));
         }
     }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
-    const float scale = 0.125f * 1.4426950408889634f;  // 1/sqrt(64) in base-2 exponent units
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+    if (tid == 0 && ok) {
+        constexpr uint32_t idesc = idesc_bf16(128, 64) | (1u << 16);  // B (V) is MN-major
 #pragma unroll
-    for (int j = 0; j < 16; j++) {
-        if (j < 2 * nkb) {
-            const int key = 8 * j + 2 * (lane & 3);
-#pragma unroll
-            for (int e = 0; e < 2; e++) {
-                const bool ok = key + e < n;
-                sc[j][e] = ok ? sc[j][e] * scale : -INFINITY;
-                sc[j][2 + e] = ok ? sc[j][2 + e] * scale : -INFINITY;
-            }
-            mx0 = fmaxf(mx0, fmaxf(sc[j][0], sc[j][1]));
-            mx1 = fmaxf(mx1, fmaxf(sc[j][2], sc[j][3]));
+        for (int ks = 0; ks < 8; ks++) {
+            const uint32_t a = smem_u32(ks < 4 ? sQ : sK) + 32 * (ks & 3);
+            mma_bf16(tbase, sw128_desc(a), sw128_mn_desc(smem_u32(sV) + 2048 * ks), idesc, ks > 0);
         }
+        mma_commit(&bars[1]);
     }
+    ok = mbar_wait(&bars[1], 1, err) && ok;
+    tc_fence_after();
+    uint32_t o0[32], o1[32];
+    tmem_ld32(trow, o0);
+    tmem_ld32(trow + 32, o1);
+    tmem_ld_wait();
+    if (ok && r < n) {
+        const float inv = 1.0f / sum;
+        uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)(s + r) * 1280 + h * 64);
 #pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        for (int q = 0; q < 4; q++)
+            dst[q] = make_uint4(pack_bf16x2(__uint_as_float(o0[8 * q]) * inv, __uint_as_float(o0[8 * q + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(o0[8 * q + 2]) * inv, __uint_as_float(o0[8 * q + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(o0[8 * q + 4]) * inv, __uint_as_float(o0[8 * q + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(o0[8 * q + 6]) * inv, __uint_as_float(o0[8 * q + 7]) * inv));
+#pragma unroll
+        for (int q = 0; q < 4; q++)
+            dst[4 + q] = make_uint4(pack_bf16x2(__uint_as_float(o1[8 * q]) * inv, __uint_as_float(o1[8 * q + 1]) * inv),
+                                    pack_bf16x2(__uint_as_float(o1[8 * q + 2]) * inv, __uint_as_float(o1[8 * q + 3]) * inv),
+                                    pack_bf16x2(__uint_as_float(o1[8 * q + 4]) * inv, __uint_as_float(o1[8 * q + 5]) * inv),
+                                    pack_bf16x2(__uint_as_float(o1[8 * q + 6]) * inv, __uint_as_float(o1[8 * q + 7]) * inv));
     }
-    float sum0 = 0.0f, sum1 = 0.0f;
-    uint32_t pa[8][4];
-#pragma unroll
-    for (int j = 0; j < 16; j++) {
-        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-        if (j < 2 * nkb) {
-            p0 = exp2f(sc[j][0] - mx0);
-            p1 = exp2f(sc[j][1] - mx0);
-            p2 = exp2f(sc[j][2] - mx1);
-            p3 = exp2f(sc[j][3] - mx1);
-        }
-        sum0 += p0 + p1;
-        sum1 += p2 + p3;
-        pa[j >> 1][(j & 1) * 2] = pack_bf16x2(p0, p1);
-        pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);
-    }
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-        sum0 += __shfl_xor_sync(0xffffffffu, sum0, o);
-        sum1 += __shfl_xor_sync(0xffffffffu, sum1, o);
-    }
-
-    float oacc[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; j++) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.0f;
-#pragma unroll
-    for (int kb = 0; kb < 8; kb++) {
-        if (kb < nkb) {
-#pragma unroll
-            for (int dp = 0; dp < 4; dp++) {
-                uint32_t b[4];
-                ldsm_x4_t(b, Vs + (kb * 16 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ATTN_PITCH + dp * 16 + 8 * (lane >> 4));
-                mma16816(oacc[2 * dp], pa[kb], b[0], b[1]);
-                mma16816(oacc[2 * dp + 1], pa[kb], b[2], b[3]);
-            }
-        }
-    }
-
-    const float inv0 = 1.0f / sum0, inv1 = 1.0f / sum1;
-    const int ra = r0 + (lane >> 2), rb = ra + 8;
-#pragma unroll
-    for (int j = 0; j < 8; j++) {
-        const int d = h * 64 + 8 * j + 2 * (lane & 3);
-        if (ra < n)
-            *reinterpret_cast<uint32_t *>(out + (size_t)(s + ra) * 1280 + d) = pack_bf16x2(oacc[j][0] * inv0, oacc[j][1] * inv0);
-        if (rb < n)
-            *reinterpret_cast<uint32_t *>(out + (size_t)(s + rb) * 1280 + d) = pack_bf16x2(oacc[j][2] * inv1, oacc[j][3] * inv1);
-    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 128);
 }
 
 }  // namespace moss

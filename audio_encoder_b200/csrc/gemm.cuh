@@ -5,9 +5,11 @@
 // One CTA per SM walks output tiles of 128 x BN.  Warp 0 (one lane) streams
 // 128x64 A and BNx64 B tiles with TMA into a ring of shared-memory stages;
 // warp 1 (one lane) issues tcgen05.mma (M=128, N=BN, K=16) into one of two
-// TMEM accumulators; warps 2-5 drain the other accumulator with tcgen05.ld
+// TMEM accumulators; warps 2-9 drain the other accumulator with tcgen05.ld
 // and apply the fused epilogue (bias, GELU, residual add, SwiGLU, conv_out
-// row packing + positions) while the next tile's mainloop runs.
+// row packing + positions) while the next tile's mainloop runs.  A warp may
+// only read the TMEM lane quarter (warp id mod 4), so two epilogue warps share
+// each quarter and split the tile's 32-column chunks between them.
 #pragma once
 
 #include "common.cuh"
@@ -23,6 +25,13 @@ enum EpiKind : int {
     EPI_F32 = 5         // out fp32 = acc + bias
 };
 
+// How the A operand is fetched.
+enum AMode : int {
+    A_PLAIN = 0,    // A [M][K] row-major, 2-D tensor map
+    A_CONV_S2 = 1   // implicit 3x3 / stride 2 / pad 1 conv over NHWC [chunk][T][F][480]:
+                    // k-block kb = tap*8 + channel block, tap = kf*3 + kt
+};
+
 struct GemmArgs {
     int M, N, K;
     int m_tiles, n_tiles;
@@ -32,11 +41,18 @@ struct GemmArgs {
     int ldo;                // output leading dimension in elements
     const float *pos;       // EPI_CONVOUT: positions [100][ldo]
     const int2 *chunk_tok;  // EPI_CONVOUT: per chunk {first packed row, rows}
+    // A_CONV_S2 only: the m-tiles to compute, each chunk * 256 + tile within
+    // the chunk; a tile is tile_t output time steps x all output frequencies.
+    const int *tile_list;
+    int rows_per_chunk;     // output rows of one chunk (T_out * F_out)
+    int tile_t;             // output time steps per 128-row tile
 };
 
 template <int BN>
 struct GemmCfg {
     static constexpr int BM = 128, BK = 64;
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     static constexpr uint32_t A_BYTES = BM * BK * 2;
     static constexpr uint32_t B_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -110,8 +126,8 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs &a, int row, int c
     }
 }
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+template <int BN, int EPI, int AMODE = A_PLAIN>
+__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmArgs args)
 {
@@ -132,7 +148,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);
+            mbar_init(&tempty[i], C::EPI_WARPS);
         }
         fence_mbar_init();
         prefetch_tmap(&tmA);
@@ -157,11 +173,24 @@ __global__ void __launch_bounds__(192, 1)
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
+                int chunk = 0, t0 = 0;
+                if constexpr (AMODE == A_CONV_S2) {
+                    const int item = args.tile_list[mt];
+                    chunk = item >> 8;
+                    t0 = (item & 255) * args.tile_t;
+                }
                 for (int kb = 0; kb < num_kb; kb++) {
                     if (!mbar_wait(&empty[s], ph ^ 1, args.err)) { ok = false; break; }
                     uint8_t *st = smem + s * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                    tma_load_2d(&tmA, &full[s], st, kb * C::BK, mt * C::BM);
+                    if constexpr (AMODE == A_CONV_S2) {
+                        // input pixels (2 t + kt - 1, 2 f + kf - 1) of the tile's outputs;
+                        // the map's traversal stride 2 on f and t does the striding
+                        const int tap = kb >> 3, kf = tap / 3, kt = tap - 3 * kf;
+                        tma_load_4d(&tmA, &full[s], st, (kb & 7) * 64, kf - 1, 2 * t0 + kt - 1, chunk);
+                    } else {
+                        tma_load_2d(&tmA, &full[s], st, kb * C::BK, mt * C::BM);
+                    }
                     tma_load_2d(&tmB, &full[s], st + C::A_BYTES, kb * C::BK, nt * BN);
                     if (++s == C::STAGES) { s = 0; ph ^= 1; }
                 }
@@ -196,7 +225,8 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
     } else {
-        const int q = warp & 3;  // this warp may read TMEM lanes 32q .. 32q+31
+        const int q = warp & 3;             // this warp may read TMEM lanes 32q .. 32q+31
+        const int half = (warp - 2) >> 2;   // which of the two warps on this quarter
         int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             const int acc = it & 1;
@@ -204,16 +234,23 @@ __global__ void __launch_bounds__(192, 1)
             if (!mbar_wait(&tfull[acc], aph, args.err)) break;
             tc_fence_after();
             const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
-            const int row = mt * C::BM + q * 32 + lane;
+            int row = mt * C::BM + q * 32 + lane;
+            bool row_ok = row < args.M;
+            if constexpr (AMODE == A_CONV_S2) {
+                const int item = args.tile_list[mt];
+                const int r_in_chunk = (item & 255) * C::BM + q * 32 + lane;
+                row_ok = r_in_chunk < args.rows_per_chunk;
+                row = (item >> 8) * args.rows_per_chunk + r_in_chunk;
+            }
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             if constexpr (EPI == EPI_SWIGLU_BF16) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 64) {
+                for (int c0 = 64 * half; c0 < BN; c0 += 128) {
                     uint32_t g[32], u[32];
                     tmem_ld32(tbase + c0, g);
                     tmem_ld32(tbase + c0 + 32, u);
                     tmem_ld_wait();
-                    if (row < args.M) {
+                    if (row_ok) {
                         const int col = nt * BN + c0;  // interleaved column of the gate block
                         const float *bg = args.bias + col, *bu = args.bias + col + 32;
                         bf16 *dst = reinterpret_cast<bf16 *>(args.out) + (size_t)row * args.ldo + col / 2;
@@ -234,11 +271,11 @@ __global__ void __launch_bounds__(192, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
+                for (int c0 = 32 * half; c0 < BN; c0 += 64) {
                     uint32_t r[32];
                     tmem_ld32(tbase + c0, r);
                     tmem_ld_wait();
-                    if (row < args.M) epilogue_store<EPI>(args, row, nt * BN + c0, r);
+                    if (row_ok) epilogue_store<EPI>(args, row, nt * BN + c0, r);
                 }
             }
             tc_fence_before();

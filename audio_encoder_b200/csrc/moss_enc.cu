@@ -27,7 +27,8 @@ namespace {
 constexpr int D = 1280, DQKV = 3840, DFF = 5120, CST = 480, DOUT = 2048, DADP = 8192;
 constexpr int CHUNK_FRAMES = 800, CHUNK_TOKENS = 100, CHUNK_SAMPLES = 128000, HOP = 160;
 constexpr int CONV_K = 9 * 512;  // conv2/conv3 patch width: 9 taps x 480 channels padded to 512
-constexpr int STEM_GROUP_DEFAULT = 16;
+constexpr int STEM_GROUP_DEFAULT = 32;
+constexpr int C2_TILES = 50, C3_TILES = 13;  // 128-row tiles per chunk of conv2 (4 t x 32 f) / conv3 (8 t x 16 f)
 
 struct LayerDev {
     float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
@@ -64,7 +65,7 @@ struct moss_enc {
     // workspace (one allocation)
     void *ws = nullptr;
     float *mel_raw = nullptr;
-    bf16 *c1out = nullptr, *a2 = nullptr, *c2out = nullptr, *a3 = nullptr, *c3out = nullptr;
+    bf16 *c1out = nullptr, *c2out = nullptr, *c3out = nullptr;
     float *X = nullptr;
     bf16 *xn = nullptr, *qkv = nullptr, *attn = nullptr, *ffn = nullptr, *hb = nullptr, *h2 = nullptr, *gu = nullptr;
     int *gmax_ord = nullptr;
@@ -193,7 +194,7 @@ static moss_enc_status gemm(moss_enc *h, const char *name, const bf16 *A, int64_
     const int grid = std::min(tiles, h->num_sms);
     const double ka = k_alg > 0 ? k_alg : K;
     Launch L(h, name, 2.0 * M * N * ka, 2.0 * M * ka + 2.0 * N * ka + epi_out_bytes(EPI) * M * N);
-    gemm_tc_kernel<BN, EPI><<<grid, 192, GemmCfg<BN>::SMEM, h->stream>>>(ta, tb, a);
+    gemm_tc_kernel<BN, EPI><<<grid, GemmCfg<BN>::THREADS, GemmCfg<BN>::SMEM, h->stream>>>(ta, tb, a);
     CUDA_TRY(h, cudaGetLastError());
     return MOSS_ENC_OK;
 }
@@ -203,6 +204,55 @@ static moss_enc_status gemm(moss_enc *h, const char *name, const bf16 *A, int64_
         moss_enc_status s_ = (x);               \
         if (s_ != MOSS_ENC_OK) return s_;       \
     } while (0)
+
+// 4-D bf16 map over NHWC [chunks][Ti][Fi][480] whose box holds the inputs of
+// one 128-row output tile of a 3x3 stride-2 conv: 64 channels x Fo
+// frequencies x tile_t time steps, both spatial axes traversed with stride 2.
+static bool tmap_conv(CUtensorMap *m, const void *ptr, int chunks, int Ti, int Fi, int tile_t)
+{
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return false;
+    const int Fo = (Fi + 1) / 2;
+    cuuint64_t dims[4] = {480, (cuuint64_t)Fi, (cuuint64_t)Ti, (cuuint64_t)chunks};
+    cuuint64_t strides[3] = {480 * 2, (cuuint64_t)Fi * 480 * 2, (cuuint64_t)Ti * Fi * 480 * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)(2 * Fo), (cuuint32_t)(2 * tile_t), 1};
+    cuuint32_t es[4] = {1, 2, 2, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// conv2/conv3 as an implicit GEMM: out [chunk][To][Fo][480] = GELU(conv(in) + b)
+// for the 128-row tiles listed in d_tiles (n_items of them).
+static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, int chunks, int Ti, int Fi,
+                                 const int *d_tiles, int n_items, const bf16 *W, const float *bias, bf16 *out)
+{
+    if (n_items <= 0) return MOSS_ENC_OK;
+    const int Fo = (Fi + 1) / 2, To = (Ti + 1) / 2, tile_t = 128 / Fo;
+    CUtensorMap ta, tb;
+    if (!tmap_conv(&ta, in, chunks, Ti, Fi, tile_t) ||
+        !tmap_2d(&tb, W, (uint64_t)CONV_K, (uint64_t)CST, (uint64_t)CONV_K * 2, 64, 160))
+        return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (conv)");
+    GemmArgs a{};
+    a.M = n_items * 128;
+    a.N = CST;
+    a.K = CONV_K;
+    a.m_tiles = n_items;
+    a.n_tiles = CST / 160;
+    a.err = h->err;
+    a.bias = bias;
+    a.out = out;
+    a.ldo = CST;
+    a.tile_list = d_tiles;
+    a.rows_per_chunk = To * Fo;
+    a.tile_t = tile_t;
+    const int grid = std::min(a.m_tiles * a.n_tiles, h->num_sms);
+    Launch L(h, name, 2.0 * 128.0 * n_items * CST * (9.0 * CST), 2.0 * 128.0 * n_items * (9.0 * CST) * 0.25 + 2.0 * 128.0 * n_items * CST);
+    gemm_tc_kernel<160, EPI_GELU_BF16, A_CONV_S2><<<grid, GemmCfg<160>::THREADS, GemmCfg<160>::SMEM, h->stream>>>(ta, tb, a);
+    CUDA_TRY(h, cudaGetLastError());
+    return MOSS_ENC_OK;
+}
 
 template <int BN, int EPI>
 static cudaError_t gemm_attr()
@@ -338,7 +388,7 @@ extern "C" const char *moss_enc_last_error(const moss_enc *h) { return h ? h->la
 
 // Table layout inside the per-call staging area.
 struct TabLayout {
-    size_t clips_main, clips_max, chunks, chunk_tok, logmax_src, total;
+    size_t clips_main, clips_max, chunks, chunk_tok, logmax_src, tiles2, tiles3, total;
 };
 
 static TabLayout tab_layout(int64_t max_clips, int64_t max_chunks)
@@ -355,6 +405,8 @@ static TabLayout tab_layout(int64_t max_clips, int64_t max_chunks)
     t.chunks = take(sizeof(StemChunk) * max_chunks);
     t.chunk_tok = take(sizeof(int2) * max_chunks);
     t.logmax_src = take(sizeof(float *) * max_clips);
+    t.tiles2 = take(sizeof(int) * max_chunks * C2_TILES);
+    t.tiles3 = take(sizeof(int) * max_chunks * C3_TILES);
     t.total = o;
     return t;
 }
@@ -376,7 +428,11 @@ extern "C" void moss_enc_destroy(moss_enc *h)
 
 static moss_enc_status set_kernel_attrs(moss_enc *h)
 {
+    CUDA_TRY(h, cudaFuncSetAttribute(gemm_tc_kernel<160, EPI_GELU_BF16, A_CONV_S2>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GemmCfg<160>::SMEM));
     CUDA_TRY(h, (gemm_attr<160, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm_attr<160, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm_attr<256, EPI_BF16>()));
     CUDA_TRY(h, (gemm_attr<128, EPI_CONVOUT_F32>()));
     CUDA_TRY(h, (gemm_attr<256, EPI_BF16>()));
     CUDA_TRY(h, (gemm_attr<256, EPI_GELU_BF16>()));
@@ -386,7 +442,7 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm_attr<256, EPI_SWIGLU_BF16>()));
     CUDA_TRY(h, (gemm_attr<128, EPI_F32>()));
     CUDA_TRY(h, (gemm_attr<128, EPI_BF16>()));
-    CUDA_TRY(h, cudaFuncSetAttribute(window_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATTN_SMEM));
+    CUDA_TRY(h, cudaFuncSetAttribute(window_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATTN_TC_SMEM));
     CUDA_TRY(h, cudaFuncSetAttribute(logmel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(MelSmem)));
     return MOSS_ENC_OK;
 }
@@ -615,9 +671,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     off = 0;
     const size_t w_mel = take(4 * (size_t)h->max_chunks * CHUNK_FRAMES * 128);
     const size_t w_c1 = take(2 * (size_t)G * 400 * 64 * CST);
-    const size_t w_a2 = take(2 * (size_t)G * 6400 * CONV_K);
     const size_t w_c2 = take(2 * (size_t)G * 6400 * CST);
-    const size_t w_a3 = take(2 * (size_t)G * 1600 * CONV_K);
     const size_t w_c3 = take(2 * (size_t)G * 1600 * CST);
     const size_t w_X = take(4 * (size_t)T * D);
     const size_t w_xn = take(2 * (size_t)T * D);
@@ -635,9 +689,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     uint8_t *S = static_cast<uint8_t *>(h->ws);
     h->mel_raw = (float *)(S + w_mel);
     h->c1out = (bf16 *)(S + w_c1);
-    h->a2 = (bf16 *)(S + w_a2);
     h->c2out = (bf16 *)(S + w_c2);
-    h->a3 = (bf16 *)(S + w_a3);
     h->c3out = (bf16 *)(S + w_c3);
     h->X = (float *)(S + w_X);
     h->xn = (bf16 *)(S + w_xn);
@@ -851,15 +903,39 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         int64_t tok = pl.tok0;
         for (int64_t c = pl.c_first; c < pl.c_last; c++, chunk++) {
             const int nf = (int)std::min<int64_t>(CHUNK_FRAMES, pl.F - c * CHUNK_FRAMES);
-            sc[chunk] = StemChunk{i, (int)(chunk * CHUNK_FRAMES), nf, 0};
             const int nt = (int)chunk_tokens(nf);
+            // the chunk's tokens need conv3 rows t < nt, conv2 rows t < 2 nt and
+            // conv1 rows t < 4 nt (kernel 3, stride 2, padding 1)
+            sc[chunk] = StemChunk{i, (int)(chunk * CHUNK_FRAMES), nf, std::min(400, 4 * nt)};
             ct[chunk] = make_int2((int)tok, nt);
             tok += nt;
+        }
+    }
+    // conv2 / conv3 tile lists per stem group (chunk index within the group)
+    int *t2 = reinterpret_cast<int *>(H + tl.tiles2);
+    int *t3 = reinterpret_cast<int *>(H + tl.tiles3);
+    std::vector<int> g_off2, g_n2, g_off3, g_n3;
+    {
+        int o2 = 0, o3 = 0;
+        for (int64_t g0 = 0; g0 < n_chunks; g0 += h->stem_group) {
+            const int gc = (int)std::min<int64_t>(h->stem_group, n_chunks - g0);
+            g_off2.push_back(o2);
+            g_off3.push_back(o3);
+            for (int j = 0; j < gc; j++) {
+                const int nt = ct[g0 + j].y;
+                const int n2 = (std::min(200, 2 * nt) + 3) / 4, n3 = (nt + 7) / 8;
+                for (int m = 0; m < n2; m++) t2[o2++] = j * 256 + m;
+                for (int m = 0; m < n3; m++) t3[o3++] = j * 256 + m;
+            }
+            g_n2.push_back(o2 - g_off2.back());
+            g_n3.push_back(o3 - g_off3.back());
         }
     }
     TRY(tab_upload(h));
     uint8_t *Dt = static_cast<uint8_t *>(h->d_tab);
     const StemChunk *d_chunks = reinterpret_cast<const StemChunk *>(Dt + tl.chunks);
+    const int *d_t2 = reinterpret_cast<const int *>(Dt + tl.tiles2);
+    const int *d_t3 = reinterpret_cast<const int *>(Dt + tl.tiles3);
     const int2 *d_ct = reinterpret_cast<const int2 *>(Dt + tl.chunk_tok);
 
     // ---- log-mel (raw) and per-clip maxima
@@ -872,33 +948,22 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), n_max_pass, max_clip_frames, nullptr, 0, max_pass_frames));
     TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_main), n_clips, max_range_frames, h->mel_raw, 1, range_frames));
 
-    // ---- conv stem, in groups of chunks
-    for (int64_t g0 = 0; g0 < n_chunks; g0 += h->stem_group) {
+    // ---- conv stem, in groups of chunks; only tiles inside the receptive
+    // field of each chunk's tokens are computed
+    for (int64_t g0 = 0, gi = 0; g0 < n_chunks; g0 += h->stem_group, gi++) {
         const int gc = (int)std::min<int64_t>(h->stem_group, n_chunks - g0);
         {
-        Launch L1(h, "conv1", 2.0 * 9 * CST * 400 * 64 * gc, 2.0 * CST * 400 * 64 * gc + 4.0 * 128 * 800 * gc);
-        conv1_kernel<<<dim3(400, gc), 240, 0, h->stream>>>(h->mel_raw, d_chunks + g0, h->gmax_ord, h->conv1_w, h->conv1_b, h->c1out);
-        CUDA_TRY(h, cudaGetLastError());
+            double px = 0.0;
+            for (int j = 0; j < gc; j++) px += 64.0 * sc[g0 + j].t1_lim;
+            Launch L1(h, "conv1", 2.0 * 9 * CST * px, 2.0 * CST * px + 4.0 * 128 * 2 * px / 64.0);
+            conv1_kernel<<<dim3(400, gc), 240, 0, h->stream>>>(h->mel_raw, d_chunks + g0, h->gmax_ord, h->conv1_w,
+                                                              h->conv1_b, h->c1out);
+            CUDA_TRY(h, cudaGetLastError());
         }
-        const int64_t r2 = (int64_t)gc * 6400, r3 = (int64_t)gc * 1600;
-        {
-        Launch L2(h, "im2col", 0.0, 2.0 * r2 * CONV_K + 2.0 * CST * 400 * 64 * gc);
-        im2col_s2_kernel<<<(int)std::min<int64_t>(65535, (r2 * 576 + 255) / 256), 256, 0, h->stream>>>(h->c1out, 400, 64, r2, h->a2);
-        CUDA_TRY(h, cudaGetLastError());
-        }
-        GemmArgs a{};
-        a.bias = h->conv2_b;
-        a.out = h->c2out;
-        a.ldo = CST;
-        TRY((gemm<160, EPI_GELU_BF16>(h, "gemm_conv2", h->a2, r2, CONV_K, h->conv2_w, CST, a, 9 * CST)));
-        {
-        Launch L3(h, "im2col", 0.0, 2.0 * r3 * CONV_K + 2.0 * CST * 200 * 32 * gc);
-        im2col_s2_kernel<<<(int)std::min<int64_t>(65535, (r3 * 576 + 255) / 256), 256, 0, h->stream>>>(h->c2out, 200, 32, r3, h->a3);
-        CUDA_TRY(h, cudaGetLastError());
-        }
-        a.bias = h->conv3_b;
-        a.out = h->c3out;
-        TRY((gemm<160, EPI_GELU_BF16>(h, "gemm_conv3", h->a3, r3, CONV_K, h->conv3_w, CST, a, 9 * CST)));
+        TRY(gemm_conv(h, "gemm_conv2", h->c1out, gc, 400, 64, d_t2 + g_off2[gi], g_n2[gi], h->conv2_w, h->conv2_b,
+                      h->c2out));
+        TRY(gemm_conv(h, "gemm_conv3", h->c2out, gc, 200, 32, d_t3 + g_off3[gi], g_n3[gi], h->conv3_w, h->conv3_b,
+                      h->c3out));
         GemmArgs co{};
         co.out = h->X;
         co.ldo = D;
@@ -915,6 +980,9 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     const int ln_grid = (int)((T + 7) / 8);
     double attn_pairs = 0.0;  // query-key pairs inside windows
     for (int64_t c = 0; c < n_chunks; c++) attn_pairs += (double)ct[c].y * ct[c].y;
+    CUtensorMap tm_qkv;  // Q, K, V slices of one window and head: 128 rows x 64
+    if (!tmap_2d(&tm_qkv, h->qkv, (uint64_t)DQKV, (uint64_t)T, (uint64_t)DQKV * 2, 64, 128))
+        return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (qkv)");
     for (size_t l = 0; l < h->layers.size(); l++) {
         const LayerDev &L = h->layers[l];
         {
@@ -929,13 +997,14 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         TRY((gemm<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
         {
             Launch Lk(h, "attention", 4.0 * 64 * 20 * attn_pairs, 2.0 * T * (DQKV + D));
-            window_attn_kernel<<<dim3((unsigned)n_chunks, 20), 256, ATTN_SMEM, h->stream>>>(h->qkv, d_ct, h->attn);
+            window_attn_tc_kernel<<<dim3((unsigned)n_chunks, 20), 128, ATTN_TC_SMEM, h->stream>>>(tm_qkv, d_ct, h->attn,
+                                                                                                 h->err);
         }
         CUDA_TRY(h, cudaGetLastError());
         a.bias = L.bo;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm<128, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a)));
+        TRY((gemm<160, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a)));
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln2_g, L.ln2_b, h->xn, (int)T);
@@ -948,7 +1017,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         a.bias = L.b2;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm<128, EPI_RESID_F32>(h, "gemm_fc2", h->ffn, T, DFF, L.w2, D, a)));
+        TRY((gemm<160, EPI_RESID_F32>(h, "gemm_fc2", h->ffn, T, DFF, L.w2, D, a)));
     }
     if (stage == MOSS_ENC_STAGE_LAYERS) {
         CUDA_TRY(h, cudaMemcpyAsync(out, h->X, sizeof(float) * T * D, cudaMemcpyDeviceToDevice, h->stream));
@@ -965,7 +1034,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     a.bias = h->bp1;
     a.out = h->hb;
     a.ldo = D;
-    TRY((gemm<128, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, D, h->wp1, D, a)));
+    TRY((gemm<160, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, D, h->wp1, D, a)));
     a.bias = h->bp2;
     a.ldo = DOUT;
     if (stage == MOSS_ENC_STAGE_HEAD) {
@@ -982,8 +1051,8 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     a.bias = h->bd;
     a.out = out;
     a.ldo = DOUT;
-    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm<128, EPI_F32>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
-    return gemm<128, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
+    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
+    return gemm<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
 }
 
 extern "C" moss_enc_status moss_enc_forward(moss_enc *h, const moss_enc_clip *clips, int n_clips, void *rows_out,
@@ -1076,6 +1145,58 @@ extern "C" int moss_enc_profile_read(moss_enc *h, moss_enc_kernel_stat *out, int
 }
 
 extern "C" int64_t moss_enc_launch_count(const moss_enc *h) { return h ? h->launches : -1; }
+
+// --------------------------------------------------------------- one GEMM
+
+template <int BN>
+static moss_enc_status gemm_one(moss_enc *h, const bf16 *A, const bf16 *B, const float *bias, void *out, int M,
+                                int N, int K, int epi)
+{
+    GemmArgs a{};
+    a.bias = bias;
+    a.out = out;
+    a.ldo = N;
+    switch (epi) {
+    case EPI_BF16: return gemm<BN, EPI_BF16>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_GELU_BF16: return gemm<BN, EPI_GELU_BF16>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_RESID_F32: return gemm<BN, EPI_RESID_F32>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_F32: return gemm<BN, EPI_F32>(h, "gemm_api", A, M, K, B, N, a);
+    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "unsupported epilogue");
+    }
+}
+
+extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const float *bias, void *out,
+                                         int M, int N, int K, int epilogue, int block_n)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (!A || !B || !bias || !out || M < 0 || N <= 0 || K <= 0 || K % 64 != 0)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad gemm arguments");
+    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A and B must be 16-byte aligned");
+    static bool attrs_done = false;
+    if (!attrs_done) {
+        CUDA_TRY(h, (gemm_attr<128, EPI_BF16>()));
+        CUDA_TRY(h, (gemm_attr<128, EPI_GELU_BF16>()));
+        CUDA_TRY(h, (gemm_attr<128, EPI_RESID_F32>()));
+        CUDA_TRY(h, (gemm_attr<128, EPI_F32>()));
+        CUDA_TRY(h, (gemm_attr<160, EPI_BF16>()));
+        CUDA_TRY(h, (gemm_attr<160, EPI_GELU_BF16>()));
+        CUDA_TRY(h, (gemm_attr<160, EPI_RESID_F32>()));
+        CUDA_TRY(h, (gemm_attr<160, EPI_F32>()));
+        CUDA_TRY(h, (gemm_attr<256, EPI_BF16>()));
+        CUDA_TRY(h, (gemm_attr<256, EPI_GELU_BF16>()));
+        CUDA_TRY(h, (gemm_attr<256, EPI_RESID_F32>()));
+        CUDA_TRY(h, (gemm_attr<256, EPI_F32>()));
+        attrs_done = true;
+    }
+    const bf16 *a = static_cast<const bf16 *>(A), *b = static_cast<const bf16 *>(B);
+    switch (block_n) {
+    case 128: return N % 128 ? fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n") : gemm_one<128>(h, a, b, bias, out, M, N, K, epilogue);
+    case 160: return N % 160 ? fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n") : gemm_one<160>(h, a, b, bias, out, M, N, K, epilogue);
+    case 256: return N % 256 ? fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n") : gemm_one<256>(h, a, b, bias, out, M, N, K, epilogue);
+    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160 or 256");
+    }
+}
 
 // ------------------------------------------------- allocation-free log-mel
 //

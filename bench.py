@@ -223,14 +223,16 @@ def run_ours(args):
     def step():
         enc.forward(xs, out=out)
 
-    for _ in range(max(args.warmup, 3)):
+    warmup = args.warmup if args.ncu else max(args.warmup, 3)
+    for _ in range(warmup):
         step()
     enc.synchronize()
 
     # ---- timed region
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     launches0 = enc.launch_count()
-    enc.profile_enable(400 * (args.steps + 1))
+    if not args.ncu:
+        enc.profile_enable(400 * (args.steps + 1))
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -245,6 +247,10 @@ def run_ours(args):
     if dist:
         dist.barrier()
     launches = enc.launch_count() - launches0
+    if args.ncu:  # a capture run: no timing report
+        print(json.dumps({"ncu_run": True, "steps": args.steps, "warmup": warmup, "gpu_launches": launches}))
+        enc.close()
+        return
     stats = enc.profile_read()
     enc.profile_enable(0)
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -317,7 +323,7 @@ def run_ours(args):
 
     line = {
         "metric": "audio-sec encoded/sec", "value": value, "unit": "audio-s/s", "n_gpus": world,
-        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
+        "steps": args.steps, "warmup": warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded PCM, random-init bf16 weights)",
         "tokens_per_s": world * tokens / (ms_per_step / 1e3),
@@ -352,6 +358,8 @@ def main():
     ap.add_argument("--workload", default="batch16_10to30s", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cpu-windows", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu", action="store_true",
+                    help="capture run for ncu: warm-up as given (may be 0), the timed steps only, no report")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

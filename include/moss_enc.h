@@ -184,6 +184,21 @@ moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host,
                                       const int64_t *n_samples, int n_clips, void *rows_host,
                                       int64_t *row_offsets);
 
+/* ------------------------------------------------------- single GEMM */
+
+/* One bf16 GEMM on the tensor cores with a fused epilogue (the kernel every
+ * linear layer and conv of the forward uses), for tuning and unit tests:
+ *   out[M][N] = epi(A[M][K] * B[N][K]^T + bias[N])
+ *  A, B       device bf16 (uint16 bits), K-major: A [M][K], B [N][K].
+ *  bias       device fp32 [N].
+ *  out        device; bf16 [M][N] for epilogue 0 (identity) and 1 (exact
+ *             GELU), fp32 [M][N] for 2 (out += result: residual add) and
+ *             5 (fp32 store).
+ *  block_n    output tile width: 128, 160 or 256; N % block_n == 0.
+ *  K % 64 == 0.  Enqueued on the handle's stream. */
+moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const float *bias, void *out,
+                              int M, int N, int K, int epilogue, int block_n);
+
 /* ------------------------------------------------- allocation-free log-mel */
 
 /* The source pages describe no such call; it exists for callers that cannot

@@ -1,0 +1,45 @@
+"""The tensor-core GEMM with each fused epilogue against a plain PyTorch
+fp32 matmul of the same bf16 operands (ragged M, several tiles, each tile
+width)."""
+import pytest
+
+from audio_encoder_b200 import binding
+from conftest import weights
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def enc():
+    e = binding.Encoder(weights(1), 1, max_samples=16000, max_clips=1)
+    yield e
+    e.close()
+
+
+@pytest.mark.parametrize("block_n", [128, 160, 256])
+@pytest.mark.parametrize("epi", [0, 1, 2, 5])
+@pytest.mark.parametrize("M,K", [(1, 64), (300, 1280), (1000, 4608)])
+def test_gemm_epilogues(enc, block_n, epi, M, K):
+    N = {128: 1280, 160: 480, 256: 2048}[block_n]
+    g = torch.Generator().manual_seed(M * 7 + K + epi + block_n)
+    A = (torch.randn(M, K, generator=g) / K ** 0.25).bfloat16()
+    B = (torch.randn(N, K, generator=g) / K ** 0.25).bfloat16()
+    bias = torch.randn(N, generator=g) * 0.1
+    ref = A.float() @ B.float().T + bias
+    if epi == 1:
+        ref = torch.nn.functional.gelu(ref)
+    base = torch.randn(M, N, generator=g)
+    if epi == 2:
+        ref = ref + base
+    if epi in (0, 1):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    else:
+        out = base.clone().cuda() if epi == 2 else torch.empty(M, N, device="cuda")
+    enc.gemm(A.cuda(), B.cuda(), bias.cuda(), out, epi, block_n)
+    enc.synchronize()
+    got = out.float().cpu()
+    tol = 2e-2 if epi in (0, 1) else 1e-3
+    err = (got - ref).abs().max().item()
+    scale = ref.abs().max().item()
+    assert err <= tol * max(scale, 1.0), (err, scale)
