@@ -102,7 +102,7 @@ def lib():
         L.moss_enc_launch_count.restype = i64
         L.moss_enc_launch_count.argtypes = [vp]
         L.moss_enc_gemm.restype = i32
-        L.moss_enc_gemm.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32]
+        L.moss_enc_gemm.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32]
         L.moss_enc_logmel_static.restype = i32
         L.moss_enc_logmel_static.argtypes = [ctypes.POINTER(Clip), i32, ctypes.POINTER(vp), vp, vp]
         _lib = L
@@ -194,12 +194,12 @@ class Encoder:
         return {arr[i].name.decode(): dict(launches=arr[i].launches, ms=arr[i].ms, flops=arr[i].flops,
                                            bytes=arr[i].bytes) for i in range(n)}
 
-    def gemm(self, A, B, bias, out, epilogue: int, block_n: int):
+    def gemm(self, A, B, bias, out, epilogue: int, block_n: int, cta_pair: bool = True):
         """out = epi(A @ B.T + bias) on the tensor cores (A [M][K], B [N][K] bf16)."""
         M, K = A.shape
         N = B.shape[0]
         self._check(lib().moss_enc_gemm(self.h, _ptr(A), _ptr(B), _ptr(bias), _ptr(out), M, N, K,
-                                        int(epilogue), int(block_n)))
+                                        int(epilogue), int(block_n), int(bool(cta_pair))))
         return out
 
     def launch_count(self) -> int:

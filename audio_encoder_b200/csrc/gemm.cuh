@@ -9,7 +9,7 @@
 // and apply the fused epilogue (bias, GELU, residual add, SwiGLU, conv_out
 // row packing + positions) while the next tile's mainloop runs.  A warp may
 // only read the TMEM lane quarter (warp id mod 4), so two epilogue warps share
-// each quarter and split the tile's 32-column chunks between them.
+// each quarter and split the tile's 64-column groups between them.
 #pragma once
 
 #include "common.cuh"
@@ -48,6 +48,13 @@ struct GemmArgs {
     int tile_t;             // output time steps per 128-row tile
 };
 
+// Each epilogue warp stages 32 rows x 128 B in shared memory (16-byte
+// chunks swizzled by row) so that global stores go out as whole 128-byte
+// lines, 4 or 8 rows per warp instruction, instead of one 16-byte piece per
+// row.
+static constexpr uint32_t EPI_STAGE_BYTES = 32 * 128;
+static constexpr size_t SMEM_LIMIT = 227 * 1024;
+
 template <int BN>
 struct GemmCfg {
     static constexpr int BM = 128, BK = 64;
@@ -56,73 +63,178 @@ struct GemmCfg {
     static constexpr uint32_t A_BYTES = BM * BK * 2;
     static constexpr uint32_t B_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES_RAW = (216 * 1024) / STAGE_BYTES;
+    static constexpr uint32_t STAGING = EPI_WARPS * EPI_STAGE_BYTES;
+    static constexpr int STAGES_RAW = (int)((SMEM_LIMIT - 1024 - 256 - STAGING) / STAGE_BYTES);
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr uint32_t TMEM_COLS = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 256;
+    static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
     static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
 };
 
-template <int EPI>
-__device__ __forceinline__ void epilogue_store(const GemmArgs &a, int row, int col,
-                                               const uint32_t (&r)[32])
+
+__device__ __forceinline__ uint4 *stage_at(uint8_t *base, int row, int chunk)
 {
-    float v[32];
+    return reinterpret_cast<uint4 *>(base + row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ float4 ld_f4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+
+// Drain the accumulator columns [c0 of this warp's groups] of one tile for the
+// 32 rows of this warp's TMEM lane quarter.  my_row / my_ok / my_aux describe
+// the output row of this lane's tile row (aux: position index for conv_out);
+// col0 is the tile's first output column in the interleaved/GEMM space.
+template <int BN, int EPI>
+__device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, int half, int lane, uint8_t *stage,
+                                           int my_row, bool my_ok, int my_aux, int col0)
+{
+    constexpr int NG = (BN + 63) / 64;
+#pragma unroll 1
+    for (int g = half; g < NG; g += 2) {
+        const int c0 = g * 64;
+        const int nc = BN - c0 < 64 ? BN - c0 : 64;  // 64, or 32 for the last group of BN = 160
+        uint32_t r[64];
+        tmem_ld32(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        if (nc == 64) tmem_ld32(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld_wait();
+        if constexpr (EPI == EPI_SWIGLU_BF16) {
+            // r[0..31] gate, r[32..63] up -> 32 outputs (64 B per row)
+            const float *bg = a.bias + col0 + c0, *bu = bg + 32;
 #pragma unroll
-    for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
+            for (int q = 0; q < 4; q++) {
+                float o[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const float gv = __uint_as_float(r[8 * q + j]) + bg[8 * q + j];
+                    const float uv = __uint_as_float(r[32 + 8 * q + j]) + bu[8 * q + j];
+                    o[j] = silu(gv) * uv;
+                }
+                *stage_at(stage, lane, q) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                                       pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+            }
+            __syncwarp();
+            bf16 *out = reinterpret_cast<bf16 *>(a.out) + (col0 + c0) / 2;
+#pragma unroll
+            for (int it = 0; it < 4; it++) {
+                const int row = it * 8 + (lane >> 2), ch = lane & 3;
+                const int grow = __shfl_sync(0xffffffffu, my_row, row);
+                const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
+                const uint4 v = *stage_at(stage, row, ch);
+                if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
+            }
+            __syncwarp();
+        } else if constexpr (EPI == EPI_BF16 || EPI == EPI_GELU_BF16) {
+            const float *b = a.bias + col0 + c0;
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                if (q * 8 < nc) {
+                    float o[8];
+                    const float4 b0 = ld_f4(b + 8 * q), b1 = ld_f4(b + 8 * q + 4);
+                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        o[j] = __uint_as_float(r[8 * q + j]) + bb[j];
+                        if constexpr (EPI == EPI_GELU_BF16) o[j] = gelu_erf(o[j]);
+                    }
+                    *stage_at(stage, lane, q) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                                           pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+                }
+            }
+            __syncwarp();
+            bf16 *out = reinterpret_cast<bf16 *>(a.out) + col0 + c0;
+            if (nc == 64) {  // 8 lanes per 128-byte row, 4 rows per instruction
+#pragma unroll
+                for (int it = 0; it < 8; it++) {
+                    const int row = it * 4 + (lane >> 3), ch = lane & 7;
+                    const int grow = __shfl_sync(0xffffffffu, my_row, row);
+                    const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
+                    const uint4 v = *stage_at(stage, row, ch);
+                    if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
+                }
+            } else {  // 32 columns: 4 lanes per 64-byte row, 8 rows per instruction
+#pragma unroll
+                for (int it = 0; it < 4; it++) {
+                    const int row = it * 8 + (lane >> 2), ch = lane & 3;
+                    const int grow = __shfl_sync(0xffffffffu, my_row, row);
+                    const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
+                    const uint4 v = *stage_at(stage, row, ch);
+                    if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
+                }
+            }
+            __syncwarp();
+        } else {
+            // fp32 results, 32 columns (128 B per row) at a time
+#pragma unroll
+            for (int hh = 0; hh < 2; hh++) {
+                if (hh * 32 < nc) {
+                    const int cc = c0 + 32 * hh;
+#pragma unroll
+                    for (int q = 0; q < 8; q++) {
+                        float4 v = make_float4(__uint_as_float(r[32 * hh + 4 * q]), __uint_as_float(r[32 * hh + 4 * q + 1]),
+                                               __uint_as_float(r[32 * hh + 4 * q + 2]), __uint_as_float(r[32 * hh + 4 * q + 3]));
+                        if constexpr (EPI != EPI_CONVOUT_F32) {
+                            const float4 bb = ld_f4(a.bias + col0 + cc + 4 * q);
+                            v.x += bb.x;
+                            v.y += bb.y;
+                            v.z += bb.z;
+                            v.w += bb.w;
+                        }
+                        *reinterpret_cast<float4 *>(stage_at(stage, lane, q)) = v;
+                    }
+                    __syncwarp();
+                    float *out = reinterpret_cast<float *>(a.out) + col0 + cc;
+                    // all loads of the pass first (residual or positions), then the stores
+                    float4 add[8];
+                    float *dst[8];
+                    bool okv[8];
+#pragma unroll
+                    for (int it = 0; it < 8; it++) {
+                        const int row = it * 4 + (lane >> 3), ch = lane & 7;
+                        const int grow = __shfl_sync(0xffffffffu, my_row, row);
+                        okv[it] = __shfl_sync(0xffffffffu, (int)my_ok, row) != 0;
+                        int t = 0;
+                        if constexpr (EPI == EPI_CONVOUT_F32) t = __shfl_sync(0xffffffffu, my_aux, row);
+                        dst[it] = out + (size_t)grow * a.ldo + ch * 4;
+                        add[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if constexpr (EPI == EPI_RESID_F32) {
+                            if (okv[it]) add[it] = ld_f4(dst[it]);
+                        } else if constexpr (EPI == EPI_CONVOUT_F32) {
+                            if (okv[it]) add[it] = ld_f4(a.pos + (size_t)t * a.ldo + col0 + cc + ch * 4);
+                        }
+                    }
+#pragma unroll
+                    for (int it = 0; it < 8; it++) {
+                        const int row = it * 4 + (lane >> 3), ch = lane & 7;
+                        float4 v = *reinterpret_cast<const float4 *>(stage_at(stage, row, ch));
+                        v.x += add[it].x;
+                        v.y += add[it].y;
+                        v.z += add[it].z;
+                        v.w += add[it].w;
+                        if (okv[it]) *reinterpret_cast<float4 *>(dst[it]) = v;
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+    }
+}
+
+// Output row of tile row `trow` for the plain and conv_out epilogues.
+template <int EPI>
+__device__ __forceinline__ void plain_row(const GemmArgs &a, int row, int &grow, bool &ok, int &aux)
+{
     if constexpr (EPI == EPI_CONVOUT_F32) {
         const int chunk = row / 100, t = row - chunk * 100;
-        const int2 ct = a.chunk_tok[chunk];
-        if (t >= ct.y) return;
-        float *dst = reinterpret_cast<float *>(a.out) + (size_t)(ct.x + t) * a.ldo + col;
-        const float *p = a.pos + (size_t)t * a.ldo + col;
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            float4 pp = *reinterpret_cast<const float4 *>(p + i);
-            float4 o = make_float4(v[i] + pp.x, v[i + 1] + pp.y, v[i + 2] + pp.z, v[i + 3] + pp.w);
-            *reinterpret_cast<float4 *>(dst + i) = o;
-        }
-        return;
+        const bool in = row < a.M;
+        const int2 ct = in ? a.chunk_tok[chunk] : make_int2(0, 0);
+        ok = in && t < ct.y;
+        grow = ct.x + t;
+        aux = t;
     } else {
-        const float *b = a.bias + col;
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            float4 bb = *reinterpret_cast<const float4 *>(b + i);
-            v[i] += bb.x;
-            v[i + 1] += bb.y;
-            v[i + 2] += bb.z;
-            v[i + 3] += bb.w;
-        }
-        if constexpr (EPI == EPI_BF16 || EPI == EPI_GELU_BF16) {
-            if constexpr (EPI == EPI_GELU_BF16) {
-#pragma unroll
-                for (int i = 0; i < 32; i++) v[i] = gelu_erf(v[i]);
-            }
-            bf16 *dst = reinterpret_cast<bf16 *>(a.out) + (size_t)row * a.ldo + col;
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-                uint4 q = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
-                                     pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
-                *reinterpret_cast<uint4 *>(dst + i) = q;
-            }
-        } else if constexpr (EPI == EPI_RESID_F32) {
-            float *dst = reinterpret_cast<float *>(a.out) + (size_t)row * a.ldo + col;
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                float4 x = *reinterpret_cast<float4 *>(dst + i);
-                x.x += v[i];
-                x.y += v[i + 1];
-                x.z += v[i + 2];
-                x.w += v[i + 3];
-                *reinterpret_cast<float4 *>(dst + i) = x;
-            }
-        } else if constexpr (EPI == EPI_F32) {
-            float *dst = reinterpret_cast<float *>(a.out) + (size_t)row * a.ldo + col;
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-        }
+        ok = row < a.M;
+        grow = row;
+        aux = 0;
     }
 }
 
@@ -134,7 +246,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     using C = GemmCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES + C::STAGING);
     uint64_t *empty = full + C::STAGES;
     uint64_t *tfull = empty + C::STAGES;
     uint64_t *tempty = tfull + 2;
@@ -227,6 +339,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     } else {
         const int q = warp & 3;             // this warp may read TMEM lanes 32q .. 32q+31
         const int half = (warp - 2) >> 2;   // which of the two warps on this quarter
+        uint8_t *stage = smem + C::STAGES * C::STAGE_BYTES + (warp - 2) * EPI_STAGE_BYTES;
         int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             const int acc = it & 1;
@@ -234,50 +347,19 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
             if (!mbar_wait(&tfull[acc], aph, args.err)) break;
             tc_fence_after();
             const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
-            int row = mt * C::BM + q * 32 + lane;
-            bool row_ok = row < args.M;
+            int grow, aux;
+            bool ok;
             if constexpr (AMODE == A_CONV_S2) {
                 const int item = args.tile_list[mt];
                 const int r_in_chunk = (item & 255) * C::BM + q * 32 + lane;
-                row_ok = r_in_chunk < args.rows_per_chunk;
-                row = (item >> 8) * args.rows_per_chunk + r_in_chunk;
+                ok = r_in_chunk < args.rows_per_chunk;
+                grow = (item >> 8) * args.rows_per_chunk + r_in_chunk;
+                aux = 0;
+            } else {
+                plain_row<EPI>(args, mt * C::BM + q * 32 + lane, grow, ok, aux);
             }
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-            if constexpr (EPI == EPI_SWIGLU_BF16) {
-#pragma unroll 1
-                for (int c0 = 64 * half; c0 < BN; c0 += 128) {
-                    uint32_t g[32], u[32];
-                    tmem_ld32(tbase + c0, g);
-                    tmem_ld32(tbase + c0 + 32, u);
-                    tmem_ld_wait();
-                    if (row_ok) {
-                        const int col = nt * BN + c0;  // interleaved column of the gate block
-                        const float *bg = args.bias + col, *bu = args.bias + col + 32;
-                        bf16 *dst = reinterpret_cast<bf16 *>(args.out) + (size_t)row * args.ldo + col / 2;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            float o[8];
-#pragma unroll
-                            for (int j = 0; j < 8; j++) {
-                                float gv = __uint_as_float(g[i + j]) + bg[i + j];
-                                float uv = __uint_as_float(u[i + j]) + bu[i + j];
-                                o[j] = silu(gv) * uv;
-                            }
-                            uint4 qv = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                                  pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
-                            *reinterpret_cast<uint4 *>(dst + i) = qv;
-                        }
-                    }
-                }
-            } else {
-#pragma unroll 1
-                for (int c0 = 32 * half; c0 < BN; c0 += 64) {
-                    uint32_t r[32];
-                    tmem_ld32(tbase + c0, r);
-                    tmem_ld_wait();
-                    if (row_ok) epilogue_store<EPI>(args, row, nt * BN + c0, r);
-                }
-            }
+            drain_tile<BN, EPI>(args, tbase, half, lane, stage, grow, ok, aux, nt * BN);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -287,6 +369,194 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// The same GEMM on CTA pairs (cluster of 2, tcgen05 cta_group::2).
+//
+// A pair computes a 256 x BN output tile: each CTA loads its own 128 rows of
+// A and its own half of B's rows per 64-wide k-block (no multicast), and the
+// even CTA's MMA thread issues M = 256 MMAs that read both CTAs' shared
+// memory and write each CTA's 128 accumulator rows into that CTA's TMEM.  Per
+// CTA a stage is 16 KB of A plus BN*64 B of B, and each CTA streams half the
+// B traffic of the single-CTA kernel.  A 320-wide tile (N = 1280 in four)
+// is two MMAs of N = 160 per k-step; the B rows of MMA j are split between
+// the CTAs as rows [j*160, j*160+80) and [j*160+80, j*160+160).
+//  - full[s] lives in the even CTA; both producers arrive on it (count 2) and
+//    both CTAs' TMA bytes complete on it.
+//  - empty[s] and tfull[acc] live in each CTA; the even CTA's MMA thread
+//    commits once to its own and once to the odd CTA's barrier.
+//  - tempty[acc] lives in the even CTA; all 16 epilogue warps of the pair
+//    arrive on it.
+template <int BN>
+struct Gemm2Cfg {
+    static constexpr int BM = 128, BK = 64;  // rows per CTA; the pair covers 256
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    // Tiles wider than one MMA (BN = 320) are two MMAs of BN/2 per k-step.
+    static constexpr int NSUB = BN > 256 ? 2 : 1;
+    static constexpr int NS = BN / NSUB;             // N of one MMA instruction
+    static constexpr uint32_t B_SUB_BYTES = (NS / 2) * BK * 2;  // this CTA's half of one MMA's B
+    static constexpr uint32_t A_BYTES = BM * BK * 2;
+    static constexpr uint32_t B_BYTES = NSUB * B_SUB_BYTES;
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr uint32_t STAGING = EPI_WARPS * EPI_STAGE_BYTES;
+    static constexpr int STAGES_RAW = (int)((SMEM_LIMIT - 1024 - 256 - STAGING) / STAGE_BYTES);
+    static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+    static constexpr int ACC = 2 * BN <= 512 ? 2 : 1;  // TMEM accumulators (double buffer when they fit)
+    static constexpr uint32_t TMEM_COLS = ACC * BN <= 128 ? 128 : ACC * BN <= 256 ? 256 : 512;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 256;
+    static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
+    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 320, "BN must be a multiple of 32 in [64, 320]");
+    static_assert(NS % 16 == 0 && NS <= 256, "MMA N");
+    static_assert(B_SUB_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+};
+
+template <int BN, int EPI, int AMODE = A_PLAIN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmArgs args)
+{
+    using C = Gemm2Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES + C::STAGING);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *tfull = empty + C::STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; s++) {
+            mbar_init(&full[s], 2);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 2 * C::EPI_WARPS);
+        }
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_tiles = args.m_tiles * args.n_tiles;  // m_tiles counts 256-row pair tiles
+    const int num_kb = args.K / C::BK;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+                const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
+                int chunk = 0, t0 = 0;
+                if constexpr (AMODE == A_CONV_S2) {
+                    const int item = args.tile_list[2 * mt + rank];  // padded list: -1 = no rows
+                    chunk = item < 0 ? 0 : item >> 8;
+                    t0 = item < 0 ? 0 : (item & 255) * args.tile_t;
+                }
+                for (int kb = 0; kb < num_kb; kb++) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, args.err)) { ok = false; break; }
+                    uint8_t *st = smem + s * C::STAGE_BYTES;
+                    const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
+                    mbar_arrive_expect_tx_remote(fb, C::STAGE_BYTES);
+                    if constexpr (AMODE == A_CONV_S2) {
+                        const int tap = kb >> 3, kf = tap / 3, kt = tap - 3 * kf;
+                        tma_load_4d_pair(&tmA, fb, st, (kb & 7) * 64, kf - 1, 2 * t0 + kt - 1, chunk);
+                    } else {
+                        tma_load_2d_pair(&tmA, fb, st, kb * C::BK, mt * 256 + (int)rank * 128);
+                    }
+#pragma unroll
+                    for (int j = 0; j < C::NSUB; j++)
+                        tma_load_2d_pair(&tmB, fb, st + C::A_BYTES + j * C::B_SUB_BYTES, kb * C::BK,
+                                         nt * BN + j * C::NS + (int)rank * (C::NS / 2));
+                    if (++s == C::STAGES) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_bf16(256, C::NS);
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            int it = 0;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++it) {
+                const int acc = it % C::ACC;
+                const uint32_t aph = (it / C::ACC) & 1;
+                if (!mbar_wait(&tempty[acc], aph ^ 1, args.err)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * BN;
+                for (int kb = 0; kb < num_kb; kb++) {
+                    if (!mbar_wait(&full[s], ph, args.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < C::BK / 16; k++)
+#pragma unroll
+                        for (int j = 0; j < C::NSUB; j++)
+                            mma_bf16_pair(d + j * C::NS, sw128_desc(a_addr + k * 32),
+                                          sw128_desc(b_addr + j * C::B_SUB_BYTES + k * 32), idesc, (kb | k) != 0);
+                    const uint32_t eb = smem_u32(&empty[s]);
+                    mma_commit_pair(map_to_rank(eb, 0));
+                    mma_commit_pair(map_to_rank(eb, 1));
+                    if (++s == C::STAGES) { s = 0; ph ^= 1; }
+                }
+                if (ok) {
+                    const uint32_t tb = smem_u32(&tfull[acc]);
+                    mma_commit_pair(map_to_rank(tb, 0));
+                    mma_commit_pair(map_to_rank(tb, 1));
+                }
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        uint8_t *stage = smem + C::STAGES * C::STAGE_BYTES + (warp - 2) * EPI_STAGE_BYTES;
+        int it = 0;
+        for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
+            const int acc = it % C::ACC;
+            const uint32_t aph = (it / C::ACC) & 1;
+            if (!mbar_wait(&tfull[acc], aph, args.err)) break;
+            tc_fence_after();
+            const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
+            int grow, aux;
+            bool ok;
+            if constexpr (AMODE == A_CONV_S2) {
+                const int item = args.tile_list[2 * mt + rank];
+                const int r_in_chunk = (item & 255) * 128 + q * 32 + lane;
+                ok = item >= 0 && r_in_chunk < args.rows_per_chunk;
+                grow = (item >> 8) * args.rows_per_chunk + r_in_chunk;
+                aux = 0;
+            } else {
+                plain_row<EPI>(args, mt * 256 + (int)rank * 128 + q * 32 + lane, grow, ok, aux);
+            }
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+            drain_tile<BN, EPI>(args, tbase, half, lane, stage, grow, ok, aux, nt * BN);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&tempty[acc]), 0));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while its partner may still touch its memory
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
 }
 
 }  // namespace moss

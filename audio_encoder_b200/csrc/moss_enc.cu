@@ -199,6 +199,40 @@ static moss_enc_status gemm(moss_enc *h, const char *name, const bf16 *A, int64_
     return MOSS_ENC_OK;
 }
 
+// The same on CTA pairs (256-row tiles, cluster of 2).
+template <int BN, int EPI>
+static moss_enc_status gemm2(moss_enc *h, const char *name, const bf16 *A, int64_t M, int K, const bf16 *B, int N,
+                             GemmArgs a, int k_alg = 0)
+{
+    if (M <= 0) return MOSS_ENC_OK;
+    if (K % 64 != 0 || N % BN != 0 || M > INT32_MAX)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "gemm shape not supported");
+    CUtensorMap ta, tb;
+    if (!tmap_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128) ||
+        !tmap_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, 64, Gemm2Cfg<BN>::NS / 2))
+        return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    a.M = (int)M;
+    a.N = N;
+    a.K = K;
+    a.m_tiles = (int)((M + 255) / 256);
+    a.n_tiles = N / BN;
+    a.err = h->err;
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int grid = 2 * std::min(tiles, h->num_sms / 2);
+    const double ka = k_alg > 0 ? k_alg : K;
+    Launch L(h, name, 2.0 * M * N * ka, 2.0 * M * ka + 2.0 * N * ka + epi_out_bytes(EPI) * M * N);
+    gemm_tc2_kernel<BN, EPI><<<grid, Gemm2Cfg<BN>::THREADS, Gemm2Cfg<BN>::SMEM, h->stream>>>(ta, tb, a);
+    CUDA_TRY(h, cudaGetLastError());
+    return MOSS_ENC_OK;
+}
+
+template <int BN, int EPI>
+static cudaError_t gemm2_attr()
+{
+    return cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Gemm2Cfg<BN>::SMEM);
+}
+
 #define TRY(x)                                  \
     do {                                        \
         moss_enc_status s_ = (x);               \
@@ -223,8 +257,9 @@ static bool tmap_conv(CUtensorMap *m, const void *ptr, int chunks, int Ti, int F
     return r == CUDA_SUCCESS;
 }
 
-// conv2/conv3 as an implicit GEMM: out [chunk][To][Fo][480] = GELU(conv(in) + b)
-// for the 128-row tiles listed in d_tiles (n_items of them).
+// conv2/conv3 as an implicit GEMM on CTA pairs: out [chunk][To][Fo][480] =
+// GELU(conv(in) + b) for the 128-row tiles listed in d_tiles (n_items of
+// them, padded with -1 to an even count; CTA r of pair p takes item 2p + r).
 static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, int chunks, int Ti, int Fi,
                                  const int *d_tiles, int n_items, const bf16 *W, const float *bias, bf16 *out)
 {
@@ -232,13 +267,13 @@ static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, 
     const int Fo = (Fi + 1) / 2, To = (Ti + 1) / 2, tile_t = 128 / Fo;
     CUtensorMap ta, tb;
     if (!tmap_conv(&ta, in, chunks, Ti, Fi, tile_t) ||
-        !tmap_2d(&tb, W, (uint64_t)CONV_K, (uint64_t)CST, (uint64_t)CONV_K * 2, 64, 160))
+        !tmap_2d(&tb, W, (uint64_t)CONV_K, (uint64_t)CST, (uint64_t)CONV_K * 2, 64, 80))
         return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (conv)");
     GemmArgs a{};
     a.M = n_items * 128;
     a.N = CST;
     a.K = CONV_K;
-    a.m_tiles = n_items;
+    a.m_tiles = (n_items + 1) / 2;
     a.n_tiles = CST / 160;
     a.err = h->err;
     a.bias = bias;
@@ -247,9 +282,9 @@ static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, 
     a.tile_list = d_tiles;
     a.rows_per_chunk = To * Fo;
     a.tile_t = tile_t;
-    const int grid = std::min(a.m_tiles * a.n_tiles, h->num_sms);
+    const int grid = 2 * std::min(a.m_tiles * a.n_tiles, h->num_sms / 2);
     Launch L(h, name, 2.0 * 128.0 * n_items * CST * (9.0 * CST), 2.0 * 128.0 * n_items * (9.0 * CST) * 0.25 + 2.0 * 128.0 * n_items * CST);
-    gemm_tc_kernel<160, EPI_GELU_BF16, A_CONV_S2><<<grid, GemmCfg<160>::THREADS, GemmCfg<160>::SMEM, h->stream>>>(ta, tb, a);
+    gemm_tc2_kernel<160, EPI_GELU_BF16, A_CONV_S2><<<grid, Gemm2Cfg<160>::THREADS, Gemm2Cfg<160>::SMEM, h->stream>>>(ta, tb, a);
     CUDA_TRY(h, cudaGetLastError());
     return MOSS_ENC_OK;
 }
@@ -405,8 +440,8 @@ static TabLayout tab_layout(int64_t max_clips, int64_t max_chunks)
     t.chunks = take(sizeof(StemChunk) * max_chunks);
     t.chunk_tok = take(sizeof(int2) * max_chunks);
     t.logmax_src = take(sizeof(float *) * max_clips);
-    t.tiles2 = take(sizeof(int) * max_chunks * C2_TILES);
-    t.tiles3 = take(sizeof(int) * max_chunks * C3_TILES);
+    t.tiles2 = take(sizeof(int) * (max_chunks * C2_TILES + max_chunks));
+    t.tiles3 = take(sizeof(int) * (max_chunks * C3_TILES + max_chunks));
     t.total = o;
     return t;
 }
@@ -428,8 +463,15 @@ extern "C" void moss_enc_destroy(moss_enc *h)
 
 static moss_enc_status set_kernel_attrs(moss_enc *h)
 {
-    CUDA_TRY(h, cudaFuncSetAttribute(gemm_tc_kernel<160, EPI_GELU_BF16, A_CONV_S2>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GemmCfg<160>::SMEM));
+    CUDA_TRY(h, cudaFuncSetAttribute(gemm_tc2_kernel<160, EPI_GELU_BF16, A_CONV_S2>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Gemm2Cfg<160>::SMEM));
+    CUDA_TRY(h, (gemm2_attr<256, EPI_BF16>()));
+    CUDA_TRY(h, (gemm2_attr<256, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm2_attr<320, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm2_attr<320, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm2_attr<256, EPI_SWIGLU_BF16>()));
+    CUDA_TRY(h, (gemm2_attr<256, EPI_F32>()));
+    CUDA_TRY(h, (gemm2_attr<320, EPI_CONVOUT_F32>()));
     CUDA_TRY(h, (gemm_attr<160, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm_attr<160, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm_attr<256, EPI_BF16>()));
@@ -927,6 +969,9 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
                 for (int m = 0; m < n2; m++) t2[o2++] = j * 256 + m;
                 for (int m = 0; m < n3; m++) t3[o3++] = j * 256 + m;
             }
+            // CTA pairs take two list entries at a time: pad to an even count
+            if ((o2 - g_off2.back()) & 1) t2[o2++] = -1;
+            if ((o3 - g_off3.back()) & 1) t3[o3++] = -1;
             g_n2.push_back(o2 - g_off2.back());
             g_n3.push_back(o3 - g_off3.back());
         }
@@ -969,7 +1014,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         co.ldo = D;
         co.pos = h->pos;
         co.chunk_tok = d_ct + g0;
-        TRY((gemm<128, EPI_CONVOUT_F32>(h, "gemm_conv_out", h->c3out, (int64_t)gc * 100, 7680, h->conv_out_w, D, co)));
+        TRY((gemm2<320, EPI_CONVOUT_F32>(h, "gemm_conv_out", h->c3out, (int64_t)gc * 100, 7680, h->conv_out_w, D, co)));
     }
     if (stage == MOSS_ENC_STAGE_STEM) {
         CUDA_TRY(h, cudaMemcpyAsync(out, h->X, sizeof(float) * T * D, cudaMemcpyDeviceToDevice, h->stream));
@@ -994,7 +1039,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         a.bias = L.bqkv;
         a.out = h->qkv;
         a.ldo = DQKV;
-        TRY((gemm<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
+        TRY((gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
         {
             Launch Lk(h, "attention", 4.0 * 64 * 20 * attn_pairs, 2.0 * T * (DQKV + D));
             window_attn_tc_kernel<<<dim3((unsigned)n_chunks, 20), 128, ATTN_TC_SMEM, h->stream>>>(tm_qkv, d_ct, h->attn,
@@ -1004,7 +1049,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         a.bias = L.bo;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm<160, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a)));
+        TRY((gemm2<320, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a)));
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln2_g, L.ln2_b, h->xn, (int)T);
@@ -1013,11 +1058,11 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         a.bias = L.b1;
         a.out = h->ffn;
         a.ldo = DFF;
-        TRY((gemm<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.w1, DFF, a)));
+        TRY((gemm2<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.w1, DFF, a)));
         a.bias = L.b2;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm<160, EPI_RESID_F32>(h, "gemm_fc2", h->ffn, T, DFF, L.w2, D, a)));
+        TRY((gemm2<320, EPI_RESID_F32>(h, "gemm_fc2", h->ffn, T, DFF, L.w2, D, a)));
     }
     if (stage == MOSS_ENC_STAGE_LAYERS) {
         CUDA_TRY(h, cudaMemcpyAsync(out, h->X, sizeof(float) * T * D, cudaMemcpyDeviceToDevice, h->stream));
@@ -1034,25 +1079,25 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     a.bias = h->bp1;
     a.out = h->hb;
     a.ldo = D;
-    TRY((gemm<160, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, D, h->wp1, D, a)));
+    TRY((gemm2<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, D, h->wp1, D, a)));
     a.bias = h->bp2;
     a.ldo = DOUT;
     if (stage == MOSS_ENC_STAGE_HEAD) {
         a.out = out;
-        return gemm<256, EPI_F32>(h, "gemm_proj2", h->hb, T, D, h->wp2, DOUT, a);
+        return gemm2<256, EPI_F32>(h, "gemm_proj2", h->hb, T, D, h->wp2, DOUT, a);
     }
     a.out = h->h2;
-    TRY((gemm<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, D, h->wp2, DOUT, a)));
+    TRY((gemm2<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, D, h->wp2, DOUT, a)));
     // ---- SwiGLU adapter
     a.bias = h->bgu;
     a.out = h->gu;
     a.ldo = DADP;
-    TRY((gemm<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, h->wgu, 2 * DADP, a)));
+    TRY((gemm2<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, h->wgu, 2 * DADP, a)));
     a.bias = h->bd;
     a.out = out;
     a.ldo = DOUT;
-    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
-    return gemm<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
+    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
+    return gemm2<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
 }
 
 extern "C" moss_enc_status moss_enc_forward(moss_enc *h, const moss_enc_clip *clips, int n_clips, void *rows_out,
@@ -1150,23 +1195,41 @@ extern "C" int64_t moss_enc_launch_count(const moss_enc *h) { return h ? h->laun
 
 template <int BN>
 static moss_enc_status gemm_one(moss_enc *h, const bf16 *A, const bf16 *B, const float *bias, void *out, int M,
-                                int N, int K, int epi)
+                                int N, int K, int epi, int pair)
 {
     GemmArgs a{};
     a.bias = bias;
     a.out = out;
     a.ldo = N;
-    switch (epi) {
-    case EPI_BF16: return gemm<BN, EPI_BF16>(h, "gemm_api", A, M, K, B, N, a);
-    case EPI_GELU_BF16: return gemm<BN, EPI_GELU_BF16>(h, "gemm_api", A, M, K, B, N, a);
-    case EPI_RESID_F32: return gemm<BN, EPI_RESID_F32>(h, "gemm_api", A, M, K, B, N, a);
-    case EPI_F32: return gemm<BN, EPI_F32>(h, "gemm_api", A, M, K, B, N, a);
+    switch (epi * 2 + (pair ? 1 : 0)) {
+    case EPI_BF16 * 2: return gemm<BN, EPI_BF16>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_GELU_BF16 * 2: return gemm<BN, EPI_GELU_BF16>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_RESID_F32 * 2: return gemm<BN, EPI_RESID_F32>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_F32 * 2: return gemm<BN, EPI_F32>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_BF16 * 2 + 1: return gemm2<BN, EPI_BF16>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_GELU_BF16 * 2 + 1: return gemm2<BN, EPI_GELU_BF16>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_RESID_F32 * 2 + 1: return gemm2<BN, EPI_RESID_F32>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_F32 * 2 + 1: return gemm2<BN, EPI_F32>(h, "gemm_api", A, M, K, B, N, a);
     default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "unsupported epilogue");
     }
 }
 
+template <int BN>
+static cudaError_t gemm_api_attrs()
+{
+    cudaError_t e;
+    if ((e = gemm_attr<BN, EPI_BF16>()) != cudaSuccess) return e;
+    if ((e = gemm_attr<BN, EPI_GELU_BF16>()) != cudaSuccess) return e;
+    if ((e = gemm_attr<BN, EPI_RESID_F32>()) != cudaSuccess) return e;
+    if ((e = gemm_attr<BN, EPI_F32>()) != cudaSuccess) return e;
+    if ((e = gemm2_attr<BN, EPI_BF16>()) != cudaSuccess) return e;
+    if ((e = gemm2_attr<BN, EPI_GELU_BF16>()) != cudaSuccess) return e;
+    if ((e = gemm2_attr<BN, EPI_RESID_F32>()) != cudaSuccess) return e;
+    return gemm2_attr<BN, EPI_F32>();
+}
+
 extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const float *bias, void *out,
-                                         int M, int N, int K, int epilogue, int block_n)
+                                         int M, int N, int K, int epilogue, int block_n, int cta_pair)
 {
     if (!h) return MOSS_ENC_ERR_INVALID_ARG;
     if (!A || !B || !bias || !out || M < 0 || N <= 0 || K <= 0 || K % 64 != 0)
@@ -1175,26 +1238,31 @@ extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void 
         return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A and B must be 16-byte aligned");
     static bool attrs_done = false;
     if (!attrs_done) {
-        CUDA_TRY(h, (gemm_attr<128, EPI_BF16>()));
-        CUDA_TRY(h, (gemm_attr<128, EPI_GELU_BF16>()));
-        CUDA_TRY(h, (gemm_attr<128, EPI_RESID_F32>()));
-        CUDA_TRY(h, (gemm_attr<128, EPI_F32>()));
-        CUDA_TRY(h, (gemm_attr<160, EPI_BF16>()));
-        CUDA_TRY(h, (gemm_attr<160, EPI_GELU_BF16>()));
-        CUDA_TRY(h, (gemm_attr<160, EPI_RESID_F32>()));
-        CUDA_TRY(h, (gemm_attr<160, EPI_F32>()));
-        CUDA_TRY(h, (gemm_attr<256, EPI_BF16>()));
-        CUDA_TRY(h, (gemm_attr<256, EPI_GELU_BF16>()));
-        CUDA_TRY(h, (gemm_attr<256, EPI_RESID_F32>()));
-        CUDA_TRY(h, (gemm_attr<256, EPI_F32>()));
+        CUDA_TRY(h, gemm_api_attrs<128>());
+        CUDA_TRY(h, gemm_api_attrs<160>());
+        CUDA_TRY(h, gemm_api_attrs<256>());
+        CUDA_TRY(h, (gemm2_attr<320, EPI_BF16>()));
+        CUDA_TRY(h, (gemm2_attr<320, EPI_GELU_BF16>()));
+        CUDA_TRY(h, (gemm2_attr<320, EPI_RESID_F32>()));
+        CUDA_TRY(h, (gemm2_attr<320, EPI_F32>()));
         attrs_done = true;
     }
     const bf16 *a = static_cast<const bf16 *>(A), *b = static_cast<const bf16 *>(B);
+    if (N % block_n != 0) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n != 0");
     switch (block_n) {
-    case 128: return N % 128 ? fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n") : gemm_one<128>(h, a, b, bias, out, M, N, K, epilogue);
-    case 160: return N % 160 ? fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n") : gemm_one<160>(h, a, b, bias, out, M, N, K, epilogue);
-    case 256: return N % 256 ? fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n") : gemm_one<256>(h, a, b, bias, out, M, N, K, epilogue);
-    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160 or 256");
+    case 128: return gemm_one<128>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
+    case 160: return gemm_one<160>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
+    case 256: return gemm_one<256>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
+    case 320:
+        if (!cta_pair) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n 320 needs cta_pair");
+        switch (epilogue) {
+        case EPI_BF16: return gemm2<320, EPI_BF16>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
+        case EPI_GELU_BF16: return gemm2<320, EPI_GELU_BF16>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
+        case EPI_RESID_F32: return gemm2<320, EPI_RESID_F32>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
+        case EPI_F32: return gemm2<320, EPI_F32>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
+        default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "unsupported epilogue");
+        }
+    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160, 256 or 320");
     }
 }
 

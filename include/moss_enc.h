@@ -186,18 +186,21 @@ moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host,
 
 /* ------------------------------------------------------- single GEMM */
 
-/* One bf16 GEMM on the tensor cores with a fused epilogue (the kernel every
- * linear layer and conv of the forward uses), for tuning and unit tests:
+/* One bf16 GEMM on the tensor cores with a fused epilogue (the kernels every
+ * linear layer and conv of the forward use), for tuning and unit tests:
  *   out[M][N] = epi(A[M][K] * B[N][K]^T + bias[N])
  *  A, B       device bf16 (uint16 bits), K-major: A [M][K], B [N][K].
  *  bias       device fp32 [N].
  *  out        device; bf16 [M][N] for epilogue 0 (identity) and 1 (exact
  *             GELU), fp32 [M][N] for 2 (out += result: residual add) and
  *             5 (fp32 store).
- *  block_n    output tile width: 128, 160 or 256; N % block_n == 0.
+ *  block_n    output tile width: 128, 160, 256, or 320 (CTA pairs only);
+ *             N % block_n == 0.
+ *  cta_pair   0: one CTA per 128 x block_n tile; 1: CTA pairs (cluster of
+ *             2) on 256 x block_n tiles, as the forward uses.
  *  K % 64 == 0.  Enqueued on the handle's stream. */
 moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const float *bias, void *out,
-                              int M, int N, int K, int epilogue, int block_n);
+                              int M, int N, int K, int epilogue, int block_n, int cta_pair);
 
 /* ------------------------------------------------- allocation-free log-mel */
 

@@ -17,11 +17,12 @@ def enc():
     e.close()
 
 
-@pytest.mark.parametrize("block_n", [128, 160, 256])
+@pytest.mark.parametrize("pair,block_n", [(False, 128), (False, 160), (False, 256), (True, 128), (True, 160),
+                                          (True, 256), (True, 320)])
 @pytest.mark.parametrize("epi", [0, 1, 2, 5])
-@pytest.mark.parametrize("M,K", [(1, 64), (300, 1280), (1000, 4608)])
-def test_gemm_epilogues(enc, block_n, epi, M, K):
-    N = {128: 1280, 160: 480, 256: 2048}[block_n]
+@pytest.mark.parametrize("M,K", [(1, 64), (300, 1280), (1000, 4608), (4608, 1280)])
+def test_gemm_epilogues(enc, pair, block_n, epi, M, K):
+    N = {128: 1280, 160: 480, 256: 2048, 320: 1280}[block_n]
     g = torch.Generator().manual_seed(M * 7 + K + epi + block_n)
     A = (torch.randn(M, K, generator=g) / K ** 0.25).bfloat16()
     B = (torch.randn(N, K, generator=g) / K ** 0.25).bfloat16()
@@ -36,7 +37,7 @@ def test_gemm_epilogues(enc, block_n, epi, M, K):
         out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     else:
         out = base.clone().cuda() if epi == 2 else torch.empty(M, N, device="cuda")
-    enc.gemm(A.cuda(), B.cuda(), bias.cuda(), out, epi, block_n)
+    enc.gemm(A.cuda(), B.cuda(), bias.cuda(), out, epi, block_n, pair)
     enc.synchronize()
     got = out.float().cpu()
     tol = 2e-2 if epi in (0, 1) else 1e-3
