@@ -88,6 +88,12 @@ struct moss_enc {
     };
     std::vector<cudaEvent_t> prof_ev;
     std::vector<Rec> prof_rec;
+
+    // CUDA graph of the last forward request (replayed while it repeats)
+    void *d_tab_graph = nullptr;
+    cudaGraphExec_t graph_exec = nullptr;
+    std::vector<uint8_t> graph_key;
+    int64_t graph_launches = 0;
 };
 
 namespace {
@@ -454,7 +460,9 @@ extern "C" void moss_enc_destroy(moss_enc *h)
     else cudaDeviceSynchronize();
     if (h->wmem) cudaFree(h->wmem);
     if (h->ws) cudaFree(h->ws);
+    if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
     if (h->d_tab) cudaFree(h->d_tab);
+    if (h->d_tab_graph) cudaFree(h->d_tab_graph);
     if (h->h_tab) cudaFreeHost(h->h_tab);
     if (h->tab_event) cudaEventDestroy(h->tab_event);
     for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
@@ -750,6 +758,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     const TabLayout tl = tab_layout(cfg->max_clips, h->max_chunks);
     h->tab_bytes = tl.total;
     if (cudaMalloc(&h->d_tab, tl.total) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
+    if (cudaMalloc(&h->d_tab_graph, tl.total) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaMallocHost(&h->h_tab, tl.total) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaEventCreateWithFlags(&h->tab_event, cudaEventDisableTiming) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
     if (cudaDeviceSynchronize() != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
@@ -888,96 +897,39 @@ extern "C" moss_enc_status moss_enc_logmel(moss_enc *h, const moss_enc_clip *cli
 
 // ----------------------------------------------------------------- forward
 
-static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int n_clips, int stage,
-                                    void *out, int64_t *row_offsets)
-{
-    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
-    if (n_clips < 0 || (n_clips > 0 && !clips) || !row_offsets) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad argument");
-    if (n_clips > h->cfg.max_clips) return fail(h, MOSS_ENC_ERR_CAPACITY, "too many clips");
-    if (stage < MOSS_ENC_STAGE_STEM || stage > MOSS_ENC_STAGE_ADAPTER) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad stage");
-
-    std::vector<ClipPlan> plans(n_clips);
-    int64_t samples = 0, T = 0, n_chunks = 0, max_range_frames = 0, max_clip_frames = 0;
-    row_offsets[0] = 0;
-    for (int i = 0; i < n_clips; i++) {
-        const moss_enc_clip &c = clips[i];
-        if (!plan_clip(c.n_samples, c.begin, c.end, &plans[i])) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad clip range");
-        if (plans[i].ntok > 0 && !c.pcm) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null pcm");
-        if (plans[i].F > INT32_MAX / 2) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "clip too long");
-        plans[i].tok0 = T;
-        T += plans[i].ntok;
-        row_offsets[i + 1] = T;
-        samples += c.end - c.begin;
-        n_chunks += plans[i].c_last - plans[i].c_first;
-        max_range_frames = std::max(max_range_frames, plans[i].f_end - plans[i].f_begin);
-        max_clip_frames = std::max(max_clip_frames, plans[i].F);
-    }
-    if (samples > h->cfg.max_samples || T > h->max_tokens || n_chunks > h->max_chunks)
-        return fail(h, MOSS_ENC_ERR_CAPACITY, "request exceeds the capacity set at create");
-    if (T > 0 && !out) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null output");
-    if (T == 0) return MOSS_ENC_OK;
-
-    // ---- tables
-    TRY(tab_begin(h));
-    const TabLayout tl = tab_layout(h->cfg.max_clips, h->max_chunks);
-    uint8_t *H = static_cast<uint8_t *>(h->h_tab);
-    const float **lsrc = reinterpret_cast<const float **>(H + tl.logmax_src);
-    MelClip *mm = reinterpret_cast<MelClip *>(H + tl.clips_main);
-    MelClip *mx = reinterpret_cast<MelClip *>(H + tl.clips_max);
-    StemChunk *sc = reinterpret_cast<StemChunk *>(H + tl.chunks);
-    int2 *ct = reinterpret_cast<int2 *>(H + tl.chunk_tok);
+// Host-side result of planning one forward: counts and the per-group conv
+// tile lists (the tables themselves sit in the staging buffer).
+struct FwdPlan {
+    int n_clips = 0;
+    int64_t n_chunks = 0, T = 0;
     int n_max_pass = 0;
-    int64_t chunk = 0, max_pass_frames = 0, range_frames = 0;
-    for (int i = 0; i < n_clips; i++) {
-        const ClipPlan &pl = plans[i];
-        const bool whole = pl.f_begin == 0 && pl.f_end == pl.F;
-        const bool own = clips[i].log_max == nullptr;
-        lsrc[i] = clips[i].log_max;
-        // main pass: frames [800 c_first, f_end) into rows of this clip's chunks
-        const int64_t fb = pl.c_first * CHUNK_FRAMES;
-        mm[i] = MelClip{clips[i].pcm, (long long)pl.n, (long long)chunk * CHUNK_FRAMES, (int)fb, (int)pl.f_end,
-                        own && whole ? i : -1, 0};
-        if (own && !whole) {
-            mx[n_max_pass++] = MelClip{clips[i].pcm, (long long)pl.n, 0, 0, (int)pl.F, i, 0};
-            max_pass_frames += pl.F;
-        }
-        range_frames += pl.f_end - fb;
-        int64_t tok = pl.tok0;
-        for (int64_t c = pl.c_first; c < pl.c_last; c++, chunk++) {
-            const int nf = (int)std::min<int64_t>(CHUNK_FRAMES, pl.F - c * CHUNK_FRAMES);
-            const int nt = (int)chunk_tokens(nf);
-            // the chunk's tokens need conv3 rows t < nt, conv2 rows t < 2 nt and
-            // conv1 rows t < 4 nt (kernel 3, stride 2, padding 1)
-            sc[chunk] = StemChunk{i, (int)(chunk * CHUNK_FRAMES), nf, std::min(400, 4 * nt)};
-            ct[chunk] = make_int2((int)tok, nt);
-            tok += nt;
-        }
-    }
-    // conv2 / conv3 tile lists per stem group (chunk index within the group)
-    int *t2 = reinterpret_cast<int *>(H + tl.tiles2);
-    int *t3 = reinterpret_cast<int *>(H + tl.tiles3);
+    int64_t max_clip_frames = 0, max_range_frames = 0, max_pass_frames = 0, range_frames = 0;
+    const StemChunk *sc = nullptr;
+    const int2 *ct = nullptr;
     std::vector<int> g_off2, g_n2, g_off3, g_n3;
-    {
-        int o2 = 0, o3 = 0;
-        for (int64_t g0 = 0; g0 < n_chunks; g0 += h->stem_group) {
-            const int gc = (int)std::min<int64_t>(h->stem_group, n_chunks - g0);
-            g_off2.push_back(o2);
-            g_off3.push_back(o3);
-            for (int j = 0; j < gc; j++) {
-                const int nt = ct[g0 + j].y;
-                const int n2 = (std::min(200, 2 * nt) + 3) / 4, n3 = (nt + 7) / 8;
-                for (int m = 0; m < n2; m++) t2[o2++] = j * 256 + m;
-                for (int m = 0; m < n3; m++) t3[o3++] = j * 256 + m;
-            }
-            // CTA pairs take two list entries at a time: pad to an even count
-            if ((o2 - g_off2.back()) & 1) t2[o2++] = -1;
-            if ((o3 - g_off3.back()) & 1) t3[o3++] = -1;
-            g_n2.push_back(o2 - g_off2.back());
-            g_n3.push_back(o3 - g_off3.back());
-        }
-    }
-    TRY(tab_upload(h));
-    uint8_t *Dt = static_cast<uint8_t *>(h->d_tab);
+};
+
+// Identity of a forward request for graph reuse.
+static std::vector<uint8_t> request_key(const moss_enc_clip *clips, int n_clips, const void *out)
+{
+    std::vector<uint8_t> k(sizeof(int) + sizeof(void *) + sizeof(moss_enc_clip) * (size_t)n_clips);
+    std::memcpy(k.data(), &n_clips, sizeof(int));
+    std::memcpy(k.data() + sizeof(int), &out, sizeof(void *));
+    if (n_clips > 0) std::memcpy(k.data() + sizeof(int) + sizeof(void *), clips, sizeof(moss_enc_clip) * (size_t)n_clips);
+    return k;
+}
+
+static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt, int stage, void *out)
+{
+    const TabLayout tl = tab_layout(h->cfg.max_clips, h->max_chunks);
+    const int n_clips = P.n_clips;
+    const int64_t n_chunks = P.n_chunks, T = P.T;
+    const int n_max_pass = P.n_max_pass;
+    const int64_t max_clip_frames = P.max_clip_frames, max_range_frames = P.max_range_frames;
+    const int64_t max_pass_frames = P.max_pass_frames, range_frames = P.range_frames;
+    const StemChunk *sc = P.sc;
+    const int2 *ct = P.ct;
+    const std::vector<int> &g_off2 = P.g_off2, &g_n2 = P.g_n2, &g_off3 = P.g_off3, &g_n3 = P.g_n3;
     const StemChunk *d_chunks = reinterpret_cast<const StemChunk *>(Dt + tl.chunks);
     const int *d_t2 = reinterpret_cast<const int *>(Dt + tl.tiles2);
     const int *d_t3 = reinterpret_cast<const int *>(Dt + tl.tiles3);
@@ -1099,6 +1051,155 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
     return gemm2<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
 }
+
+static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int n_clips, int stage,
+                                    void *out, int64_t *row_offsets)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (n_clips < 0 || (n_clips > 0 && !clips) || !row_offsets) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad argument");
+    if (n_clips > h->cfg.max_clips) return fail(h, MOSS_ENC_ERR_CAPACITY, "too many clips");
+    if (stage < MOSS_ENC_STAGE_STEM || stage > MOSS_ENC_STAGE_ADAPTER) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad stage");
+
+    std::vector<ClipPlan> plans(n_clips);
+    int64_t samples = 0, T = 0, n_chunks = 0, max_range_frames = 0, max_clip_frames = 0;
+    row_offsets[0] = 0;
+    for (int i = 0; i < n_clips; i++) {
+        const moss_enc_clip &c = clips[i];
+        if (!plan_clip(c.n_samples, c.begin, c.end, &plans[i])) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad clip range");
+        if (plans[i].ntok > 0 && !c.pcm) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null pcm");
+        if (plans[i].F > INT32_MAX / 2) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "clip too long");
+        plans[i].tok0 = T;
+        T += plans[i].ntok;
+        row_offsets[i + 1] = T;
+        samples += c.end - c.begin;
+        n_chunks += plans[i].c_last - plans[i].c_first;
+        max_range_frames = std::max(max_range_frames, plans[i].f_end - plans[i].f_begin);
+        max_clip_frames = std::max(max_clip_frames, plans[i].F);
+    }
+    if (samples > h->cfg.max_samples || T > h->max_tokens || n_chunks > h->max_chunks)
+        return fail(h, MOSS_ENC_ERR_CAPACITY, "request exceeds the capacity set at create");
+    if (T > 0 && !out) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null output");
+    if (T == 0) return MOSS_ENC_OK;
+
+    // ---- tables
+    TRY(tab_begin(h));
+    const TabLayout tl = tab_layout(h->cfg.max_clips, h->max_chunks);
+    uint8_t *H = static_cast<uint8_t *>(h->h_tab);
+    const float **lsrc = reinterpret_cast<const float **>(H + tl.logmax_src);
+    MelClip *mm = reinterpret_cast<MelClip *>(H + tl.clips_main);
+    MelClip *mx = reinterpret_cast<MelClip *>(H + tl.clips_max);
+    StemChunk *sc = reinterpret_cast<StemChunk *>(H + tl.chunks);
+    int2 *ct = reinterpret_cast<int2 *>(H + tl.chunk_tok);
+    int n_max_pass = 0;
+    int64_t chunk = 0, max_pass_frames = 0, range_frames = 0;
+    for (int i = 0; i < n_clips; i++) {
+        const ClipPlan &pl = plans[i];
+        const bool whole = pl.f_begin == 0 && pl.f_end == pl.F;
+        const bool own = clips[i].log_max == nullptr;
+        lsrc[i] = clips[i].log_max;
+        // main pass: frames [800 c_first, f_end) into rows of this clip's chunks
+        const int64_t fb = pl.c_first * CHUNK_FRAMES;
+        mm[i] = MelClip{clips[i].pcm, (long long)pl.n, (long long)chunk * CHUNK_FRAMES, (int)fb, (int)pl.f_end,
+                        own && whole ? i : -1, 0};
+        if (own && !whole) {
+            mx[n_max_pass++] = MelClip{clips[i].pcm, (long long)pl.n, 0, 0, (int)pl.F, i, 0};
+            max_pass_frames += pl.F;
+        }
+        range_frames += pl.f_end - fb;
+        int64_t tok = pl.tok0;
+        for (int64_t c = pl.c_first; c < pl.c_last; c++, chunk++) {
+            const int nf = (int)std::min<int64_t>(CHUNK_FRAMES, pl.F - c * CHUNK_FRAMES);
+            const int nt = (int)chunk_tokens(nf);
+            // the chunk's tokens need conv3 rows t < nt, conv2 rows t < 2 nt and
+            // conv1 rows t < 4 nt (kernel 3, stride 2, padding 1)
+            sc[chunk] = StemChunk{i, (int)(chunk * CHUNK_FRAMES), nf, std::min(400, 4 * nt)};
+            ct[chunk] = make_int2((int)tok, nt);
+            tok += nt;
+        }
+    }
+    // conv2 / conv3 tile lists per stem group (chunk index within the group)
+    int *t2 = reinterpret_cast<int *>(H + tl.tiles2);
+    int *t3 = reinterpret_cast<int *>(H + tl.tiles3);
+    std::vector<int> g_off2, g_n2, g_off3, g_n3;
+    {
+        int o2 = 0, o3 = 0;
+        for (int64_t g0 = 0; g0 < n_chunks; g0 += h->stem_group) {
+            const int gc = (int)std::min<int64_t>(h->stem_group, n_chunks - g0);
+            g_off2.push_back(o2);
+            g_off3.push_back(o3);
+            for (int j = 0; j < gc; j++) {
+                const int nt = ct[g0 + j].y;
+                const int n2 = (std::min(200, 2 * nt) + 3) / 4, n3 = (nt + 7) / 8;
+                for (int m = 0; m < n2; m++) t2[o2++] = j * 256 + m;
+                for (int m = 0; m < n3; m++) t3[o3++] = j * 256 + m;
+            }
+            // CTA pairs take two list entries at a time: pad to an even count
+            if ((o2 - g_off2.back()) & 1) t2[o2++] = -1;
+            if ((o3 - g_off3.back()) & 1) t3[o3++] = -1;
+            g_n2.push_back(o2 - g_off2.back());
+            g_n3.push_back(o3 - g_off3.back());
+        }
+    }
+    FwdPlan P;
+    P.n_clips = n_clips;
+    P.n_chunks = n_chunks;
+    P.T = T;
+    P.n_max_pass = n_max_pass;
+    P.max_clip_frames = max_clip_frames;
+    P.max_range_frames = max_range_frames;
+    P.max_pass_frames = max_pass_frames;
+    P.range_frames = range_frames;
+    P.sc = sc;
+    P.ct = ct;
+    P.g_off2 = std::move(g_off2);
+    P.g_n2 = std::move(g_n2);
+    P.g_off3 = std::move(g_off3);
+    P.g_n3 = std::move(g_n3);
+
+    // Whole forwards run as one CUDA graph: captured the first time a request
+    // is seen, replayed while the same request (clips, ranges, output, stage)
+    // comes back.  The graph reads its own copy of the tables.
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    CUDA_TRY(h, cudaStreamIsCapturing(h->stream, &cs));
+    const bool graphable = stage == MOSS_ENC_STAGE_ADAPTER && !h->profiling && h->stream != nullptr &&
+                           cs == cudaStreamCaptureStatusNone;
+    if (!graphable) {
+        TRY(tab_upload(h));
+        return forward_launch(h, P, static_cast<uint8_t *>(h->d_tab), stage, out);
+    }
+    if (h->graph_exec && h->graph_key == request_key(clips, n_clips, out)) {
+        h->launches += h->graph_launches;
+        CUDA_TRY(h, cudaGraphLaunch(h->graph_exec, h->stream));
+        return MOSS_ENC_OK;
+    }
+    if (h->graph_exec) {
+        cudaGraphExecDestroy(h->graph_exec);
+        h->graph_exec = nullptr;
+    }
+    CUDA_TRY(h, cudaMemcpyAsync(h->d_tab_graph, h->h_tab, h->tab_bytes, cudaMemcpyHostToDevice, h->stream));
+    CUDA_TRY(h, cudaEventRecord(h->tab_event, h->stream));
+    const int64_t launches0 = h->launches;
+    CUDA_TRY(h, cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
+    const moss_enc_status st = forward_launch(h, P, static_cast<uint8_t *>(h->d_tab_graph), stage, out);
+    cudaGraph_t g = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(h->stream, &g);
+    if (st != MOSS_ENC_OK || ce != cudaSuccess) {
+        if (g) cudaGraphDestroy(g);
+        cudaGetLastError();
+        return st != MOSS_ENC_OK ? st : fail(h, MOSS_ENC_ERR_CUDA, std::string("graph capture: ") + cudaGetErrorString(ce));
+    }
+    const cudaError_t ie = cudaGraphInstantiate(&h->graph_exec, g, 0);
+    cudaGraphDestroy(g);
+    if (ie != cudaSuccess) {
+        h->graph_exec = nullptr;
+        return fail(h, MOSS_ENC_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(ie));
+    }
+    h->graph_key = request_key(clips, n_clips, out);
+    h->graph_launches = h->launches - launches0;
+    CUDA_TRY(h, cudaGraphLaunch(h->graph_exec, h->stream));
+    return MOSS_ENC_OK;
+}
+
 
 extern "C" moss_enc_status moss_enc_forward(moss_enc *h, const moss_enc_clip *clips, int n_clips, void *rows_out,
                                             int64_t *row_offsets)

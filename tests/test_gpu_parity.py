@@ -259,3 +259,28 @@ def test_capacity_and_range_errors():
         enc.forward([x[:1000]] * 3)
     assert e.value.status == 2
     enc.synchronize()
+
+
+def test_graph_replay_matches_eager_launches(tiny_case):
+    # On a non-default stream a repeated request replays one captured CUDA
+    # graph; with profiling on the same request runs launch by launch.
+    pcm, out, _ = tiny_case
+    s = torch.cuda.Stream()
+    enc = binding.Encoder(weights(4), 4, 600_000, 2, stream=s)
+    xa, xb = dev(pcm), dev(synth.pcm_tones(8, 40000))
+    torch.cuda.synchronize()
+    ya1, _ = enc.forward([xa])        # captured
+    ya2, _ = enc.forward([xa])        # replayed
+    yb1, _ = enc.forward([xa, xb])    # another request: captured again
+    enc.profile_enable(2000)
+    ya3, _ = enc.forward([xa])        # launched one by one
+    yb2, _ = enc.forward([xa, xb])
+    stats = enc.profile_read()
+    enc.profile_enable(0)
+    enc.synchronize()
+    assert torch.equal(ya1, ya2) and torch.equal(ya1, ya3)
+    assert torch.equal(yb1, yb2)
+    assert torch.equal(yb1[:13], ya1)
+    assert "gemm_fc1" in stats and stats["gemm_fc1"]["launches"] == 2 * 4
+    assert_rows_close(ya1.cpu().numpy(), out, "graph rows")
+    enc.close()
