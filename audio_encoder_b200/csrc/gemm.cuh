@@ -46,6 +46,10 @@ struct GemmArgs {
     const int *tile_list;
     int rows_per_chunk;     // output rows of one chunk (T_out * F_out)
     int tile_t;             // output time steps per 128-row tile
+    // bf16 outputs only: when nonzero, each value v is also written as the pair
+    // hi = bf16(v) at column c and lo = bf16(v - hi) at column c + split_off,
+    // so that a following GEMM over [hi | lo] x [W | W] sees v to ~16 bits.
+    int split_off;
 };
 
 // Each epilogue warp stages 32 rows x 128 B in shared memory (16-byte
@@ -98,71 +102,80 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
         tmem_ld32(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         if (nc == 64) tmem_ld32(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_ld_wait();
-        if constexpr (EPI == EPI_SWIGLU_BF16) {
-            // r[0..31] gate, r[32..63] up -> 32 outputs (64 B per row)
-            const float *bg = a.bias + col0 + c0, *bu = bg + 32;
+        if constexpr (EPI == EPI_SWIGLU_BF16 || EPI == EPI_BF16 || EPI == EPI_GELU_BF16) {
+            // values in place (fp32 bits in r), then one or two bf16 passes
+            int nv;  // values of this lane's row in this group
+            if constexpr (EPI == EPI_SWIGLU_BF16) {
+                // r[0..31] gate, r[32..63] up -> 32 outputs
+                const float *bg = a.bias + col0 + c0, *bu = bg + 32;
 #pragma unroll
-            for (int q = 0; q < 4; q++) {
-                float o[8];
-#pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    const float gv = __uint_as_float(r[8 * q + j]) + bg[8 * q + j];
-                    const float uv = __uint_as_float(r[32 + 8 * q + j]) + bu[8 * q + j];
-                    o[j] = silu(gv) * uv;
+                for (int j = 0; j < 32; j++) {
+                    const float gv = __uint_as_float(r[j]) + bg[j];
+                    const float uv = __uint_as_float(r[32 + j]) + bu[j];
+                    r[j] = __float_as_uint(silu(gv) * uv);
                 }
-                *stage_at(stage, lane, q) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                                       pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
-            }
-            __syncwarp();
-            bf16 *out = reinterpret_cast<bf16 *>(a.out) + (col0 + c0) / 2;
+                nv = 32;
+            } else {
+                const float *b = a.bias + col0 + c0;
 #pragma unroll
-            for (int it = 0; it < 4; it++) {
-                const int row = it * 8 + (lane >> 2), ch = lane & 3;
-                const int grow = __shfl_sync(0xffffffffu, my_row, row);
-                const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
-                const uint4 v = *stage_at(stage, row, ch);
-                if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
-            }
-            __syncwarp();
-        } else if constexpr (EPI == EPI_BF16 || EPI == EPI_GELU_BF16) {
-            const float *b = a.bias + col0 + c0;
+                for (int q = 0; q < 8; q++) {
+                    if (q * 8 < nc) {
+                        const float4 b0 = ld_f4(b + 8 * q), b1 = ld_f4(b + 8 * q + 4);
+                        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int q = 0; q < 8; q++) {
-                if (q * 8 < nc) {
-                    float o[8];
-                    const float4 b0 = ld_f4(b + 8 * q), b1 = ld_f4(b + 8 * q + 4);
-                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-                    for (int j = 0; j < 8; j++) {
-                        o[j] = __uint_as_float(r[8 * q + j]) + bb[j];
-                        if constexpr (EPI == EPI_GELU_BF16) o[j] = gelu_erf(o[j]);
+                        for (int j = 0; j < 8; j++) {
+                            float o = __uint_as_float(r[8 * q + j]) + bb[j];
+                            if constexpr (EPI == EPI_GELU_BF16) o = gelu_fast(o);
+                            r[8 * q + j] = __float_as_uint(o);
+                        }
                     }
-                    *stage_at(stage, lane, q) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                                           pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
                 }
+                nv = nc;
             }
-            __syncwarp();
-            bf16 *out = reinterpret_cast<bf16 *>(a.out) + col0 + c0;
-            if (nc == 64) {  // 8 lanes per 128-byte row, 4 rows per instruction
+            const int ocol = EPI == EPI_SWIGLU_BF16 ? (col0 + c0) / 2 : col0 + c0;
+            const int parts = a.split_off ? 2 : 1;
+#pragma unroll 1
+            for (int part = 0; part < parts; part++) {
 #pragma unroll
-                for (int it = 0; it < 8; it++) {
-                    const int row = it * 4 + (lane >> 3), ch = lane & 7;
-                    const int grow = __shfl_sync(0xffffffffu, my_row, row);
-                    const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
-                    const uint4 v = *stage_at(stage, row, ch);
-                    if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
-                }
-            } else {  // 32 columns: 4 lanes per 64-byte row, 8 rows per instruction
+                for (int q = 0; q < 8; q++) {
+                    if (q * 8 < nv) {
+                        uint32_t w[4];
 #pragma unroll
-                for (int it = 0; it < 4; it++) {
-                    const int row = it * 8 + (lane >> 2), ch = lane & 3;
-                    const int grow = __shfl_sync(0xffffffffu, my_row, row);
-                    const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
-                    const uint4 v = *stage_at(stage, row, ch);
-                    if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
+                        for (int j = 0; j < 4; j++) {
+                            const float x0 = __uint_as_float(r[8 * q + 2 * j]), x1 = __uint_as_float(r[8 * q + 2 * j + 1]);
+                            if (part == 0) {
+                                w[j] = pack_bf16x2(x0, x1);
+                            } else {
+                                const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
+                                w[j] = pack_bf16x2(x0 - __low2float(hi), x1 - __high2float(hi));
+                            }
+                        }
+                        *stage_at(stage, lane, q) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
                 }
+                __syncwarp();
+                bf16 *out = reinterpret_cast<bf16 *>(a.out) + ocol + part * a.split_off;
+                if (nv == 64) {  // 8 lanes per 128-byte row, 4 rows per instruction
+#pragma unroll
+                    for (int it = 0; it < 8; it++) {
+                        const int row = it * 4 + (lane >> 3), ch = lane & 7;
+                        const int grow = __shfl_sync(0xffffffffu, my_row, row);
+                        const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
+                        const uint4 v = *stage_at(stage, row, ch);
+                        if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
+                    }
+                } else {  // 32 values: 4 lanes per 64-byte row, 8 rows per instruction
+#pragma unroll
+                    for (int it = 0; it < 4; it++) {
+                        const int row = it * 8 + (lane >> 2), ch = lane & 3;
+                        const int grow = __shfl_sync(0xffffffffu, my_row, row);
+                        const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
+                        const uint4 v = *stage_at(stage, row, ch);
+                        if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
+                    }
+                }
+                __syncwarp();
             }
-            __syncwarp();
         } else {
             // fp32 results, 32 columns (128 B per row) at a time
 #pragma unroll

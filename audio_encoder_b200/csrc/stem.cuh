@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(240) conv1_kernel(const float *__restrict__ me
                 sa += wa[kf * 3 + kt] * x;
                 sb += wb[kf * 3 + kt] * x;
             }
-        *reinterpret_cast<uint32_t *>(dst + (size_t)f * 480) = pack_bf16x2(gelu_erf(sa), gelu_erf(sb));
+        *reinterpret_cast<uint32_t *>(dst + (size_t)f * 480) = pack_bf16x2(gelu_fast(sa), gelu_fast(sb));
     }
 }
 

@@ -44,3 +44,8 @@ def test_gemm_epilogues(enc, pair, block_n, epi, M, K):
     err = (got - ref).abs().max().item()
     scale = ref.abs().max().item()
     assert err <= tol * max(scale, 1.0), (err, scale)
+
+
+def test_fast_gelu_matches_erff(enc):
+    # Abramowitz & Stegun 7.1.26 erf against CUDA's erff
+    assert enc.selftest_gelu() <= 1e-6
