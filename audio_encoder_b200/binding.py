@@ -27,7 +27,7 @@ EXPORTED = [
     "moss_enc_status_string", "moss_enc_last_error", "moss_enc_logmel", "moss_enc_log_max",
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
-    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_selftest_gelu",
+    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_selftest_gelu", "moss_enc_selftest_timeout",
 ]
 STATIC_MAX_CLIPS = 64
 
@@ -101,6 +101,8 @@ def lib():
         L.moss_enc_profile_read.argtypes = [vp, ctypes.POINTER(KernelStat), i32]
         L.moss_enc_launch_count.restype = i64
         L.moss_enc_launch_count.argtypes = [vp]
+        L.moss_enc_selftest_timeout.restype = i32
+        L.moss_enc_selftest_timeout.argtypes = [vp, i32]
         L.moss_enc_selftest_gelu.restype = i32
         L.moss_enc_selftest_gelu.argtypes = [vp, ctypes.POINTER(ctypes.c_float)]
         L.moss_enc_gemm.restype = i32
@@ -203,6 +205,9 @@ class Encoder:
         self._check(lib().moss_enc_gemm(self.h, _ptr(A), _ptr(B), _ptr(bias), _ptr(out), M, N, K,
                                         int(epilogue), int(block_n), int(bool(cta_pair))))
         return out
+
+    def selftest_timeout(self, limit_ms: int = 50):
+        self._check(lib().moss_enc_selftest_timeout(self.h, int(limit_ms)))
 
     def selftest_gelu(self) -> float:
         e = ctypes.c_float()

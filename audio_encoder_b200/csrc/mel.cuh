@@ -2,12 +2,12 @@
 //
 // One CTA takes a block of up to 32 consecutive frames of one clip.  The PCM
 // span those frames cover (160*31 + 400 samples) is read once, coalesced, into
-// shared memory, with reflect padding applied only at the true clip ends.  Each
-// warp then transforms two frames at a time: frame a as the real part and
-// frame b as the imaginary part of one 400-point complex DFT, computed as
-// 20 x 20 (two passes of 20-point DFTs, each a 4-point and a 5-point stage,
-// with the 400-point twiddles between the passes).  The two real spectra are
-// separated with X_a[k] = (Z[k] + conj Z[-k]) / 2, X_b[k] = (Z[k] - conj Z[-k]) / 2i,
+// shared memory, with reflect padding applied only at the true clip ends.
+// Frames are transformed two at a time: frame a as the real part and frame b
+// as the imaginary part of one 400-point complex DFT, computed as 20 x 20
+// (two passes of 20-point DFTs, each a 4-point and a 5-point stage, with the
+// 400-point twiddles between the passes).  The two real spectra are separated
+// with X_a[k] = (Z[k] + conj Z[-k]) / 2, X_b[k] = (Z[k] - conj Z[-k]) / 2i,
 // squared, pushed through the banded mel filterbank, and log10'd.  The block's
 // maximum goes to the clip's maximum with one ordered-integer atomicMax.
 #pragma once
@@ -16,9 +16,7 @@
 
 namespace moss {
 
-static constexpr int MEL_FRAMES_PER_BLOCK = 32;
 static constexpr int MEL_BAND = 16;  // max nonzero FFT bins of one mel filter
-static constexpr int MEL_SPAN = 160 * (MEL_FRAMES_PER_BLOCK - 1) + 400;
 
 // One clip's frame range for a logmel launch.  Block (x, y) of the grid
 // takes frames f_begin + 32x .. of clip y; frame f goes to output row
@@ -39,18 +37,7 @@ struct MelTables {
     float hann[400];              // periodic Hann
     int band_lo[128];             // first nonzero bin of each filter
     float band_w[128][MEL_BAND];  // filter weights on bins band_lo .. band_lo+15
-};
-
-// Shared memory of one logmel CTA (dynamic; about 74 KB).
-struct MelSmem {
-    float2 tw[400];
-    float2 zbuf[8][400];   // per warp: the 20 x 20 exchange, then Z
-    float xs[MEL_SPAN];    // the PCM span of the block
-    float hann[400];
-    int band_lo[128];
-    float band_w[128][MEL_BAND];
-    float pw[8][2][204];   // per warp: power of frames a and b
-    float wmax[8];
+    int band_n[128];              // nonzero bins of each filter (<= MEL_BAND)
 };
 
 __device__ __forceinline__ float2 cmul(float2 a, float2 b)
@@ -110,141 +97,133 @@ __device__ __forceinline__ long long reflect_index(long long j, long long n)
     return j;
 }
 
-// out: rows of 128 fp32 log10 mel values (not normalised) when write_out.
-// gmax_ord: per-clip ordered-int maxima (atomicMax) when do_max.
-__global__ void __launch_bounds__(256) logmel_kernel(const MelClip *__restrict__ clips,
-                                                     const MelTables *__restrict__ tab,
-                                                     float *__restrict__ out, int *gmax_ord,
-                                                     int write_out)
+// A CTA of 320 threads
+// takes up to 32 frames (16 frame pairs).  The 400-point complex DFT of a
+// frame pair is split as 20 x 20: pass 1 gives each thread one (pair, n1)
+// 20-point DFT over samples n1 + 20 n2, pass 2 one (pair, k2) DFT over n1, so
+// all 320 lanes work in both passes; the exchange goes through shared memory
+// with rows padded to 21 entries.  Power, banded mel and log10 then run over
+// (frame, bin) and (frame, filter) items.  Registers stay near 100, so two
+// CTAs share an SM.
+static constexpr int MEL2_FRAMES = 32;
+static constexpr int MEL2_THREADS = 320;
+static constexpr int MEL2_SPAN = 160 * (MEL2_FRAMES - 1) + 400;  // 5360 samples
+
+struct Mel2Smem {
+    float2 tw[400];
+    float hann[400];
+    int band_lo[128];
+    int band_n[128];
+    float band_w[128][MEL_BAND];
+    float2 y[MEL2_FRAMES / 2][20 * 21];      // pass-1 output / pass-2 output per pair
+    float xs[MEL2_FRAMES * 204 > MEL2_SPAN ? MEL2_FRAMES * 204 : MEL2_SPAN];  // PCM, then power [32][204]
+    float wmax[MEL2_THREADS / 32];
+};
+
+__global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip *__restrict__ clips,
+                                                                  const MelTables *__restrict__ tab,
+                                                                  float *__restrict__ out, int *gmax_ord,
+                                                                  int write_out)
 {
-    extern __shared__ __align__(16) uint8_t mel_smem[];
-    MelSmem &S = *reinterpret_cast<MelSmem *>(mel_smem);
-    float *xs = S.xs;
-    float2 *tw = S.tw;
-    float *hann = S.hann;
-    int *band_lo = S.band_lo;
-    float (*band_w)[MEL_BAND] = S.band_w;
-    float2 (*zbuf)[400] = S.zbuf;
-    float (*pw)[2][204] = S.pw;
-    float *wmax = S.wmax;
-
+    extern __shared__ __align__(16) uint8_t mel2_smem[];
+    Mel2Smem &S = *reinterpret_cast<Mel2Smem *>(mel2_smem);
     const MelClip clip = clips[blockIdx.y];
-    struct { int frame0, nframes; long long out_row; } blk;
-    blk.frame0 = clip.f_begin + MEL_FRAMES_PER_BLOCK * blockIdx.x;
-    if (blk.frame0 >= clip.f_end) return;
-    blk.nframes = min(MEL_FRAMES_PER_BLOCK, clip.f_end - blk.frame0);
-    blk.out_row = clip.out_row0 + (blk.frame0 - clip.f_begin);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int frame0 = clip.f_begin + MEL2_FRAMES * blockIdx.x;
+    if (frame0 >= clip.f_end) return;
+    const int nf = min(MEL2_FRAMES, clip.f_end - frame0);
+    const long long out_row = clip.out_row0 + (frame0 - clip.f_begin);
+    const int tid = threadIdx.x;
 
-    for (int i = tid; i < 400; i += 256) {
-        tw[i] = tab->tw400[i];
-        hann[i] = tab->hann[i];
+    for (int i = tid; i < 400; i += MEL2_THREADS) {
+        S.tw[i] = tab->tw400[i];
+        S.hann[i] = tab->hann[i];
     }
-    for (int i = tid; i < 128; i += 256) band_lo[i] = tab->band_lo[i];
-    for (int i = tid; i < 128 * MEL_BAND; i += 256) band_w[i / MEL_BAND][i % MEL_BAND] = tab->band_w[i / MEL_BAND][i % MEL_BAND];
+    for (int i = tid; i < 128; i += MEL2_THREADS) {
+        S.band_lo[i] = tab->band_lo[i];
+        S.band_n[i] = tab->band_n[i];
+    }
+    for (int i = tid; i < 128 * MEL_BAND; i += MEL2_THREADS) S.band_w[i / MEL_BAND][i % MEL_BAND] = tab->band_w[i / MEL_BAND][i % MEL_BAND];
 
-    const long long s0 = 160LL * blk.frame0 - 200;
-    const int span = 160 * (blk.nframes - 1) + 400;
-    const bool interior = s0 >= 0 && s0 + span <= clip.n;
-    if (interior && (s0 & 3) == 0 && ((reinterpret_cast<uintptr_t>(clip.pcm) & 15) == 0)) {
-        const float4 *src = reinterpret_cast<const float4 *>(clip.pcm + s0);
-        for (int i = tid; i < (span + 3) / 4; i += 256) {
-            if (4 * i + 3 < span) {
-                float4 v = __ldg(src + i);
-                xs[4 * i] = v.x;
-                xs[4 * i + 1] = v.y;
-                xs[4 * i + 2] = v.z;
-                xs[4 * i + 3] = v.w;
-            } else {
-                for (int j = 4 * i; j < span; j++) xs[j] = clip.pcm[s0 + j];
-            }
-        }
+    // the block's PCM span, reflect-padded only at the clip ends
+    const long long s0 = 160LL * frame0 - 200;
+    const int span = 160 * (nf - 1) + 400;
+    if (s0 >= 0 && s0 + span <= clip.n && ((reinterpret_cast<uintptr_t>(clip.pcm) & 15) == 0)) {
+        const float4 *src = reinterpret_cast<const float4 *>(clip.pcm + s0);  // s0 = 160 f - 200 is a multiple of 4
+        for (int i = tid; i < span / 4; i += MEL2_THREADS) reinterpret_cast<float4 *>(S.xs)[i] = __ldg(src + i);
     } else {
-        for (int i = tid; i < span; i += 256) xs[i] = __ldg(clip.pcm + reflect_index(s0 + i, clip.n));
+        for (int i = tid; i < span; i += MEL2_THREADS) S.xs[i] = __ldg(clip.pcm + reflect_index(s0 + i, clip.n));
     }
     __syncthreads();
 
+    const int npairs = (nf + 1) / 2;
+    // pass 1: task (pair p, n1): 20-point DFT over n2 of the windowed samples
+    // n = n1 + 20 n2 of frame a (real part) and frame b (imaginary part)
+    for (int task = tid; task < npairs * 20; task += MEL2_THREADS) {
+        const int p = task / 20, n1 = task - 20 * p;
+        const int fa = 2 * p, fb = 2 * p + 1;
+        const bool has_b = fb < nf;
+        const float *xa = S.xs + 160 * fa, *xb = S.xs + 160 * (has_b ? fb : fa);
+        float2 v[20];
+#pragma unroll
+        for (int n2 = 0; n2 < 20; n2++) {
+            const int n = n1 + 20 * n2;
+            const float w = S.hann[n];
+            v[n2] = make_float2(w * xa[n], has_b ? w * xb[n] : 0.0f);
+        }
+        dft20(v, S.tw);
+        float2 *yr = S.y[p] + n1 * 21;
+#pragma unroll
+        for (int k2 = 0; k2 < 20; k2++) yr[k2] = (k2 == 0 || n1 == 0) ? v[k2] : cmul(v[k2], S.tw[n1 * k2]);
+    }
+    __syncthreads();
+    // pass 2: task (pair p, k2): 20-point DFT over n1 -> Z[20 k1 + k2], in place
+    for (int task = tid; task < npairs * 20; task += MEL2_THREADS) {
+        const int p = task / 20, k2 = task - 20 * p;
+        float2 v[20];
+#pragma unroll
+        for (int n1 = 0; n1 < 20; n1++) v[n1] = S.y[p][n1 * 21 + k2];
+        dft20(v, S.tw);
+#pragma unroll
+        for (int k1 = 0; k1 < 20; k1++) S.y[p][k1 * 21 + k2] = v[k1];
+    }
+    __syncthreads();
+    // power of both frames of each pair, bins 0..200, into S.xs as [frame][204]
+    float *pw = S.xs;
+    for (int task = tid; task < npairs * 201; task += MEL2_THREADS) {
+        const int p = task / 201, k = task - 201 * p;
+        const int kn = (400 - k) % 400;
+        const float2 zk = S.y[p][(k / 20) * 21 + (k % 20)], zn = S.y[p][(kn / 20) * 21 + (kn % 20)];
+        const float ar = 0.5f * (zk.x + zn.x), ai = 0.5f * (zk.y - zn.y);
+        const float br = 0.5f * (zk.y + zn.y), bi = -0.5f * (zk.x - zn.x);
+        pw[(2 * p) * 204 + k] = ar * ar + ai * ai;
+        pw[(2 * p + 1) * 204 + k] = br * br + bi * bi;
+    }
+    __syncthreads();
+    // banded mel, log10, block max; thread takes 4 consecutive filters of a frame
     float lmax = -INFINITY;
-    const int npairs = (blk.nframes + 1) / 2;
-    for (int pr = warp; pr < npairs; pr += 8) {
-        const int fa = 2 * pr, fb = 2 * pr + 1;
-        const bool has_b = fb < blk.nframes;
-        const float *xa = xs + 160 * fa;
-        const float *xb = xs + 160 * (has_b ? fb : fa);
-        float2 *z = zbuf[warp];
-        // pass 1: lane n1 < 20 takes samples n1 + 20 n2
-        if (lane < 20) {
-            float2 v[20];
+    for (int task = tid; task < nf * 32; task += MEL2_THREADS) {
+        const int f = task >> 5, q = task & 31;
+        const float *P = pw + f * 204;
+        float r[4];
 #pragma unroll
-            for (int n2 = 0; n2 < 20; n2++) {
-                const int nidx = lane + 20 * n2;
-                const float w = hann[nidx];
-                v[n2] = make_float2(w * xa[nidx], has_b ? w * xb[nidx] : 0.0f);
-            }
-            dft20(v, tw);
-#pragma unroll
-            for (int k2 = 0; k2 < 20; k2++) {
-                float2 t = k2 == 0 || lane == 0 ? v[k2] : cmul(v[k2], tw[(lane * k2) % 400]);
-                z[lane * 20 + k2] = t;
-            }
+        for (int j = 0; j < 4; j++) {
+            const int m = 4 * q + j;
+            const int lo = S.band_lo[m], cnt = S.band_n[m];
+            float acc = 0.0f;
+            for (int b = 0; b < cnt; b++) acc = fmaf(S.band_w[m][b], P[lo + b], acc);
+            r[j] = log10f(fmaxf(acc, 1e-10f));
+            lmax = fmaxf(lmax, r[j]);
         }
-        __syncwarp();
-        // pass 2: lane k2 < 20 takes column k2 -> Z[20 k1 + k2]
-        float2 v2[20];
-        if (lane < 20) {
-#pragma unroll
-            for (int n1 = 0; n1 < 20; n1++) v2[n1] = z[n1 * 20 + lane];
-            dft20(v2, tw);
-        }
-        __syncwarp();
-        if (lane < 20) {
-#pragma unroll
-            for (int k1 = 0; k1 < 20; k1++) z[20 * k1 + lane] = v2[k1];
-        }
-        __syncwarp();
-        // split the two real spectra and take the power
-        for (int k = lane; k <= 200; k += 32) {
-            const float2 zk = z[k], zn = z[(400 - k) % 400];
-            const float ar = 0.5f * (zk.x + zn.x), ai = 0.5f * (zk.y - zn.y);
-            const float br = 0.5f * (zk.y + zn.y), bi = -0.5f * (zk.x - zn.x);
-            pw[warp][0][k] = ar * ar + ai * ai;
-            pw[warp][1][k] = br * br + bi * bi;
-        }
-        __syncwarp();
-        // mel: lane handles filters 4 lane .. 4 lane + 3 of both frames
-#pragma unroll
-        for (int f = 0; f < 2; f++) {
-            if (f == 1 && !has_b) break;
-            float r[4];
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int m = 4 * lane + j;
-                const int lo = band_lo[m];
-                float acc = 0.0f;
-#pragma unroll
-                for (int b = 0; b < MEL_BAND; b++) {
-                    const int k = lo + b;
-                    acc += band_w[m][b] * (k <= 200 ? pw[warp][f][k] : 0.0f);
-                }
-                r[j] = log10f(fmaxf(acc, 1e-10f));
-                lmax = fmaxf(lmax, r[j]);
-            }
-            if (write_out) {
-                const int frame = f == 0 ? fa : fb;
-                float4 *dst = reinterpret_cast<float4 *>(out + (size_t)(blk.out_row + frame) * 128) + lane;
-                *dst = make_float4(r[0], r[1], r[2], r[3]);
-            }
-        }
-        __syncwarp();
+        if (write_out)
+            reinterpret_cast<float4 *>(out + (size_t)(out_row + f) * 128)[q] = make_float4(r[0], r[1], r[2], r[3]);
     }
     if (clip.gslot >= 0) {
-#pragma unroll
         for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-        if (lane == 0) wmax[warp] = lmax;
+        if ((tid & 31) == 0) S.wmax[tid >> 5] = lmax;
         __syncthreads();
         if (tid == 0) {
-            float m = wmax[0];
-            for (int i = 1; i < 8; i++) m = fmaxf(m, wmax[i]);
+            float m = S.wmax[0];
+            for (int i = 1; i < MEL2_THREADS / 32; i++) m = fmaxf(m, S.wmax[i]);
             atomicMax(gmax_ord + clip.gslot, float_to_ordered(m));
         }
     }

@@ -354,6 +354,7 @@ static bool build_mel_tables(MelTables *t)
         if (lo < 0) lo = hi = 0;
         if (hi - lo + 1 > MEL_BAND) return false;
         t->band_lo[m] = lo;
+        t->band_n[m] = hi - lo + 1;
         for (int b = 0; b < MEL_BAND; b++) t->band_w[m][b] = (lo + b <= 200) ? (float)w[lo + b] : 0.0f;
     }
     return true;
@@ -494,7 +495,8 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm_attr<128, EPI_F32>()));
     CUDA_TRY(h, (gemm_attr<128, EPI_BF16>()));
     CUDA_TRY(h, cudaFuncSetAttribute(window_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATTN_TC_SMEM));
-    CUDA_TRY(h, cudaFuncSetAttribute(logmel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(MelSmem)));
+    CUDA_TRY(h, cudaFuncSetAttribute(logmel2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel2Smem)));
+    CUDA_TRY(h, cudaFuncSetAttribute(logmel2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     return MOSS_ENC_OK;
 }
 
@@ -814,7 +816,7 @@ static moss_enc_status tab_upload(moss_enc *h)
     return MOSS_ENC_OK;
 }
 
-static int mel_grid_x(int64_t max_frames) { return (int)std::max<int64_t>(1, (max_frames + MEL_FRAMES_PER_BLOCK - 1) / MEL_FRAMES_PER_BLOCK); }
+static int mel_grid_x(int64_t max_frames) { return (int)std::max<int64_t>(1, (max_frames + MEL2_FRAMES - 1) / MEL2_FRAMES); }
 
 static moss_enc_status launch_logmel(moss_enc *h, const MelClip *d_clips, int n_clips, int64_t max_frames,
                                      float *out, int write_out, int64_t total_frames)
@@ -822,7 +824,7 @@ static moss_enc_status launch_logmel(moss_enc *h, const MelClip *d_clips, int n_
     if (n_clips <= 0 || max_frames <= 0) return MOSS_ENC_OK;
     dim3 grid(mel_grid_x(max_frames), n_clips);
     Launch L(h, write_out ? "logmel" : "logmel_max", 0.0, 4.0 * 160 * (double)total_frames + (write_out ? 512.0 * total_frames : 0.0));
-    logmel_kernel<<<grid, 256, sizeof(MelSmem), h->stream>>>(d_clips, h->mel_tab, out, h->gmax_ord, write_out);
+    logmel2_kernel<<<grid, MEL2_THREADS, sizeof(Mel2Smem), h->stream>>>(d_clips, h->mel_tab, out, h->gmax_ord, write_out);
     CUDA_TRY(h, cudaGetLastError());
     return MOSS_ENC_OK;
 }
@@ -1412,6 +1414,34 @@ extern "C" moss_enc_status moss_enc_selftest_gelu(moss_enc *h, float *max_rel_er
     return MOSS_ENC_OK;
 }
 
+// ------------------------------------------------ bounded-wait self-test
+
+// One thread waits on an mbarrier that nothing arrives at, with the given
+// limit, the way every pipeline wait in the kernels is bounded.  The wait
+// gives up, raises the timeout bit of the handle's device flag, and returns.
+__global__ void wait_timeout_check_kernel(int *err, unsigned long long limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&bar, 0)) {
+        if (globaltimer_ns() - t0 > limit_ns) {
+            atomicOr(err, DEV_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
+extern "C" moss_enc_status moss_enc_selftest_timeout(moss_enc *h, int limit_ms)
+{
+    if (!h || limit_ms < 1 || limit_ms > 2000) return MOSS_ENC_ERR_INVALID_ARG;
+    wait_timeout_check_kernel<<<1, 32, 0, h->stream>>>(h->err, (unsigned long long)limit_ms * 1000000ull);
+    CUDA_TRY(h, cudaGetLastError());
+    return MOSS_ENC_OK;
+}
+
 // ------------------------------------------------- allocation-free log-mel
 //
 // Scratch for moss_enc_logmel_static: a fixed-size device array, laid out as
@@ -1453,7 +1483,7 @@ static moss_enc_status static_scratch(uint8_t **out)
     if (!g_static_ptr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_logmel_scratch) != cudaSuccess || !p) return MOSS_ENC_ERR_CUDA;
-        if (cudaFuncSetAttribute(logmel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(MelSmem)) !=
+        if (cudaFuncSetAttribute(logmel2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel2Smem)) !=
             cudaSuccess)
             return MOSS_ENC_ERR_CUDA;
         MelTables tab;
@@ -1508,11 +1538,11 @@ extern "C" moss_enc_status moss_enc_logmel_static(const moss_enc_clip *clips, in
     // the maxima start at -inf or at the caller's value
     gmax_init_kernel<<<1, STATIC_MAX_CLIPS, 0, st>>>(d_gmax, d_src, n_clips);
     if (n_max > 0)
-        logmel_kernel<<<dim3(mel_grid_x(max_clip), n_max), 256, sizeof(MelSmem), st>>>(d_maxp, d_tab, nullptr, d_gmax, 0);
+        logmel2_kernel<<<dim3(mel_grid_x(max_clip), n_max), MEL2_THREADS, sizeof(Mel2Smem), st>>>(d_maxp, d_tab, nullptr, d_gmax, 0);
     for (int i = 0; i < n_clips; i++) {
         const int nf = stage.main[i].f_end - stage.main[i].f_begin;
         if (nf <= 0) continue;
-        logmel_kernel<<<dim3(mel_grid_x(nf), 1), 256, sizeof(MelSmem), st>>>(d_main + i, d_tab, mel_out[i], d_gmax, 1);
+        logmel2_kernel<<<dim3(mel_grid_x(nf), 1), MEL2_THREADS, sizeof(Mel2Smem), st>>>(d_main + i, d_tab, mel_out[i], d_gmax, 1);
     }
     for (int i = 0; i < n_clips; i++) {
         const int64_t nf = stage.main[i].f_end - stage.main[i].f_begin;

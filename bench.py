@@ -70,7 +70,7 @@ class Clocks:
     def __enter__(self):
         try:
             self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
                                       stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.p = None
@@ -210,8 +210,9 @@ def run_ours(args):
     blob = synth.make_weights(n_layers)
     total_samples = sum(c.size for c in clips)
     stream = torch.cuda.Stream()
-    enc = binding.Encoder(blob, n_layers, max_samples=total_samples + 4 * len(clips), max_clips=len(clips),
-                          out_dtype=binding.OUT_BF16, stream=stream)
+    mel_samples = 9_600_000  # the 10-min clip, for the log-mel roofline
+    enc = binding.Encoder(blob, n_layers, max_samples=max(total_samples + 4 * len(clips), mel_samples),
+                          max_clips=len(clips), out_dtype=binding.OUT_BF16, stream=stream)
     with torch.cuda.stream(stream):
         xs = [torch.from_numpy(c).to(dev) for c in clips]
         tokens = sum(binding.num_tokens(c.size) for c in clips)
@@ -293,6 +294,33 @@ def run_ours(args):
             dist.destroy_process_group()
         return
 
+    # log-mel kernel alone on the 10-min clip (inputs resident, L2 flushed
+    # between launches): algorithmic bytes = 4 B per sample read + 512 B per
+    # frame written
+    mel_roof = None
+    if rank == 0:
+        with torch.cuda.stream(stream):
+            pcm10 = torch.from_numpy(synth.pcm_long(2, mel_samples)).to(dev)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            enc.logmel(pcm10)
+        enc.profile_enable(400)
+        for i in range(10):
+            with torch.cuda.stream(stream):
+                flush.fill_(float(i))
+                enc.logmel(pcm10)
+        mst = enc.profile_read()
+        enc.profile_enable(0)
+        if "logmel" in mst:
+            m = mst["logmel"]
+            gbs = m["bytes"] / (m["ms"] / 1e3) / 1e9
+            hbm = peaks()["hbm"]
+            mel_roof = {"kernel": "logmel", "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                        "frac": gbs / hbm, "ms_per_launch": m["ms"] / m["launches"],
+                        "bytes_per_launch": m["bytes"] / m["launches"],
+                        "workload": "one 10-min clip, 9.6M samples, 60000 frames"}
+        del pcm10
+
     pk = peaks()
     ms_per_step = total_ms / args.steps
     value = world * audio_s / (ms_per_step / 1e3)
@@ -342,6 +370,7 @@ def run_ours(args):
                    "out_dtype": "bf16", "l2": "512 MB buffer written between timed steps (outside the events)",
                    "parallelism": f"dp{world}" if world > 1 else "single"},
         "roofline": roof,
+        "mel_roofline": mel_roof,
         "kernels": kernels,
         "kernel_ms_per_step_eager": kernel_ms / args.steps,
         "gpu_launches": launches,
@@ -360,7 +389,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="batch16_10to30s", choices=sorted(synth.WORKLOADS))

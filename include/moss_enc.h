@@ -208,6 +208,12 @@ moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const f
  * |difference| / max(1, |x|) of the GELU values.  Synchronises. */
 moss_enc_status moss_enc_selftest_gelu(moss_enc *h, float *max_rel_err);
 
+/* Failure-path check: enqueues a kernel whose one bounded wait can never be
+ * satisfied, with a limit of limit_ms (1..2000).  The next
+ * moss_enc_synchronize returns MOSS_ENC_ERR_DEVICE_TIMEOUT and clears the
+ * flag; the context stays usable. */
+moss_enc_status moss_enc_selftest_timeout(moss_enc *h, int limit_ms);
+
 /* ------------------------------------------------- allocation-free log-mel */
 
 /* The source pages describe no such call; it exists for callers that cannot

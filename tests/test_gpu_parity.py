@@ -284,3 +284,15 @@ def test_graph_replay_matches_eager_launches(tiny_case):
     assert "gemm_fc1" in stats and stats["gemm_fc1"]["launches"] == 2 * 4
     assert_rows_close(ya1.cpu().numpy(), out, "graph rows")
     enc.close()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(tiny_case):
+    pcm, out, _ = tiny_case
+    enc = encoder(4, 600_000)
+    enc.selftest_timeout(50)
+    with pytest.raises(binding.MossEncError) as e:
+        enc.synchronize()
+    assert e.value.status == 5
+    enc.synchronize()  # flag cleared
+    y, _ = enc.forward([dev(pcm)])
+    assert_rows_close(y.cpu().numpy(), out, "rows after a device timeout")
