@@ -205,27 +205,31 @@ __device__ __forceinline__ float gelu_erf(float x)
 }
 
 // erf after Abramowitz & Stegun, Handbook of Mathematical Functions, formula
-// 7.1.26: for x >= 0, erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5)
-// exp(-x^2) with t = 1 / (1 + p x); the approximation error is at most
-// 1.5e-7.  erf is odd.  Two special-function instructions (reciprocal and
-// exponential) and a short polynomial, instead of erff's longer sequence.
-__device__ __forceinline__ float erf_as7126(float x)
+// 7.1.28: for x >= 0, erf(x) = 1 - (1 + a1 x + a2 x^2 + ... + a6 x^6)^-16,
+// with an approximation error of at most 3e-7; erf is odd.  The reciprocal
+// is taken once and raised to the 16th power by squaring, so one
+// special-function instruction per value (erff needs a longer sequence).
+__device__ __forceinline__ float erf_as7128(float x)
 {
     const float ax = fabsf(x);
-    const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
-    float poly = fmaf(1.061405429f, t, -1.453152027f);
-    poly = fmaf(poly, t, 1.421413741f);
-    poly = fmaf(poly, t, -0.284496736f);
-    poly = fmaf(poly, t, 0.254829592f);
-    poly *= t;
-    const float r = fmaf(-poly, __expf(-ax * ax), 1.0f);
-    return copysignf(r, x);
+    float p = fmaf(4.30638e-5f, ax, 2.765672e-4f);
+    p = fmaf(p, ax, 1.520143e-4f);
+    p = fmaf(p, ax, 9.2705272e-3f);
+    p = fmaf(p, ax, 4.22820123e-2f);
+    p = fmaf(p, ax, 7.05230784e-2f);
+    p = fmaf(p, ax, 1.0f);
+    float r = __fdividef(1.0f, p);
+    r = r * r;
+    r = r * r;
+    r = r * r;
+    r = r * r;
+    return copysignf(1.0f - r, x);
 }
 
 // Exact-form GELU, 0.5 x (1 + erf(x / sqrt 2)), with the erf above.
 __device__ __forceinline__ float gelu_fast(float x)
 {
-    return 0.5f * x * (1.0f + erf_as7126(x * 0.70710678118654752f));
+    return 0.5f * x * (1.0f + erf_as7128(x * 0.70710678118654752f));
 }
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }

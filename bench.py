@@ -107,6 +107,22 @@ class Clocks:
                 "samples": len(sm)}
 
 
+def reduce_max(value, dist, device):
+    """Max of a float over all ranks (the value itself on one process)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_throughput(world, units_per_rank, ms_per_step):
+    """Whole-job throughput: every rank processes its own units each step,
+    and the step takes as long as the slowest rank."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def dist_setup(n_gpus):
     if n_gpus <= 1 or "RANK" not in os.environ:
         return 0, 1, None
@@ -261,11 +277,7 @@ def run_ours(args):
     stats = enc.profile_read()
     enc.profile_enable(0)
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = float(sum(step_ms))
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(float(sum(step_ms)), dist, dev)
     enc.synchronize()
 
     # ---- end to end through the host API: pinned PCM in, rows out to host
@@ -282,11 +294,7 @@ def run_ours(args):
         b.record(stream)
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    e2e_step = float(np.mean(e2e_ms))
-    if dist:
-        t = torch.tensor([e2e_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_step = float(t.item())
+    e2e_step = reduce_max(float(np.mean(e2e_ms)), dist, dev)
 
     if rank != 0:
         enc.close()
@@ -323,7 +331,7 @@ def run_ours(args):
 
     pk = peaks()
     ms_per_step = total_ms / args.steps
-    value = world * audio_s / (ms_per_step / 1e3)
+    value = weak_scaling_throughput(world, audio_s, ms_per_step)
     flops_step = model_flops(tokens, n_layers)
     tflops = flops_step / (ms_per_step / 1e3) / 1e12
     # dominant kernel: the category with the most device time
@@ -361,7 +369,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded PCM, random-init bf16 weights)",
-        "tokens_per_s": world * tokens / (ms_per_step / 1e3),
+        "tokens_per_s": weak_scaling_throughput(world, tokens, ms_per_step),
         "model_tflops": tflops,
         "tc_roofline_frac": tflops / pk["bf16"],
         "tc_roofline_frac_sustained": tflops / pk["bf16_sus"],
@@ -374,7 +382,7 @@ def run_ours(args):
         "kernels": kernels,
         "kernel_ms_per_step_eager": kernel_ms / args.steps,
         "gpu_launches": launches,
-        "e2e": {"value": world * audio_s / (e2e_step / 1e3), "unit": "audio-s/s",
+        "e2e": {"value": weak_scaling_throughput(world, audio_s, e2e_step), "unit": "audio-s/s",
                 "h2d_bytes_per_step": 4 * total_samples, "d2h_bytes_per_step": 2 * tokens * 2048,
                 "ms_per_step": e2e_step},
         "cpu_baseline": cpu,

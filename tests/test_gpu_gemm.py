@@ -47,5 +47,5 @@ def test_gemm_epilogues(enc, pair, block_n, epi, M, K):
 
 
 def test_fast_gelu_matches_erff(enc):
-    # Abramowitz & Stegun 7.1.26 erf against CUDA's erff
+    # Abramowitz & Stegun 7.1.28 erf against CUDA's erff
     assert enc.selftest_gelu() <= 1e-6
