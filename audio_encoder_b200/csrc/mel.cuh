@@ -40,6 +40,12 @@ struct MelTables {
     int band_n[128];              // nonzero bins of each filter (<= MEL_BAND)
 };
 
+// The filterbank weights transposed, [bin offset][filter]: consecutive
+// filters are consecutive words (read by logmel3_kernel).
+struct MelBandT {
+    float w[MEL_BAND][128];
+};
+
 __device__ __forceinline__ float2 cmul(float2 a, float2 b)
 {
     return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
@@ -227,6 +233,207 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip 
             atomicMax(gmax_ord + clip.gslot, float_to_ordered(m));
         }
     }
+}
+
+// Persistent form of the same computation (the one the library launches).
+// Two CTAs per SM walk the (clip, 32-frame block) items of the launch; each
+// loads the twiddle, window and filterbank tables once, and while it
+// transforms one block it already fetches the next block's PCM span into the
+// other buffer with cp.async (blocks at the clip ends, which need reflect
+// padding, are loaded synchronously).  The power spectrum is written back
+// into the exchange buffer, and log10 uses the hardware log2.
+static constexpr int MEL3_MAX_CLIPS = 128;  // clips per launch (the host splits larger batches)
+
+struct Mel3Smem {
+    float2 tw[400];
+    float hann[400];
+    int band_lo[128];
+    int band_n[128];
+    float band_wt[MEL_BAND][128];
+    float2 y[MEL2_FRAMES / 2][20 * 21];  // pass outputs; then power: pair p holds frame 2p at [0..200], 2p+1 at [420..620]
+    float xs[2][MEL2_SPAN];              // PCM spans of the current and the next block
+    int first_block[MEL3_MAX_CLIPS + 1];  // prefix of blocks per clip
+    float wmax[MEL2_THREADS / 32];
+};
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Locate item `item` among the clips' blocks: returns false past the end.
+__device__ __forceinline__ bool mel3_item(const Mel3Smem &S, const MelClip *clips, int n_clips, int item, int &c,
+                                          int &frame0, int &nf)
+{
+    if (item >= S.first_block[n_clips]) return false;
+    c = 0;
+    while (S.first_block[c + 1] <= item) ++c;
+    const MelClip &cl = clips[c];
+    frame0 = cl.f_begin + MEL2_FRAMES * (item - S.first_block[c]);
+    nf = min(MEL2_FRAMES, cl.f_end - frame0);
+    return true;
+}
+
+// Whether the span of a block lies inside the clip and can be copied as is.
+__device__ __forceinline__ bool mel3_interior(const MelClip &cl, int frame0, int nf)
+{
+    const long long s0 = 160LL * frame0 - 200;
+    return s0 >= 0 && s0 + 160LL * (nf - 1) + 400 <= cl.n && ((reinterpret_cast<uintptr_t>(cl.pcm) & 15) == 0);
+}
+
+__global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip *__restrict__ clips, int n_clips,
+                                                                  const MelTables *__restrict__ tab,
+                                                                  const MelBandT *__restrict__ tabt,
+                                                                  float *__restrict__ out, int *gmax_ord,
+                                                                  int write_out)
+{
+    extern __shared__ __align__(16) uint8_t mel3_smem[];
+    Mel3Smem &S = *reinterpret_cast<Mel3Smem *>(mel3_smem);
+    const int tid = threadIdx.x;
+    for (int i = tid; i < 400; i += MEL2_THREADS) {
+        S.tw[i] = tab->tw400[i];
+        S.hann[i] = tab->hann[i];
+    }
+    for (int i = tid; i < 128; i += MEL2_THREADS) {
+        S.band_lo[i] = tab->band_lo[i];
+        S.band_n[i] = tab->band_n[i];
+    }
+    for (int i = tid; i < 128 * MEL_BAND; i += MEL2_THREADS) S.band_wt[i / 128][i % 128] = tabt->w[i / 128][i % 128];
+    if (tid == 0) {
+        int acc = 0;
+        for (int c = 0; c < n_clips; c++) {
+            S.first_block[c] = acc;
+            const int f = clips[c].f_end - clips[c].f_begin;
+            acc += f > 0 ? (f + MEL2_FRAMES - 1) / MEL2_FRAMES : 0;
+        }
+        S.first_block[n_clips] = acc;
+    }
+    __syncthreads();
+
+    // span loader: async 16-byte copies for interior blocks (returns true),
+    // nothing for edge blocks (loaded synchronously when their turn comes)
+    auto prefetch = [&](int item, int buf) -> bool {
+        int c, frame0, nf;
+        if (!mel3_item(S, clips, n_clips, item, c, frame0, nf)) return true;
+        const MelClip &cl = clips[c];
+        if (!mel3_interior(cl, frame0, nf)) return false;
+        const float4 *src = reinterpret_cast<const float4 *>(cl.pcm + (160LL * frame0 - 200));
+        const int n4 = (160 * (nf - 1) + 400) / 4;
+        for (int i = tid; i < n4; i += MEL2_THREADS) cp_async16(reinterpret_cast<float4 *>(S.xs[buf]) + i, src + i);
+        return true;
+    };
+
+    const float log10_2 = 0.30102999566398120f;
+    int it = 0;
+    bool ready = prefetch(blockIdx.x, 0);
+    cp_async_commit();
+    for (int item = blockIdx.x;; item += gridDim.x, ++it) {
+        int c, frame0, nf;
+        if (!mel3_item(S, clips, n_clips, item, c, frame0, nf)) break;
+        const MelClip cl = clips[c];
+        const int cur = it & 1;
+        if (!ready) {  // edge block: reflect-padded load now
+            const long long s0 = 160LL * frame0 - 200;
+            const int span = 160 * (nf - 1) + 400;
+            for (int i = tid; i < span; i += MEL2_THREADS) S.xs[cur][i] = __ldg(cl.pcm + reflect_index(s0 + i, cl.n));
+        }
+        ready = prefetch(item + gridDim.x, cur ^ 1);
+        cp_async_commit();
+        cp_async_wait_1();  // this block's span has landed (the next one may still be in flight)
+        __syncthreads();
+
+        const float *xsb = S.xs[cur];
+        const int npairs = (nf + 1) / 2;
+        for (int task = tid; task < npairs * 20; task += MEL2_THREADS) {
+            const int p = task / 20, n1 = task - 20 * p;
+            const int fa = 2 * p, fb = 2 * p + 1;
+            const bool has_b = fb < nf;
+            const float *xa = xsb + 160 * fa, *xb = xsb + 160 * (has_b ? fb : fa);
+            float2 v[20];
+#pragma unroll
+            for (int n2 = 0; n2 < 20; n2++) {
+                const int n = n1 + 20 * n2;
+                const float w = S.hann[n];
+                v[n2] = make_float2(w * xa[n], has_b ? w * xb[n] : 0.0f);
+            }
+            dft20(v, S.tw);
+            float2 *yr = S.y[p] + n1 * 21;
+#pragma unroll
+            for (int k2 = 0; k2 < 20; k2++) yr[k2] = (k2 == 0 || n1 == 0) ? v[k2] : cmul(v[k2], S.tw[n1 * k2]);
+        }
+        __syncthreads();
+        for (int task = tid; task < npairs * 20; task += MEL2_THREADS) {
+            const int p = task / 20, k2 = task - 20 * p;
+            float2 v[20];
+#pragma unroll
+            for (int n1 = 0; n1 < 20; n1++) v[n1] = S.y[p][n1 * 21 + k2];
+            dft20(v, S.tw);
+#pragma unroll
+            for (int k1 = 0; k1 < 20; k1++) S.y[p][k1 * 21 + k2] = v[k1];
+        }
+        __syncthreads();
+        // power of both frames: read all of this thread's bins, then write them in place
+        constexpr int PT = (MEL2_FRAMES / 2 * 201 + MEL2_THREADS - 1) / MEL2_THREADS;  // 11
+        float pa[PT], pb[PT];
+#pragma unroll
+        for (int i = 0; i < PT; i++) {
+            const int task = tid + i * MEL2_THREADS;
+            pa[i] = pb[i] = 0.0f;
+            if (task < npairs * 201) {
+                const int p = task / 201, k = task - 201 * p;
+                const int kn = (400 - k) % 400;
+                const float2 zk = S.y[p][(k / 20) * 21 + (k % 20)], zn = S.y[p][(kn / 20) * 21 + (kn % 20)];
+                const float ar = 0.5f * (zk.x + zn.x), ai = 0.5f * (zk.y - zn.y);
+                const float br = 0.5f * (zk.y + zn.y), bi = -0.5f * (zk.x - zn.x);
+                pa[i] = ar * ar + ai * ai;
+                pb[i] = br * br + bi * bi;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < PT; i++) {
+            const int task = tid + i * MEL2_THREADS;
+            if (task < npairs * 201) {
+                const int p = task / 201, k = task - 201 * p;
+                float *pw = reinterpret_cast<float *>(S.y[p]);
+                pw[k] = pa[i];
+                pw[420 + k] = pb[i];
+            }
+        }
+        __syncthreads();
+        float lmax = -INFINITY;
+        const long long out_row = cl.out_row0 + (frame0 - cl.f_begin);
+        // lane q of a frame's 32 lanes takes filters q, q+32, q+64, q+96, so that
+        // the lanes read consecutive words of the transposed filterbank
+        for (int task = tid; task < nf * 32; task += MEL2_THREADS) {
+            const int f = task >> 5, q = task & 31;
+            const float *P = reinterpret_cast<const float *>(S.y[f >> 1]) + (f & 1) * 420;
+            float *orow = out + (size_t)(out_row + f) * 128;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int m = q + 32 * j;
+                const int lo = S.band_lo[m], cnt = S.band_n[m];
+                float acc = 0.0f;
+                for (int b = 0; b < cnt; b++) acc = fmaf(S.band_wt[b][m], P[lo + b], acc);
+                const float r = __log2f(fmaxf(acc, 1e-10f)) * log10_2;
+                lmax = fmaxf(lmax, r);
+                if (write_out) orow[m] = r;
+            }
+        }
+        if (cl.gslot >= 0) {
+            for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+            if ((tid & 31) == 0) S.wmax[tid >> 5] = lmax;
+        }
+        __syncthreads();  // power read and buffers free for the next item
+        if (cl.gslot >= 0 && tid == 0) {
+            float m = S.wmax[0];
+            for (int i = 1; i < MEL2_THREADS / 32; i++) m = fmaxf(m, S.wmax[i]);
+            atomicMax(gmax_ord + cl.gslot, float_to_ordered(m));
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // In-place Whisper normalisation of rows [n_rows][128]: (max(x, g - 8) + 4) / 4.

@@ -57,6 +57,7 @@ struct moss_enc {
     bf16 *wp1 = nullptr, *wp2 = nullptr, *wgu = nullptr, *wd = nullptr;
     float *pos = nullptr;
     MelTables *mel_tab = nullptr;
+    MelBandT *mel_tabt = nullptr;
 
     // capacity
     int64_t max_tokens = 0, max_chunks = 0;
@@ -495,8 +496,8 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm_attr<128, EPI_F32>()));
     CUDA_TRY(h, (gemm_attr<128, EPI_BF16>()));
     CUDA_TRY(h, cudaFuncSetAttribute(window_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATTN_TC_SMEM));
-    CUDA_TRY(h, cudaFuncSetAttribute(logmel2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel2Smem)));
-    CUDA_TRY(h, cudaFuncSetAttribute(logmel2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+    CUDA_TRY(h, cudaFuncSetAttribute(logmel3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel3Smem)));
+    CUDA_TRY(h, cudaFuncSetAttribute(logmel3_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     return MOSS_ENC_OK;
 }
 
@@ -560,6 +561,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     const size_t o_gu = take(2 * (size_t)2 * DADP * 2 * DOUT), o_bgu = take(4 * 2 * DADP);
     const size_t o_wd = take(2 * (size_t)DOUT * 2 * DADP), o_bd = take(4 * DOUT);
     const size_t o_pos = take(4 * (size_t)CHUNK_TOKENS * D), o_mel = take(sizeof(MelTables));
+    const size_t o_melt = take(sizeof(MelBandT));
     const size_t wtotal = off;
 
     std::vector<uint8_t> pk(wtotal, 0);
@@ -684,6 +686,12 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
             F32(o_pos)[t * D + D / 2 + i] = (float)std::cos(t * inv);
         }
     if (!build_mel_tables(reinterpret_cast<MelTables *>(pk.data() + o_mel))) return bail(MOSS_ENC_ERR_INVALID_ARG);
+    {
+        const MelTables *mt = reinterpret_cast<const MelTables *>(pk.data() + o_mel);
+        MelBandT *bt = reinterpret_cast<MelBandT *>(pk.data() + o_melt);
+        for (int m = 0; m < 128; m++)
+            for (int b = 0; b < MEL_BAND; b++) bt->w[b][m] = mt->band_w[m][b];
+    }
 
     if (cudaMalloc(&h->wmem, wtotal) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaMemcpy(h->wmem, pk.data(), wtotal, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
@@ -723,6 +731,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     h->bd = (float *)(W + o_bd);
     h->pos = (float *)(W + o_pos);
     h->mel_tab = (MelTables *)(W + o_mel);
+    h->mel_tabt = (MelBandT *)(W + o_melt);
 
     // ---- workspace
     h->max_tokens = cfg->max_samples / 1280 + cfg->max_clips + 1;
@@ -822,10 +831,16 @@ static moss_enc_status launch_logmel(moss_enc *h, const MelClip *d_clips, int n_
                                      float *out, int write_out, int64_t total_frames)
 {
     if (n_clips <= 0 || max_frames <= 0) return MOSS_ENC_OK;
-    dim3 grid(mel_grid_x(max_frames), n_clips);
-    Launch L(h, write_out ? "logmel" : "logmel_max", 0.0, 4.0 * 160 * (double)total_frames + (write_out ? 512.0 * total_frames : 0.0));
-    logmel2_kernel<<<grid, MEL2_THREADS, sizeof(Mel2Smem), h->stream>>>(d_clips, h->mel_tab, out, h->gmax_ord, write_out);
-    CUDA_TRY(h, cudaGetLastError());
+    for (int c0 = 0; c0 < n_clips; c0 += MEL3_MAX_CLIPS) {
+        const int nc = std::min(MEL3_MAX_CLIPS, n_clips - c0);
+        const int64_t blocks = (int64_t)nc * ((max_frames + MEL2_FRAMES - 1) / MEL2_FRAMES);  // upper bound
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks, 2 * h->num_sms));
+        Launch L(h, write_out ? "logmel" : "logmel_max", 0.0,
+                 c0 == 0 ? 4.0 * 160 * (double)total_frames + (write_out ? 512.0 * total_frames : 0.0) : 0.0);
+        logmel3_kernel<<<grid, MEL2_THREADS, sizeof(Mel3Smem), h->stream>>>(d_clips + c0, nc, h->mel_tab, h->mel_tabt, out,
+                                                                          h->gmax_ord, write_out);
+        CUDA_TRY(h, cudaGetLastError());
+    }
     return MOSS_ENC_OK;
 }
 
