@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(128) window_attn_tc_kernel(const __grid_consta
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 49152);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
     const int h = blockIdx.y;
-    const int2 win = windows[blockIdx.x];
+    const int2 win = windows[blockIdx.x];  // host-written table
     const int s = win.x, n = win.y;
     const int tid = threadIdx.x, warp = tid >> 5;
 
@@ -62,6 +62,10 @@ __global__ void __launch_bounds__(128) window_attn_tc_kernel(const __grid_consta
     tc_fence_after();
     const uint32_t tbase = *tslot;
     const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
+    // the TMEM of this CTA is held: later kernels may start (they never wait
+    // for TMEM that an unstarted CTA of this grid would need)
+    grid_dep_launch();
+    grid_dep_wait();
 
     if (tid == 0) {
         mbar_arrive_expect_tx(&bars[0], 3 * 16384);

@@ -290,9 +290,11 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 
     const int num_tiles = args.m_tiles * args.n_tiles;
     const int num_kb = args.K / C::BK;
+    if (threadIdx.x == 0) grid_dep_launch();
 
     if (warp == 0) {
         if (lane == 0) {
+            grid_dep_wait();
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -353,6 +355,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
         const int q = warp & 3;             // this warp may read TMEM lanes 32q .. 32q+31
         const int half = (warp - 2) >> 2;   // which of the two warps on this quarter
         uint8_t *stage = smem + C::STAGES * C::STAGE_BYTES + (warp - 2) * EPI_STAGE_BYTES;
+        grid_dep_wait();
         int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             const int acc = it & 1;
@@ -467,9 +470,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
     const int num_tiles = args.m_tiles * args.n_tiles;  // m_tiles counts 256-row pair tiles
     const int num_kb = args.K / C::BK;
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    // TMEM is held by every started CTA of this grid: the next kernel may start
+    if (threadIdx.x == 0) grid_dep_launch();
 
     if (warp == 0) {
         if (lane == 0) {
+            auto load_b = [&](uint8_t *st, uint32_t fb, int kb, int nt) {
+#pragma unroll
+                for (int j = 0; j < C::NSUB; j++)
+                    tma_load_2d_pair(&tmB, fb, st + C::A_BYTES + j * C::B_SUB_BYTES, kb * C::BK,
+                                     nt * BN + j * C::NS + (int)rank * (C::NS / 2));
+            };
+            // The weights do not depend on earlier kernels: the first tile's
+            // first stages of B are requested before waiting for them (each
+            // stage's first use needs no wait on its empty barrier).
+            const int npre = pair < num_tiles ? (num_kb < C::STAGES ? num_kb : C::STAGES) : 0;
+            for (int kb = 0; kb < npre; kb++) {
+                const uint32_t fb = map_to_rank(smem_u32(&full[kb]), 0);
+                mbar_arrive_expect_tx_remote(fb, C::STAGE_BYTES);
+                load_b(smem + kb * C::STAGE_BYTES, fb, kb, pair / args.m_tiles);
+            }
+            grid_dep_wait();
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -482,20 +503,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
                     t0 = item < 0 ? 0 : (item & 255) * args.tile_t;
                 }
                 for (int kb = 0; kb < num_kb; kb++) {
-                    if (!mbar_wait(&empty[s], ph ^ 1, args.err)) { ok = false; break; }
+                    const bool pre = tile == pair && kb < npre;  // B already requested
                     uint8_t *st = smem + s * C::STAGE_BYTES;
                     const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
-                    mbar_arrive_expect_tx_remote(fb, C::STAGE_BYTES);
+                    if (!pre) {
+                        if (!mbar_wait(&empty[s], ph ^ 1, args.err)) { ok = false; break; }
+                        mbar_arrive_expect_tx_remote(fb, C::STAGE_BYTES);
+                    }
                     if constexpr (AMODE == A_CONV_S2) {
                         const int tap = kb >> 3, kf = tap / 3, kt = tap - 3 * kf;
                         tma_load_4d_pair(&tmA, fb, st, (kb & 7) * 64, kf - 1, 2 * t0 + kt - 1, chunk);
                     } else {
                         tma_load_2d_pair(&tmA, fb, st, kb * C::BK, mt * 256 + (int)rank * 128);
                     }
-#pragma unroll
-                    for (int j = 0; j < C::NSUB; j++)
-                        tma_load_2d_pair(&tmB, fb, st + C::A_BYTES + j * C::B_SUB_BYTES, kb * C::BK,
-                                         nt * BN + j * C::NS + (int)rank * (C::NS / 2));
+                    if (!pre) load_b(st, fb, kb, nt);
                     if (++s == C::STAGES) { s = 0; ph ^= 1; }
                 }
             }
@@ -540,13 +561,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
         uint8_t *stage = smem + C::STAGES * C::STAGE_BYTES + (warp - 2) * EPI_STAGE_BYTES;
+        grid_dep_wait();
         int it = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
             const int acc = it % C::ACC;
             const uint32_t aph = (it / C::ACC) & 1;
+            const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
+            if constexpr (EPI == EPI_RESID_F32) {
+                // the residual rows this tile adds to go to L2 while the mainloop runs
+                const int row = mt * 256 + (int)rank * 128 + q * 32 + lane;
+                if (half == 0 && row < args.M)
+                    prefetch_l2(reinterpret_cast<const float *>(args.out) + (size_t)row * args.ldo + nt * BN, BN * 4);
+            }
             if (!mbar_wait(&tfull[acc], aph, args.err)) break;
             tc_fence_after();
-            const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
             int grow, aux;
             bool ok;
             if constexpr (AMODE == A_CONV_S2) {

@@ -301,6 +301,8 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
         S.band_n[i] = tab->band_n[i];
     }
     for (int i = tid; i < 128 * MEL_BAND; i += MEL2_THREADS) S.band_wt[i / 128][i % 128] = tabt->w[i / 128][i % 128];
+    grid_dep_wait();
+    grid_dep_launch();
     if (tid == 0) {
         int acc = 0;
         for (int c = 0; c < n_clips; c++) {
@@ -448,6 +450,8 @@ __global__ void mel_normalize_kernel(float *mel, long long count, const int *gma
 // gmax slots from caller-given device floats (or -inf to start an atomicMax).
 __global__ void gmax_init_kernel(int *gmax_ord, const float *const *src, int n)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) gmax_ord[i] = float_to_ordered(src[i] ? *src[i] : -INFINITY);
 }

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <mutex>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -79,6 +80,10 @@ struct moss_enc {
     void *d_tab = nullptr, *h_tab = nullptr;
     cudaEvent_t tab_event = nullptr;
 
+    // launches may overlap the previous kernel's tail (programmatic dependent
+    // launch); MOSS_ENC_PDL=0 in the environment at create turns it off
+    bool pdl = true;
+
     // measurement: launch counter and optional per-launch CUDA events
     int64_t launches = 0;
     bool profiling = false;
@@ -124,6 +129,26 @@ struct Launch {
 }  // namespace
 
 // ------------------------------------------------------------ small helpers
+
+// Launch `kern` on the handle's stream.  With h->pdl the launch carries
+// programmatic stream serialisation: the kernel may start while the previous
+// one finishes, and waits for it (griddepcontrol.wait) before touching its
+// results; every kernel launched here does so.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_k(moss_enc *h, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = h->stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = h->pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 static moss_enc_status fail(moss_enc *h, moss_enc_status s, const std::string &msg)
 {
@@ -228,8 +253,8 @@ static moss_enc_status gemm2(moss_enc *h, const char *name, const bf16 *A, int64
     const int grid = 2 * std::min(tiles, h->num_sms / 2);
     const double ka = k_alg > 0 ? k_alg : K;
     Launch L(h, name, 2.0 * M * N * ka, 2.0 * M * ka + 2.0 * N * ka + epi_out_bytes(EPI) * M * N);
-    gemm_tc2_kernel<BN, EPI><<<grid, Gemm2Cfg<BN>::THREADS, Gemm2Cfg<BN>::SMEM, h->stream>>>(ta, tb, a);
-    CUDA_TRY(h, cudaGetLastError());
+    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN>, dim3(grid), dim3(Gemm2Cfg<BN>::THREADS), Gemm2Cfg<BN>::SMEM,
+                         ta, tb, a));
     return MOSS_ENC_OK;
 }
 
@@ -291,8 +316,8 @@ static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, 
     a.tile_t = tile_t;
     const int grid = 2 * std::min(a.m_tiles * a.n_tiles, h->num_sms / 2);
     Launch L(h, name, 2.0 * 128.0 * n_items * CST * (9.0 * CST), 2.0 * 128.0 * n_items * (9.0 * CST) * 0.25 + 2.0 * 128.0 * n_items * CST);
-    gemm_tc2_kernel<160, EPI_GELU_BF16, A_CONV_S2><<<grid, Gemm2Cfg<160>::THREADS, Gemm2Cfg<160>::SMEM, h->stream>>>(ta, tb, a);
-    CUDA_TRY(h, cudaGetLastError());
+    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<160, EPI_GELU_BF16, A_CONV_S2>, dim3(grid), dim3(Gemm2Cfg<160>::THREADS),
+                         Gemm2Cfg<160>::SMEM, ta, tb, a));
     return MOSS_ENC_OK;
 }
 
@@ -526,6 +551,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     if (cudaGetDeviceProperties(&prop, h->device) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
     if (prop.major != 10) return bail(MOSS_ENC_ERR_CUDA);  // built for sm_100a only
     h->num_sms = prop.multiProcessorCount;
+    if (const char *e = std::getenv("MOSS_ENC_PDL")) h->pdl = std::strcmp(e, "0") != 0;
     if (!encode_fn()) return bail(MOSS_ENC_ERR_CUDA);
     if ((st = set_kernel_attrs(h)) != MOSS_ENC_OK) return bail(st);
 
@@ -837,9 +863,8 @@ static moss_enc_status launch_logmel(moss_enc *h, const MelClip *d_clips, int n_
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks, 2 * h->num_sms));
         Launch L(h, write_out ? "logmel" : "logmel_max", 0.0,
                  c0 == 0 ? 4.0 * 160 * (double)total_frames + (write_out ? 512.0 * total_frames : 0.0) : 0.0);
-        logmel3_kernel<<<grid, MEL2_THREADS, sizeof(Mel3Smem), h->stream>>>(d_clips + c0, nc, h->mel_tab, h->mel_tabt, out,
-                                                                          h->gmax_ord, write_out);
-        CUDA_TRY(h, cudaGetLastError());
+        CUDA_TRY(h, launch_k(h, logmel3_kernel, dim3(grid), dim3(MEL2_THREADS), sizeof(Mel3Smem), d_clips + c0, nc,
+                             (const MelTables *)h->mel_tab, (const MelBandT *)h->mel_tabt, out, h->gmax_ord, write_out));
     }
     return MOSS_ENC_OK;
 }
@@ -964,9 +989,9 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
     // ---- log-mel (raw) and per-clip maxima
     {
         Launch Lk(h, "gmax", 0.0, 0.0);
-        gmax_init_kernel<<<(n_clips + 127) / 128, 128, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), n_clips);
+        CUDA_TRY(h, launch_k(h, gmax_init_kernel, dim3((n_clips + 127) / 128), dim3(128), 0, h->gmax_ord,
+                             reinterpret_cast<const float *const *>(Dt + tl.logmax_src), n_clips));
     }
-    CUDA_TRY(h, cudaGetLastError());
     if (n_max_pass > 0)
         TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), n_max_pass, max_clip_frames, nullptr, 0, max_pass_frames));
     TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_main), n_clips, max_range_frames, h->mel_raw, 1, range_frames));
@@ -979,9 +1004,8 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
             double px = 0.0;
             for (int j = 0; j < gc; j++) px += 64.0 * sc[g0 + j].t1_lim;
             Launch L1(h, "conv1", 2.0 * 9 * CST * px, 2.0 * CST * px + 4.0 * 128 * 2 * px / 64.0);
-            conv1_kernel<<<dim3(400, gc), 240, 0, h->stream>>>(h->mel_raw, d_chunks + g0, h->gmax_ord, h->conv1_w,
-                                                              h->conv1_b, h->c1out);
-            CUDA_TRY(h, cudaGetLastError());
+            CUDA_TRY(h, launch_k(h, conv1_kernel, dim3(400, gc), dim3(240), 0, (const float *)h->mel_raw, d_chunks + g0,
+                                 (const int *)h->gmax_ord, (const float *)h->conv1_w, (const float *)h->conv1_b, h->c1out));
         }
         TRY(gemm_conv(h, "gemm_conv2", h->c1out, gc, 400, 64, d_t2 + g_off2[gi], g_n2[gi], h->conv2_w, h->conv2_b,
                       h->c2out));
@@ -1010,9 +1034,9 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         const LayerDev &L = h->layers[l];
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
-            layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln1_g, L.ln1_b, h->xn, (int)T, D, 0);
+            CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln1_g, L.ln1_b,
+                                 h->xn, (int)T, D, 0));
         }
-        CUDA_TRY(h, cudaGetLastError());
         GemmArgs a{};
         a.bias = L.bqkv;
         a.out = h->qkv;
@@ -1020,19 +1044,18 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         TRY((gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
         {
             Launch Lk(h, "attention", 4.0 * 64 * 20 * attn_pairs, 2.0 * T * (DQKV + D));
-            window_attn_tc_kernel<<<dim3((unsigned)n_chunks, 20), 128, ATTN_TC_SMEM, h->stream>>>(tm_qkv, d_ct, h->attn,
-                                                                                                 h->err);
+            CUDA_TRY(h, launch_k(h, window_attn_tc_kernel, dim3((unsigned)n_chunks, 20), dim3(128), ATTN_TC_SMEM, tm_qkv,
+                                 d_ct, h->attn, h->err));
         }
-        CUDA_TRY(h, cudaGetLastError());
         a.bias = L.bo;
         a.out = h->X;
         a.ldo = D;
         TRY((gemm2<320, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a)));
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
-            layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, L.ln2_g, L.ln2_b, h->xn, (int)T, D, 0);
+            CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln2_g, L.ln2_b,
+                                 h->xn, (int)T, D, 0));
         }
-        CUDA_TRY(h, cudaGetLastError());
         a.bias = L.b1;
         a.out = h->ffn;
         a.ldo = DFF;
@@ -1050,9 +1073,9 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
     // ---- head: ln_post -> proj1 -> GELU -> proj2
     {
         Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
-        layernorm1280_kernel<<<ln_grid, 256, 0, h->stream>>>(h->X, h->lnp_g, h->lnp_b, h->xn, (int)T, 2 * D, 1);
+        CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X,
+                             (const float *)h->lnp_g, (const float *)h->lnp_b, h->xn, (int)T, 2 * D, 1));
     }
-    CUDA_TRY(h, cudaGetLastError());
     // The head and adapter GEMMs take split operands [hi | lo] (bf16 pairs that
     // carry ~16 bits) against weights repeated along K: 6 % of the flops, and
     // it keeps the SwiGLU from amplifying bf16 rounding of its inputs.

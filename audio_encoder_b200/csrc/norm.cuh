@@ -16,6 +16,8 @@ __global__ void __launch_bounds__(256) layernorm1280_kernel(const float *__restr
                                                             bf16 *__restrict__ y, int rows, int ldy,
                                                             int split)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= rows) return;

@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(240) conv1_kernel(const float *__restrict__ me
                                                     bf16 *__restrict__ out)
 {
     __shared__ float in[3][130];  // 3 time rows x (128 freq + 2 zero pads)
+    grid_dep_wait();
+    grid_dep_launch();
     const int t = blockIdx.x, ci = blockIdx.y;
     const StemChunk ch = chunks[ci];
     if (t >= ch.t1_lim) return;  // outside the receptive field of the chunk's tokens
