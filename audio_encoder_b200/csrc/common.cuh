@@ -112,6 +112,38 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 
+// Bulk-async output of a box held in shared memory (layout as the map's
+// swizzle wants it).  The store writes the box; the reduce adds it, element
+// by element, to what global memory holds (the add happens in L2, so the
+// issuing thread never waits for a load).  Elements outside the map's
+// bounds are skipped.  Both are tracked as bulk groups of the issuing thread.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, const void *src, int x, int y)
+{
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Every committed bulk group of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Every committed bulk group of this thread has completed its global writes.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Orders this thread's ordinary shared-memory writes before later bulk-async
+// (TMA) reads of them.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // Bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
 {
@@ -245,6 +277,29 @@ __device__ __forceinline__ float erf_as7128(float x)
 __device__ __forceinline__ float gelu_fast(float x)
 {
     return 0.5f * x * (1.0f + erf_as7128(x * 0.70710678118654752f));
+}
+
+// The same GELU on two values at once with the paired fp32 instructions of
+// sm_100 (add/mul/fma on float2): the same formula and error bound, half the
+// instructions for the polynomial and the squarings.
+__device__ __forceinline__ float2 gelu2(float2 x)
+{
+    const float2 z = __fmul2_rn(x, make_float2(0.70710678118654752f, 0.70710678118654752f));
+    const float2 az = make_float2(fabsf(z.x), fabsf(z.y));
+    float2 p = __ffma2_rn(make_float2(4.30638e-5f, 4.30638e-5f), az, make_float2(2.765672e-4f, 2.765672e-4f));
+    p = __ffma2_rn(p, az, make_float2(1.520143e-4f, 1.520143e-4f));
+    p = __ffma2_rn(p, az, make_float2(9.2705272e-3f, 9.2705272e-3f));
+    p = __ffma2_rn(p, az, make_float2(4.22820123e-2f, 4.22820123e-2f));
+    p = __ffma2_rn(p, az, make_float2(7.05230784e-2f, 7.05230784e-2f));
+    p = __ffma2_rn(p, az, make_float2(1.0f, 1.0f));
+    float2 r = make_float2(__fdividef(1.0f, p.x), __fdividef(1.0f, p.y));
+    r = __fmul2_rn(r, r);
+    r = __fmul2_rn(r, r);
+    r = __fmul2_rn(r, r);
+    r = __fmul2_rn(r, r);
+    const float2 e = make_float2(copysignf(1.0f - r.x, z.x), copysignf(1.0f - r.y, z.y));
+    const float2 hx = __fmul2_rn(x, make_float2(0.5f, 0.5f));
+    return __ffma2_rn(hx, e, hx);  // 0.5 x (1 + erf)
 }
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }

@@ -123,10 +123,12 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
                         const float4 b0 = ld_f4(b + 8 * q), b1 = ld_f4(b + 8 * q + 4);
                         const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-                        for (int j = 0; j < 8; j++) {
-                            float o = __uint_as_float(r[8 * q + j]) + bb[j];
-                            if constexpr (EPI == EPI_GELU_BF16) o = gelu_fast(o);
-                            r[8 * q + j] = __float_as_uint(o);
+                        for (int j = 0; j < 8; j += 2) {
+                            float2 o = __fadd2_rn(make_float2(__uint_as_float(r[8 * q + j]), __uint_as_float(r[8 * q + j + 1])),
+                                                  make_float2(bb[j], bb[j + 1]));
+                            if constexpr (EPI == EPI_GELU_BF16) o = gelu2(o);
+                            r[8 * q + j] = __float_as_uint(o.x);
+                            r[8 * q + j + 1] = __float_as_uint(o.y);
                         }
                     }
                 }
@@ -227,6 +229,101 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
                         if (okv[it]) *reinterpret_cast<float4 *>(dst[it]) = v;
                     }
                     __syncwarp();
+                }
+            }
+        }
+    }
+}
+
+// Output through the bulk-async (TMA) unit, for plain row-major outputs:
+// the 32-row slab of this warp starts at output row `row0`.  bf16 outputs
+// leave in boxes of 32 rows x 64 columns (tma_store_2d); fp32 outputs in
+// boxes of 32 rows x 32 columns, stored (EPI_F32) or added to the residual
+// stream in L2 (EPI_RESID_F32, tma_reduce_add_2d: X + (acc + bias), the same
+// single rounding as a load-add-store, with no load latency in the warp).
+// The staging buffer is reused once the previous box has been read out of it.
+template <int BN, int EPI>
+__device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensorMap *tmC, uint32_t tbase, int half,
+                                               int lane, uint8_t *stage, int row0, int col0)
+{
+    static_assert(BN % 64 == 0, "TMA output needs 64-column groups");
+    static_assert(EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 || EPI == EPI_F32, "epilogue");
+    constexpr int NG = BN / 64;
+    const bool live = row0 < a.M;  // whole slab outside the output: nothing to write
+#pragma unroll 1
+    for (int g = half; g < NG; g += 2) {
+        const int c0 = g * 64;
+        uint32_t r[64];
+        tmem_ld32(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld_wait();
+        const float *b = a.bias + col0 + c0;
+        if constexpr (EPI == EPI_BF16 || EPI == EPI_GELU_BF16) {
+#pragma unroll
+            for (int q = 0; q < 16; q++) {
+                const float4 bb = ld_f4(b + 4 * q);
+                float2 v0 = make_float2(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]));
+                float2 v1 = make_float2(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+                v0 = __fadd2_rn(v0, make_float2(bb.x, bb.y));
+                v1 = __fadd2_rn(v1, make_float2(bb.z, bb.w));
+                if constexpr (EPI == EPI_GELU_BF16) {
+                    v0 = gelu2(v0);
+                    v1 = gelu2(v1);
+                }
+                r[4 * q] = __float_as_uint(v0.x);
+                r[4 * q + 1] = __float_as_uint(v0.y);
+                r[4 * q + 2] = __float_as_uint(v1.x);
+                r[4 * q + 3] = __float_as_uint(v1.y);
+            }
+            const int parts = a.split_off ? 2 : 1;
+#pragma unroll 1
+            for (int part = 0; part < parts; part++) {
+                if (lane == 0) bulk_wait_read();
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const float x0 = __uint_as_float(r[8 * q + 2 * j]), x1 = __uint_as_float(r[8 * q + 2 * j + 1]);
+                        if (part == 0) {
+                            w[j] = pack_bf16x2(x0, x1);
+                        } else {
+                            const __nv_bfloat162 hi = __floats2bfloat162_rn(x0, x1);
+                            w[j] = pack_bf16x2(x0 - __low2float(hi), x1 - __high2float(hi));
+                        }
+                    }
+                    *stage_at(stage, lane, q) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0 && live) {
+                    tma_store_2d(tmC, stage, col0 + c0 + part * a.split_off, row0);
+                    bulk_commit();
+                }
+            }
+        } else {
+#pragma unroll
+            for (int hh = 0; hh < 2; hh++) {
+                if (lane == 0) bulk_wait_read();
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    const float4 bb = ld_f4(b + 32 * hh + 4 * q);
+                    float2 v0 = make_float2(__uint_as_float(r[32 * hh + 4 * q]), __uint_as_float(r[32 * hh + 4 * q + 1]));
+                    float2 v1 = make_float2(__uint_as_float(r[32 * hh + 4 * q + 2]), __uint_as_float(r[32 * hh + 4 * q + 3]));
+                    v0 = __fadd2_rn(v0, make_float2(bb.x, bb.y));
+                    v1 = __fadd2_rn(v1, make_float2(bb.z, bb.w));
+                    *reinterpret_cast<float4 *>(stage_at(stage, lane, q)) = make_float4(v0.x, v0.y, v1.x, v1.y);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0 && live) {
+                    if constexpr (EPI == EPI_RESID_F32)
+                        tma_reduce_add_2d(tmC, stage, col0 + c0 + 32 * hh, row0);
+                    else
+                        tma_store_2d(tmC, stage, col0 + c0 + 32 * hh, row0);
+                    bulk_commit();
                 }
             }
         }
@@ -431,9 +528,13 @@ struct Gemm2Cfg {
 template <int BN, int EPI, int AMODE = A_PLAIN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const GemmArgs args)
+                    const __grid_constant__ CUtensorMap tmC, const GemmArgs args)
 {
     using C = Gemm2Cfg<BN>;
+    // plain row-major outputs leave through TMA boxes (tmC); the conv and
+    // conv_out row mappings and SwiGLU keep per-row stores
+    constexpr bool TMA_OUT = AMODE == A_PLAIN && BN % 64 == 0 &&
+                             (EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 || EPI == EPI_F32);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES + C::STAGING);
@@ -456,6 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        if constexpr (TMA_OUT) prefetch_tmap(&tmC);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -587,10 +689,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
                 plain_row<EPI>(args, mt * 256 + (int)rank * 128 + q * 32 + lane, grow, ok, aux);
             }
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-            drain_tile<BN, EPI>(args, tbase, half, lane, stage, grow, ok, aux, nt * BN);
+            if constexpr (TMA_OUT)
+                drain_tile_tma<BN, EPI>(args, &tmC, tbase, half, lane, stage, mt * 256 + (int)rank * 128 + q * 32, nt * BN);
+            else
+                drain_tile<BN, EPI>(args, tbase, half, lane, stage, grow, ok, aux, nt * BN);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&tempty[acc]), 0));
+        }
+        if constexpr (TMA_OUT) {
+            if (lane == 0) bulk_wait_all();  // this warp's output boxes are written before the grid ends
         }
     }
     tc_fence_before();
