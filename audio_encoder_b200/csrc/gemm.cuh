@@ -97,10 +97,14 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
 #pragma unroll 1
     for (int g = half; g < NG; g += 2) {
         const int c0 = g * 64;
-        const int nc = BN - c0 < 64 ? BN - c0 : 64;  // 64, or 32 for the last group of BN = 160
+        // 64 columns, or the last group's rest: 32 (BN = 160) or 48 (BN = 240)
+        constexpr int REST = BN % 64;
+        static_assert(REST == 0 || REST == 32 || REST == 48, "BN % 64 must be 0, 32 or 48");
+        const int nc = BN - c0 < 64 ? REST : 64;
         uint32_t r[64];
         tmem_ld32(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         if (nc == 64) tmem_ld32(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        if (REST == 48 && nc == 48) tmem_ld16(tbase + c0 + 32, &r[32]);
         tmem_ld_wait();
         if constexpr (EPI == EPI_SWIGLU_BF16 || EPI == EPI_BF16 || EPI == EPI_GELU_BF16) {
             // values in place (fp32 bits in r), then one or two bf16 passes
@@ -157,14 +161,14 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
                 }
                 __syncwarp();
                 bf16 *out = reinterpret_cast<bf16 *>(a.out) + ocol + part * a.split_off;
-                if (nv == 64) {  // 8 lanes per 128-byte row, 4 rows per instruction
+                if (nv > 32) {  // 8 lanes per 128-byte row (6 of them for 48 values), 4 rows per instruction
 #pragma unroll
                     for (int it = 0; it < 8; it++) {
                         const int row = it * 4 + (lane >> 3), ch = lane & 7;
                         const int grow = __shfl_sync(0xffffffffu, my_row, row);
                         const bool ok = __shfl_sync(0xffffffffu, (int)my_ok, row);
                         const uint4 v = *stage_at(stage, row, ch);
-                        if (ok) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
+                        if (ok && ch * 8 < nv) *reinterpret_cast<uint4 *>(out + (size_t)grow * a.ldo + ch * 8) = v;
                     }
                 } else {  // 32 values: 4 lanes per 64-byte row, 8 rows per instruction
 #pragma unroll
@@ -179,6 +183,7 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
                 __syncwarp();
             }
         } else {
+            static_assert(REST != 48, "fp32 epilogues take BN % 64 of 0 or 32");
             // fp32 results, 32 columns (128 B per row) at a time
 #pragma unroll
             for (int hh = 0; hh < 2; hh++) {
@@ -520,7 +525,7 @@ struct Gemm2Cfg {
     static constexpr uint32_t TMEM_COLS = ACC * BN <= 128 ? 128 : ACC * BN <= 256 ? 256 : 512;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 256;
     static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
-    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 320, "BN must be a multiple of 32 in [64, 320]");
+    static_assert(BN % 16 == 0 && BN >= 64 && BN <= 320, "BN must be a multiple of 16 in [64, 320]");
     static_assert(NS % 16 == 0 && NS <= 256, "MMA N");
     static_assert(B_SUB_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
 };
@@ -641,12 +646,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + s * C::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + C::A_BYTES;
+                    // conv: the last channel block of a tap holds channels 448..479 and
+                    // 32 zeros (past the 480 channels); its zero half is not multiplied
+                    const int nk = (AMODE == A_CONV_S2 && (kb & 7) == 7) ? 2 : C::BK / 16;
 #pragma unroll
                     for (int k = 0; k < C::BK / 16; k++)
 #pragma unroll
                         for (int j = 0; j < C::NSUB; j++)
-                            mma_bf16_pair(d + j * C::NS, sw128_desc(a_addr + k * 32),
-                                          sw128_desc(b_addr + j * C::B_SUB_BYTES + k * 32), idesc, (kb | k) != 0);
+                            if (k < nk)
+                                mma_bf16_pair(d + j * C::NS, sw128_desc(a_addr + k * 32),
+                                              sw128_desc(b_addr + j * C::B_SUB_BYTES + k * 32), idesc, (kb | k) != 0);
                     const uint32_t eb = smem_u32(&empty[s]);
                     mma_commit_pair(map_to_rank(eb, 0));
                     mma_commit_pair(map_to_rank(eb, 1));

@@ -28,6 +28,7 @@ namespace {
 constexpr int D = 1280, DQKV = 3840, DFF = 5120, CST = 480, DOUT = 2048, DADP = 8192;
 constexpr int CHUNK_FRAMES = 800, CHUNK_TOKENS = 100, CHUNK_SAMPLES = 128000, HOP = 160;
 constexpr int CONV_K = 9 * 512;  // conv2/conv3 patch width: 9 taps x 480 channels padded to 512
+constexpr int CONV_BN = 240;     // conv2/conv3 output channels per pair tile (480 in two)
 constexpr int STEM_GROUP_DEFAULT = 32;
 constexpr int C2_TILES = 50, C3_TILES = 13;  // 128-row tiles per chunk of conv2 (4 t x 32 f) / conv3 (8 t x 16 f)
 
@@ -327,14 +328,14 @@ static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, 
     const int Fo = (Fi + 1) / 2, To = (Ti + 1) / 2, tile_t = 128 / Fo;
     CUtensorMap ta, tb;
     if (!tmap_conv(&ta, in, chunks, Ti, Fi, tile_t) ||
-        !tmap_2d(&tb, W, (uint64_t)CONV_K, (uint64_t)CST, (uint64_t)CONV_K * 2, 64, 80))
+        !tmap_2d(&tb, W, (uint64_t)CONV_K, (uint64_t)CST, (uint64_t)CONV_K * 2, 64, CONV_BN / 2))
         return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (conv)");
     GemmArgs a{};
     a.M = n_items * 128;
     a.N = CST;
     a.K = CONV_K;
     a.m_tiles = (n_items + 1) / 2;
-    a.n_tiles = CST / 160;
+    a.n_tiles = CST / CONV_BN;
     a.err = h->err;
     a.bias = bias;
     a.out = out;
@@ -344,8 +345,8 @@ static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, 
     a.tile_t = tile_t;
     const int grid = 2 * std::min(a.m_tiles * a.n_tiles, h->num_sms / 2);
     Launch L(h, name, 2.0 * 128.0 * n_items * CST * (9.0 * CST), 2.0 * 128.0 * n_items * (9.0 * CST) * 0.25 + 2.0 * 128.0 * n_items * CST);
-    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<160, EPI_GELU_BF16, A_CONV_S2>, dim3(grid), dim3(Gemm2Cfg<160>::THREADS),
-                         Gemm2Cfg<160>::SMEM, ta, tb, tb, a));
+    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<CONV_BN, EPI_GELU_BF16, A_CONV_S2>, dim3(grid),
+                         dim3(Gemm2Cfg<CONV_BN>::THREADS), Gemm2Cfg<CONV_BN>::SMEM, ta, tb, tb, a));
     return MOSS_ENC_OK;
 }
 
@@ -526,8 +527,8 @@ extern "C" void moss_enc_destroy(moss_enc *h)
 
 static moss_enc_status set_kernel_attrs(moss_enc *h)
 {
-    CUDA_TRY(h, cudaFuncSetAttribute(gemm_tc2_kernel<160, EPI_GELU_BF16, A_CONV_S2>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Gemm2Cfg<160>::SMEM));
+    CUDA_TRY(h, cudaFuncSetAttribute(gemm_tc2_kernel<CONV_BN, EPI_GELU_BF16, A_CONV_S2>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Gemm2Cfg<CONV_BN>::SMEM));
     CUDA_TRY(h, (gemm2_attr<256, EPI_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_RESID_F32>()));
@@ -1055,8 +1056,9 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
     const int ln_grid = (int)((T + 7) / 8);
     double attn_pairs = 0.0;  // query-key pairs inside windows
     for (int64_t c = 0; c < n_chunks; c++) attn_pairs += (double)ct[c].y * ct[c].y;
-    CUtensorMap tm_qkv;  // Q, K, V slices of one window and head: 128 rows x 64
-    if (!tmap_2d(&tm_qkv, h->qkv, (uint64_t)DQKV, (uint64_t)T, (uint64_t)DQKV * 2, 64, 128))
+    static_assert(CHUNK_TOKENS <= ATTN_ROWS, "a window must fit the attention kernel's slices");
+    CUtensorMap tm_qkv;  // Q, K, V slices of one window and head: ATTN_ROWS rows x 64
+    if (!tmap_2d(&tm_qkv, h->qkv, (uint64_t)DQKV, (uint64_t)T, (uint64_t)DQKV * 2, 64, ATTN_ROWS))
         return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (qkv)");
     for (size_t l = 0; l < h->layers.size(); l++) {
         const LayerDev &L = h->layers[l];

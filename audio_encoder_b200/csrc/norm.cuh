@@ -10,7 +10,7 @@
 
 namespace moss {
 
-__global__ void __launch_bounds__(256) layernorm1280_kernel(const float *__restrict__ x,
+__global__ void __launch_bounds__(256, 4) layernorm1280_kernel(const float *__restrict__ x,
                                                             const float *__restrict__ gamma,
                                                             const float *__restrict__ beta,
                                                             bf16 *__restrict__ y, int rows, int ldy,

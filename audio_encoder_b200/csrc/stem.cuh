@@ -46,27 +46,25 @@ __global__ void __launch_bounds__(240) conv1_kernel(const float *__restrict__ me
         in[kt][i % 130] = v;
     }
     __syncthreads();
+    // channels c, c + 1 side by side in the paired fp32 instructions
     const int c = 2 * threadIdx.x;
-    float wa[9], wb[9];
+    float2 w[9];
 #pragma unroll
-    for (int k = 0; k < 9; k++) {
-        wa[k] = w1[c * 9 + k];
-        wb[k] = w1[(c + 1) * 9 + k];
-    }
-    const float ba = b1[c], bb = b1[c + 1];
+    for (int k = 0; k < 9; k++) w[k] = make_float2(w1[c * 9 + k], w1[(c + 1) * 9 + k]);
+    const float2 b = make_float2(b1[c], b1[c + 1]);
     bf16 *dst = out + ((size_t)ci * 400 + t) * 64 * 480 + c;
 #pragma unroll 4
     for (int f = 0; f < 64; f++) {
-        float sa = ba, sb = bb;
+        float2 acc = b;
 #pragma unroll
         for (int kf = 0; kf < 3; kf++)
 #pragma unroll
             for (int kt = 0; kt < 3; kt++) {
                 const float x = in[kt][2 * f + kf];  // freq index 2f + kf - 1, shifted by the pad
-                sa += wa[kf * 3 + kt] * x;
-                sb += wb[kf * 3 + kt] * x;
+                acc = __ffma2_rn(w[kf * 3 + kt], make_float2(x, x), acc);
             }
-        *reinterpret_cast<uint32_t *>(dst + (size_t)f * 480) = pack_bf16x2(gelu_fast(sa), gelu_fast(sb));
+        const float2 g = gelu2(acc);
+        *reinterpret_cast<uint32_t *>(dst + (size_t)f * 480) = pack_bf16x2(g.x, g.y);
     }
 }
 
