@@ -246,15 +246,29 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
 // boxes of 32 rows x 32 columns, stored (EPI_F32) or added to the residual
 // stream in L2 (EPI_RESID_F32, tma_reduce_add_2d: X + (acc + bias), the same
 // single rounding as a load-add-store, with no load latency in the warp).
-// The staging buffer is reused once the previous box has been read out of it.
+// Boxes are staged in `nbuf` 4 KB buffers used in turn (1024-byte aligned,
+// EPI_STAGE_BYTES apart); a buffer is rewritten only after the boxes in
+// flight have been read out of shared memory.
 template <int BN, int EPI>
 __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensorMap *tmC, uint32_t tbase, int half,
-                                               int lane, uint8_t *stage, int row0, int col0)
+                                               int lane, uint8_t *stage_base, int nbuf, int row0, int col0)
 {
     static_assert(BN % 64 == 0, "TMA output needs 64-column groups");
     static_assert(EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 || EPI == EPI_F32, "epilogue");
     constexpr int NG = BN / 64;
     const bool live = row0 < a.M;  // whole slab outside the output: nothing to write
+    // boxes of the previous tile may still be reading the staging buffer
+    if (lane == 0) bulk_wait_read();
+    int bi = 0;  // next staging buffer
+    // the buffer for the next box; waits for the earlier boxes' reads when the ring wraps
+    auto next_stage = [&]() -> uint8_t * {
+        if (bi == nbuf) {
+            bi = 0;
+            if (lane == 0) bulk_wait_read();
+        }
+        __syncwarp();
+        return stage_base + (bi++) * EPI_STAGE_BYTES;
+    };
 #pragma unroll 1
     for (int g = half; g < NG; g += 2) {
         const int c0 = g * 64;
@@ -283,8 +297,7 @@ __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensor
             const int parts = a.split_off ? 2 : 1;
 #pragma unroll 1
             for (int part = 0; part < parts; part++) {
-                if (lane == 0) bulk_wait_read();
-                __syncwarp();
+                uint8_t *stage = next_stage();
 #pragma unroll
                 for (int q = 0; q < 8; q++) {
                     uint32_t w[4];
@@ -310,8 +323,7 @@ __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensor
         } else {
 #pragma unroll
             for (int hh = 0; hh < 2; hh++) {
-                if (lane == 0) bulk_wait_read();
-                __syncwarp();
+                uint8_t *stage = next_stage();
 #pragma unroll
                 for (int q = 0; q < 8; q++) {
                     const float4 bb = ld_f4(b + 32 * hh + 4 * q);
@@ -631,6 +643,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             constexpr uint32_t idesc = idesc_bf16(256, C::NS);
+            // Descriptors and barrier addresses are formed once: the issue loop
+            // shares its SM sub-partition with epilogue warps, and every
+            // instruction it saves brings the next MMA to the tensor pipe sooner.
+            // A descriptor's start-address field is the byte address / 16, so
+            // stage s and k-step k add (s * STAGE_BYTES + 32 k) / 16 to stage 0's.
+            const uint64_t a_desc0 = sw128_desc(smem_u32(smem));
+            const uint32_t emp0 = map_to_rank(smem_u32(&empty[0]), 0), emp1 = map_to_rank(smem_u32(&empty[0]), 1);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -644,8 +663,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
                 for (int kb = 0; kb < num_kb; kb++) {
                     if (!mbar_wait(&full[s], ph, args.err)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + C::A_BYTES;
+                    const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                    const uint64_t bd = ad + (C::A_BYTES >> 4);
                     // conv: the last channel block of a tap holds channels 448..479 and
                     // 32 zeros (past the 480 channels); its zero half is not multiplied
                     const int nk = (AMODE == A_CONV_S2 && (kb & 7) == 7) ? 2 : C::BK / 16;
@@ -654,11 +673,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
 #pragma unroll
                         for (int j = 0; j < C::NSUB; j++)
                             if (k < nk)
-                                mma_bf16_pair(d + j * C::NS, sw128_desc(a_addr + k * 32),
-                                              sw128_desc(b_addr + j * C::B_SUB_BYTES + k * 32), idesc, (kb | k) != 0);
-                    const uint32_t eb = smem_u32(&empty[s]);
-                    mma_commit_pair(map_to_rank(eb, 0));
-                    mma_commit_pair(map_to_rank(eb, 1));
+                                mma_bf16_pair(d + j * C::NS, ad + 2 * k, bd + j * (C::B_SUB_BYTES >> 4) + 2 * k, idesc,
+                                              (kb | k) != 0);
+                    mma_commit_pair(emp0 + 8 * s);
+                    mma_commit_pair(emp1 + 8 * s);
                     if (++s == C::STAGES) { s = 0; ph ^= 1; }
                 }
                 if (ok) {
@@ -698,9 +716,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
                 plain_row<EPI>(args, mt * 256 + (int)rank * 128 + q * 32 + lane, grow, ok, aux);
             }
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-            if constexpr (TMA_OUT)
-                drain_tile_tma<BN, EPI>(args, &tmC, tbase, half, lane, stage, mt * 256 + (int)rank * 128 + q * 32, nt * BN);
-            else
+            if constexpr (TMA_OUT) {
+                // On the CTA's last tile the stage ring is idle once the
+                // accumulator is full (every load of this CTA has been consumed),
+                // so each epilogue warp stages through its eighth of the ring and
+                // keeps several boxes in flight; otherwise one 4 KB buffer.
+                constexpr int RING_BUFS = (int)(C::STAGES * C::STAGE_BYTES / C::EPI_WARPS / EPI_STAGE_BYTES);
+                const bool last = tile + npairs >= num_tiles;
+                uint8_t *stg = last ? smem + (warp - 2) * RING_BUFS * EPI_STAGE_BYTES : stage;
+                drain_tile_tma<BN, EPI>(args, &tmC, tbase, half, lane, stg, last ? RING_BUFS : 1,
+                                        mt * 256 + (int)rank * 128 + q * 32, nt * BN);
+            } else
                 drain_tile<BN, EPI>(args, tbase, half, lane, stage, grow, ok, aux, nt * BN);
             tc_fence_before();
             __syncwarp();
