@@ -518,17 +518,22 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 //    commits once to its own and once to the odd CTA's barrier.
 //  - tempty[acc] lives in the even CTA; all 16 epilogue warps of the pair
 //    arrive on it.
-template <int BN>
+template <int BN, int KSUB = 1>
 struct Gemm2Cfg {
-    static constexpr int BM = 128, BK = 64;  // rows per CTA; the pair covers 256
+    // A stage holds KSUB k sub-blocks of 64 (one 128-byte swizzle atom each):
+    // larger stages halve the stage hand-offs between the producer, the MMA
+    // lane and the barriers, which measurably idle the tensor pipe.
+    static constexpr int BM = 128, BK = 64 * KSUB;  // rows per CTA; the pair covers 256
     static constexpr int EPI_WARPS = 8;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     // Tiles wider than one MMA (BN = 320) are two MMAs of BN/2 per k-step.
     static constexpr int NSUB = BN > 256 ? 2 : 1;
-    static constexpr int NS = BN / NSUB;             // N of one MMA instruction
-    static constexpr uint32_t B_SUB_BYTES = (NS / 2) * BK * 2;  // this CTA's half of one MMA's B
-    static constexpr uint32_t A_BYTES = BM * BK * 2;
-    static constexpr uint32_t B_BYTES = NSUB * B_SUB_BYTES;
+    static constexpr int NS = BN / NSUB;                        // N of one MMA instruction
+    static constexpr uint32_t B_SUB_BYTES = (NS / 2) * 64 * 2;  // this CTA's half of one MMA's B, one k sub-block
+    static constexpr uint32_t A_SUB = BM * 64 * 2;              // this CTA's A rows, one k sub-block
+    static constexpr uint32_t A_BYTES = KSUB * A_SUB;
+    static constexpr uint32_t B_KS = NSUB * B_SUB_BYTES;        // B bytes of one k sub-block
+    static constexpr uint32_t B_BYTES = KSUB * B_KS;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr uint32_t STAGING = EPI_WARPS * EPI_STAGE_BYTES;
     static constexpr int STAGES_RAW = (int)((SMEM_LIMIT - 1024 - 256 - STAGING) / STAGE_BYTES);
@@ -537,17 +542,19 @@ struct Gemm2Cfg {
     static constexpr uint32_t TMEM_COLS = ACC * BN <= 128 ? 128 : ACC * BN <= 256 ? 256 : 512;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 256;
     static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
+    static_assert(STAGES >= 2, "at least two pipeline stages");
+    static_assert(KSUB == 1 || KSUB == 2, "k sub-blocks per stage");
     static_assert(BN % 16 == 0 && BN >= 64 && BN <= 320, "BN must be a multiple of 16 in [64, 320]");
     static_assert(NS % 16 == 0 && NS <= 256, "MMA N");
     static_assert(B_SUB_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
 };
 
-template <int BN, int EPI, int AMODE = A_PLAIN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREADS, 1)
+template <int BN, int EPI, int AMODE = A_PLAIN, int KSUB = 1>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const GemmArgs args)
 {
-    using C = Gemm2Cfg<BN>;
+    using C = Gemm2Cfg<BN, KSUB>;
     // plain row-major outputs leave through TMA boxes (tmC); the conv and
     // conv_out row mappings and SwiGLU keep per-row stores
     constexpr bool TMA_OUT = AMODE == A_PLAIN && BN % 64 == 0 &&
@@ -596,9 +603,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
         if (lane == 0) {
             auto load_b = [&](uint8_t *st, uint32_t fb, int kb, int nt) {
 #pragma unroll
-                for (int j = 0; j < C::NSUB; j++)
-                    tma_load_2d_pair(&tmB, fb, st + C::A_BYTES + j * C::B_SUB_BYTES, kb * C::BK,
-                                     nt * BN + j * C::NS + (int)rank * (C::NS / 2));
+                for (int ks = 0; ks < KSUB; ks++)
+#pragma unroll
+                    for (int j = 0; j < C::NSUB; j++)
+                        tma_load_2d_pair(&tmB, fb, st + C::A_BYTES + ks * C::B_KS + j * C::B_SUB_BYTES,
+                                         kb * C::BK + ks * 64, nt * BN + j * C::NS + (int)rank * (C::NS / 2));
             };
             // The weights do not depend on earlier kernels: the first tile's
             // first stages of B are requested before waiting for them (each
@@ -629,11 +638,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
                         if (!mbar_wait(&empty[s], ph ^ 1, args.err)) { ok = false; break; }
                         mbar_arrive_expect_tx_remote(fb, C::STAGE_BYTES);
                     }
-                    if constexpr (AMODE == A_CONV_S2) {
-                        const int tap = kb >> 3, kf = tap / 3, kt = tap - 3 * kf;
-                        tma_load_4d_pair(&tmA, fb, st, (kb & 7) * 64, kf - 1, 2 * t0 + kt - 1, chunk);
-                    } else {
-                        tma_load_2d_pair(&tmA, fb, st, kb * C::BK, mt * 256 + (int)rank * 128);
+#pragma unroll
+                    for (int ks = 0; ks < KSUB; ks++) {
+                        if constexpr (AMODE == A_CONV_S2) {
+                            // 64-wide k block b = tap * 8 + channel block
+                            const int b = kb * KSUB + ks, tap = b >> 3, kf = tap / 3, kt = tap - 3 * kf;
+                            tma_load_4d_pair(&tmA, fb, st + ks * C::A_SUB, (b & 7) * 64, kf - 1, 2 * t0 + kt - 1, chunk);
+                        } else {
+                            tma_load_2d_pair(&tmA, fb, st + ks * C::A_SUB, kb * C::BK + ks * 64, mt * 256 + (int)rank * 128);
+                        }
                     }
                     if (!pre) load_b(st, fb, kb, nt);
                     if (++s == C::STAGES) { s = 0; ph ^= 1; }
@@ -665,16 +678,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN>::THREAD
                     tc_fence_after();
                     const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
                     const uint64_t bd = ad + (C::A_BYTES >> 4);
-                    // conv: the last channel block of a tap holds channels 448..479 and
-                    // 32 zeros (past the 480 channels); its zero half is not multiplied
-                    const int nk = (AMODE == A_CONV_S2 && (kb & 7) == 7) ? 2 : C::BK / 16;
 #pragma unroll
-                    for (int k = 0; k < C::BK / 16; k++)
+                    for (int ks = 0; ks < KSUB; ks++) {
+                        // conv: the last channel block of a tap holds channels 448..479 and
+                        // 32 zeros (past the 480 channels); its zero half is not multiplied
+                        const int nk = (AMODE == A_CONV_S2 && ((kb * KSUB + ks) & 7) == 7) ? 2 : 4;
 #pragma unroll
-                        for (int j = 0; j < C::NSUB; j++)
-                            if (k < nk)
-                                mma_bf16_pair(d + j * C::NS, ad + 2 * k, bd + j * (C::B_SUB_BYTES >> 4) + 2 * k, idesc,
-                                              (kb | k) != 0);
+                        for (int k = 0; k < 4; k++)
+#pragma unroll
+                            for (int j = 0; j < C::NSUB; j++)
+                                if (k < nk)
+                                    mma_bf16_pair(d + j * C::NS, ad + ks * (C::A_SUB >> 4) + 2 * k,
+                                                  bd + ks * (C::B_KS >> 4) + j * (C::B_SUB_BYTES >> 4) + 2 * k, idesc,
+                                                  (kb | ks | k) != 0);
+                    }
                     mma_commit_pair(emp0 + 8 * s);
                     mma_commit_pair(emp1 + 8 * s);
                     if (++s == C::STAGES) { s = 0; ph ^= 1; }

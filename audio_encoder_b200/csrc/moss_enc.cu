@@ -258,10 +258,12 @@ static moss_enc_status gemm(moss_enc *h, const char *name, const bf16 *A, int64_
     return MOSS_ENC_OK;
 }
 
-// The same on CTA pairs (256-row tiles, cluster of 2).
+// The same on CTA pairs (256-row tiles, cluster of 2).  ksub: 64-wide k
+// sub-blocks per pipeline stage (2 when K allows it and the stages still fit
+// at least three deep, i.e. BN <= 256; callers may ask for 1 or 2).
 template <int BN, int EPI>
 static moss_enc_status gemm2(moss_enc *h, const char *name, const bf16 *A, int64_t M, int K, const bf16 *B, int N,
-                             GemmArgs a, int k_alg = 0)
+                             GemmArgs a, int k_alg = 0, int ksub = BN <= 256 ? 2 : 1)
 {
     if (M <= 0) return MOSS_ENC_OK;
     if (K % 64 != 0 || N % BN != 0 || M > INT32_MAX)
@@ -282,16 +284,23 @@ static moss_enc_status gemm2(moss_enc *h, const char *name, const bf16 *A, int64
     const int grid = 2 * std::min(tiles, h->num_sms / 2);
     const double ka = k_alg > 0 ? k_alg : K;
     Launch L(h, name, 2.0 * M * N * ka, 2.0 * M * ka + 2.0 * N * ka + epi_out_bytes(EPI) * M * N);
-    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN>, dim3(grid), dim3(Gemm2Cfg<BN>::THREADS), Gemm2Cfg<BN>::SMEM,
-                         ta, tb, tc, a));
+    if (ksub == 2 && K % 128 == 0)
+        CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 2>, dim3(grid), dim3(Gemm2Cfg<BN, 2>::THREADS),
+                             Gemm2Cfg<BN, 2>::SMEM, ta, tb, tc, a));
+    else
+        CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 1>, dim3(grid), dim3(Gemm2Cfg<BN, 1>::THREADS),
+                             Gemm2Cfg<BN, 1>::SMEM, ta, tb, tc, a));
     return MOSS_ENC_OK;
 }
 
 template <int BN, int EPI>
 static cudaError_t gemm2_attr()
 {
-    return cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)Gemm2Cfg<BN>::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI, A_PLAIN, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Gemm2Cfg<BN, 1>::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI, A_PLAIN, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Gemm2Cfg<BN, 2>::SMEM);
 }
 
 #define TRY(x)                                  \
@@ -345,8 +354,8 @@ static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, 
     a.tile_t = tile_t;
     const int grid = 2 * std::min(a.m_tiles * a.n_tiles, h->num_sms / 2);
     Launch L(h, name, 2.0 * 128.0 * n_items * CST * (9.0 * CST), 2.0 * 128.0 * n_items * (9.0 * CST) * 0.25 + 2.0 * 128.0 * n_items * CST);
-    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<CONV_BN, EPI_GELU_BF16, A_CONV_S2>, dim3(grid),
-                         dim3(Gemm2Cfg<CONV_BN>::THREADS), Gemm2Cfg<CONV_BN>::SMEM, ta, tb, tb, a));
+    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<CONV_BN, EPI_GELU_BF16, A_CONV_S2, 2>, dim3(grid),
+                         dim3(Gemm2Cfg<CONV_BN, 2>::THREADS), Gemm2Cfg<CONV_BN, 2>::SMEM, ta, tb, tb, a));
     return MOSS_ENC_OK;
 }
 
@@ -527,8 +536,8 @@ extern "C" void moss_enc_destroy(moss_enc *h)
 
 static moss_enc_status set_kernel_attrs(moss_enc *h)
 {
-    CUDA_TRY(h, cudaFuncSetAttribute(gemm_tc2_kernel<CONV_BN, EPI_GELU_BF16, A_CONV_S2>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Gemm2Cfg<CONV_BN>::SMEM));
+    CUDA_TRY(h, cudaFuncSetAttribute(gemm_tc2_kernel<CONV_BN, EPI_GELU_BF16, A_CONV_S2, 2>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Gemm2Cfg<CONV_BN, 2>::SMEM));
     CUDA_TRY(h, (gemm2_attr<256, EPI_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_RESID_F32>()));
@@ -1033,7 +1042,7 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
             double px = 0.0;
             for (int j = 0; j < gc; j++) px += 64.0 * sc[g0 + j].t1_lim;
             Launch L1(h, "conv1", 2.0 * 9 * CST * px, 2.0 * CST * px + 4.0 * 128 * 2 * px / 64.0);
-            CUDA_TRY(h, launch_k(h, conv1_kernel, dim3(400, gc), dim3(240), 0, (const float *)h->mel_raw, d_chunks + g0,
+            CUDA_TRY(h, launch_k(h, conv1_kernel, dim3(200, gc), dim3(240), 0, (const float *)h->mel_raw, d_chunks + g0,
                                  (const int *)h->gmax_ord, (const float *)h->conv1_w, (const float *)h->conv1_b, h->c1out));
         }
         TRY(gemm_conv(h, "gemm_conv2", h->c1out, gc, 400, 64, d_t2 + g_off2[gi], g_n2[gi], h->conv2_w, h->conv2_b,
@@ -1080,7 +1089,7 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.bo;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm2<320, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a)));
+        TRY((gemm2<320, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a, 0, 2)));
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln2_g, L.ln2_b,
