@@ -19,8 +19,13 @@ struct StemChunk {
 
 // conv1 over the normalised log-mel of a chunk.  Input plane (freq 128, time
 // 800), with frames >= nframes zero (the tail padding) and conv padding 1.
-// Output [chunk][400][64][480] bf16.  One CTA per (time step, chunk); thread
-// j owns channels 2j, 2j+1.
+// Output [chunk][400][64][480] bf16.  One CTA of 240 threads per (pair of
+// time steps, chunk): thread j takes time step 2 blockIdx.x + j / 120 and the
+// four channels 4 (j % 120) .. +3, two by two in the paired fp32
+// instructions.  The five input frames the pair reads sit in shared memory,
+// normalised on load, column 2 + f holding frequency f and column 1 the
+// conv's zero pad, so that each output frequency step reads its two new
+// input columns of a row as one 8-byte word.
 __global__ void __launch_bounds__(240) conv1_kernel(const float *__restrict__ mel_raw,
                                                     const StemChunk *__restrict__ chunks,
                                                     const int *__restrict__ gmax_ord,
@@ -28,43 +33,60 @@ __global__ void __launch_bounds__(240) conv1_kernel(const float *__restrict__ me
                                                     const float *__restrict__ b1,  // [480]
                                                     bf16 *__restrict__ out)
 {
-    __shared__ float in[3][130];  // 3 time rows x (128 freq + 2 zero pads)
+    __shared__ __align__(16) float in[5][132];  // row r = frame 2 t0 - 1 + r
     grid_dep_wait();
     grid_dep_launch();
-    const int t = blockIdx.x, ci = blockIdx.y;
+    const int t0 = 2 * blockIdx.x, ci = blockIdx.y;
     const StemChunk ch = chunks[ci];
-    if (t >= ch.t1_lim) return;  // outside the receptive field of the chunk's tokens
+    if (t0 >= ch.t1_lim) return;  // outside the receptive field of the chunk's tokens
     const float floor_v = ordered_to_float(gmax_ord[ch.clip]) - 8.0f;
-    for (int i = threadIdx.x; i < 3 * 130; i += blockDim.x) {
-        const int kt = i / 130, f = i % 130 - 1;
-        const int ti = 2 * t + kt - 1;
+    for (int i = threadIdx.x; i < 5 * 132; i += blockDim.x) {
+        const int r = i / 132, col = i - 132 * r, f = col - 2;
+        const int ti = 2 * t0 - 1 + r;
         float v = 0.0f;
         if (f >= 0 && f < 128 && ti >= 0 && ti < ch.nframes) {
             const float x = mel_raw[(size_t)(ch.mel_row + ti) * 128 + f];
             v = (fmaxf(x, floor_v) + 4.0f) * 0.25f;
         }
-        in[kt][i % 130] = v;
+        in[r][col] = v;
     }
     __syncthreads();
-    // channels c, c + 1 side by side in the paired fp32 instructions
-    const int c = 2 * threadIdx.x;
-    float2 w[9];
+    const int tl = threadIdx.x / 120, t = t0 + tl;
+    if (t >= ch.t1_lim) return;  // no barrier follows
+    const int c = 4 * (threadIdx.x - 120 * tl);
+    float2 wa[9], wb[9];  // channels (c, c+1) and (c+2, c+3)
 #pragma unroll
-    for (int k = 0; k < 9; k++) w[k] = make_float2(w1[c * 9 + k], w1[(c + 1) * 9 + k]);
-    const float2 b = make_float2(b1[c], b1[c + 1]);
+    for (int k = 0; k < 9; k++) {
+        wa[k] = make_float2(w1[c * 9 + k], w1[(c + 1) * 9 + k]);
+        wb[k] = make_float2(w1[(c + 2) * 9 + k], w1[(c + 3) * 9 + k]);
+    }
+    const float2 ba = make_float2(b1[c], b1[c + 1]), bb = make_float2(b1[c + 2], b1[c + 3]);
+    const float *row[3] = {in[2 * tl], in[2 * tl + 1], in[2 * tl + 2]};  // frames 2t - 1 + kt
     bf16 *dst = out + ((size_t)ci * 400 + t) * 64 * 480 + c;
-#pragma unroll 4
+    // window of output frequency f: columns 2f+1, 2f+2, 2f+3 (frequencies 2f-1 .. 2f+1)
+    float x0[3], x1[3], x2[3];
+#pragma unroll
+    for (int kt = 0; kt < 3; kt++) x2[kt] = row[kt][1];
+#pragma unroll 2
     for (int f = 0; f < 64; f++) {
-        float2 acc = b;
+#pragma unroll
+        for (int kt = 0; kt < 3; kt++) {
+            x0[kt] = x2[kt];
+            const float2 n = *reinterpret_cast<const float2 *>(row[kt] + 2 * f + 2);
+            x1[kt] = n.x;
+            x2[kt] = n.y;
+        }
+        float2 sa = ba, sb = bb;
 #pragma unroll
         for (int kf = 0; kf < 3; kf++)
 #pragma unroll
             for (int kt = 0; kt < 3; kt++) {
-                const float x = in[kt][2 * f + kf];  // freq index 2f + kf - 1, shifted by the pad
-                acc = __ffma2_rn(w[kf * 3 + kt], make_float2(x, x), acc);
+                const float x = kf == 0 ? x0[kt] : kf == 1 ? x1[kt] : x2[kt];
+                sa = __ffma2_rn(wa[kf * 3 + kt], make_float2(x, x), sa);
+                sb = __ffma2_rn(wb[kf * 3 + kt], make_float2(x, x), sb);
             }
-        const float2 g = gelu2(acc);
-        *reinterpret_cast<uint32_t *>(dst + (size_t)f * 480) = pack_bf16x2(g.x, g.y);
+        const float2 ga = gelu2(sa), gb = gelu2(sb);
+        *reinterpret_cast<uint2 *>(dst + (size_t)f * 480) = make_uint2(pack_bf16x2(ga.x, ga.y), pack_bf16x2(gb.x, gb.y));
     }
 }
 
