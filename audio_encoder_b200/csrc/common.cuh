@@ -291,26 +291,29 @@ __device__ __forceinline__ float gelu_fast(float x)
 }
 
 // The same GELU on two values at once with the paired fp32 instructions of
-// sm_100 (add/mul/fma on float2): the same formula and error bound, half the
-// instructions for the polynomial and the squarings.
+// sm_100 (add/mul/fma on float2), with the constants folded: the polynomial
+// is taken in |x| directly (a_k scaled by 2^(-k/2), which absorbs the 1/sqrt 2
+// of the argument) and every coefficient is scaled by 2^(1/16), so that
+// (1/p)^16 comes out as (1 - erf)/2 = Phi(-|x|) with no further multiply.
+// Then Phi(x) = 1 - that for x >= 0, and GELU = x Phi(x).  Same formula and
+// error class as gelu_fast (at most 5.5e-7 absolute per unit |x| in fp32),
+// four fewer fp32 operations.
 __device__ __forceinline__ float2 gelu2(float2 x)
 {
-    const float2 z = __fmul2_rn(x, make_float2(0.70710678118654752f, 0.70710678118654752f));
-    const float2 az = make_float2(fabsf(z.x), fabsf(z.y));
-    float2 p = __ffma2_rn(make_float2(4.30638e-5f, 4.30638e-5f), az, make_float2(2.765672e-4f, 2.765672e-4f));
-    p = __ffma2_rn(p, az, make_float2(1.520143e-4f, 1.520143e-4f));
-    p = __ffma2_rn(p, az, make_float2(9.2705272e-3f, 9.2705272e-3f));
-    p = __ffma2_rn(p, az, make_float2(4.22820123e-2f, 4.22820123e-2f));
-    p = __ffma2_rn(p, az, make_float2(7.05230784e-2f, 7.05230784e-2f));
-    p = __ffma2_rn(p, az, make_float2(1.0f, 1.0f));
+    const float2 ax = make_float2(fabsf(x.x), fabsf(x.y));
+    float2 p = __ffma2_rn(make_float2(5.62129981e-6f, 5.62129981e-6f), ax, make_float2(5.10552090e-5f, 5.10552090e-5f));
+    p = __ffma2_rn(p, ax, make_float2(3.96861360e-5f, 3.96861360e-5f));
+    p = __ffma2_rn(p, ax, make_float2(3.42273922e-3f, 3.42273922e-3f));
+    p = __ffma2_rn(p, ax, make_float2(2.20769979e-2f, 2.20769979e-2f));
+    p = __ffma2_rn(p, ax, make_float2(5.20751625e-2f, 5.20751625e-2f));
+    p = __ffma2_rn(p, ax, make_float2(1.04427373f, 1.04427373f));
     float2 r = make_float2(__fdividef(1.0f, p.x), __fdividef(1.0f, p.y));
     r = __fmul2_rn(r, r);
     r = __fmul2_rn(r, r);
     r = __fmul2_rn(r, r);
-    r = __fmul2_rn(r, r);
-    const float2 e = make_float2(copysignf(1.0f - r.x, z.x), copysignf(1.0f - r.y, z.y));
-    const float2 hx = __fmul2_rn(x, make_float2(0.5f, 0.5f));
-    return __ffma2_rn(hx, e, hx);  // 0.5 x (1 + erf)
+    r = __fmul2_rn(r, r);  // Phi(-|x|)
+    const float2 phi = make_float2(x.x >= 0.0f ? 1.0f - r.x : r.x, x.y >= 0.0f ? 1.0f - r.y : r.y);
+    return __fmul2_rn(x, phi);
 }
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
