@@ -1083,7 +1083,7 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         TRY((gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
         {
             Launch Lk(h, "attention", 4.0 * 64 * 20 * attn_pairs, 2.0 * T * (DQKV + D));
-            CUDA_TRY(h, launch_k(h, window_attn_tc_kernel, dim3((unsigned)n_chunks, 20), dim3(ATTN_THREADS), ATTN_TC_SMEM, tm_qkv,
+            CUDA_TRY(h, launch_k(h, window_attn_tc_kernel, dim3((unsigned)n_chunks, 20), dim3(128), ATTN_TC_SMEM, tm_qkv,
                                  d_ct, h->attn, h->err));
         }
         a.bias = L.bo;
