@@ -53,9 +53,16 @@ __device__ __forceinline__ float2 cmul(float2 a, float2 b)
 
 // 20-point DFT in registers: X[k] = sum_n x[n] exp(-2 pi i n k / 20).
 // n = nb + 5 na, k = 4 kb + ka:  4-point DFTs over na, twiddle
-// exp(-2 pi i nb ka / 20), then 5-point DFTs over nb.
-__device__ __forceinline__ void dft20(float2 (&x)[20], const float2 *tw400)
+// exp(-2 pi i nb ka / 20) (compile-time constants), then 5-point DFTs over nb.
+__device__ __forceinline__ void dft20(float2 (&x)[20])
 {
+    // cos and sin of 2 pi m / 20, m = 0..12
+    constexpr float C20[13] = {1.0f, 9.510565163e-01f, 8.090169944e-01f, 5.877852523e-01f, 3.090169944e-01f, 0.0f,
+                               -3.090169944e-01f, -5.877852523e-01f, -8.090169944e-01f, -9.510565163e-01f, -1.0f,
+                               -9.510565163e-01f, -8.090169944e-01f};
+    constexpr float S20[13] = {0.0f, 3.090169944e-01f, 5.877852523e-01f, 8.090169944e-01f, 9.510565163e-01f, 1.0f,
+                               9.510565163e-01f, 8.090169944e-01f, 5.877852523e-01f, 3.090169944e-01f, 0.0f,
+                               -3.090169944e-01f, -5.877852523e-01f};
     float2 A[5][4];
 #pragma unroll
     for (int nb = 0; nb < 5; nb++) {
@@ -71,7 +78,7 @@ __device__ __forceinline__ void dft20(float2 (&x)[20], const float2 *tw400)
 #pragma unroll
     for (int nb = 1; nb < 5; nb++)
 #pragma unroll
-        for (int ka = 1; ka < 4; ka++) A[nb][ka] = cmul(A[nb][ka], tw400[20 * nb * ka]);
+        for (int ka = 1; ka < 4; ka++) A[nb][ka] = cmul(A[nb][ka], make_float2(C20[nb * ka], -S20[nb * ka]));
     // 5-point DFT with c1 = cos(2pi/5), c2 = cos(4pi/5), s1 = sin(2pi/5), s2 = sin(4pi/5)
     const float c1 = 0.30901699437494742f, c2 = -0.80901699437494742f;
     const float s1 = 0.95105651629515357f, s2 = 0.58778525229247313f;
@@ -176,7 +183,7 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip 
             const float w = S.hann[n];
             v[n2] = make_float2(w * xa[n], has_b ? w * xb[n] : 0.0f);
         }
-        dft20(v, S.tw);
+        dft20(v);
         float2 *yr = S.y[p] + n1 * 21;
 #pragma unroll
         for (int k2 = 0; k2 < 20; k2++) yr[k2] = (k2 == 0 || n1 == 0) ? v[k2] : cmul(v[k2], S.tw[n1 * k2]);
@@ -188,7 +195,7 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip 
         float2 v[20];
 #pragma unroll
         for (int n1 = 0; n1 < 20; n1++) v[n1] = S.y[p][n1 * 21 + k2];
-        dft20(v, S.tw);
+        dft20(v);
 #pragma unroll
         for (int k1 = 0; k1 < 20; k1++) S.y[p][k1 * 21 + k2] = v[k1];
     }
@@ -328,6 +335,13 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
     };
 
     const float log10_2 = 0.30102999566398120f;
+    // Every DFT task of this thread has the same pair and row: pass 1 takes
+    // (pair tp, n1 = tj), pass 2 (tp, k2 = tj), and the power step the bins
+    // k = tj + 20 i of pair tp; the window values it multiplies stay in registers.
+    const int tp = tid / 20, tj = tid - 20 * tp;
+    float hw[20];
+#pragma unroll
+    for (int n2 = 0; n2 < 20; n2++) hw[n2] = S.hann[tj + 20 * n2];
     int it = 0;
     bool ready = prefetch(blockIdx.x, 0);
     cp_async_commit();
@@ -348,60 +362,56 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
 
         const float *xsb = S.xs[cur];
         const int npairs = (nf + 1) / 2;
-        for (int task = tid; task < npairs * 20; task += MEL2_THREADS) {
-            const int p = task / 20, n1 = task - 20 * p;
-            const int fa = 2 * p, fb = 2 * p + 1;
-            const bool has_b = fb < nf;
-            const float *xa = xsb + 160 * fa, *xb = xsb + 160 * (has_b ? fb : fa);
+        if (tp < npairs) {
+            // pass 1: 20-point DFT over n2 of the windowed samples n = tj + 20 n2
+            // of frame 2 tp (real part) and frame 2 tp + 1 (imaginary part)
+            const bool has_b = 2 * tp + 1 < nf;
+            const float *xa = xsb + 320 * tp + tj, *xb = has_b ? xa + 160 : xa;
             float2 v[20];
 #pragma unroll
-            for (int n2 = 0; n2 < 20; n2++) {
-                const int n = n1 + 20 * n2;
-                const float w = S.hann[n];
-                v[n2] = make_float2(w * xa[n], has_b ? w * xb[n] : 0.0f);
-            }
-            dft20(v, S.tw);
-            float2 *yr = S.y[p] + n1 * 21;
+            for (int n2 = 0; n2 < 20; n2++) v[n2] = make_float2(hw[n2] * xa[20 * n2], has_b ? hw[n2] * xb[20 * n2] : 0.0f);
+            dft20(v);
+            float2 *yr = S.y[tp] + tj * 21;
 #pragma unroll
-            for (int k2 = 0; k2 < 20; k2++) yr[k2] = (k2 == 0 || n1 == 0) ? v[k2] : cmul(v[k2], S.tw[n1 * k2]);
+            for (int k2 = 0; k2 < 20; k2++) yr[k2] = (k2 == 0 || tj == 0) ? v[k2] : cmul(v[k2], S.tw[tj * k2]);
         }
         __syncthreads();
-        for (int task = tid; task < npairs * 20; task += MEL2_THREADS) {
-            const int p = task / 20, k2 = task - 20 * p;
+        if (tp < npairs) {
+            // pass 2: 20-point DFT over n1 -> Z[20 k1 + tj], in place
             float2 v[20];
 #pragma unroll
-            for (int n1 = 0; n1 < 20; n1++) v[n1] = S.y[p][n1 * 21 + k2];
-            dft20(v, S.tw);
+            for (int n1 = 0; n1 < 20; n1++) v[n1] = S.y[tp][n1 * 21 + tj];
+            dft20(v);
 #pragma unroll
-            for (int k1 = 0; k1 < 20; k1++) S.y[p][k1 * 21 + k2] = v[k1];
+            for (int k1 = 0; k1 < 20; k1++) S.y[tp][k1 * 21 + tj] = v[k1];
         }
         __syncthreads();
-        // power of both frames: read all of this thread's bins, then write them in place
-        constexpr int PT = (MEL2_FRAMES / 2 * 201 + MEL2_THREADS - 1) / MEL2_THREADS;  // 11
-        float pa[PT], pb[PT];
+        // power of both frames at bins k = tj + 20 i: X_a[k] = (Z[k] + conj Z[400-k]) / 2,
+        // X_b[k] = (Z[k] - conj Z[400-k]) / 2i, with Z[20 k1 + k2] at y[k1 * 21 + k2];
+        // read all of this thread's bins, then write them in place
+        float pa[11], pb[11];
+        if (tp < npairs) {
 #pragma unroll
-        for (int i = 0; i < PT; i++) {
-            const int task = tid + i * MEL2_THREADS;
-            pa[i] = pb[i] = 0.0f;
-            if (task < npairs * 201) {
-                const int p = task / 201, k = task - 201 * p;
-                const int kn = (400 - k) % 400;
-                const float2 zk = S.y[p][(k / 20) * 21 + (k % 20)], zn = S.y[p][(kn / 20) * 21 + (kn % 20)];
-                const float ar = 0.5f * (zk.x + zn.x), ai = 0.5f * (zk.y - zn.y);
-                const float br = 0.5f * (zk.y + zn.y), bi = -0.5f * (zk.x - zn.x);
-                pa[i] = ar * ar + ai * ai;
-                pb[i] = br * br + bi * bi;
+            for (int i = 0; i < 11; i++) {
+                if (i < 10 || tj == 0) {
+                    const float2 zk = S.y[tp][i * 21 + tj];
+                    const float2 zn = tj == 0 ? S.y[tp][(i == 0 ? 0 : 20 - i) * 21] : S.y[tp][(19 - i) * 21 + 20 - tj];
+                    const float ar = 0.5f * (zk.x + zn.x), ai = 0.5f * (zk.y - zn.y);
+                    const float br = 0.5f * (zk.y + zn.y), bi = -0.5f * (zk.x - zn.x);
+                    pa[i] = ar * ar + ai * ai;
+                    pb[i] = br * br + bi * bi;
+                }
             }
         }
         __syncthreads();
+        if (tp < npairs) {
+            float *pw = reinterpret_cast<float *>(S.y[tp]);
 #pragma unroll
-        for (int i = 0; i < PT; i++) {
-            const int task = tid + i * MEL2_THREADS;
-            if (task < npairs * 201) {
-                const int p = task / 201, k = task - 201 * p;
-                float *pw = reinterpret_cast<float *>(S.y[p]);
-                pw[k] = pa[i];
-                pw[420 + k] = pb[i];
+            for (int i = 0; i < 11; i++) {
+                if (i < 10 || tj == 0) {
+                    pw[tj + 20 * i] = pa[i];
+                    pw[420 + tj + 20 * i] = pb[i];
+                }
             }
         }
         __syncthreads();
