@@ -251,15 +251,26 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip 
 // into the exchange buffer, and log10 uses the hardware log2.
 static constexpr int MEL3_MAX_CLIPS = 128;  // clips per launch (the host splits larger batches)
 
+// A block's PCM span sits in shared memory with 20 unused words after every
+// 320 samples (one frame pair): sample s of the span is word mel3_pad(s).
+// Pass-1 task t reads sample 20 n2 + (t mod 20) of pair t / 20, i.e. word
+// 340 (t / 20) + (t mod 20) + 20 n2 + (0 or 20), whose bank is
+// t + 20 n2 (mod 32): distinct across a warp, so the loads are conflict-free.
+__host__ __device__ constexpr int mel3_pad(int s) { return s + 20 * (s / 320); }
+static constexpr int MEL3_SPAN = mel3_pad(MEL2_SPAN - 1) + 1;  // 5680 words
+static constexpr int MEL3_OUT_LD = 132;  // row pitch of the staged log-mel rows (float4-aligned)
+
 struct Mel3Smem {
     float2 tw[400];
     float hann[400];
     int band_lo[128];
     int band_n[128];
     float band_wt[MEL_BAND][128];
-    float2 y[MEL2_FRAMES / 2][20 * 21];  // pass outputs; then power: pair p holds frame 2p at [0..200], 2p+1 at [420..620]
-    float xs[2][MEL2_SPAN];              // PCM spans of the current and the next block
+    float2 y[MEL2_FRAMES / 2][20 * 21];  // pass outputs; then the power spectra, frame f at floats [201 f, 201 f + 201)
+    float xs[2][MEL3_SPAN];              // PCM spans of the current and the next block (padded, see mel3_pad);
+                                         // the current one then stages the block's log-mel rows
     int first_block[MEL3_MAX_CLIPS + 1];  // prefix of blocks per clip
+    int mpart[MEL2_THREADS / 32 + 1];     // filters of warp w: [mpart[w], mpart[w+1])
     float wmax[MEL2_THREADS / 32];
 };
 
@@ -310,6 +321,7 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
     for (int i = tid; i < 128 * MEL_BAND; i += MEL2_THREADS) S.band_wt[i / 128][i % 128] = tabt->w[i / 128][i % 128];
     grid_dep_wait();
     grid_dep_launch();
+    __syncthreads();  // the filter table is in place before thread 0 reads it
     if (tid == 0) {
         int acc = 0;
         for (int c = 0; c < n_clips; c++) {
@@ -318,6 +330,16 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
             acc += f > 0 ? (f + MEL2_FRAMES - 1) / MEL2_FRAMES : 0;
         }
         S.first_block[n_clips] = acc;
+        // filters per warp for the filterbank stage, balanced by their bins
+        int total = 0;
+        for (int m = 0; m < 128; m++) total += S.band_n[m];
+        int w = 0, run = 0;
+        S.mpart[0] = 0;
+        for (int m = 0; m < 128; m++) {
+            run += S.band_n[m];
+            while (w + 1 < MEL2_THREADS / 32 && run * (MEL2_THREADS / 32) >= total * (w + 1)) S.mpart[++w] = m + 1;
+        }
+        while (w + 1 <= MEL2_THREADS / 32) S.mpart[++w] = 128;
     }
     __syncthreads();
 
@@ -330,18 +352,17 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
         if (!mel3_interior(cl, frame0, nf)) return false;
         const float4 *src = reinterpret_cast<const float4 *>(cl.pcm + (160LL * frame0 - 200));
         const int n4 = (160 * (nf - 1) + 400) / 4;
-        for (int i = tid; i < n4; i += MEL2_THREADS) cp_async16(reinterpret_cast<float4 *>(S.xs[buf]) + i, src + i);
+        for (int i = tid; i < n4; i += MEL2_THREADS)
+            cp_async16(reinterpret_cast<float4 *>(S.xs[buf]) + i + 5 * (i / 80), src + i);
         return true;
     };
 
     const float log10_2 = 0.30102999566398120f;
     // Every DFT task of this thread has the same pair and row: pass 1 takes
     // (pair tp, n1 = tj), pass 2 (tp, k2 = tj), and the power step the bins
-    // k = tj + 20 i of pair tp; the window values it multiplies stay in registers.
+    // k = tj + 20 i of pair tp.
     const int tp = tid / 20, tj = tid - 20 * tp;
-    float hw[20];
-#pragma unroll
-    for (int n2 = 0; n2 < 20; n2++) hw[n2] = S.hann[tj + 20 * n2];
+    const float *hw = S.hann + tj;  // window value of sample tj + 20 n2: hw[20 n2]
     int it = 0;
     bool ready = prefetch(blockIdx.x, 0);
     cp_async_commit();
@@ -353,7 +374,7 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
         if (!ready) {  // edge block: reflect-padded load now
             const long long s0 = 160LL * frame0 - 200;
             const int span = 160 * (nf - 1) + 400;
-            for (int i = tid; i < span; i += MEL2_THREADS) S.xs[cur][i] = __ldg(cl.pcm + reflect_index(s0 + i, cl.n));
+            for (int i = tid; i < span; i += MEL2_THREADS) S.xs[cur][mel3_pad(i)] = __ldg(cl.pcm + reflect_index(s0 + i, cl.n));
         }
         ready = prefetch(item + gridDim.x, cur ^ 1);
         cp_async_commit();
@@ -366,10 +387,15 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
             // pass 1: 20-point DFT over n2 of the windowed samples n = tj + 20 n2
             // of frame 2 tp (real part) and frame 2 tp + 1 (imaginary part)
             const bool has_b = 2 * tp + 1 < nf;
-            const float *xa = xsb + 320 * tp + tj, *xb = has_b ? xa + 160 : xa;
+            // frame 2 tp starts at span sample 320 tp, frame 2 tp + 1 at 320 tp + 160
+            const float *xa = xsb + 340 * tp + tj, *xb = has_b ? xa + 160 : xa;
             float2 v[20];
 #pragma unroll
-            for (int n2 = 0; n2 < 20; n2++) v[n2] = make_float2(hw[n2] * xa[20 * n2], has_b ? hw[n2] * xb[20 * n2] : 0.0f);
+            for (int n2 = 0; n2 < 20; n2++) {
+                const float a = xa[20 * n2 + (n2 >= 16 ? 20 : 0)];
+                const float b = has_b ? xb[20 * n2 + (n2 >= 8 ? 20 : 0)] : 0.0f;
+                v[n2] = make_float2(hw[20 * n2] * a, hw[20 * n2] * b);
+            }
             dft20(v);
             float2 *yr = S.y[tp] + tj * 21;
 #pragma unroll
@@ -405,33 +431,61 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
         }
         __syncthreads();
         if (tp < npairs) {
-            float *pw = reinterpret_cast<float *>(S.y[tp]);
+            float *pw = reinterpret_cast<float *>(S.y) + 402 * tp;  // frames 2 tp, 2 tp + 1: rows of 201
 #pragma unroll
             for (int i = 0; i < 11; i++) {
                 if (i < 10 || tj == 0) {
                     pw[tj + 20 * i] = pa[i];
-                    pw[420 + tj + 20 * i] = pb[i];
+                    pw[201 + tj + 20 * i] = pb[i];
                 }
             }
         }
         __syncthreads();
+        // banded filterbank: warp w takes filters mpart[w] .. mpart[w+1] - 1 for
+        // all frames, lane = frame; the filter's bins and weights are the same
+        // across the warp, and the power rows' odd pitch (201) puts the lanes'
+        // reads in distinct banks.  The block's log-mel rows are staged in the
+        // (now unused) span buffer and then stored whole.
         float lmax = -INFINITY;
-        const long long out_row = cl.out_row0 + (frame0 - cl.f_begin);
-        // lane q of a frame's 32 lanes takes filters q, q+32, q+64, q+96, so that
-        // the lanes read consecutive words of the transposed filterbank
-        for (int task = tid; task < nf * 32; task += MEL2_THREADS) {
-            const int f = task >> 5, q = task & 31;
-            const float *P = reinterpret_cast<const float *>(S.y[f >> 1]) + (f & 1) * 420;
-            float *orow = out + (size_t)(out_row + f) * 128;
+        {
+            const int f = tid & 31, w = tid >> 5;
+            const float *P = reinterpret_cast<const float *>(S.y) + 201 * f;
+            float *ost = S.xs[cur] + MEL3_OUT_LD * f;
+            const int m1 = S.mpart[w + 1];
+            // four filters at a time (four independent sums); neighbouring
+            // filters have nearly equal widths, so little of the padding runs
+            for (int m0 = S.mpart[w]; m0 < m1; m0 += 4) {
+                int lo[4], cnt[4], cmax = 0;
 #pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int m = q + 32 * j;
-                const int lo = S.band_lo[m], cnt = S.band_n[m];
-                float acc = 0.0f;
-                for (int b = 0; b < cnt; b++) acc = fmaf(S.band_wt[b][m], P[lo + b], acc);
-                const float r = __log2f(fmaxf(acc, 1e-10f)) * log10_2;
-                lmax = fmaxf(lmax, r);
-                if (write_out) orow[m] = r;
+                for (int j = 0; j < 4; j++) {
+                    const bool in = m0 + j < m1;
+                    lo[j] = in ? S.band_lo[m0 + j] : 0;
+                    cnt[j] = in ? S.band_n[m0 + j] : 0;
+                    cmax = max(cmax, cnt[j]);
+                }
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                for (int b = 0; b < cmax; b++) {
+#pragma unroll
+                    for (int j = 0; j < 4; j++)
+                        if (b < cnt[j]) acc[j] = fmaf(S.band_wt[b][m0 + j], P[lo[j] + b], acc[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    if (m0 + j < m1) {
+                        const float r = __log2f(fmaxf(acc[j], 1e-10f)) * log10_2;
+                        if (f < nf) lmax = fmaxf(lmax, r);
+                        ost[m0 + j] = r;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (write_out) {
+            const long long out_row = cl.out_row0 + (frame0 - cl.f_begin);
+            for (int i = tid; i < nf * 32; i += MEL2_THREADS) {
+                const int f = i >> 5, q = i & 31;
+                const float4 v = *reinterpret_cast<const float4 *>(S.xs[cur] + MEL3_OUT_LD * f + 4 * q);
+                reinterpret_cast<float4 *>(out + (size_t)(out_row + f) * 128)[q] = v;
             }
         }
         if (cl.gslot >= 0) {
