@@ -25,6 +25,7 @@ EXPORTED = [
     "moss_enc_weight_count", "moss_enc_num_frames", "moss_enc_num_tokens", "moss_enc_range_tokens",
     "moss_enc_create", "moss_enc_set_stream", "moss_enc_synchronize", "moss_enc_destroy",
     "moss_enc_status_string", "moss_enc_last_error", "moss_enc_logmel", "moss_enc_log_max",
+    "moss_enc_range_log_max",
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
     "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_selftest_gelu", "moss_enc_selftest_timeout",
@@ -88,6 +89,8 @@ def lib():
         L.moss_enc_logmel.argtypes = [vp, ctypes.POINTER(Clip), vp, ctypes.POINTER(i64), vp]
         L.moss_enc_log_max.restype = i32
         L.moss_enc_log_max.argtypes = [vp, vp, i64, vp]
+        L.moss_enc_range_log_max.restype = i32
+        L.moss_enc_range_log_max.argtypes = [vp, vp, i64, i64, i64, vp]
         L.moss_enc_forward.restype = i32
         L.moss_enc_forward.argtypes = [vp, ctypes.POINTER(Clip), i32, vp, ctypes.POINTER(i64)]
         L.moss_enc_forward_stage.restype = i32
@@ -226,6 +229,14 @@ class Encoder:
     def log_max(self, pcm):
         out = self.torch.empty(1, dtype=self.torch.float32, device=pcm.device)
         self._check(lib().moss_enc_log_max(self.h, _ptr(pcm), pcm.numel(), _ptr(out)))
+        return out
+
+    def range_log_max(self, pcm, begin=0, end=None):
+        """Log-mel maximum over the frames of samples [begin, end) (device [1])."""
+        n = pcm.numel()
+        out = self.torch.empty(1, dtype=self.torch.float32, device=pcm.device)
+        self._check(lib().moss_enc_range_log_max(self.h, _ptr(pcm), n, int(begin), int(n if end is None else end),
+                                                 _ptr(out)))
         return out
 
     def logmel(self, pcm, begin=0, end=None, log_max=None):

@@ -936,6 +936,37 @@ extern "C" moss_enc_status moss_enc_log_max(moss_enc *h, const float *pcm, int64
     return MOSS_ENC_OK;
 }
 
+extern "C" moss_enc_status moss_enc_range_log_max(moss_enc *h, const float *pcm, int64_t n_samples, int64_t begin,
+                                                  int64_t end, float *out)
+{
+    if (!h || !pcm || !out || n_samples < 0) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad argument");
+    if (begin < 0 || end < begin || end > n_samples || begin % HOP != 0 || (end != n_samples && end % HOP != 0))
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad range");
+    if (n_samples / HOP > INT32_MAX) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "clip too long");
+    const int64_t f_begin = begin / HOP, f_end = end == n_samples ? n_samples / HOP : end / HOP;
+    TRY(tab_begin(h));
+    const TabLayout tl = tab_layout(h->cfg.max_clips, h->max_chunks);
+    uint8_t *H = static_cast<uint8_t *>(h->h_tab);
+    reinterpret_cast<const float **>(H + tl.logmax_src)[0] = nullptr;
+    MelClip *mc = reinterpret_cast<MelClip *>(H + tl.clips_max);
+    mc[0] = MelClip{pcm, (long long)n_samples, 0, (int)f_begin, (int)f_end, 0, 0};
+    TRY(tab_upload(h));
+    uint8_t *Dt = static_cast<uint8_t *>(h->d_tab);
+    {
+        Launch Lk(h, "gmax", 0.0, 0.0);
+        gmax_init_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, reinterpret_cast<const float *const *>(Dt + tl.logmax_src), 1);
+    }
+    CUDA_TRY(h, cudaGetLastError());
+    TRY(launch_logmel(h, reinterpret_cast<const MelClip *>(Dt + tl.clips_max), 1, f_end - f_begin, nullptr, 0,
+                      f_end - f_begin));
+    {
+        Launch Lk(h, "gmax", 0.0, 0.0);
+        gmax_export_kernel<<<1, 32, 0, h->stream>>>(h->gmax_ord, out);
+    }
+    CUDA_TRY(h, cudaGetLastError());
+    return MOSS_ENC_OK;
+}
+
 extern "C" moss_enc_status moss_enc_logmel(moss_enc *h, const moss_enc_clip *clip, float *mel_out,
                                            int64_t *n_frames, float *log_max_out)
 {

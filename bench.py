@@ -394,6 +394,85 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_sharded(args):
+    """One long clip split over the ranks by whole 800-frame chunks
+    (audio_encoder_b200.shard): a step is each rank's log-mel maximum over its
+    range, one all-reduce(max) of that float over NCCL (the path's only
+    exchange), and the rank's range encoded against the common maximum.
+    Strong scaling: the same clip at every N; value = clip audio-seconds per
+    step time (max over ranks)."""
+    import torch
+
+    from audio_encoder_b200 import binding, shard
+
+    rank, world, dist = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    name = args.workload if args.workload in ("clip_10min", "clip_60min_streamed") else "clip_10min"
+    desc, clips, n_layers = workload_clips(name)
+    pcm = clips[0]
+    n = pcm.size
+    b, e = shard.chunk_ranges(n, world)[rank]
+    stream = torch.cuda.Stream()
+    enc = binding.Encoder(synth.make_weights(n_layers), n_layers, max_samples=max(e - b, 1), max_clips=1,
+                          out_dtype=binding.OUT_BF16, stream=stream)
+    with torch.cuda.stream(stream):
+        x = torch.from_numpy(pcm).to(dev)
+        rows_n = binding.range_tokens(n, b, e) if e > b else 0
+        out = torch.empty((max(rows_n, 1), 2048), dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    def max_reduce(t):
+        if dist:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+
+    def step():
+        with torch.cuda.stream(stream):
+            shard.encode_range(enc, x, rank, world, max_reduce, out=out[:rows_n] if rows_n else None)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(dev.index) as clk:
+        for i in range(args.steps):
+            with torch.cuda.stream(stream):
+                flush.fill_(float(i))
+                ev[i][0].record(stream)
+            step()
+            with torch.cuda.stream(stream):
+                ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    total_ms = reduce_max(float(sum(a.elapsed_time(c) for a, c in ev)), dist, dev)
+    ms = total_ms / args.steps
+    audio_s = n / 16000.0
+    tokens = binding.num_tokens(n)
+    if rank == 0:
+        line = {
+            "metric": "audio-sec encoded/sec", "value": audio_s / (ms / 1e3), "unit": "audio-s/s",
+            "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded PCM, random-init bf16 weights)",
+            "tokens_per_s": tokens / (ms / 1e3),
+            "model_tflops": model_flops(tokens, n_layers) / (ms / 1e3) / 1e12,
+            "config": {"workload": name + "_sharded", "description": desc + ", chunk ranges split over ranks",
+                       "audio_s": audio_s, "tokens": tokens, "layers": n_layers,
+                       "l2": "512 MB buffer written between timed steps (outside the events)",
+                       "parallelism": f"windows{world}" if world > 1 else "single"},
+            "e2e": None,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    enc.close()
+    if dist:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -403,11 +482,15 @@ def main():
     ap.add_argument("--workload", default="batch16_10to30s", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cpu-windows", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard-clip", action="store_true",
+                    help="one long clip (10 or 60 min) split over the ranks by chunk ranges (strong scaling)")
     ap.add_argument("--ncu", action="store_true",
                     help="capture run for ncu: warm-up as given (may be 0), the timed steps only, no report")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard_clip:
+        run_sharded(args)
     else:
         run_ours(args)
 

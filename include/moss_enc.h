@@ -157,6 +157,19 @@ moss_enc_status moss_enc_logmel(moss_enc *h, const moss_enc_clip *clip, float *m
  *  pcm device [n_samples]; out device float.  Any length is accepted. */
 moss_enc_status moss_enc_log_max(moss_enc *h, const float *pcm, int64_t n_samples, float *out);
 
+/* Log-mel maximum over the frames of the sample range [begin, end) of a clip
+ * (frames t with 160 t in [begin, end); end == n_samples: t < n_samples/160),
+ * each frame computed as in the whole clip (reflect padding only at its true
+ * ends).  The maximum of the values for ranges that cover a clip is the
+ * clip's log_max, so ranks that each encode one range of a long clip agree on
+ * the Whisper floor with one max-reduction of a float (page "Ossicle-4B",
+ * "Long Audio": pieces use the whole clip's log-mel).
+ *  pcm  device [n_samples]; out device float (-inf for an empty range).
+ *  begin and end are multiples of 160 (end may also equal n_samples).
+ * Nothing else is written. */
+moss_enc_status moss_enc_range_log_max(moss_enc *h, const float *pcm, int64_t n_samples, int64_t begin,
+                                       int64_t end, float *out);
+
 /* Encode n_clips clips (or pieces) into embedding rows.
  *  clips        host array [n_clips].
  *  rows_out     device [sum of tokens][2048] of cfg.out_dtype; the rows of

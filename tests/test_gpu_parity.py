@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import oracle
-from audio_encoder_b200 import binding, synth
+from audio_encoder_b200 import binding, shard, synth
 from conftest import oracle_model, weights
 from metrics import MEL_ATOL, assert_rows_close
 
@@ -214,6 +214,29 @@ def test_60min_streamed_equals_whole_clip_and_oracle():
 
 
 # ---------------------------------------------------------------- edge cases
+
+def test_long_clip_split_over_ranks_equals_whole_clip():
+    # three ranks simulated on one GPU: each takes its range's log-mel maximum,
+    # the maxima are max-reduced (here on the host, over NCCL/gloo across
+    # processes), each range is encoded against the common maximum, and the
+    # ranks' rows, in rank order, are the whole clip's rows bit for bit
+    n = 5 * 128000 + 37000
+    pcm = synth.pcm_long(3, n)
+    enc = encoder(4, 1_024_000)
+    x = dev(pcm)
+    whole, _ = enc.forward([x])
+    whole = whole.cpu().numpy()
+    world = 3
+    maxima = [float(enc.range_log_max(x, b, e).item()) for b, e in shard.chunk_ranges(n, world)]
+    gmax = max(maxima)
+    assert gmax == float(enc.log_max(x).item())
+    parts = []
+    for r in range(world):
+        rows, first = shard.encode_range(enc, x, r, world, lambda t: t.fill_(gmax))
+        assert first == sum(p.shape[0] for p in parts)
+        parts.append(rows.cpu().numpy())
+    np.testing.assert_array_equal(np.concatenate(parts), whole)
+
 
 def test_ragged_batch_with_empty_and_tiny_clips():
     enc = encoder(4, 600_000, 8)
