@@ -89,13 +89,13 @@ __device__ __forceinline__ float4 ld_f4(const float *p) { return *reinterpret_ca
 // 32 rows of this warp's TMEM lane quarter.  my_row / my_ok / my_aux describe
 // the output row of this lane's tile row (aux: position index for conv_out);
 // col0 is the tile's first output column in the interleaved/GEMM space.
-template <int BN, int EPI>
+template <int BN, int EPI, int NHALF = 2>
 __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, int half, int lane, uint8_t *stage,
                                            int my_row, bool my_ok, int my_aux, int col0)
 {
     constexpr int NG = (BN + 63) / 64;
 #pragma unroll 1
-    for (int g = half; g < NG; g += 2) {
+    for (int g = half; g < NG; g += NHALF) {
         const int c0 = g * 64;
         // 64 columns, or the last group's rest: 32 (BN = 160) or 48 (BN = 240)
         constexpr int REST = BN % 64;
@@ -249,7 +249,7 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
 // Boxes are staged in `nbuf` 4 KB buffers used in turn (1024-byte aligned,
 // EPI_STAGE_BYTES apart); a buffer is rewritten only after the boxes in
 // flight have been read out of shared memory.
-template <int BN, int EPI>
+template <int BN, int EPI, int NHALF = 2>
 __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensorMap *tmC, uint32_t tbase, int half,
                                                int lane, uint8_t *stage_base, int nbuf, int row0, int col0)
 {
@@ -270,7 +270,7 @@ __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensor
         return stage_base + (bi++) * EPI_STAGE_BYTES;
     };
 #pragma unroll 1
-    for (int g = half; g < NG; g += 2) {
+    for (int g = half; g < NG; g += NHALF) {
         const int c0 = g * 64;
         uint32_t r[64];
         tmem_ld32(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
@@ -524,6 +524,8 @@ struct Gemm2Cfg {
     // larger stages halve the stage hand-offs between the producer, the MMA
     // lane and the barriers, which measurably idle the tensor pipe.
     static constexpr int BM = 128, BK = 64 * KSUB;  // rows per CTA; the pair covers 256
+    // a multiple of 4 (the TMEM lane quarters); 8 measured faster than 4 on
+    // the layer GEMMs (FC1 45 vs 48-50 us, out-proj 21.5 vs 24.5-25 us)
     static constexpr int EPI_WARPS = 8;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     // Tiles wider than one MMA (BN = 320) are two MMAs of BN/2 per k-step.
@@ -705,7 +707,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
         }
     } else {
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;
+        const int half = (warp - 2) >> 2;  // which of the warps on this lane quarter
         uint8_t *stage = smem + C::STAGES * C::STAGE_BYTES + (warp - 2) * EPI_STAGE_BYTES;
         grid_dep_wait();
         int it = 0;
@@ -741,10 +743,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
                 constexpr int RING_BUFS = (int)(C::STAGES * C::STAGE_BYTES / C::EPI_WARPS / EPI_STAGE_BYTES);
                 const bool last = tile + npairs >= num_tiles;
                 uint8_t *stg = last ? smem + (warp - 2) * RING_BUFS * EPI_STAGE_BYTES : stage;
-                drain_tile_tma<BN, EPI>(args, &tmC, tbase, half, lane, stg, last ? RING_BUFS : 1,
+                drain_tile_tma<BN, EPI, C::EPI_WARPS / 4>(args, &tmC, tbase, half, lane, stg, last ? RING_BUFS : 1,
                                         mt * 256 + (int)rank * 128 + q * 32, nt * BN);
             } else
-                drain_tile<BN, EPI>(args, tbase, half, lane, stage, grow, ok, aux, nt * BN);
+                drain_tile<BN, EPI, C::EPI_WARPS / 4>(args, tbase, half, lane, stage, grow, ok, aux, nt * BN);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&tempty[acc]), 0));

@@ -1473,6 +1473,7 @@ extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void 
     if (!attrs_done) {
         CUDA_TRY(h, gemm_api_attrs<128>());
         CUDA_TRY(h, gemm_api_attrs<160>());
+        CUDA_TRY(h, gemm_api_attrs<192>());
         CUDA_TRY(h, gemm_api_attrs<256>());
         CUDA_TRY(h, (gemm2_attr<320, EPI_BF16>()));
         CUDA_TRY(h, (gemm2_attr<320, EPI_GELU_BF16>()));
@@ -1485,6 +1486,7 @@ extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void 
     switch (block_n) {
     case 128: return gemm_one<128>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
     case 160: return gemm_one<160>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
+    case 192: return gemm_one<192>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
     case 256: return gemm_one<256>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
     case 320:
         if (!cta_pair) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n 320 needs cta_pair");
@@ -1495,7 +1497,7 @@ extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void 
         case EPI_F32: return gemm2<320, EPI_F32>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
         default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "unsupported epilogue");
         }
-    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160, 256 or 320");
+    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160, 192, 256 or 320");
     }
 }
 

@@ -207,7 +207,7 @@ moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host,
  *  out        device; bf16 [M][N] for epilogue 0 (identity) and 1 (exact
  *             GELU), fp32 [M][N] for 2 (out += result: residual add) and
  *             5 (fp32 store).
- *  block_n    output tile width: 128, 160, 256, or 320 (CTA pairs only);
+ *  block_n    output tile width: 128, 160, 192, 256, or 320 (CTA pairs only);
  *             N % block_n == 0.
  *  cta_pair   0: one CTA per 128 x block_n tile; 1: CTA pairs (cluster of
  *             2) on 256 x block_n tiles, as the forward uses.
