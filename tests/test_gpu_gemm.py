@@ -17,12 +17,12 @@ def enc():
     e.close()
 
 
-@pytest.mark.parametrize("pair,block_n", [(False, 128), (False, 160), (False, 256), (True, 128), (True, 160),
-                                          (True, 256), (True, 320)])
+@pytest.mark.parametrize("pair,block_n", [(False, 128), (False, 160), (False, 192), (False, 256), (True, 128),
+                                          (True, 160), (True, 192), (True, 256), (True, 320)])
 @pytest.mark.parametrize("epi", [0, 1, 2, 5])
 @pytest.mark.parametrize("M,K", [(1, 64), (300, 1280), (1000, 4608), (4608, 1280)])
 def test_gemm_epilogues(enc, pair, block_n, epi, M, K):
-    N = {128: 1280, 160: 480, 256: 2048, 320: 1280}[block_n]
+    N = {128: 1280, 160: 480, 192: 3840, 256: 2048, 320: 1280}[block_n]
     g = torch.Generator().manual_seed(M * 7 + K + epi + block_n)
     A = (torch.randn(M, K, generator=g) / K ** 0.25).bfloat16()
     B = (torch.randn(N, K, generator=g) / K ** 0.25).bfloat16()
