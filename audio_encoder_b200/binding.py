@@ -27,6 +27,7 @@ EXPORTED = [
     "moss_enc_status_string", "moss_enc_last_error", "moss_enc_logmel", "moss_enc_log_max",
     "moss_enc_range_log_max",
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
+    "moss_enc_tap_weight_count", "moss_enc_set_taps", "moss_enc_forward_taps",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
     "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_selftest_gelu", "moss_enc_selftest_timeout",
 ]
@@ -98,6 +99,13 @@ def lib():
         L.moss_enc_forward_host.restype = i32
         L.moss_enc_forward_host.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(i64), i32, vp,
                                             ctypes.POINTER(i64)]
+        L.moss_enc_tap_weight_count.restype = i64
+        L.moss_enc_tap_weight_count.argtypes = []
+        L.moss_enc_set_taps.restype = i32
+        L.moss_enc_set_taps.argtypes = [vp, ctypes.POINTER(i32), i32, vp, ctypes.c_size_t, i32]
+        L.moss_enc_forward_taps.restype = i32
+        L.moss_enc_forward_taps.argtypes = [vp, ctypes.POINTER(Clip), i32, vp, ctypes.POINTER(vp),
+                                            ctypes.POINTER(i64)]
         L.moss_enc_profile_enable.restype = i32
         L.moss_enc_profile_enable.argtypes = [vp, i32]
         L.moss_enc_profile_read.restype = i32
@@ -130,6 +138,10 @@ def num_tokens(n: int) -> int:
 
 def range_tokens(n: int, begin: int, end: int) -> int:
     return int(lib().moss_enc_range_tokens(n, begin, end))
+
+
+def tap_weight_count() -> int:
+    return int(lib().moss_enc_tap_weight_count())
 
 
 def _ptr(t):
@@ -291,6 +303,43 @@ class Encoder:
             st = lib().moss_enc_forward_stage(self.h, arr, len(clips), stage, _ptr(out) if T else None, offs)
         self._check(st)
         return out, list(offs)
+
+    def set_taps(self, layers, weights=None):
+        """Layer taps: 0-based encoder layers, each with its own head + adapter
+        set (``weights``: uint16 numpy array or torch uint16/int16 CUDA tensor
+        of len(layers) * tap_weight_count() bf16 bits), or None to share the
+        encoder's own head and adapter."""
+        n = len(layers)
+        arr = (ctypes.c_int * max(n, 1))(*[int(l) for l in layers])
+        if weights is None:
+            st = lib().moss_enc_set_taps(self.h, arr, n, None, 0, 0)
+        elif isinstance(weights, np.ndarray):
+            w = np.ascontiguousarray(weights, dtype=np.uint16)
+            st = lib().moss_enc_set_taps(self.h, arr, n, w.ctypes.data_as(ctypes.c_void_p), w.nbytes, 0)
+        else:
+            st = lib().moss_enc_set_taps(self.h, arr, n, ctypes.c_void_p(weights.data_ptr()),
+                                         weights.numel() * 2, 1)
+        self._check(st)
+        self.n_taps = n
+
+    def forward_taps(self, clips, out=None, taps=None):
+        """Final rows plus one [T][2048] tensor per tap set by set_taps.
+
+        Returns (rows, [tap rows], row_offsets)."""
+        torch = self.torch
+        arr, T = self._clips(clips)
+        dt = torch.float32 if self.out_dtype == OUT_F32 else torch.bfloat16
+        dev = clips[0][0].device if isinstance(clips[0], tuple) else clips[0].device
+        n = getattr(self, "n_taps", 0)
+        if out is None:
+            out = torch.empty((T, D_OUT), dtype=dt, device=dev)
+        if taps is None:
+            taps = [torch.empty((T, D_OUT), dtype=dt, device=dev) for _ in range(n)]
+        ptrs = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in taps])
+        offs = (ctypes.c_int64 * (len(clips) + 1))()
+        self._check(lib().moss_enc_forward_taps(self.h, arr, len(clips), _ptr(out) if T else None,
+                                                ptrs if n else None, offs))
+        return out, taps, list(offs)
 
     def forward_host(self, clips_host, rows_host=None):
         """End-to-end from host fp32 arrays to host rows (synchronises)."""

@@ -38,6 +38,13 @@ struct LayerDev {
     float *bqkv, *bo, *b1, *b2;
 };
 
+// ln_post, proj1, proj2 and the SwiGLU adapter: the encoder's own set, and
+// one per layer tap (the cross-layer taps each have their own projector)
+struct HeadDev {
+    float *lnp_g, *lnp_b, *bp1, *bp2, *bgu, *bd;
+    bf16 *wp1, *wp2, *wgu, *wd;
+};
+
 struct ClipPlan {
     int64_t n, F, f_begin, f_end, c_first, c_last, tok0, ntok;
 };
@@ -55,11 +62,15 @@ struct moss_enc {
     float *conv1_w = nullptr, *conv1_b = nullptr, *conv2_b = nullptr, *conv3_b = nullptr;
     bf16 *conv2_w = nullptr, *conv3_w = nullptr, *conv_out_w = nullptr;
     std::vector<LayerDev> layers;
-    float *lnp_g = nullptr, *lnp_b = nullptr, *bp1 = nullptr, *bp2 = nullptr, *bgu = nullptr, *bd = nullptr;
-    bf16 *wp1 = nullptr, *wp2 = nullptr, *wgu = nullptr, *wd = nullptr;
+    HeadDev head{};
     float *pos = nullptr;
     MelTables *mel_tab = nullptr;
     MelBandT *mel_tabt = nullptr;
+
+    // layer taps (moss_enc_set_taps): encoder layer per tap and its head set
+    void *tap_wmem = nullptr;
+    std::vector<int> tap_layers;
+    std::vector<HeadDev> tap_heads;
 
     // capacity
     int64_t max_tokens = 0, max_chunks = 0;
@@ -524,6 +535,7 @@ extern "C" void moss_enc_destroy(moss_enc *h)
     if (h->stream) cudaStreamSynchronize(h->stream);
     else cudaDeviceSynchronize();
     if (h->wmem) cudaFree(h->wmem);
+    if (h->tap_wmem) cudaFree(h->tap_wmem);
     if (h->ws) cudaFree(h->ws);
     if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
     if (h->d_tab) cudaFree(h->d_tab);
@@ -532,6 +544,94 @@ extern "C" void moss_enc_destroy(moss_enc *h)
     if (h->tab_event) cudaEventDestroy(h->tab_event);
     for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
     delete h;
+}
+
+// Packed layout of one head + adapter set (ln_post, proj1, proj2, gate/up,
+// down).  proj1, proj2 and gate/up are stored twice along K ([W | W]) for
+// the split [hi | lo] operands; gate and up are interleaved in blocks of 32
+// output rows: g[0:32], u[0:32], g[32:64], ...
+struct HeadOff {
+    size_t lnp, p1, bp1, p2, bp2, gu, bgu, wd, bd;
+};
+
+template <class Take>
+static HeadOff head_take(Take &take)
+{
+    HeadOff o;
+    o.lnp = take(4 * 2 * D);
+    o.p1 = take(2 * (size_t)D * 2 * D);
+    o.bp1 = take(4 * D);
+    o.p2 = take(2 * (size_t)DOUT * 2 * D);
+    o.bp2 = take(4 * DOUT);
+    o.gu = take(2 * (size_t)2 * DADP * 2 * DOUT);
+    o.bgu = take(4 * 2 * DADP);
+    o.wd = take(2 * (size_t)DOUT * DADP);
+    o.bd = take(4 * DOUT);
+    return o;
+}
+
+// bf16 elements of one head + adapter set in the blob order: ln_post.g,
+// ln_post.b, proj1.w, proj1.b, proj2.w, proj2.b, gate.w, gate.b, up.w, up.b,
+// down.w, down.b.
+static int64_t head_count()
+{
+    return 2 * (int64_t)D + (int64_t)D * D + D + (int64_t)DOUT * D + DOUT + 2 * ((int64_t)DADP * DOUT + DADP) +
+           (int64_t)DOUT * DADP + DOUT;
+}
+
+// Repacks one set from the blob order at p into pk; returns the end of it.
+static const uint16_t *head_pack(const HeadOff &o, uint8_t *pk, const uint16_t *p)
+{
+    auto F32 = [&](size_t off) { return reinterpret_cast<float *>(pk + off); };
+    auto U16 = [&](size_t off) { return reinterpret_cast<uint16_t *>(pk + off); };
+    auto copy_twice = [&](uint16_t *dst, const uint16_t *src_rows, int rows, int k) {
+        for (int r = 0; r < rows; r++) {
+            std::memcpy(dst + (size_t)r * 2 * k, src_rows + (size_t)r * k, 2 * (size_t)k);
+            std::memcpy(dst + (size_t)r * 2 * k + k, src_rows + (size_t)r * k, 2 * (size_t)k);
+        }
+    };
+    for (int i = 0; i < 2 * D; i++) F32(o.lnp)[i] = bf16_bits_to_float(p[i]);
+    p += 2 * D;
+    copy_twice(U16(o.p1), p, D, D);
+    p += (size_t)D * D;
+    for (int i = 0; i < D; i++) F32(o.bp1)[i] = bf16_bits_to_float(p[i]);
+    p += D;
+    copy_twice(U16(o.p2), p, DOUT, D);
+    p += (size_t)DOUT * D;
+    for (int i = 0; i < DOUT; i++) F32(o.bp2)[i] = bf16_bits_to_float(p[i]);
+    p += DOUT;
+    const uint16_t *gw = p;
+    const uint16_t *gb = gw + (size_t)DADP * DOUT;
+    const uint16_t *uw = gb + DADP;
+    const uint16_t *ub = uw + (size_t)DADP * DOUT;
+    for (int j = 0; j < DADP / 32; j++)
+        for (int r = 0; r < 32; r++) {
+            copy_twice(U16(o.gu) + ((size_t)(64 * j + r)) * 2 * DOUT, gw + (size_t)(32 * j + r) * DOUT, 1, DOUT);
+            copy_twice(U16(o.gu) + ((size_t)(64 * j + 32 + r)) * 2 * DOUT, uw + (size_t)(32 * j + r) * DOUT, 1, DOUT);
+            F32(o.bgu)[64 * j + r] = bf16_bits_to_float(gb[32 * j + r]);
+            F32(o.bgu)[64 * j + 32 + r] = bf16_bits_to_float(ub[32 * j + r]);
+        }
+    p = ub + DADP;
+    std::memcpy(U16(o.wd), p, 2 * (size_t)DOUT * DADP);
+    p += (size_t)DOUT * DADP;
+    for (int i = 0; i < DOUT; i++) F32(o.bd)[i] = bf16_bits_to_float(p[i]);
+    return p + DOUT;
+}
+
+static HeadDev head_bind(const HeadOff &o, uint8_t *W)
+{
+    HeadDev d;
+    d.lnp_g = (float *)(W + o.lnp);
+    d.lnp_b = d.lnp_g + D;
+    d.wp1 = (bf16 *)(W + o.p1);
+    d.bp1 = (float *)(W + o.bp1);
+    d.wp2 = (bf16 *)(W + o.p2);
+    d.bp2 = (float *)(W + o.bp2);
+    d.wgu = (bf16 *)(W + o.gu);
+    d.bgu = (float *)(W + o.bgu);
+    d.wd = (bf16 *)(W + o.wd);
+    d.bd = (float *)(W + o.bd);
+    return d;
 }
 
 static moss_enc_status set_kernel_attrs(moss_enc *h)
@@ -618,12 +718,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     const size_t layer_bytes = 4 * 4 * D + 2 * ((size_t)DQKV * D + (size_t)D * D + (size_t)DFF * D + (size_t)D * DFF) +
                                4 * (DQKV + D + DFF + D) + 8 * 256;
     for (int l = 0; l < L; l++) o_layer[l] = take(layer_bytes);
-    // head and adapter weights are stored twice along K ([W | W]) for the
-    // split [hi | lo] operands
-    const size_t o_lnp = take(4 * 2 * D), o_p1 = take(2 * (size_t)D * 2 * D), o_bp1 = take(4 * D);
-    const size_t o_p2 = take(2 * (size_t)DOUT * 2 * D), o_bp2 = take(4 * DOUT);
-    const size_t o_gu = take(2 * (size_t)2 * DADP * 2 * DOUT), o_bgu = take(4 * 2 * DADP);
-    const size_t o_wd = take(2 * (size_t)DOUT * DADP), o_bd = take(4 * DOUT);
+    const HeadOff o_head = head_take(take);
     const size_t o_pos = take(4 * (size_t)CHUNK_TOKENS * D), o_mel = take(sizeof(MelTables));
     const size_t o_melt = take(sizeof(MelBandT));
     const size_t wtotal = off;
@@ -701,45 +796,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         for (int i = 0; i < D; i++) F32(b2)[i] = bf16_bits_to_float(p[i]);
         p += D;
     }
-    for (int i = 0; i < D; i++) F32(o_lnp)[i] = bf16_bits_to_float(p[i]);
-    p += D;
-    for (int i = 0; i < D; i++) F32(o_lnp)[D + i] = bf16_bits_to_float(p[i]);
-    p += D;
-    auto copy_twice = [&](uint16_t *dst, const uint16_t *src_rows, int rows, int k) {
-        for (int r = 0; r < rows; r++) {
-            std::memcpy(dst + (size_t)r * 2 * k, src_rows + (size_t)r * k, 2 * (size_t)k);
-            std::memcpy(dst + (size_t)r * 2 * k + k, src_rows + (size_t)r * k, 2 * (size_t)k);
-        }
-    };
-    copy_twice(U16(o_p1), p, D, D);
-    p += (size_t)D * D;
-    for (int i = 0; i < D; i++) F32(o_bp1)[i] = bf16_bits_to_float(p[i]);
-    p += D;
-    copy_twice(U16(o_p2), p, DOUT, D);
-    p += (size_t)DOUT * D;
-    for (int i = 0; i < DOUT; i++) F32(o_bp2)[i] = bf16_bits_to_float(p[i]);
-    p += DOUT;
-    // gate and up interleaved in blocks of 32 output rows: g[0:32], u[0:32], g[32:64], ...
-    {
-        const uint16_t *gw = p;
-        const uint16_t *gb = gw + (size_t)DADP * DOUT;
-        const uint16_t *uw = gb + DADP;
-        const uint16_t *ub = uw + (size_t)DADP * DOUT;
-        uint16_t *dst = U16(o_gu);
-        float *bdst = F32(o_bgu);
-        for (int j = 0; j < DADP / 32; j++)
-            for (int r = 0; r < 32; r++) {
-                copy_twice(dst + ((size_t)(64 * j + r)) * 2 * DOUT, gw + (size_t)(32 * j + r) * DOUT, 1, DOUT);
-                copy_twice(dst + ((size_t)(64 * j + 32 + r)) * 2 * DOUT, uw + (size_t)(32 * j + r) * DOUT, 1, DOUT);
-                bdst[64 * j + r] = bf16_bits_to_float(gb[32 * j + r]);
-                bdst[64 * j + 32 + r] = bf16_bits_to_float(ub[32 * j + r]);
-            }
-        p = ub + DADP;
-    }
-    std::memcpy(U16(o_wd), p, 2 * (size_t)DOUT * DADP);
-    p += (size_t)DOUT * DADP;
-    for (int i = 0; i < DOUT; i++) F32(o_bd)[i] = bf16_bits_to_float(p[i]);
-    p += DOUT;
+    p = head_pack(o_head, pk.data(), p);
     if (p - src != count) return bail(MOSS_ENC_ERR_INVALID_ARG);
     // sinusoidal positions 0..99: 640 sin channels then 640 cos channels,
     // inv_timescale_i = exp(-i ln(10000) / 639)
@@ -783,16 +840,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         d.w2 = (bf16 *)(W + L12[10]);
         d.b2 = (float *)(W + L12[11]);
     }
-    h->lnp_g = (float *)(W + o_lnp);
-    h->lnp_b = h->lnp_g + D;
-    h->wp1 = (bf16 *)(W + o_p1);
-    h->bp1 = (float *)(W + o_bp1);
-    h->wp2 = (bf16 *)(W + o_p2);
-    h->bp2 = (float *)(W + o_bp2);
-    h->wgu = (bf16 *)(W + o_gu);
-    h->bgu = (float *)(W + o_bgu);
-    h->wd = (bf16 *)(W + o_wd);
-    h->bd = (float *)(W + o_bd);
+    h->head = head_bind(o_head, W);
     h->pos = (float *)(W + o_pos);
     h->mel_tab = (MelTables *)(W + o_mel);
     h->mel_tabt = (MelBandT *)(W + o_melt);
@@ -1029,17 +1077,78 @@ struct FwdPlan {
     std::vector<int> g_off2, g_n2, g_off3, g_n3;
 };
 
-// Identity of a forward request for graph reuse.
-static std::vector<uint8_t> request_key(const moss_enc_clip *clips, int n_clips, const void *out)
+// Identity of a forward request for graph reuse: clips, output and the tap
+// outputs (the tap layers and weights are fixed between set_taps calls, which
+// drop the graph).
+static std::vector<uint8_t> request_key(const moss_enc_clip *clips, int n_clips, const void *out,
+                                        void *const *tap_out, int n_taps)
 {
-    std::vector<uint8_t> k(sizeof(int) + sizeof(void *) + sizeof(moss_enc_clip) * (size_t)n_clips);
-    std::memcpy(k.data(), &n_clips, sizeof(int));
-    std::memcpy(k.data() + sizeof(int), &out, sizeof(void *));
-    if (n_clips > 0) std::memcpy(k.data() + sizeof(int) + sizeof(void *), clips, sizeof(moss_enc_clip) * (size_t)n_clips);
+    const int nt = tap_out ? n_taps : 0;
+    std::vector<uint8_t> k(2 * sizeof(int) + sizeof(void *) * (1 + (size_t)nt) + sizeof(moss_enc_clip) * (size_t)n_clips);
+    uint8_t *q = k.data();
+    std::memcpy(q, &n_clips, sizeof(int));
+    q += sizeof(int);
+    std::memcpy(q, &nt, sizeof(int));
+    q += sizeof(int);
+    std::memcpy(q, &out, sizeof(void *));
+    q += sizeof(void *);
+    if (nt > 0) std::memcpy(q, tap_out, sizeof(void *) * (size_t)nt);
+    q += sizeof(void *) * (size_t)nt;
+    if (n_clips > 0) std::memcpy(q, clips, sizeof(moss_enc_clip) * (size_t)n_clips);
     return k;
 }
 
-static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt, int stage, void *out)
+// ln_post -> proj1 -> GELU -> proj2 -> SwiGLU adapter on the residual stream
+// X [T][1280], with the head set W; stops after proj2 (fp32 rows) when stage
+// is MOSS_ENC_STAGE_HEAD, else writes the adapter rows (cfg.out_dtype).
+static moss_enc_status head_launch(moss_enc *h, const HeadDev &W, int64_t T, int stage, void *out)
+{
+    const int ln_grid = (int)((T + 7) / 8);
+    {
+        Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
+        CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X,
+                             (const float *)W.lnp_g, (const float *)W.lnp_b, h->xn, (int)T, 2 * D, 1));
+    }
+    // The head GEMMs and the gate/up GEMM take split operands [hi | lo] (bf16
+    // pairs that carry ~16 bits) against weights repeated along K, which keeps
+    // the SwiGLU from amplifying bf16 rounding of its inputs; the SwiGLU
+    // product itself goes to the down-projection as plain bf16 (splitting it
+    // too would double the largest adapter GEMM for a small gain: on the 30 s
+    // clip the final rows' max err/rms is 0.0179 without that split, 0.0158
+    // with it, against a bound of 0.03).
+    GemmArgs a{};
+    a.bias = W.bp1;
+    a.out = h->hb;
+    a.ldo = 2 * D;
+    a.split_off = D;
+    TRY((gemm2<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, W.wp1, D, a, D)));
+    a.bias = W.bp2;
+    if (stage == MOSS_ENC_STAGE_HEAD) {
+        a.out = out;
+        a.ldo = DOUT;
+        a.split_off = 0;
+        return gemm2<256, EPI_F32>(h, "gemm_proj2", h->hb, T, 2 * D, W.wp2, DOUT, a, D);
+    }
+    a.out = h->h2;
+    a.ldo = 2 * DOUT;
+    a.split_off = DOUT;
+    TRY((gemm2<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, 2 * D, W.wp2, DOUT, a, D)));
+    // ---- SwiGLU adapter
+    a.bias = W.bgu;
+    a.out = h->gu;
+    a.ldo = DADP;
+    a.split_off = 0;
+    TRY((gemm2<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, 2 * DOUT, W.wgu, 2 * DADP, a, DOUT)));
+    a.bias = W.bd;
+    a.out = out;
+    a.ldo = DOUT;
+    a.split_off = 0;
+    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
+    return gemm2<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
+}
+
+static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt, int stage, void *out,
+                                     void *const *tap_out)
 {
     const TabLayout tl = tab_layout(h->cfg.max_clips, h->max_chunks);
     const int n_clips = P.n_clips;
@@ -1134,58 +1243,22 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.out = h->X;
         a.ldo = D;
         TRY((gemm2<320, EPI_RESID_F32>(h, "gemm_fc2", h->ffn, T, DFF, L.w2, D, a)));
+        // layer taps: this layer's hidden states through the tap's own head set
+        // (xn, hb, h2 and gu are free between layers)
+        if (tap_out)
+            for (size_t t = 0; t < h->tap_layers.size(); t++)
+                if (h->tap_layers[t] == (int)l) TRY(head_launch(h, h->tap_heads[t], T, MOSS_ENC_STAGE_ADAPTER, tap_out[t]));
     }
     if (stage == MOSS_ENC_STAGE_LAYERS) {
         CUDA_TRY(h, cudaMemcpyAsync(out, h->X, sizeof(float) * T * D, cudaMemcpyDeviceToDevice, h->stream));
         return MOSS_ENC_OK;
     }
 
-    // ---- head: ln_post -> proj1 -> GELU -> proj2
-    {
-        Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
-        CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X,
-                             (const float *)h->lnp_g, (const float *)h->lnp_b, h->xn, (int)T, 2 * D, 1));
-    }
-    // The head GEMMs and the gate/up GEMM take split operands [hi | lo] (bf16
-    // pairs that carry ~16 bits) against weights repeated along K, which keeps
-    // the SwiGLU from amplifying bf16 rounding of its inputs; the SwiGLU
-    // product itself goes to the down-projection as plain bf16 (splitting it
-    // too would double the largest adapter GEMM for a small gain: on the 30 s
-    // clip the final rows' max err/rms is 0.0179 without that split, 0.0158
-    // with it, against a bound of 0.03).
-    GemmArgs a{};
-    a.bias = h->bp1;
-    a.out = h->hb;
-    a.ldo = 2 * D;
-    a.split_off = D;
-    TRY((gemm2<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, h->wp1, D, a, D)));
-    a.bias = h->bp2;
-    if (stage == MOSS_ENC_STAGE_HEAD) {
-        a.out = out;
-        a.ldo = DOUT;
-        a.split_off = 0;
-        return gemm2<256, EPI_F32>(h, "gemm_proj2", h->hb, T, 2 * D, h->wp2, DOUT, a, D);
-    }
-    a.out = h->h2;
-    a.ldo = 2 * DOUT;
-    a.split_off = DOUT;
-    TRY((gemm2<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, 2 * D, h->wp2, DOUT, a, D)));
-    // ---- SwiGLU adapter
-    a.bias = h->bgu;
-    a.out = h->gu;
-    a.ldo = DADP;
-    a.split_off = 0;
-    TRY((gemm2<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, 2 * DOUT, h->wgu, 2 * DADP, a, DOUT)));
-    a.bias = h->bd;
-    a.out = out;
-    a.ldo = DOUT;
-    a.split_off = 0;
-    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
-    return gemm2<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, h->wd, DOUT, a);
+    return head_launch(h, h->head, T, stage, out);
 }
 
 static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int n_clips, int stage,
-                                    void *out, int64_t *row_offsets)
+                                    void *out, int64_t *row_offsets, void *const *tap_out = nullptr)
 {
     if (!h) return MOSS_ENC_ERR_INVALID_ARG;
     if (n_clips < 0 || (n_clips > 0 && !clips) || !row_offsets) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad argument");
@@ -1211,6 +1284,9 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     if (samples > h->cfg.max_samples || T > h->max_tokens || n_chunks > h->max_chunks)
         return fail(h, MOSS_ENC_ERR_CAPACITY, "request exceeds the capacity set at create");
     if (T > 0 && !out) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null output");
+    if (T > 0 && tap_out)
+        for (size_t t = 0; t < h->tap_layers.size(); t++)
+            if (!tap_out[t]) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null tap output");
     if (T == 0) return MOSS_ENC_OK;
 
     // ---- tables
@@ -1297,9 +1373,10 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
                            cs == cudaStreamCaptureStatusNone;
     if (!graphable) {
         TRY(tab_upload(h));
-        return forward_launch(h, P, static_cast<uint8_t *>(h->d_tab), stage, out);
+        return forward_launch(h, P, static_cast<uint8_t *>(h->d_tab), stage, out, tap_out);
     }
-    if (h->graph_exec && h->graph_key == request_key(clips, n_clips, out)) {
+    const int n_taps = (int)h->tap_layers.size();
+    if (h->graph_exec && h->graph_key == request_key(clips, n_clips, out, tap_out, n_taps)) {
         h->launches += h->graph_launches;
         CUDA_TRY(h, cudaGraphLaunch(h->graph_exec, h->stream));
         return MOSS_ENC_OK;
@@ -1312,7 +1389,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     CUDA_TRY(h, cudaEventRecord(h->tab_event, h->stream));
     const int64_t launches0 = h->launches;
     CUDA_TRY(h, cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
-    const moss_enc_status st = forward_launch(h, P, static_cast<uint8_t *>(h->d_tab_graph), stage, out);
+    const moss_enc_status st = forward_launch(h, P, static_cast<uint8_t *>(h->d_tab_graph), stage, out, tap_out);
     cudaGraph_t g = nullptr;
     const cudaError_t ce = cudaStreamEndCapture(h->stream, &g);
     if (st != MOSS_ENC_OK || ce != cudaSuccess) {
@@ -1326,7 +1403,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         h->graph_exec = nullptr;
         return fail(h, MOSS_ENC_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(ie));
     }
-    h->graph_key = request_key(clips, n_clips, out);
+    h->graph_key = request_key(clips, n_clips, out, tap_out, n_taps);
     h->graph_launches = h->launches - launches0;
     CUDA_TRY(h, cudaGraphLaunch(h->graph_exec, h->stream));
     return MOSS_ENC_OK;
@@ -1343,6 +1420,72 @@ extern "C" moss_enc_status moss_enc_forward_stage(moss_enc *h, const moss_enc_cl
                                                   void *out, int64_t *row_offsets)
 {
     return forward_impl(h, clips, n_clips, stage, out, row_offsets);
+}
+
+extern "C" int64_t moss_enc_tap_weight_count(void) { return head_count(); }
+
+extern "C" moss_enc_status moss_enc_set_taps(moss_enc *h, const int *layers, int n_taps, const void *weights,
+                                             size_t bytes, int weights_on_device)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (n_taps < 0 || n_taps > MOSS_ENC_MAX_TAPS || (n_taps > 0 && !layers))
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad tap list");
+    for (int t = 0; t < n_taps; t++)
+        if (layers[t] < 0 || layers[t] >= h->cfg.n_layers) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "tap layer out of range");
+    if (weights && (int64_t)bytes != 2 * head_count() * n_taps)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "tap weight blob has the wrong size");
+    // pending work may still read the old tap weights
+    CUDA_TRY(h, cudaStreamSynchronize(h->stream));
+    if (h->graph_exec) {
+        cudaGraphExecDestroy(h->graph_exec);
+        h->graph_exec = nullptr;
+        h->graph_key.clear();
+    }
+    if (h->tap_wmem) {
+        cudaFree(h->tap_wmem);
+        h->tap_wmem = nullptr;
+    }
+    h->tap_layers.clear();
+    h->tap_heads.clear();
+    if (n_taps == 0) return MOSS_ENC_OK;
+    std::vector<HeadDev> heads(n_taps, h->head);
+    if (weights) {
+        size_t off = 0;
+        auto take = [&](size_t b) {
+            size_t r = off;
+            off += (b + 255) & ~size_t(255);
+            return r;
+        };
+        std::vector<HeadOff> o(n_taps);
+        for (int t = 0; t < n_taps; t++) o[t] = head_take(take);
+        std::vector<uint16_t> host;
+        const uint16_t *p = static_cast<const uint16_t *>(weights);
+        if (weights_on_device) {
+            host.resize((size_t)head_count() * n_taps);
+            CUDA_TRY(h, cudaMemcpy(host.data(), weights, bytes, cudaMemcpyDeviceToHost));
+            p = host.data();
+        }
+        std::vector<uint8_t> pk(off, 0);
+        for (int t = 0; t < n_taps; t++) p = head_pack(o[t], pk.data(), p);
+        if (cudaMalloc(&h->tap_wmem, off) != cudaSuccess) {
+            h->tap_wmem = nullptr;
+            return fail(h, MOSS_ENC_ERR_OOM, "tap weights");
+        }
+        CUDA_TRY(h, cudaMemcpy(h->tap_wmem, pk.data(), off, cudaMemcpyHostToDevice));
+        for (int t = 0; t < n_taps; t++) heads[t] = head_bind(o[t], static_cast<uint8_t *>(h->tap_wmem));
+    }
+    h->tap_layers.assign(layers, layers + n_taps);
+    h->tap_heads = std::move(heads);
+    return MOSS_ENC_OK;
+}
+
+extern "C" moss_enc_status moss_enc_forward_taps(moss_enc *h, const moss_enc_clip *clips, int n_clips, void *rows_out,
+                                                 void *const *tap_rows, int64_t *row_offsets)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (!h->tap_layers.empty() && !tap_rows) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "null tap_rows");
+    return forward_impl(h, clips, n_clips, MOSS_ENC_STAGE_ADAPTER, rows_out, row_offsets,
+                        h->tap_layers.empty() ? nullptr : tap_rows);
 }
 
 extern "C" moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host, const int64_t *n_samples,

@@ -135,6 +135,35 @@ def make_weights(n_layers: int, seed: int = 1234) -> np.ndarray:
     return blob
 
 
+def head_manifest():
+    """(name, shape, kind) of one head + adapter set: the tail of the blob
+    after the layers, which is also the layout of one layer tap's set."""
+    m = weight_manifest(0)
+    first = [name for name, _, _ in m].index("ln_post.weight")
+    return m[first:]
+
+
+def make_tap_weights(n_taps: int, seed: int = 4321) -> np.ndarray:
+    """n_taps consecutive head + adapter sets (bf16 bits), initialised like
+    the blob's own: N(0, 1/fan_in) matrices, N(0, 0.01^2) biases, LayerNorm
+    gamma 1 and beta 0."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    parts = []
+    for _ in range(n_taps):
+        for _name, shape, kind in head_manifest():
+            n = int(np.prod(shape))
+            if kind == "w":
+                v = rng.standard_normal(n, dtype=np.float32) * np.float32(1.0 / np.sqrt(int(np.prod(shape[1:]))))
+            elif kind == "b":
+                v = rng.standard_normal(n, dtype=np.float32) * np.float32(0.01)
+            elif kind == "g":
+                v = np.ones(n, dtype=np.float32)
+            else:
+                v = np.zeros(n, dtype=np.float32)
+            parts.append(f32_to_bf16_bits(v))
+    return np.concatenate(parts) if parts else np.empty(0, dtype=np.uint16)
+
+
 def _tones(rng, n: int, t0: int = 0) -> np.ndarray:
     t = (np.arange(n, dtype=np.float64) + t0) / SAMPLE_RATE
     freqs = rng.uniform(100.0, 6000.0, size=3)

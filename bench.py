@@ -51,9 +51,10 @@ def workload_clips(name):
     return desc, make(), n_layers
 
 
-def model_flops(tokens, n_layers):
-    # stem 353.6 + 39.83 per layer + head/adapter 109.2 MFLOP per token
-    return tokens * (353.6e6 + 39.83e6 * n_layers + 109.2e6)
+def model_flops(tokens, n_layers, n_taps=0):
+    # stem 353.6 + 39.83 per layer + head/adapter 109.2 MFLOP per token; each
+    # layer tap runs one more head/adapter set
+    return tokens * (353.6e6 + 39.83e6 * n_layers + 109.2e6 * (1 + n_taps))
 
 
 class Clocks:
@@ -229,16 +230,23 @@ def run_ours(args):
     mel_samples = 9_600_000  # the 10-min clip, for the log-mel roofline
     enc = binding.Encoder(blob, n_layers, max_samples=max(total_samples + 4 * len(clips), mel_samples),
                           max_clips=len(clips), out_dtype=binding.OUT_BF16, stream=stream)
+    tap_layers = [int(v) for v in args.taps.split(",")] if args.taps else []
     with torch.cuda.stream(stream):
         xs = [torch.from_numpy(c).to(dev) for c in clips]
         tokens = sum(binding.num_tokens(c.size) for c in clips)
         out = torch.empty((tokens, 2048), dtype=torch.bfloat16, device=dev)
+        tap_out = [torch.empty((tokens, 2048), dtype=torch.bfloat16, device=dev) for _ in tap_layers]
         flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    if tap_layers:
+        enc.set_taps(tap_layers, synth.make_tap_weights(len(tap_layers)))
     audio_s = total_samples / 16000.0
     torch.cuda.synchronize()
 
     def step():
-        enc.forward(xs, out=out)
+        if tap_layers:
+            enc.forward_taps(xs, out=out, taps=tap_out)
+        else:
+            enc.forward(xs, out=out)
 
     warmup = args.warmup if args.ncu else max(args.warmup, 3)
     for _ in range(warmup):
@@ -281,19 +289,23 @@ def run_ours(args):
     enc.synchronize()
 
     # ---- end to end through the host API: pinned PCM in, rows out to host
-    pinned = [torch.from_numpy(c).pin_memory() for c in clips]
-    rows_host = torch.empty((tokens, 2048), dtype=torch.bfloat16).pin_memory()
-    enc.forward_host(pinned, rows_host)
-    e2e_ms = []
-    for i in range(max(2, min(args.steps, 10))):
-        flush.fill_(float(i))
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+    # (the host API returns the final rows only, so a run with layer taps
+    # reports no end-to-end figure)
+    e2e_ms = [float("nan")]
+    if not tap_layers:
+        pinned = [torch.from_numpy(c).pin_memory() for c in clips]
+        rows_host = torch.empty((tokens, 2048), dtype=torch.bfloat16).pin_memory()
         enc.forward_host(pinned, rows_host)
-        b.record(stream)
-        b.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
+        e2e_ms = []
+        for i in range(max(2, min(args.steps, 10))):
+            flush.fill_(float(i))
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            enc.forward_host(pinned, rows_host)
+            b.record(stream)
+            b.synchronize()
+            e2e_ms.append(a.elapsed_time(b))
     e2e_step = reduce_max(float(np.mean(e2e_ms)), dist, dev)
 
     if rank != 0:
@@ -332,7 +344,7 @@ def run_ours(args):
     pk = peaks()
     ms_per_step = total_ms / args.steps
     value = weak_scaling_throughput(world, audio_s, ms_per_step)
-    flops_step = model_flops(tokens, n_layers)
+    flops_step = model_flops(tokens, n_layers, len(tap_layers))
     tflops = flops_step / (ms_per_step / 1e3) / 1e12
     # dominant kernel: the category with the most device time
     dom_name, dom = max(stats.items(), key=lambda kv: kv[1]["ms"])
@@ -376,15 +388,17 @@ def run_ours(args):
         "config": {"workload": args.workload, "description": desc, "clips_per_gpu": len(clips),
                    "audio_s_per_gpu": audio_s, "tokens_per_gpu": tokens, "layers": n_layers,
                    "out_dtype": "bf16", "l2": "512 MB buffer written between timed steps (outside the events)",
-                   "parallelism": f"dp{world}" if world > 1 else "single"},
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   **({"tap_layers": tap_layers} if tap_layers else {})},
         "roofline": roof,
         "mel_roofline": mel_roof,
         "kernels": kernels,
         "kernel_ms_per_step_eager": kernel_ms / args.steps,
         "gpu_launches": launches,
-        "e2e": {"value": weak_scaling_throughput(world, audio_s, e2e_step), "unit": "audio-s/s",
-                "h2d_bytes_per_step": 4 * total_samples, "d2h_bytes_per_step": 2 * tokens * 2048,
-                "ms_per_step": e2e_step},
+        "e2e": None if tap_layers else {
+            "value": weak_scaling_throughput(world, audio_s, e2e_step), "unit": "audio-s/s",
+            "h2d_bytes_per_step": 4 * total_samples, "d2h_bytes_per_step": 2 * tokens * 2048,
+            "ms_per_step": e2e_step},
         "cpu_baseline": cpu,
         "clocks": clk.summary(),
     }
@@ -484,6 +498,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shard-clip", action="store_true",
                     help="one long clip (10 or 60 min) split over the ranks by chunk ranges (strong scaling)")
+    ap.add_argument("--taps", default="",
+                    help="comma-separated encoder layers (0-based) whose hidden states also go through a "
+                         "head + adapter set of their own (layer taps); the step is forward_taps")
     ap.add_argument("--ncu", action="store_true",
                     help="capture run for ncu: warm-up as given (may be 0), the timed steps only, no report")
     args = ap.parse_args()

@@ -186,6 +186,47 @@ moss_enc_status moss_enc_forward(moss_enc *h, const moss_enc_clip *clips, int n_
 moss_enc_status moss_enc_forward_stage(moss_enc *h, const moss_enc_clip *clips, int n_clips,
                                        int stage, void *out, int64_t *row_offsets);
 
+/* ------------------------------------------------------- layer taps */
+
+/* Cross-layer taps (page "MOSS-Audio-4B-Instruct on an RTX 5070", opening
+ * paragraph: a DeepStack-inspired cross-layer adapter; page
+ * "MOSS-Music-8B-Instruct-GGUF", files section: deepstack injection wiring).
+ * A tap takes the residual stream after one encoder layer and runs it through
+ * a head + adapter set of its own (ln_post -> proj1 -> GELU -> proj2 ->
+ * SwiGLU adapter, the same computation as the encoder's final path), giving
+ * [T][2048] rows per tap beside the final rows.  The pages name the idea but
+ * not its wiring; this is the plainest reading of it. */
+#define MOSS_ENC_MAX_TAPS 8
+
+/* bf16 elements of one tap's head + adapter set, in the order of the tail of
+ * the main blob: ln_post.g, ln_post.b [1280], proj1.w [1280][1280], proj1.b,
+ * proj2.w [2048][1280], proj2.b [2048], gate.w [8192][2048], gate.b [8192],
+ * up.w, up.b, down.w [2048][8192], down.b [2048].  Pure. */
+int64_t moss_enc_tap_weight_count(void);
+
+/* Set the taps used by moss_enc_forward_taps (replaces any earlier set).
+ *  layers      host int [n_taps]: 0-based encoder layer after which each tap
+ *              reads the residual stream (0 <= layer < cfg.n_layers; repeats
+ *              allowed).  n_taps 0..MOSS_ENC_MAX_TAPS; 0 removes the taps.
+ *  weights     n_taps consecutive sets of moss_enc_tap_weight_count() bf16
+ *              elements, host or device memory as weights_on_device says,
+ *              copied and repacked (the caller may free it); or NULL to make
+ *              every tap use the encoder's own ln_post/proj/adapter weights.
+ *  bytes       size of weights in bytes (checked unless weights is NULL).
+ * Synchronises the handle's stream and allocates the packed tap weights
+ * (about 185 MB per set); forward calls still allocate nothing.
+ * Errors: INVALID_ARG (bad list, layer out of range, wrong size), OOM. */
+moss_enc_status moss_enc_set_taps(moss_enc *h, const int *layers, int n_taps, const void *weights,
+                                  size_t bytes, int weights_on_device);
+
+/* moss_enc_forward plus the tap rows.
+ *  tap_rows     host array of n_taps device pointers, tap t's rows
+ *               [sum of tokens][2048] of cfg.out_dtype, clip i at rows
+ *               row_offsets[i] ..; ignored (may be NULL) with no taps set.
+ * Same clips, rows_out, row_offsets and errors as moss_enc_forward. */
+moss_enc_status moss_enc_forward_taps(moss_enc *h, const moss_enc_clip *clips, int n_clips,
+                                      void *rows_out, void *const *tap_rows, int64_t *row_offsets);
+
 /* End-to-end from host memory: copies each clip's samples host->device,
  * encodes, copies the rows device->host and synchronises.
  *  pcm_host     host array of n_clips pointers to fp32 [n_samples[i]].
