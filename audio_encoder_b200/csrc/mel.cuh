@@ -40,12 +40,6 @@ struct MelTables {
     int band_n[128];              // nonzero bins of each filter (<= MEL_BAND)
 };
 
-// The filterbank weights transposed, [bin offset][filter]: consecutive
-// filters are consecutive words (read by logmel3_kernel).
-struct MelBandT {
-    float w[MEL_BAND][128];
-};
-
 __device__ __forceinline__ float2 cmul(float2 a, float2 b)
 {
     return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
@@ -243,35 +237,62 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip 
 }
 
 // Persistent form of the same computation (the one the library launches).
-// Two CTAs per SM walk the (clip, 32-frame block) items of the launch; each
-// loads the twiddle, window and filterbank tables once, and while it
-// transforms one block it already fetches the next block's PCM span into the
-// other buffer with cp.async (blocks at the clip ends, which need reflect
-// padding, are loaded synchronously).  The power spectrum is written back
-// into the exchange buffer, and log10 uses the hardware log2.
-static constexpr int MEL3_MAX_CLIPS = 128;  // clips per launch (the host splits larger batches)
+// Four CTAs of 160 threads per SM walk the (clip, 16-frame block) items of
+// the launch, 5 barriers per item.  Thread t takes pair tp = t % 8 and row or
+// column tj = t / 8 in every transform phase, so a warp covers 8 pairs x 4
+// columns and its shared-memory accesses spread over the banks.
+//  pass 1: 20-point DFT over n2 of the windowed samples tj + 20 n2 of both
+//          frames of pair tp (frame a real, frame b imaginary), times the
+//          400-point twiddle w^(tj k2), into row tj of the pair's buffer
+//          (row pitch 20: Z[20 k1 + k2] ends up at element 20 k1 + k2);
+//          the block's PCM span is then dead, and the next block's span is
+//          fetched into it with cp.async while this block finishes;
+//  pass 2: 20-point DFT over the rows of column tj, in place;
+//  power:  bins k = tj + 20 i of both frames from Z[k] and Z[400 - k]; the
+//          power pair (a, b) replaces Z[k] in place (the locations a thread
+//          reads are its own, so the phase needs no inner barrier);
+//  mel:    lane = frame (16), the two half-warps take the even and odd bins
+//          of the same filters (one shuffle adds them), warp w a range of
+//          filters balanced by their bins; log-mel rows are staged in the
+//          pair's dead upper half (Z[k], k > 200) and stored whole.
+static constexpr int MEL_MAX_CLIPS = 128;  // clips per launch (the host splits larger batches)
+static constexpr int MEL4_FRAMES = 16;
+static constexpr int MEL4_THREADS = 160;
+static constexpr int MEL4_WARPS = MEL4_THREADS / 32;
+static constexpr int MEL4_PAIRS = MEL4_FRAMES / 2;
+static constexpr int MEL4_SPAN_SAMPLES = 160 * (MEL4_FRAMES - 1) + 400;  // 2800
 
 // A block's PCM span sits in shared memory with 20 unused words after every
-// 320 samples (one frame pair): sample s of the span is word mel3_pad(s).
-// Pass-1 task t reads sample 20 n2 + (t mod 20) of pair t / 20, i.e. word
-// 340 (t / 20) + (t mod 20) + 20 n2 + (0 or 20), whose bank is
-// t + 20 n2 (mod 32): distinct across a warp, so the loads are conflict-free.
-__host__ __device__ constexpr int mel3_pad(int s) { return s + 20 * (s / 320); }
-static constexpr int MEL3_SPAN = mel3_pad(MEL2_SPAN - 1) + 1;  // 5680 words
-static constexpr int MEL3_OUT_LD = 132;  // row pitch of the staged log-mel rows (float4-aligned)
+// 320 samples (one frame pair): sample s of the span is word mel_span_pad(s).
+// Pass-1 thread (tp, tj) reads sample 20 n2 + tj of pair tp, i.e. word
+// 340 tp + tj + 20 n2 (+ 20), whose bank is 20 tp + tj + 20 n2 (mod 32):
+// distinct across a warp's 8 pairs x 4 columns.
+__host__ __device__ constexpr int mel_span_pad(int s) { return s + 20 * (s / 320); }
+static constexpr int MEL4_SPAN = mel_span_pad(MEL4_SPAN_SAMPLES - 1) + 1;  // 2960 words
+// Pair pitch of the exchange buffer (float2): 402 = 4 words mod 32 between
+// consecutive pairs, so a half-warp's 8 pairs x 2 columns hit distinct banks.
+static constexpr int MEL4_YP = 402;
+static constexpr int MEL4_STAGE = 416;  // float offset of the staged log-mel rows inside a pair (Z[208] on)
 
-struct Mel3Smem {
-    float2 tw[400];
+// Constant tables of the kernel, built on the host in their shared-memory
+// layout and copied in whole at the start.
+struct alignas(16) Mel4Tab {
+    float2 tw[20][21];  // w^(n1 k2) at [k2][n1], w = exp(-2 pi i / 400)
     float hann[400];
-    int band_lo[128];
-    int band_n[128];
-    float band_wt[MEL_BAND][128];
-    float2 y[MEL2_FRAMES / 2][20 * 21];  // pass outputs; then the power spectra, frame f at floats [201 f, 201 f + 201)
-    float xs[2][MEL3_SPAN];              // PCM spans of the current and the next block (padded, see mel3_pad);
-                                         // the current one then stages the block's log-mel rows
-    int first_block[MEL3_MAX_CLIPS + 1];  // prefix of blocks per clip
-    int mpart[MEL2_THREADS / 32 + 1];     // filters of warp w: [mpart[w], mpart[w+1])
-    float wmax[MEL2_THREADS / 32];
+    int band_lo[128];   // first nonzero bin of filter m
+    int band_n[128];    // nonzero bins of filter m (<= MEL_BAND)
+    float band_wt[MEL_BAND][129];  // weight of bin band_lo[m] + b at [b][m] (odd pitch: rows b, b + 1 on different banks)
+    int mpart[8];       // filters of warp w: [mpart[w], mpart[w+1])
+};
+static_assert(sizeof(Mel4Tab) % 16 == 0, "the tables are copied in 16-byte pieces");
+
+struct Mel4Smem {
+    Mel4Tab t;
+    alignas(16) float2 y[MEL4_PAIRS][MEL4_YP];  // exchange buffer; 16-byte aligned rows (staged rows are read as float4)
+    alignas(16) float xs[MEL4_SPAN];            // the block's PCM span (padded); cp.async target
+    int first_block[MEL_MAX_CLIPS + 1];
+    int scan[MEL4_WARPS];
+    float wmax[MEL4_WARPS];
 };
 
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
@@ -279,116 +300,107 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Locate item `item` among the clips' blocks: returns false past the end.
-__device__ __forceinline__ bool mel3_item(const Mel3Smem &S, const MelClip *clips, int n_clips, int item, int &c,
+__device__ __forceinline__ bool mel4_item(const int *first_block, const MelClip *clips, int n_clips, int item, int &c,
                                           int &frame0, int &nf)
 {
-    if (item >= S.first_block[n_clips]) return false;
-    c = 0;
-    while (S.first_block[c + 1] <= item) ++c;
+    if (item >= first_block[n_clips]) return false;
+    int lo = 0, hi = n_clips - 1;  // the last clip whose first block is <= item
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (first_block[mid] <= item) lo = mid;
+        else hi = mid - 1;
+    }
+    c = lo;
     const MelClip &cl = clips[c];
-    frame0 = cl.f_begin + MEL2_FRAMES * (item - S.first_block[c]);
-    nf = min(MEL2_FRAMES, cl.f_end - frame0);
+    frame0 = cl.f_begin + MEL4_FRAMES * (item - first_block[c]);
+    nf = min(MEL4_FRAMES, cl.f_end - frame0);
     return true;
 }
 
 // Whether the span of a block lies inside the clip and can be copied as is.
-__device__ __forceinline__ bool mel3_interior(const MelClip &cl, int frame0, int nf)
+__device__ __forceinline__ bool mel_span_interior(const MelClip &cl, int frame0, int nf)
 {
     const long long s0 = 160LL * frame0 - 200;
     return s0 >= 0 && s0 + 160LL * (nf - 1) + 400 <= cl.n && ((reinterpret_cast<uintptr_t>(cl.pcm) & 15) == 0);
 }
 
-__global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip *__restrict__ clips, int n_clips,
-                                                                  const MelTables *__restrict__ tab,
-                                                                  const MelBandT *__restrict__ tabt,
+__global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip *__restrict__ clips, int n_clips,
+                                                                  const Mel4Tab *__restrict__ tab,
                                                                   float *__restrict__ out, int *gmax_ord,
                                                                   int write_out)
 {
-    extern __shared__ __align__(16) uint8_t mel3_smem[];
-    Mel3Smem &S = *reinterpret_cast<Mel3Smem *>(mel3_smem);
-    const int tid = threadIdx.x;
-    for (int i = tid; i < 400; i += MEL2_THREADS) {
-        S.tw[i] = tab->tw400[i];
-        S.hann[i] = tab->hann[i];
-    }
-    for (int i = tid; i < 128; i += MEL2_THREADS) {
-        S.band_lo[i] = tab->band_lo[i];
-        S.band_n[i] = tab->band_n[i];
-    }
-    for (int i = tid; i < 128 * MEL_BAND; i += MEL2_THREADS) S.band_wt[i / 128][i % 128] = tabt->w[i / 128][i % 128];
+    extern __shared__ __align__(16) uint8_t mel4_smem[];
+    Mel4Smem &S = *reinterpret_cast<Mel4Smem *>(mel4_smem);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // the tables: one round of 16-byte copies
+    for (int i = tid; i < (int)(sizeof(Mel4Tab) / 16); i += MEL4_THREADS)
+        cp_async16(reinterpret_cast<float4 *>(&S.t) + i, reinterpret_cast<const float4 *>(tab) + i);
+    cp_async_commit();
     grid_dep_wait();
     grid_dep_launch();
-    __syncthreads();  // the filter table is in place before thread 0 reads it
-    if (tid == 0) {
-        int acc = 0;
-        for (int c = 0; c < n_clips; c++) {
-            S.first_block[c] = acc;
-            const int f = clips[c].f_end - clips[c].f_begin;
-            acc += f > 0 ? (f + MEL2_FRAMES - 1) / MEL2_FRAMES : 0;
+    // blocks per clip -> prefix (thread c takes clip c; n_clips <= MEL_MAX_CLIPS <= MEL4_THREADS)
+    {
+        int nb = 0;
+        if (tid < n_clips) {
+            const int f = clips[tid].f_end - clips[tid].f_begin;
+            nb = f > 0 ? (f + MEL4_FRAMES - 1) / MEL4_FRAMES : 0;
         }
-        S.first_block[n_clips] = acc;
-        // filters per warp for the filterbank stage, balanced by their bins
-        int total = 0;
-        for (int m = 0; m < 128; m++) total += S.band_n[m];
-        int w = 0, run = 0;
-        S.mpart[0] = 0;
-        for (int m = 0; m < 128; m++) {
-            run += S.band_n[m];
-            while (w + 1 < MEL2_THREADS / 32 && run * (MEL2_THREADS / 32) >= total * (w + 1)) S.mpart[++w] = m + 1;
+        int incl = nb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        while (w + 1 <= MEL2_THREADS / 32) S.mpart[++w] = 128;
+        if (lane == 31) S.scan[warp] = incl;
+        __syncthreads();
+        int base = 0;
+        for (int w = 0; w < warp; w++) base += S.scan[w];
+        if (tid <= n_clips) S.first_block[tid] = base + incl - nb;  // exclusive prefix; [n_clips] = total
+        cp_async_wait_all();
+        __syncthreads();
     }
-    __syncthreads();
 
     // span loader: async 16-byte copies for interior blocks (returns true),
     // nothing for edge blocks (loaded synchronously when their turn comes)
-    auto prefetch = [&](int item, int buf) -> bool {
+    auto prefetch = [&](int item) -> bool {
         int c, frame0, nf;
-        if (!mel3_item(S, clips, n_clips, item, c, frame0, nf)) return true;
+        if (!mel4_item(S.first_block, clips, n_clips, item, c, frame0, nf)) return true;
         const MelClip &cl = clips[c];
-        if (!mel3_interior(cl, frame0, nf)) return false;
+        if (!mel_span_interior(cl, frame0, nf)) return false;
         const float4 *src = reinterpret_cast<const float4 *>(cl.pcm + (160LL * frame0 - 200));
         const int n4 = (160 * (nf - 1) + 400) / 4;
-        for (int i = tid; i < n4; i += MEL2_THREADS)
-            cp_async16(reinterpret_cast<float4 *>(S.xs[buf]) + i + 5 * (i / 80), src + i);
+        for (int i = tid; i < n4; i += MEL4_THREADS)
+            cp_async16(reinterpret_cast<float4 *>(S.xs) + i + 5 * (i / 80), src + i);
         return true;
     };
 
     const float log10_2 = 0.30102999566398120f;
-    // Every DFT task of this thread has the same pair and row: pass 1 takes
-    // (pair tp, n1 = tj), pass 2 (tp, k2 = tj), and the power step the bins
-    // k = tj + 20 i of pair tp.
-    const int tp = tid / 20, tj = tid - 20 * tp;
-    const float *hw = S.hann + tj;  // window value of sample tj + 20 n2: hw[20 n2]
-    int it = 0;
-    bool ready = prefetch(blockIdx.x, 0);
+    const int tp = tid & 7, tj = tid >> 3;
+    const float *hw = S.t.hann + tj;  // window value of sample tj + 20 n2: hw[20 n2]
+    bool ready = prefetch(blockIdx.x);
     cp_async_commit();
-    for (int item = blockIdx.x;; item += gridDim.x, ++it) {
+    for (int item = blockIdx.x;; item += gridDim.x) {
         int c, frame0, nf;
-        if (!mel3_item(S, clips, n_clips, item, c, frame0, nf)) break;
+        if (!mel4_item(S.first_block, clips, n_clips, item, c, frame0, nf)) break;
         const MelClip cl = clips[c];
-        const int cur = it & 1;
-        if (!ready) {  // edge block: reflect-padded load now
+        if (!ready) {  // edge block: reflect-padded load now (nothing is in flight into the span)
             const long long s0 = 160LL * frame0 - 200;
             const int span = 160 * (nf - 1) + 400;
-            for (int i = tid; i < span; i += MEL2_THREADS) S.xs[cur][mel3_pad(i)] = __ldg(cl.pcm + reflect_index(s0 + i, cl.n));
+            for (int i = tid; i < span; i += MEL4_THREADS)
+                S.xs[mel_span_pad(i)] = __ldg(cl.pcm + reflect_index(s0 + i, cl.n));
         }
-        ready = prefetch(item + gridDim.x, cur ^ 1);
-        cp_async_commit();
-        cp_async_wait_1();  // this block's span has landed (the next one may still be in flight)
-        __syncthreads();
+        cp_async_wait_all();
+        __syncthreads();  // B0: span in place; the previous block's staged rows are stored
 
-        const float *xsb = S.xs[cur];
         const int npairs = (nf + 1) / 2;
+        float2 *Y = S.y[tp];
         if (tp < npairs) {
-            // pass 1: 20-point DFT over n2 of the windowed samples n = tj + 20 n2
-            // of frame 2 tp (real part) and frame 2 tp + 1 (imaginary part)
+            // pass 1 (frame 2 tp starts at span sample 320 tp, frame 2 tp + 1 at 320 tp + 160)
             const bool has_b = 2 * tp + 1 < nf;
-            // frame 2 tp starts at span sample 320 tp, frame 2 tp + 1 at 320 tp + 160
-            const float *xa = xsb + 340 * tp + tj, *xb = has_b ? xa + 160 : xa;
+            const float *xa = S.xs + 340 * tp + tj, *xb = xa + 160;
             float2 v[20];
 #pragma unroll
             for (int n2 = 0; n2 < 20; n2++) {
@@ -397,109 +409,106 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel3_kernel(const MelClip 
                 v[n2] = make_float2(hw[20 * n2] * a, hw[20 * n2] * b);
             }
             dft20(v);
-            float2 *yr = S.y[tp] + tj * 21;
+            float2 *yr = Y + tj * 20;
+            yr[0] = v[0];
 #pragma unroll
-            for (int k2 = 0; k2 < 20; k2++) yr[k2] = (k2 == 0 || tj == 0) ? v[k2] : cmul(v[k2], S.tw[tj * k2]);
+            for (int k2 = 1; k2 < 20; k2++) yr[k2] = cmul(v[k2], S.t.tw[k2][tj]);  // w^0 = 1 exactly for tj = 0
         }
-        __syncthreads();
+        __syncthreads();  // B1: pass-1 rows written; the span is dead
+        ready = prefetch(item + gridDim.x);
+        cp_async_commit();
         if (tp < npairs) {
-            // pass 2: 20-point DFT over n1 -> Z[20 k1 + tj], in place
+            // pass 2: 20-point DFT over n1 -> Z[20 k1 + tj], in place (own column)
             float2 v[20];
 #pragma unroll
-            for (int n1 = 0; n1 < 20; n1++) v[n1] = S.y[tp][n1 * 21 + tj];
+            for (int n1 = 0; n1 < 20; n1++) v[n1] = Y[n1 * 20 + tj];
             dft20(v);
 #pragma unroll
-            for (int k1 = 0; k1 < 20; k1++) S.y[tp][k1 * 21 + tj] = v[k1];
+            for (int k1 = 0; k1 < 20; k1++) Y[k1 * 20 + tj] = v[k1];
         }
-        __syncthreads();
-        // power of both frames at bins k = tj + 20 i: X_a[k] = (Z[k] + conj Z[400-k]) / 2,
-        // X_b[k] = (Z[k] - conj Z[400-k]) / 2i, with Z[20 k1 + k2] at y[k1 * 21 + k2];
-        // read all of this thread's bins, then write them in place
-        float pa[11], pb[11];
+        __syncthreads();  // B2: the pair's spectrum Z is complete
         if (tp < npairs) {
+            // X_a[k] = (Z[k] + conj Z[400-k]) / 2, X_b[k] = (Z[k] - conj Z[400-k]) / 2i, k = tj + 20 i
+            float2 zk[11], zn[11];
 #pragma unroll
             for (int i = 0; i < 11; i++) {
-                if (i < 10 || tj == 0) {
-                    const float2 zk = S.y[tp][i * 21 + tj];
-                    const float2 zn = tj == 0 ? S.y[tp][(i == 0 ? 0 : 20 - i) * 21] : S.y[tp][(19 - i) * 21 + 20 - tj];
-                    const float ar = 0.5f * (zk.x + zn.x), ai = 0.5f * (zk.y - zn.y);
-                    const float br = 0.5f * (zk.y + zn.y), bi = -0.5f * (zk.x - zn.x);
-                    pa[i] = ar * ar + ai * ai;
-                    pb[i] = br * br + bi * bi;
+                const int k = tj + 20 * i;
+                if (k <= 200) {
+                    zk[i] = Y[k];
+                    zn[i] = Y[k == 0 ? 0 : 400 - k];
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 11; i++) {
+                const int k = tj + 20 * i;
+                if (k <= 200) {
+                    const float ar = zk[i].x + zn[i].x, ai = zk[i].y - zn[i].y;
+                    const float br = zk[i].y + zn[i].y, bi = zk[i].x - zn[i].x;
+                    Y[k] = make_float2(0.25f * (ar * ar + ai * ai), 0.25f * (br * br + bi * bi));
                 }
             }
         }
-        __syncthreads();
-        if (tp < npairs) {
-            float *pw = reinterpret_cast<float *>(S.y) + 402 * tp;  // frames 2 tp, 2 tp + 1: rows of 201
-#pragma unroll
-            for (int i = 0; i < 11; i++) {
-                if (i < 10 || tj == 0) {
-                    pw[tj + 20 * i] = pa[i];
-                    pw[201 + tj + 20 * i] = pb[i];
-                }
-            }
-        }
-        __syncthreads();
-        // banded filterbank: warp w takes filters mpart[w] .. mpart[w+1] - 1 for
-        // all frames, lane = frame; the filter's bins and weights are the same
-        // across the warp, and the power rows' odd pitch (201) puts the lanes'
-        // reads in distinct banks.  The block's log-mel rows are staged in the
-        // (now unused) span buffer and then stored whole.
+        __syncthreads();  // B3: power of every frame in place: frame f, bin k at float 2 k + (f & 1) of pair f / 2
         float lmax = -INFINITY;
         {
-            const int f = tid & 31, w = tid >> 5;
-            const float *P = reinterpret_cast<const float *>(S.y) + 201 * f;
-            float *ost = S.xs[cur] + MEL3_OUT_LD * f;
-            const int m1 = S.mpart[w + 1];
-            // four filters at a time (four independent sums); neighbouring
-            // filters have nearly equal widths, so little of the padding runs
-            for (int m0 = S.mpart[w]; m0 < m1; m0 += 4) {
-                int lo[4], cnt[4], cmax = 0;
+            const int f = lane & 15, h = lane >> 4;
+            const float *P = reinterpret_cast<const float *>(S.y[f >> 1]) + (f & 1);
+            float *ost = reinterpret_cast<float *>(S.y[f >> 1]) + MEL4_STAGE + 128 * (f & 1);
+            const int swz = 2 * (f & 1);  // odd frames' columns XOR 2: the pair's two rows on different banks
+            const int m1 = S.t.mpart[warp + 1];
+            for (int m0 = S.t.mpart[warp]; m0 < m1; m0 += 4) {
+                int lo[4], cnt[4], nit = 0;
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     const bool in = m0 + j < m1;
-                    lo[j] = in ? S.band_lo[m0 + j] : 0;
-                    cnt[j] = in ? S.band_n[m0 + j] : 0;
-                    cmax = max(cmax, cnt[j]);
+                    lo[j] = in ? S.t.band_lo[m0 + j] : 0;
+                    cnt[j] = in ? S.t.band_n[m0 + j] : 0;
+                    nit = max(nit, cnt[j]);
                 }
                 float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                for (int b = 0; b < cmax; b++) {
+                // half-warp h takes bins b = h, h + 2, ... of each filter
+                for (int b = h; b < nit; b += 2) {
 #pragma unroll
                     for (int j = 0; j < 4; j++)
-                        if (b < cnt[j]) acc[j] = fmaf(S.band_wt[b][m0 + j], P[lo[j] + b], acc[j]);
+                        if (b < cnt[j]) acc[j] = fmaf(S.t.band_wt[b][m0 + j], P[2 * (lo[j] + b)], acc[j]);
                 }
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
+                for (int j = 0; j < 4; j++) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 16);
+                // half 0 emits filters j = 0, 1, half 1 filters j = 2, 3
+#pragma unroll
+                for (int jj = 0; jj < 2; jj++) {
+                    const int j = 2 * h + jj;
+                    const float a = h ? acc[2 + jj] : acc[jj];
                     if (m0 + j < m1) {
-                        const float r = __log2f(fmaxf(acc[j], 1e-10f)) * log10_2;
+                        const float r = __log2f(fmaxf(a, 1e-10f)) * log10_2;
                         if (f < nf) lmax = fmaxf(lmax, r);
-                        ost[m0 + j] = r;
+                        ost[(m0 + j) ^ swz] = r;
                     }
                 }
             }
         }
-        __syncthreads();
+        if (cl.gslot >= 0) {
+            for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+            if (lane == 0) S.wmax[warp] = lmax;
+        }
+        __syncthreads();  // B4: staged rows and warp maxima written
         if (write_out) {
             const long long out_row = cl.out_row0 + (frame0 - cl.f_begin);
-            for (int i = tid; i < nf * 32; i += MEL2_THREADS) {
+            for (int i = tid; i < nf * 32; i += MEL4_THREADS) {
                 const int f = i >> 5, q = i & 31;
-                const float4 v = *reinterpret_cast<const float4 *>(S.xs[cur] + MEL3_OUT_LD * f + 4 * q);
+                float4 v = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(S.y[f >> 1]) + MEL4_STAGE +
+                                                             128 * (f & 1) + 4 * q);
+                if (f & 1) v = make_float4(v.z, v.w, v.x, v.y);
                 reinterpret_cast<float4 *>(out + (size_t)(out_row + f) * 128)[q] = v;
             }
         }
-        if (cl.gslot >= 0) {
-            for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-            if ((tid & 31) == 0) S.wmax[tid >> 5] = lmax;
-        }
-        __syncthreads();  // power read and buffers free for the next item
         if (cl.gslot >= 0 && tid == 0) {
             float m = S.wmax[0];
-            for (int i = 1; i < MEL2_THREADS / 32; i++) m = fmaxf(m, S.wmax[i]);
+            for (int i = 1; i < MEL4_WARPS; i++) m = fmaxf(m, S.wmax[i]);
             atomicMax(gmax_ord + cl.gslot, float_to_ordered(m));
         }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    cp_async_wait_all();
 }
 
 // In-place Whisper normalisation of rows [n_rows][128]: (max(x, g - 8) + 4) / 4.

@@ -65,7 +65,7 @@ struct moss_enc {
     HeadDev head{};
     float *pos = nullptr;
     MelTables *mel_tab = nullptr;
-    MelBandT *mel_tabt = nullptr;
+    Mel4Tab *mel4_tab = nullptr;
 
     // layer taps (moss_enc_set_taps): encoder layer per tap and its head set
     void *tap_wmem = nullptr;
@@ -435,6 +435,34 @@ static bool build_mel_tables(MelTables *t)
     return true;
 }
 
+// The persistent log-mel kernel's tables in its shared-memory layout: the
+// twiddles w^(n1 k2) at [k2][n1], the window, the filters' bin ranges and
+// weights (transposed), and the filter range of each warp, balanced by the
+// work of a filter in the kernel (its bins split over two half-warps, plus
+// the log and the store).
+static void build_mel4_tab(const MelTables &t, Mel4Tab *o)
+{
+    std::memset(o, 0, sizeof(Mel4Tab));
+    for (int k2 = 0; k2 < 20; k2++)
+        for (int n1 = 0; n1 < 21; n1++) o->tw[k2][n1] = n1 < 20 ? t.tw400[(n1 * k2) % 400] : make_float2(0.0f, 0.0f);
+    for (int i = 0; i < 400; i++) o->hann[i] = t.hann[i];
+    int cost[128], total = 0;
+    for (int m = 0; m < 128; m++) {
+        o->band_lo[m] = t.band_lo[m];
+        o->band_n[m] = t.band_n[m];
+        for (int b = 0; b < MEL_BAND; b++) o->band_wt[b][m] = t.band_w[m][b];
+        cost[m] = (t.band_n[m] + 1) / 2 + 2;
+        total += cost[m];
+    }
+    int w = 0, run = 0;
+    o->mpart[0] = 0;
+    for (int m = 0; m < 128; m++) {
+        run += cost[m];
+        while (w + 1 < MEL4_WARPS && run * MEL4_WARPS >= total * (w + 1)) o->mpart[++w] = m + 1;
+    }
+    while (w + 1 <= MEL4_WARPS) o->mpart[++w] = 128;
+}
+
 // ----------------------------------------------------------------- sizes
 
 extern "C" int64_t moss_enc_weight_count(int n_layers)
@@ -659,8 +687,8 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm_attr<128, EPI_F32>()));
     CUDA_TRY(h, (gemm_attr<128, EPI_BF16>()));
     CUDA_TRY(h, cudaFuncSetAttribute(window_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATTN_TC_SMEM));
-    CUDA_TRY(h, cudaFuncSetAttribute(logmel3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel3Smem)));
-    CUDA_TRY(h, cudaFuncSetAttribute(logmel3_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+    CUDA_TRY(h, cudaFuncSetAttribute(logmel4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel4Smem)));
+    CUDA_TRY(h, cudaFuncSetAttribute(logmel4_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     return MOSS_ENC_OK;
 }
 
@@ -720,7 +748,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     for (int l = 0; l < L; l++) o_layer[l] = take(layer_bytes);
     const HeadOff o_head = head_take(take);
     const size_t o_pos = take(4 * (size_t)CHUNK_TOKENS * D), o_mel = take(sizeof(MelTables));
-    const size_t o_melt = take(sizeof(MelBandT));
+    const size_t o_mel4 = take(sizeof(Mel4Tab));
     const size_t wtotal = off;
 
     std::vector<uint8_t> pk(wtotal, 0);
@@ -807,12 +835,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
             F32(o_pos)[t * D + D / 2 + i] = (float)std::cos(t * inv);
         }
     if (!build_mel_tables(reinterpret_cast<MelTables *>(pk.data() + o_mel))) return bail(MOSS_ENC_ERR_INVALID_ARG);
-    {
-        const MelTables *mt = reinterpret_cast<const MelTables *>(pk.data() + o_mel);
-        MelBandT *bt = reinterpret_cast<MelBandT *>(pk.data() + o_melt);
-        for (int m = 0; m < 128; m++)
-            for (int b = 0; b < MEL_BAND; b++) bt->w[b][m] = mt->band_w[m][b];
-    }
+    build_mel4_tab(*reinterpret_cast<const MelTables *>(pk.data() + o_mel), reinterpret_cast<Mel4Tab *>(pk.data() + o_mel4));
 
     if (cudaMalloc(&h->wmem, wtotal) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaMemcpy(h->wmem, pk.data(), wtotal, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
@@ -843,7 +866,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     h->head = head_bind(o_head, W);
     h->pos = (float *)(W + o_pos);
     h->mel_tab = (MelTables *)(W + o_mel);
-    h->mel_tabt = (MelBandT *)(W + o_melt);
+    h->mel4_tab = (Mel4Tab *)(W + o_mel4);
 
     // ---- workspace
     h->max_tokens = cfg->max_samples / 1280 + cfg->max_clips + 1;
@@ -943,14 +966,14 @@ static moss_enc_status launch_logmel(moss_enc *h, const MelClip *d_clips, int n_
                                      float *out, int write_out, int64_t total_frames)
 {
     if (n_clips <= 0 || max_frames <= 0) return MOSS_ENC_OK;
-    for (int c0 = 0; c0 < n_clips; c0 += MEL3_MAX_CLIPS) {
-        const int nc = std::min(MEL3_MAX_CLIPS, n_clips - c0);
-        const int64_t blocks = (int64_t)nc * ((max_frames + MEL2_FRAMES - 1) / MEL2_FRAMES);  // upper bound
-        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks, 2 * h->num_sms));
+    for (int c0 = 0; c0 < n_clips; c0 += MEL_MAX_CLIPS) {
+        const int nc = std::min(MEL_MAX_CLIPS, n_clips - c0);
+        const int64_t blocks = (int64_t)nc * ((max_frames + MEL4_FRAMES - 1) / MEL4_FRAMES);  // upper bound
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks, 4 * h->num_sms));
         Launch L(h, write_out ? "logmel" : "logmel_max", 0.0,
                  c0 == 0 ? 4.0 * 160 * (double)total_frames + (write_out ? 512.0 * total_frames : 0.0) : 0.0);
-        CUDA_TRY(h, launch_k(h, logmel3_kernel, dim3(grid), dim3(MEL2_THREADS), sizeof(Mel3Smem), d_clips + c0, nc,
-                             (const MelTables *)h->mel_tab, (const MelBandT *)h->mel_tabt, out, h->gmax_ord, write_out));
+        CUDA_TRY(h, launch_k(h, logmel4_kernel, dim3(grid), dim3(MEL4_THREADS), sizeof(Mel4Smem), d_clips + c0, nc,
+                             (const Mel4Tab *)h->mel4_tab, out, h->gmax_ord, write_out));
     }
     return MOSS_ENC_OK;
 }
