@@ -274,15 +274,27 @@ static constexpr int MEL4_SPAN = mel_span_pad(MEL4_SPAN_SAMPLES - 1) + 1;  // 29
 static constexpr int MEL4_YP = 402;
 static constexpr int MEL4_STAGE = 416;  // float offset of the staged log-mel rows inside a pair (Z[208] on)
 
+// The filterbank runs over groups of 4 consecutive filters (32 groups); a
+// warp takes a contiguous run of groups, balanced by their work.  Group g:
+// lo[j] = first bin of filter 4 g + j, nit = bin pairs to visit (the widest
+// filter's bins, two per step: one per half-warp), and w4[woff + 2 it + h] =
+// the four filters' weights of bin lo[j] + 2 it + h (zero past a filter's
+// last bin).
+static constexpr int MEL4_GROUPS = 32;
+static constexpr int MEL4_MAXIT = (MEL_BAND + 1) / 2;
+struct Mel4Group {
+    int lo[4];
+    int nit, woff, pad0, pad1;
+};
+
 // Constant tables of the kernel, built on the host in their shared-memory
 // layout and copied in whole at the start.
 struct alignas(16) Mel4Tab {
     float2 tw[20][21];  // w^(n1 k2) at [k2][n1], w = exp(-2 pi i / 400)
     float hann[400];
-    int band_lo[128];   // first nonzero bin of filter m
-    int band_n[128];    // nonzero bins of filter m (<= MEL_BAND)
-    float band_wt[MEL_BAND][129];  // weight of bin band_lo[m] + b at [b][m] (odd pitch: rows b, b + 1 on different banks)
-    int mpart[8];       // filters of warp w: [mpart[w], mpart[w+1])
+    Mel4Group grp[MEL4_GROUPS];
+    float4 w4[MEL4_GROUPS * MEL4_MAXIT * 2];
+    int gpart[8];  // groups of warp w: [gpart[w], gpart[w+1])
 };
 static_assert(sizeof(Mel4Tab) % 16 == 0, "the tables are copied in 16-byte pieces");
 
@@ -451,40 +463,40 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
         __syncthreads();  // B3: power of every frame in place: frame f, bin k at float 2 k + (f & 1) of pair f / 2
         float lmax = -INFINITY;
         {
+            // lane = frame f, half-warp h takes bins lo + 2 it + h of each filter
+            // of the group; bins a little past a filter's last one carry zero
+            // weight and read finite spectrum values (Z[k], k > 200, is written
+            // by pass 2 of every active pair)
             const int f = lane & 15, h = lane >> 4;
-            const float *P = reinterpret_cast<const float *>(S.y[f >> 1]) + (f & 1);
+            const float *P = reinterpret_cast<const float *>(S.y[f >> 1]) + (f & 1) + 2 * h;
             float *ost = reinterpret_cast<float *>(S.y[f >> 1]) + MEL4_STAGE + 128 * (f & 1);
             const int swz = 2 * (f & 1);  // odd frames' columns XOR 2: the pair's two rows on different banks
-            const int m1 = S.t.mpart[warp + 1];
-            for (int m0 = S.t.mpart[warp]; m0 < m1; m0 += 4) {
-                int lo[4], cnt[4], nit = 0;
+            const int g1 = S.t.gpart[warp + 1];
+            for (int g = S.t.gpart[warp]; g < g1; g++) {
+                const Mel4Group G = S.t.grp[g];
+                const float *p0 = P + 2 * G.lo[0], *p1 = P + 2 * G.lo[1], *p2 = P + 2 * G.lo[2], *p3 = P + 2 * G.lo[3];
+                const float4 *wv = S.t.w4 + G.woff + h;
+                float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const bool in = m0 + j < m1;
-                    lo[j] = in ? S.t.band_lo[m0 + j] : 0;
-                    cnt[j] = in ? S.t.band_n[m0 + j] : 0;
-                    nit = max(nit, cnt[j]);
+                for (int it = 0; it < MEL4_MAXIT; it++) {
+                    if (it >= G.nit) break;
+                    const float4 w = wv[2 * it];
+                    a0 = fmaf(w.x, p0[4 * it], a0);
+                    a1 = fmaf(w.y, p1[4 * it], a1);
+                    a2 = fmaf(w.z, p2[4 * it], a2);
+                    a3 = fmaf(w.w, p3[4 * it], a3);
                 }
-                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                // half-warp h takes bins b = h, h + 2, ... of each filter
-                for (int b = h; b < nit; b += 2) {
-#pragma unroll
-                    for (int j = 0; j < 4; j++)
-                        if (b < cnt[j]) acc[j] = fmaf(S.t.band_wt[b][m0 + j], P[2 * (lo[j] + b)], acc[j]);
-                }
-#pragma unroll
-                for (int j = 0; j < 4; j++) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 16);
-                // half 0 emits filters j = 0, 1, half 1 filters j = 2, 3
-#pragma unroll
-                for (int jj = 0; jj < 2; jj++) {
-                    const int j = 2 * h + jj;
-                    const float a = h ? acc[2 + jj] : acc[jj];
-                    if (m0 + j < m1) {
-                        const float r = __log2f(fmaxf(a, 1e-10f)) * log10_2;
-                        if (f < nf) lmax = fmaxf(lmax, r);
-                        ost[(m0 + j) ^ swz] = r;
-                    }
-                }
+                a0 += __shfl_xor_sync(0xffffffffu, a0, 16);
+                a1 += __shfl_xor_sync(0xffffffffu, a1, 16);
+                a2 += __shfl_xor_sync(0xffffffffu, a2, 16);
+                a3 += __shfl_xor_sync(0xffffffffu, a3, 16);
+                // half 0 emits filters 4 g, 4 g + 1, half 1 filters 4 g + 2, 4 g + 3
+                const float e0 = h ? a2 : a0, e1 = h ? a3 : a1;
+                const float r0 = __log2f(fmaxf(e0, 1e-10f)) * log10_2, r1 = __log2f(fmaxf(e1, 1e-10f)) * log10_2;
+                if (f < nf) lmax = fmaxf(lmax, fmaxf(r0, r1));
+                const int m = 4 * g + 2 * h;
+                ost[m ^ swz] = r0;
+                ost[(m + 1) ^ swz] = r1;
             }
         }
         if (cl.gslot >= 0) {

@@ -436,31 +436,49 @@ static bool build_mel_tables(MelTables *t)
 }
 
 // The persistent log-mel kernel's tables in its shared-memory layout: the
-// twiddles w^(n1 k2) at [k2][n1], the window, the filters' bin ranges and
-// weights (transposed), and the filter range of each warp, balanced by the
-// work of a filter in the kernel (its bins split over two half-warps, plus
-// the log and the store).
-static void build_mel4_tab(const MelTables &t, Mel4Tab *o)
+// twiddles w^(n1 k2) at [k2][n1], the window, the filterbank as 32 groups of
+// 4 filters (first bins, bin pairs to visit, the weights of each bin pair as
+// float4 over the group's filters), and the groups of each warp, balanced by
+// their work in the kernel (a fixed part for the shuffles, logs and stores,
+// plus the bin pairs).
+static bool build_mel4_tab(const MelTables &t, Mel4Tab *o)
 {
     std::memset(o, 0, sizeof(Mel4Tab));
     for (int k2 = 0; k2 < 20; k2++)
         for (int n1 = 0; n1 < 21; n1++) o->tw[k2][n1] = n1 < 20 ? t.tw400[(n1 * k2) % 400] : make_float2(0.0f, 0.0f);
     for (int i = 0; i < 400; i++) o->hann[i] = t.hann[i];
-    int cost[128], total = 0;
-    for (int m = 0; m < 128; m++) {
-        o->band_lo[m] = t.band_lo[m];
-        o->band_n[m] = t.band_n[m];
-        for (int b = 0; b < MEL_BAND; b++) o->band_wt[b][m] = t.band_w[m][b];
-        cost[m] = (t.band_n[m] + 1) / 2 + 2;
-        total += cost[m];
+    int cost[MEL4_GROUPS], total = 0, woff = 0;
+    for (int g = 0; g < MEL4_GROUPS; g++) {
+        Mel4Group &G = o->grp[g];
+        int nmax = 0;
+        for (int j = 0; j < 4; j++) {
+            G.lo[j] = t.band_lo[4 * g + j];
+            nmax = std::max(nmax, t.band_n[4 * g + j]);
+        }
+        G.nit = (nmax + 1) / 2;
+        G.woff = woff;
+        for (int it = 0; it < G.nit; it++)
+            for (int h = 0; h < 2; h++) {
+                float w[4];
+                for (int j = 0; j < 4; j++) {
+                    const int b = 2 * it + h, m = 4 * g + j;
+                    w[j] = b < t.band_n[m] ? t.band_w[m][b] : 0.0f;
+                }
+                o->w4[woff + 2 * it + h] = make_float4(w[0], w[1], w[2], w[3]);
+            }
+        woff += 2 * G.nit;
+        if (woff > MEL4_GROUPS * MEL4_MAXIT * 2) return false;
+        cost[g] = 40 + 10 * G.nit;
+        total += cost[g];
     }
     int w = 0, run = 0;
-    o->mpart[0] = 0;
-    for (int m = 0; m < 128; m++) {
-        run += cost[m];
-        while (w + 1 < MEL4_WARPS && run * MEL4_WARPS >= total * (w + 1)) o->mpart[++w] = m + 1;
+    o->gpart[0] = 0;
+    for (int g = 0; g < MEL4_GROUPS; g++) {
+        run += cost[g];
+        while (w + 1 < MEL4_WARPS && run * MEL4_WARPS >= total * (w + 1)) o->gpart[++w] = g + 1;
     }
-    while (w + 1 <= MEL4_WARPS) o->mpart[++w] = 128;
+    while (w + 1 <= MEL4_WARPS) o->gpart[++w] = MEL4_GROUPS;
+    return true;
 }
 
 // ----------------------------------------------------------------- sizes
@@ -835,7 +853,8 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
             F32(o_pos)[t * D + D / 2 + i] = (float)std::cos(t * inv);
         }
     if (!build_mel_tables(reinterpret_cast<MelTables *>(pk.data() + o_mel))) return bail(MOSS_ENC_ERR_INVALID_ARG);
-    build_mel4_tab(*reinterpret_cast<const MelTables *>(pk.data() + o_mel), reinterpret_cast<Mel4Tab *>(pk.data() + o_mel4));
+    if (!build_mel4_tab(*reinterpret_cast<const MelTables *>(pk.data() + o_mel), reinterpret_cast<Mel4Tab *>(pk.data() + o_mel4)))
+        return bail(MOSS_ENC_ERR_INVALID_ARG);
 
     if (cudaMalloc(&h->wmem, wtotal) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaMemcpy(h->wmem, pk.data(), wtotal, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
