@@ -254,7 +254,8 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip 
 //  mel:    lane = frame (16), the two half-warps take the even and odd bins
 //          of the same filters (one shuffle adds them), warp w a range of
 //          filters balanced by their bins; log-mel rows are staged in the
-//          pair's dead upper half (Z[k], k > 200) and stored whole.
+//          pair's dead upper half (Z[k], k > 200), the pair's two rows
+//          together, and leave as one bulk copy per pair.
 static constexpr int MEL_MAX_CLIPS = 128;  // clips per launch (the host splits larger batches)
 static constexpr int MEL4_FRAMES = 16;
 static constexpr int MEL4_THREADS = 160;
@@ -272,7 +273,7 @@ static constexpr int MEL4_SPAN = mel_span_pad(MEL4_SPAN_SAMPLES - 1) + 1;  // 29
 // Pair pitch of the exchange buffer (float2): 402 = 4 words mod 32 between
 // consecutive pairs, so a half-warp's 8 pairs x 2 columns hit distinct banks.
 static constexpr int MEL4_YP = 402;
-static constexpr int MEL4_STAGE = 416;  // float offset of the staged log-mel rows inside a pair (Z[208] on)
+static constexpr int MEL4_STAGE = 416;  // float offset of the staged log-mel rows inside a pair (Z[208] on; 16-byte aligned)
 
 // The filterbank runs over groups of 4 consecutive filters (32 groups); a
 // warp takes a contiguous run of groups, balanced by their work.  Group g:
@@ -313,6 +314,15 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from
+// shared to global memory by the async proxy, in this thread's bulk group.
+__device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst), "r"(smem_u32(smem_src)),
+                 "r"(bytes)
+                 : "memory");
+}
 
 // Locate item `item` among the clips' blocks: returns false past the end.
 __device__ __forceinline__ bool mel4_item(const int *first_block, const MelClip *clips, int n_clips, int item, int &c,
@@ -375,11 +385,15 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
         __syncthreads();
     }
 
-    // span loader: async 16-byte copies for interior blocks (returns true),
-    // nothing for edge blocks (loaded synchronously when their turn comes)
-    auto prefetch = [&](int item) -> bool {
-        int c, frame0, nf;
-        if (!mel4_item(S.first_block, clips, n_clips, item, c, frame0, nf)) return true;
+    // span loader: locates `item` (nc < 0 past the end) and starts async
+    // 16-byte copies of its span if it lies inside the clip (returns true);
+    // edge blocks are loaded synchronously when their turn comes
+    auto prefetch = [&](int item, int &nc, int &nframe0, int &nnf) -> bool {
+        if (!mel4_item(S.first_block, clips, n_clips, item, nc, nframe0, nnf)) {
+            nc = -1;
+            return true;
+        }
+        const int c = nc, frame0 = nframe0, nf = nnf;
         const MelClip &cl = clips[c];
         if (!mel_span_interior(cl, frame0, nf)) return false;
         const float4 *src = reinterpret_cast<const float4 *>(cl.pcm + (160LL * frame0 - 200));
@@ -390,13 +404,13 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
     };
 
     const float log10_2 = 0.30102999566398120f;
+    const bool out_aligned = (reinterpret_cast<uintptr_t>(out) & 15) == 0;
     const int tp = tid & 7, tj = tid >> 3;
     const float *hw = S.t.hann + tj;  // window value of sample tj + 20 n2: hw[20 n2]
-    bool ready = prefetch(blockIdx.x);
+    int c, frame0, nf;
+    bool ready = prefetch(blockIdx.x, c, frame0, nf);
     cp_async_commit();
-    for (int item = blockIdx.x;; item += gridDim.x) {
-        int c, frame0, nf;
-        if (!mel4_item(S.first_block, clips, n_clips, item, c, frame0, nf)) break;
+    for (int item = blockIdx.x; c >= 0; item += gridDim.x) {
         const MelClip cl = clips[c];
         if (!ready) {  // edge block: reflect-padded load now (nothing is in flight into the span)
             const long long s0 = 160LL * frame0 - 200;
@@ -405,7 +419,8 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
                 S.xs[mel_span_pad(i)] = __ldg(cl.pcm + reflect_index(s0 + i, cl.n));
         }
         cp_async_wait_all();
-        __syncthreads();  // B0: span in place; the previous block's staged rows are stored
+        if (write_out && out_aligned && tid < MEL4_PAIRS) bulk_wait_read();  // the previous rows have left the staging area
+        __syncthreads();  // B0: span in place; staging area free
 
         const int npairs = (nf + 1) / 2;
         float2 *Y = S.y[tp];
@@ -427,7 +442,8 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
             for (int k2 = 1; k2 < 20; k2++) yr[k2] = cmul(v[k2], S.t.tw[k2][tj]);  // w^0 = 1 exactly for tj = 0
         }
         __syncthreads();  // B1: pass-1 rows written; the span is dead
-        ready = prefetch(item + gridDim.x);
+        int c_next, frame0_next, nf_next;
+        ready = prefetch(item + gridDim.x, c_next, frame0_next, nf_next);
         cp_async_commit();
         if (tp < npairs) {
             // pass 2: 20-point DFT over n1 -> Z[20 k1 + tj], in place (own column)
@@ -470,7 +486,6 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
             const int f = lane & 15, h = lane >> 4;
             const float *P = reinterpret_cast<const float *>(S.y[f >> 1]) + (f & 1) + 2 * h;
             float *ost = reinterpret_cast<float *>(S.y[f >> 1]) + MEL4_STAGE + 128 * (f & 1);
-            const int swz = 2 * (f & 1);  // odd frames' columns XOR 2: the pair's two rows on different banks
             const int g1 = S.t.gpart[warp + 1];
             for (int g = S.t.gpart[warp]; g < g1; g++) {
                 const Mel4Group G = S.t.grp[g];
@@ -495,23 +510,30 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
                 const float r0 = __log2f(fmaxf(e0, 1e-10f)) * log10_2, r1 = __log2f(fmaxf(e1, 1e-10f)) * log10_2;
                 if (f < nf) lmax = fmaxf(lmax, fmaxf(r0, r1));
                 const int m = 4 * g + 2 * h;
-                ost[m ^ swz] = r0;
-                ost[(m + 1) ^ swz] = r1;
+                ost[m] = r0;
+                ost[m + 1] = r1;
             }
         }
         if (cl.gslot >= 0) {
             for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
             if (lane == 0) S.wmax[warp] = lmax;
         }
+        fence_async_smem();  // the staged rows are read by the bulk copies below
         __syncthreads();  // B4: staged rows and warp maxima written
-        if (write_out) {
+        if (write_out && out_aligned) {
+            if (tid < npairs) {
+                // frames 2 tid, 2 tid + 1: consecutive output rows, staged back to back
+                const long long row = cl.out_row0 + (frame0 - cl.f_begin) + 2 * tid;
+                const uint32_t bytes = (2 * tid + 1 < nf ? 2 : 1) * 128 * 4;
+                bulk_store(out + (size_t)row * 128, reinterpret_cast<const float *>(S.y[tid]) + MEL4_STAGE, bytes);
+                bulk_commit();
+            }
+        } else if (write_out) {  // an output buffer without 16-byte alignment: plain stores
             const long long out_row = cl.out_row0 + (frame0 - cl.f_begin);
-            for (int i = tid; i < nf * 32; i += MEL4_THREADS) {
-                const int f = i >> 5, q = i & 31;
-                float4 v = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(S.y[f >> 1]) + MEL4_STAGE +
-                                                             128 * (f & 1) + 4 * q);
-                if (f & 1) v = make_float4(v.z, v.w, v.x, v.y);
-                reinterpret_cast<float4 *>(out + (size_t)(out_row + f) * 128)[q] = v;
+            for (int i = tid; i < nf * 128; i += MEL4_THREADS) {
+                const int f = i >> 7;
+                out[(size_t)(out_row + f) * 128 + (i & 127)] =
+                    reinterpret_cast<const float *>(S.y[f >> 1])[MEL4_STAGE + 128 * (f & 1) + (i & 127)];
             }
         }
         if (cl.gslot >= 0 && tid == 0) {
@@ -519,8 +541,12 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
             for (int i = 1; i < MEL4_WARPS; i++) m = fmaxf(m, S.wmax[i]);
             atomicMax(gmax_ord + cl.gslot, float_to_ordered(m));
         }
+        c = c_next;
+        frame0 = frame0_next;
+        nf = nf_next;
     }
     cp_async_wait_all();
+    if (write_out && out_aligned && tid < MEL4_PAIRS) bulk_wait_all();
 }
 
 // In-place Whisper normalisation of rows [n_rows][128]: (max(x, g - 8) + 4) / 4.

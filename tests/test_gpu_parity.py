@@ -56,6 +56,25 @@ def test_logmel_silence_and_empty():
     assert mel.shape == (0, 128)
 
 
+def test_logmel_output_without_16_byte_alignment():
+    # the rows leave by bulk copies only when the output buffer allows them;
+    # a float buffer at a 4-byte offset takes the plain-store path, same values
+    import ctypes
+    enc = encoder(1, 600_000)
+    pcm = dev(synth.pcm_tones(3, 48000))
+    ref, _ = enc.logmel(pcm)
+    buf = torch.zeros(300 * 128 + 1, dtype=torch.float32, device="cuda")
+    view = buf[1:]
+    mx = torch.empty(1, dtype=torch.float32, device="cuda")
+    c = enc._clip(pcm)
+    nf = ctypes.c_int64()
+    enc._check(binding.lib().moss_enc_logmel(enc.h, ctypes.byref(c), ctypes.c_void_p(view.data_ptr()),
+                                             ctypes.byref(nf), ctypes.c_void_p(mx.data_ptr())))
+    torch.cuda.synchronize()
+    assert nf.value == 300 and float(buf[0]) == 0.0
+    np.testing.assert_array_equal(view.view(300, 128).cpu().numpy(), ref.cpu().numpy())
+
+
 def test_logmel_range_uses_whole_clip_max():
     enc = encoder(1, 600_000)
     n = 128000 * 3 + 5000
