@@ -246,14 +246,16 @@ __global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip 
 //          400-point twiddle w^(tj k2), into row tj of the pair's buffer
 //          (row pitch 20: Z[20 k1 + k2] ends up at element 20 k1 + k2);
 //          the block's PCM span is then dead, and the next block's span is
-//          fetched into it with cp.async while this block finishes;
+//          fetched into it with cp.async while this block finishes (blocks
+//          at the clip ends copy each sample from its reflected source, so
+//          no block waits on a synchronous load);
 //  pass 2: 20-point DFT over the rows of column tj, in place;
 //  power:  bins k = tj + 20 i of both frames from Z[k] and Z[400 - k]; the
 //          power pair (a, b) replaces Z[k] in place (the locations a thread
 //          reads are its own, so the phase needs no inner barrier);
 //  mel:    lane = frame (16), the two half-warps take the even and odd bins
-//          of the same filters (one shuffle adds them), warp w a range of
-//          filters balanced by their bins; log-mel rows are staged in the
+//          of the same group of 4 filters (one shuffle adds them), warp w a
+//          run of groups balanced by their work; log-mel rows are staged in the
 //          pair's dead upper half (Z[k], k > 200), the pair's two rows
 //          together, and leave as one bulk copy per pair.
 static constexpr int MEL_MAX_CLIPS = 128;  // clips per launch (the host splits larger batches)
@@ -349,6 +351,31 @@ __device__ __forceinline__ bool mel_span_interior(const MelClip &cl, int frame0,
     return s0 >= 0 && s0 + 160LL * (nf - 1) + 400 <= cl.n && ((reinterpret_cast<uintptr_t>(cl.pcm) & 15) == 0);
 }
 
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+
+// Starts the asynchronous copy of the PCM span of frames frame0 .. frame0 +
+// nf - 1 into xs (padded layout): 16-byte pieces when the span lies inside
+// the clip, else one 4-byte copy per sample from its reflect-padded source.
+template <int THREADS>
+__device__ __forceinline__ void mel_span_fetch(float *xs, const MelClip &cl, int frame0, int nf, int tid)
+{
+    const long long s0 = 160LL * frame0 - 200;
+    const int span = 160 * (nf - 1) + 400;
+    if (mel_span_interior(cl, frame0, nf)) {
+        const float4 *src = reinterpret_cast<const float4 *>(cl.pcm + s0);
+        for (int i = tid; i < span / 4; i += THREADS) cp_async16(reinterpret_cast<float4 *>(xs) + i + 5 * (i / 80), src + i);
+    } else {
+        for (int i = tid; i < span; i += THREADS) {
+            long long j = s0 + i;
+            if (j < 0 || j >= cl.n) j = reflect_index(j, cl.n);
+            cp_async4(xs + mel_span_pad(i), cl.pcm + j);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip *__restrict__ clips, int n_clips,
                                                                   const Mel4Tab *__restrict__ tab,
                                                                   float *__restrict__ out, int *gmax_ord,
@@ -385,22 +412,14 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
         __syncthreads();
     }
 
-    // span loader: locates `item` (nc < 0 past the end) and starts async
-    // 16-byte copies of its span if it lies inside the clip (returns true);
-    // edge blocks are loaded synchronously when their turn comes
-    auto prefetch = [&](int item, int &nc, int &nframe0, int &nnf) -> bool {
+    // span loader: locates `item` (nc < 0 past the end) and starts the
+    // asynchronous copy of its span
+    auto prefetch = [&](int item, int &nc, int &nframe0, int &nnf) {
         if (!mel4_item(S.first_block, clips, n_clips, item, nc, nframe0, nnf)) {
             nc = -1;
-            return true;
+            return;
         }
-        const int c = nc, frame0 = nframe0, nf = nnf;
-        const MelClip &cl = clips[c];
-        if (!mel_span_interior(cl, frame0, nf)) return false;
-        const float4 *src = reinterpret_cast<const float4 *>(cl.pcm + (160LL * frame0 - 200));
-        const int n4 = (160 * (nf - 1) + 400) / 4;
-        for (int i = tid; i < n4; i += MEL4_THREADS)
-            cp_async16(reinterpret_cast<float4 *>(S.xs) + i + 5 * (i / 80), src + i);
-        return true;
+        mel_span_fetch<MEL4_THREADS>(S.xs, clips[nc], nframe0, nnf, tid);
     };
 
     const float log10_2 = 0.30102999566398120f;
@@ -408,16 +427,10 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
     const int tp = tid & 7, tj = tid >> 3;
     const float *hw = S.t.hann + tj;  // window value of sample tj + 20 n2: hw[20 n2]
     int c, frame0, nf;
-    bool ready = prefetch(blockIdx.x, c, frame0, nf);
+    prefetch(blockIdx.x, c, frame0, nf);
     cp_async_commit();
     for (int item = blockIdx.x; c >= 0; item += gridDim.x) {
         const MelClip cl = clips[c];
-        if (!ready) {  // edge block: reflect-padded load now (nothing is in flight into the span)
-            const long long s0 = 160LL * frame0 - 200;
-            const int span = 160 * (nf - 1) + 400;
-            for (int i = tid; i < span; i += MEL4_THREADS)
-                S.xs[mel_span_pad(i)] = __ldg(cl.pcm + reflect_index(s0 + i, cl.n));
-        }
         cp_async_wait_all();
         if (write_out && out_aligned && tid < MEL4_PAIRS) bulk_wait_read();  // the previous rows have left the staging area
         __syncthreads();  // B0: span in place; staging area free
@@ -443,7 +456,7 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
         }
         __syncthreads();  // B1: pass-1 rows written; the span is dead
         int c_next, frame0_next, nf_next;
-        ready = prefetch(item + gridDim.x, c_next, frame0_next, nf_next);
+        prefetch(item + gridDim.x, c_next, frame0_next, nf_next);
         cp_async_commit();
         if (tp < npairs) {
             // pass 2: 20-point DFT over n1 -> Z[20 k1 + tj], in place (own column)
