@@ -111,6 +111,7 @@ struct moss_enc {
     void *d_tab_graph = nullptr;
     cudaGraphExec_t graph_exec = nullptr;
     std::vector<uint8_t> graph_key;
+    std::vector<uint8_t> last_key;  // the previous graphable request (run launch by launch)
     int64_t graph_launches = 0;
 };
 
@@ -1406,22 +1407,27 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     P.g_off3 = std::move(g_off3);
     P.g_n3 = std::move(g_n3);
 
-    // Whole forwards run as one CUDA graph: captured the first time a request
-    // is seen, replayed while the same request (clips, ranges, output, stage)
-    // comes back.  The graph reads its own copy of the tables.
+    // Whole forwards run as one CUDA graph once a request repeats: the second
+    // consecutive call with the same request (clips, ranges, output, taps)
+    // captures it, later ones replay it.  A stream of different requests (the
+    // pieces of a long clip) runs launch by launch and never pays for a
+    // capture.  The graph reads its own copy of the tables.
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     CUDA_TRY(h, cudaStreamIsCapturing(h->stream, &cs));
+    const int n_taps = (int)h->tap_layers.size();
     const bool graphable = stage == MOSS_ENC_STAGE_ADAPTER && !h->profiling && h->stream != nullptr &&
                            cs == cudaStreamCaptureStatusNone;
-    if (!graphable) {
-        TRY(tab_upload(h));
-        return forward_launch(h, P, static_cast<uint8_t *>(h->d_tab), stage, out, tap_out);
-    }
-    const int n_taps = (int)h->tap_layers.size();
-    if (h->graph_exec && h->graph_key == request_key(clips, n_clips, out, tap_out, n_taps)) {
+    std::vector<uint8_t> key;
+    if (graphable) key = request_key(clips, n_clips, out, tap_out, n_taps);
+    if (graphable && h->graph_exec && h->graph_key == key) {
         h->launches += h->graph_launches;
         CUDA_TRY(h, cudaGraphLaunch(h->graph_exec, h->stream));
         return MOSS_ENC_OK;
+    }
+    if (!graphable || key != h->last_key) {
+        if (graphable) h->last_key = std::move(key);
+        TRY(tab_upload(h));
+        return forward_launch(h, P, static_cast<uint8_t *>(h->d_tab), stage, out, tap_out);
     }
     if (h->graph_exec) {
         cudaGraphExecDestroy(h->graph_exec);
@@ -1445,7 +1451,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         h->graph_exec = nullptr;
         return fail(h, MOSS_ENC_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(ie));
     }
-    h->graph_key = request_key(clips, n_clips, out, tap_out, n_taps);
+    h->graph_key = std::move(key);
     h->graph_launches = h->launches - launches0;
     CUDA_TRY(h, cudaGraphLaunch(h->graph_exec, h->stream));
     return MOSS_ENC_OK;
@@ -1482,6 +1488,7 @@ extern "C" moss_enc_status moss_enc_set_taps(moss_enc *h, const int *layers, int
         cudaGraphExecDestroy(h->graph_exec);
         h->graph_exec = nullptr;
         h->graph_key.clear();
+        h->last_key.clear();
     }
     if (h->tap_wmem) {
         cudaFree(h->tap_wmem);

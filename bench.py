@@ -408,6 +408,102 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_streamed(args):
+    """The 60-min clip encoded as a stream of 64 s pieces (1,024,000 samples,
+    the last 256,000): a step is the whole-clip log-mel maximum (one pass)
+    and the 57 piece forwards against it, each piece reading its 200-sample
+    halo from the whole clip.  Reports sustained audio-seconds per second and
+    the device memory the encoder holds (weights + workspace for one piece)
+    beside the resident clip and its rows.  Weak scaling: every rank streams
+    its own clip."""
+    import torch
+
+    from audio_encoder_b200 import binding
+
+    rank, world, dist = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    desc, clips, n_layers = workload_clips("clip_60min_streamed")
+    pcm = clips[0]
+    n = pcm.size
+    piece = 1_024_000
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    stream = torch.cuda.Stream()
+    enc = binding.Encoder(synth.make_weights(n_layers), n_layers, max_samples=piece, max_clips=1,
+                          out_dtype=binding.OUT_BF16, stream=stream)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    tokens = binding.num_tokens(n)
+    with torch.cuda.stream(stream):
+        x = torch.from_numpy(pcm).to(dev)
+        out = torch.empty((tokens, 2048), dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    ranges = []
+    r0 = 0
+    for b in range(0, n, piece):
+        e = min(b + piece, n)
+        t = binding.range_tokens(n, b, e)
+        ranges.append((b, e, r0, r0 + t))
+        r0 += t
+    assert r0 == tokens
+    torch.cuda.synchronize()
+
+    def step():
+        with torch.cuda.stream(stream):
+            lm = enc.log_max(x)
+            for b, e, o0, o1 in ranges:
+                enc.forward([(x, b, e, lm)], out=out[o0:o1])
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    enc.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = enc.launch_count()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(dev.index) as clk:
+        for i in range(args.steps):
+            with torch.cuda.stream(stream):
+                flush.fill_(float(i))
+                ev[i][0].record(stream)
+            step()
+            with torch.cuda.stream(stream):
+                ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    launches = enc.launch_count() - launches0
+    total_ms = reduce_max(float(sum(a.elapsed_time(c) for a, c in ev)), dist, dev)
+    ms = total_ms / args.steps
+    audio_s = n / 16000.0
+    pk = peaks()
+    tflops = model_flops(tokens, n_layers) / (ms / 1e3) / 1e12
+    if rank == 0:
+        line = {
+            "metric": "audio-sec encoded/sec", "value": weak_scaling_throughput(world, audio_s, ms),
+            "unit": "audio-s/s", "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded PCM, random-init bf16 weights)",
+            "tokens_per_s": weak_scaling_throughput(world, tokens, ms),
+            "model_tflops": tflops, "tc_roofline_frac_sustained": tflops / pk["bf16_sus"],
+            "config": {"workload": "clip_60min_streamed", "description": desc, "pieces": len(ranges),
+                       "piece_samples": piece, "audio_s_per_gpu": audio_s, "tokens_per_gpu": tokens,
+                       "layers": n_layers, "out_dtype": "bf16",
+                       "encoder_device_bytes": int(free0 - free1),
+                       "clip_and_rows_device_bytes": int(4 * n + 2 * tokens * 2048),
+                       "l2": "512 MB buffer written between timed steps (outside the events)",
+                       "parallelism": f"dp{world}" if world > 1 else "single"},
+            "gpu_launches": launches,
+            "e2e": None,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    enc.close()
+    if dist:
+        dist.destroy_process_group()
+
+
 def run_sharded(args):
     """One long clip split over the ranks by whole 800-frame chunks
     (audio_encoder_b200.shard): a step is each rank's log-mel maximum over its
@@ -508,6 +604,8 @@ def main():
         run_reference(args)
     elif args.shard_clip:
         run_sharded(args)
+    elif args.workload == "clip_60min_streamed":
+        run_streamed(args)
     else:
         run_ours(args)
 

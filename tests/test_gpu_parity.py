@@ -304,27 +304,41 @@ def test_capacity_and_range_errors():
 
 
 def test_graph_replay_matches_eager_launches(tiny_case):
-    # On a non-default stream a repeated request replays one captured CUDA
-    # graph; with profiling on the same request runs launch by launch.
+    # On a non-default stream a request that repeats the previous one is
+    # captured as one CUDA graph and replayed after that; a new request runs
+    # launch by launch (no capture for a stream of distinct requests); with
+    # profiling on, every request runs launch by launch.
     pcm, out, _ = tiny_case
     s = torch.cuda.Stream()
     enc = binding.Encoder(weights(4), 4, 600_000, 2, stream=s)
     xa, xb = dev(pcm), dev(synth.pcm_tones(8, 40000))
+    with torch.cuda.stream(s):
+        ya = torch.empty((13, 2048), dtype=torch.float32, device="cuda")
+        yb = torch.empty((13 + binding.num_tokens(40000), 2048), dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
-    ya1, _ = enc.forward([xa])        # captured
-    ya2, _ = enc.forward([xa])        # replayed
-    yb1, _ = enc.forward([xa, xb])    # another request: captured again
-    enc.profile_enable(2000)
-    ya3, _ = enc.forward([xa])        # launched one by one
-    yb2, _ = enc.forward([xa, xb])
-    stats = enc.profile_read()
-    enc.profile_enable(0)
+    got = []
+    with torch.cuda.stream(s):        # the copies below follow the forwards on their stream
+        for _ in range(3):            # launched, captured, replayed
+            enc.forward([xa], out=ya)
+            got.append(ya.clone())
+        enc.forward([xa, xb], out=yb)  # a new request: launched
+        yb1 = yb.clone()
+        enc.forward([xa], out=ya)     # the captured request again: replayed
+        got.append(ya.clone())
+        enc.profile_enable(2000)
+        enc.forward([xa], out=ya)     # launched one by one
+        got.append(ya.clone())
+        enc.forward([xa, xb], out=yb)
+        stats = enc.profile_read()
+        enc.profile_enable(0)
     enc.synchronize()
-    assert torch.equal(ya1, ya2) and torch.equal(ya1, ya3)
-    assert torch.equal(yb1, yb2)
-    assert torch.equal(yb1[:13], ya1)
+    torch.cuda.synchronize()
+    for g in got[1:]:
+        assert torch.equal(got[0], g)
+    assert torch.equal(yb1, yb)
+    assert torch.equal(yb1[:13], got[0])
     assert "gemm_fc1" in stats and stats["gemm_fc1"]["launches"] == 2 * 4
-    assert_rows_close(ya1.cpu().numpy(), out, "graph rows")
+    assert_rows_close(got[0].cpu().numpy(), out, "graph rows")
     enc.close()
 
 

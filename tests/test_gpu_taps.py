@@ -96,8 +96,8 @@ def test_taps_shared_weights_equal_final_rows_at_last_layer():
 
 def test_taps_batch_ragged_and_graph_replay():
     # two clips (3 + 2 windows, ragged tails: 588 rows over three 256-row
-    # tiles), own weights, on a side stream so that the forward runs as a
-    # CUDA graph; the second call replays it
+    # tiles), own weights, on a side stream: the first call runs launch by
+    # launch, the repeated one is captured as a CUDA graph and run from it
     n_layers, layers = 4, [1, 3]
     clips = [synth.pcm_30s(1, 480000), synth.pcm_tones(5, 17 * 16000 + 123)]
     s = torch.cuda.Stream()
