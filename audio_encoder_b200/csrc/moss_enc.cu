@@ -688,6 +688,7 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm2_attr<256, EPI_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm2_attr<128, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_SWIGLU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_F32>()));
@@ -1252,6 +1253,15 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
     CUtensorMap tm_qkv;  // Q, K, V slices of one window and head: ATTN_ROWS rows x 64
     if (!tmap_2d(&tm_qkv, h->qkv, (uint64_t)DQKV, (uint64_t)T, (uint64_t)DQKV * 2, 64, ATTN_ROWS))
         return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (qkv)");
+    // The N = 1280 residual GEMMs (out-proj, FC2) on a small batch have few
+    // 320-wide tiles (ceil(T / 256) x 4) for the SMs; 128-wide tiles give them
+    // 2.5 times as many.  The tile width does not change any output element's
+    // arithmetic, so a clip's rows are the same at every batch size.
+    const bool narrow = 4 * ((T + 255) / 256) < h->num_sms / 4;
+    auto resid_gemm = [&](const char *name, const bf16 *Ain, int K, const bf16 *W, GemmArgs a) -> moss_enc_status {
+        if (narrow) return gemm2<128, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, 2);
+        return gemm2<320, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, K == D ? 2 : 1);
+    };
     for (size_t l = 0; l < h->layers.size(); l++) {
         const LayerDev &L = h->layers[l];
         {
@@ -1272,7 +1282,7 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.bo;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm2<320, EPI_RESID_F32>(h, "gemm_out", h->attn, T, D, L.wo, D, a, 0, 2)));
+        TRY(resid_gemm("gemm_out", h->attn, D, L.wo, a));
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln2_g, L.ln2_b,
@@ -1285,7 +1295,7 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.b2;
         a.out = h->X;
         a.ldo = D;
-        TRY((gemm2<320, EPI_RESID_F32>(h, "gemm_fc2", h->ffn, T, DFF, L.w2, D, a)));
+        TRY(resid_gemm("gemm_fc2", h->ffn, DFF, L.w2, a));
         // layer taps: this layer's hidden states through the tap's own head set
         // (xn, hb, h2 and gu are free between layers)
         if (tap_out)
