@@ -1,15 +1,15 @@
 // Whisper-style log-mel front end (fp32, CUDA cores).
 //
-// One CTA takes a block of up to 32 consecutive frames of one clip.  The PCM
-// span those frames cover (160*31 + 400 samples) is read once, coalesced, into
-// shared memory, with reflect padding applied only at the true clip ends.
-// Frames are transformed two at a time: frame a as the real part and frame b
-// as the imaginary part of one 400-point complex DFT, computed as 20 x 20
-// (two passes of 20-point DFTs, each a 4-point and a 5-point stage, with the
-// 400-point twiddles between the passes).  The two real spectra are separated
-// with X_a[k] = (Z[k] + conj Z[-k]) / 2, X_b[k] = (Z[k] - conj Z[-k]) / 2i,
-// squared, pushed through the banded mel filterbank, and log10'd.  The block's
-// maximum goes to the clip's maximum with one ordered-integer atomicMax.
+// Blocks of 16 consecutive frames of a clip: the PCM span those frames cover
+// (160*15 + 400 samples) is copied once into shared memory, with reflect
+// padding applied only at the true clip ends.  Frames are transformed two at
+// a time: frame a as the real part and frame b as the imaginary part of one
+// 400-point complex DFT, computed as 20 x 20 (two passes of 20-point DFTs,
+// each a 4-point and a 5-point stage, with the 400-point twiddles between the
+// passes).  The two real spectra are separated with X_a[k] = (Z[k] + conj
+// Z[-k]) / 2, X_b[k] = (Z[k] - conj Z[-k]) / 2i, squared, pushed through the
+// banded mel filterbank, and log10'd.  A block's maximum goes to the clip's
+// maximum with one ordered-integer atomicMax.
 #pragma once
 
 #include "common.cuh"
@@ -18,10 +18,9 @@ namespace moss {
 
 static constexpr int MEL_BAND = 16;  // max nonzero FFT bins of one mel filter
 
-// One clip's frame range for a logmel launch.  Block (x, y) of the grid
-// takes frames f_begin + 32x .. of clip y; frame f goes to output row
-// out_row0 + (f - f_begin).  gslot >= 0 names the per-clip maximum this
-// range folds into (atomicMax); -1 folds into nothing.
+// One clip's frame range for a log-mel launch: frames [f_begin, f_end), frame
+// f to output row out_row0 + (f - f_begin).  gslot >= 0 names the per-clip
+// maximum this range folds into (atomicMax); -1 folds into nothing.
 struct MelClip {
     const float *pcm;
     long long n;
@@ -31,7 +30,8 @@ struct MelClip {
     int pad;
 };
 
-// Device tables shared by every mel launch (filled at create).
+// The transform and filterbank in their plain form (built on the host from
+// the definitions; the kernel's tables, Mel4Tab, are derived from them).
 struct MelTables {
     float2 tw400[400];            // exp(-2 pi i k / 400)
     float hann[400];              // periodic Hann
@@ -104,139 +104,7 @@ __device__ __forceinline__ long long reflect_index(long long j, long long n)
     return j;
 }
 
-// A CTA of 320 threads
-// takes up to 32 frames (16 frame pairs).  The 400-point complex DFT of a
-// frame pair is split as 20 x 20: pass 1 gives each thread one (pair, n1)
-// 20-point DFT over samples n1 + 20 n2, pass 2 one (pair, k2) DFT over n1, so
-// all 320 lanes work in both passes; the exchange goes through shared memory
-// with rows padded to 21 entries.  Power, banded mel and log10 then run over
-// (frame, bin) and (frame, filter) items.  Registers stay near 100, so two
-// CTAs share an SM.
-static constexpr int MEL2_FRAMES = 32;
-static constexpr int MEL2_THREADS = 320;
-static constexpr int MEL2_SPAN = 160 * (MEL2_FRAMES - 1) + 400;  // 5360 samples
-
-struct Mel2Smem {
-    float2 tw[400];
-    float hann[400];
-    int band_lo[128];
-    int band_n[128];
-    float band_w[128][MEL_BAND];
-    float2 y[MEL2_FRAMES / 2][20 * 21];      // pass-1 output / pass-2 output per pair
-    float xs[MEL2_FRAMES * 204 > MEL2_SPAN ? MEL2_FRAMES * 204 : MEL2_SPAN];  // PCM, then power [32][204]
-    float wmax[MEL2_THREADS / 32];
-};
-
-__global__ void __launch_bounds__(MEL2_THREADS, 2) logmel2_kernel(const MelClip *__restrict__ clips,
-                                                                  const MelTables *__restrict__ tab,
-                                                                  float *__restrict__ out, int *gmax_ord,
-                                                                  int write_out)
-{
-    extern __shared__ __align__(16) uint8_t mel2_smem[];
-    Mel2Smem &S = *reinterpret_cast<Mel2Smem *>(mel2_smem);
-    const MelClip clip = clips[blockIdx.y];
-    const int frame0 = clip.f_begin + MEL2_FRAMES * blockIdx.x;
-    if (frame0 >= clip.f_end) return;
-    const int nf = min(MEL2_FRAMES, clip.f_end - frame0);
-    const long long out_row = clip.out_row0 + (frame0 - clip.f_begin);
-    const int tid = threadIdx.x;
-
-    for (int i = tid; i < 400; i += MEL2_THREADS) {
-        S.tw[i] = tab->tw400[i];
-        S.hann[i] = tab->hann[i];
-    }
-    for (int i = tid; i < 128; i += MEL2_THREADS) {
-        S.band_lo[i] = tab->band_lo[i];
-        S.band_n[i] = tab->band_n[i];
-    }
-    for (int i = tid; i < 128 * MEL_BAND; i += MEL2_THREADS) S.band_w[i / MEL_BAND][i % MEL_BAND] = tab->band_w[i / MEL_BAND][i % MEL_BAND];
-
-    // the block's PCM span, reflect-padded only at the clip ends
-    const long long s0 = 160LL * frame0 - 200;
-    const int span = 160 * (nf - 1) + 400;
-    if (s0 >= 0 && s0 + span <= clip.n && ((reinterpret_cast<uintptr_t>(clip.pcm) & 15) == 0)) {
-        const float4 *src = reinterpret_cast<const float4 *>(clip.pcm + s0);  // s0 = 160 f - 200 is a multiple of 4
-        for (int i = tid; i < span / 4; i += MEL2_THREADS) reinterpret_cast<float4 *>(S.xs)[i] = __ldg(src + i);
-    } else {
-        for (int i = tid; i < span; i += MEL2_THREADS) S.xs[i] = __ldg(clip.pcm + reflect_index(s0 + i, clip.n));
-    }
-    __syncthreads();
-
-    const int npairs = (nf + 1) / 2;
-    // pass 1: task (pair p, n1): 20-point DFT over n2 of the windowed samples
-    // n = n1 + 20 n2 of frame a (real part) and frame b (imaginary part)
-    for (int task = tid; task < npairs * 20; task += MEL2_THREADS) {
-        const int p = task / 20, n1 = task - 20 * p;
-        const int fa = 2 * p, fb = 2 * p + 1;
-        const bool has_b = fb < nf;
-        const float *xa = S.xs + 160 * fa, *xb = S.xs + 160 * (has_b ? fb : fa);
-        float2 v[20];
-#pragma unroll
-        for (int n2 = 0; n2 < 20; n2++) {
-            const int n = n1 + 20 * n2;
-            const float w = S.hann[n];
-            v[n2] = make_float2(w * xa[n], has_b ? w * xb[n] : 0.0f);
-        }
-        dft20(v);
-        float2 *yr = S.y[p] + n1 * 21;
-#pragma unroll
-        for (int k2 = 0; k2 < 20; k2++) yr[k2] = (k2 == 0 || n1 == 0) ? v[k2] : cmul(v[k2], S.tw[n1 * k2]);
-    }
-    __syncthreads();
-    // pass 2: task (pair p, k2): 20-point DFT over n1 -> Z[20 k1 + k2], in place
-    for (int task = tid; task < npairs * 20; task += MEL2_THREADS) {
-        const int p = task / 20, k2 = task - 20 * p;
-        float2 v[20];
-#pragma unroll
-        for (int n1 = 0; n1 < 20; n1++) v[n1] = S.y[p][n1 * 21 + k2];
-        dft20(v);
-#pragma unroll
-        for (int k1 = 0; k1 < 20; k1++) S.y[p][k1 * 21 + k2] = v[k1];
-    }
-    __syncthreads();
-    // power of both frames of each pair, bins 0..200, into S.xs as [frame][204]
-    float *pw = S.xs;
-    for (int task = tid; task < npairs * 201; task += MEL2_THREADS) {
-        const int p = task / 201, k = task - 201 * p;
-        const int kn = (400 - k) % 400;
-        const float2 zk = S.y[p][(k / 20) * 21 + (k % 20)], zn = S.y[p][(kn / 20) * 21 + (kn % 20)];
-        const float ar = 0.5f * (zk.x + zn.x), ai = 0.5f * (zk.y - zn.y);
-        const float br = 0.5f * (zk.y + zn.y), bi = -0.5f * (zk.x - zn.x);
-        pw[(2 * p) * 204 + k] = ar * ar + ai * ai;
-        pw[(2 * p + 1) * 204 + k] = br * br + bi * bi;
-    }
-    __syncthreads();
-    // banded mel, log10, block max; thread takes 4 consecutive filters of a frame
-    float lmax = -INFINITY;
-    for (int task = tid; task < nf * 32; task += MEL2_THREADS) {
-        const int f = task >> 5, q = task & 31;
-        const float *P = pw + f * 204;
-        float r[4];
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const int m = 4 * q + j;
-            const int lo = S.band_lo[m], cnt = S.band_n[m];
-            float acc = 0.0f;
-            for (int b = 0; b < cnt; b++) acc = fmaf(S.band_w[m][b], P[lo + b], acc);
-            r[j] = log10f(fmaxf(acc, 1e-10f));
-            lmax = fmaxf(lmax, r[j]);
-        }
-        if (write_out)
-            reinterpret_cast<float4 *>(out + (size_t)(out_row + f) * 128)[q] = make_float4(r[0], r[1], r[2], r[3]);
-    }
-    if (clip.gslot >= 0) {
-        for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-        if ((tid & 31) == 0) S.wmax[tid >> 5] = lmax;
-        __syncthreads();
-        if (tid == 0) {
-            float m = S.wmax[0];
-            for (int i = 1; i < MEL2_THREADS / 32; i++) m = fmaxf(m, S.wmax[i]);
-            atomicMax(gmax_ord + clip.gslot, float_to_ordered(m));
-        }
-    }
-}
-
-// Persistent form of the same computation (the one the library launches).
+// The log-mel kernel (every log-mel launch of the library).
 // Four CTAs of 160 threads per SM walk the (clip, 16-frame block) items of
 // the launch, 5 barriers per item.  Thread t takes pair tp = t % 8 and row or
 // column tj = t / 8 in every transform phase, so a warp covers 8 pairs x 4

@@ -64,7 +64,6 @@ struct moss_enc {
     std::vector<LayerDev> layers;
     HeadDev head{};
     float *pos = nullptr;
-    MelTables *mel_tab = nullptr;
     Mel4Tab *mel4_tab = nullptr;
 
     // layer taps (moss_enc_set_taps): encoder layer per tap and its head set
@@ -767,7 +766,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
                                4 * (DQKV + D + DFF + D) + 8 * 256;
     for (int l = 0; l < L; l++) o_layer[l] = take(layer_bytes);
     const HeadOff o_head = head_take(take);
-    const size_t o_pos = take(4 * (size_t)CHUNK_TOKENS * D), o_mel = take(sizeof(MelTables));
+    const size_t o_pos = take(4 * (size_t)CHUNK_TOKENS * D);
     const size_t o_mel4 = take(sizeof(Mel4Tab));
     const size_t wtotal = off;
 
@@ -854,9 +853,11 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
             F32(o_pos)[t * D + i] = (float)std::sin(t * inv);
             F32(o_pos)[t * D + D / 2 + i] = (float)std::cos(t * inv);
         }
-    if (!build_mel_tables(reinterpret_cast<MelTables *>(pk.data() + o_mel))) return bail(MOSS_ENC_ERR_INVALID_ARG);
-    if (!build_mel4_tab(*reinterpret_cast<const MelTables *>(pk.data() + o_mel), reinterpret_cast<Mel4Tab *>(pk.data() + o_mel4)))
-        return bail(MOSS_ENC_ERR_INVALID_ARG);
+    {
+        MelTables mt;
+        if (!build_mel_tables(&mt) || !build_mel4_tab(mt, reinterpret_cast<Mel4Tab *>(pk.data() + o_mel4)))
+            return bail(MOSS_ENC_ERR_INVALID_ARG);
+    }
 
     if (cudaMalloc(&h->wmem, wtotal) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaMemcpy(h->wmem, pk.data(), wtotal, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
@@ -886,7 +887,6 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     }
     h->head = head_bind(o_head, W);
     h->pos = (float *)(W + o_pos);
-    h->mel_tab = (MelTables *)(W + o_mel);
     h->mel4_tab = (Mel4Tab *)(W + o_mel4);
 
     // ---- workspace
@@ -981,7 +981,6 @@ static moss_enc_status tab_upload(moss_enc *h)
     return MOSS_ENC_OK;
 }
 
-static int mel_grid_x(int64_t max_frames) { return (int)std::max<int64_t>(1, (max_frames + MEL2_FRAMES - 1) / MEL2_FRAMES); }
 
 static moss_enc_status launch_logmel(moss_enc *h, const MelClip *d_clips, int n_clips, int64_t max_frames,
                                      float *out, int write_out, int64_t total_frames)
@@ -1762,18 +1761,19 @@ extern "C" moss_enc_status moss_enc_selftest_timeout(moss_enc *h, int limit_ms)
 // ------------------------------------------------- allocation-free log-mel
 //
 // Scratch for moss_enc_logmel_static: a fixed-size device array, laid out as
-// [MelTables | main-pass MelClip x 64 | max-pass MelClip x 64 | log_max
+// [log-mel kernel tables (Mel4Tab) | main-pass MelClip x 64 | max-pass
+// MelClip x 64 | log_max
 // source pointers x 64 | ordered-int maxima x 64].  Nothing here allocates.
 
 namespace {
 constexpr int STATIC_MAX_CLIPS = MOSS_ENC_STATIC_MAX_CLIPS;
 constexpr size_t ST_TABLES = 0;
-constexpr size_t ST_MAIN = (sizeof(MelTables) + 255) & ~size_t(255);
+constexpr size_t ST_MAIN = (sizeof(Mel4Tab) + 255) & ~size_t(255);
 constexpr size_t ST_MAXP = ST_MAIN + ((sizeof(MelClip) * STATIC_MAX_CLIPS + 255) & ~size_t(255));
 constexpr size_t ST_SRC = ST_MAXP + ((sizeof(MelClip) * STATIC_MAX_CLIPS + 255) & ~size_t(255));
 constexpr size_t ST_GMAX = ST_SRC + ((sizeof(float *) * STATIC_MAX_CLIPS + 255) & ~size_t(255));
 constexpr size_t ST_USED = ST_GMAX + sizeof(int) * STATIC_MAX_CLIPS;
-constexpr size_t ST_BYTES = 20480;
+constexpr size_t ST_BYTES = 24576;
 static_assert(ST_USED <= ST_BYTES, "static log-mel scratch too small");
 
 // Per-call descriptors staged on the host before one copy into the array.
@@ -1786,6 +1786,7 @@ struct StaticStage {
 constexpr int STATIC_MAX_DEVICES = 64;
 std::mutex g_static_mu;
 uint8_t *g_static_ptr[STATIC_MAX_DEVICES] = {};
+int g_static_sms[STATIC_MAX_DEVICES] = {};
 }  // namespace
 
 static __device__ __align__(256) uint8_t g_logmel_scratch[ST_BYTES];
@@ -1800,12 +1801,16 @@ static moss_enc_status static_scratch(uint8_t **out)
     if (!g_static_ptr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_logmel_scratch) != cudaSuccess || !p) return MOSS_ENC_ERR_CUDA;
-        if (cudaFuncSetAttribute(logmel2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel2Smem)) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(logmel4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel4Smem)) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(logmel4_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
             return MOSS_ENC_ERR_CUDA;
         MelTables tab;
-        if (!build_mel_tables(&tab)) return MOSS_ENC_ERR_INVALID_ARG;
-        if (cudaMemcpy(static_cast<uint8_t *>(p) + ST_TABLES, &tab, sizeof(tab), cudaMemcpyHostToDevice) != cudaSuccess)
+        static Mel4Tab tab4;  // built once under the lock (too large for the stack)
+        if (!build_mel_tables(&tab) || !build_mel4_tab(tab, &tab4)) return MOSS_ENC_ERR_INVALID_ARG;
+        if (cudaMemcpy(static_cast<uint8_t *>(p) + ST_TABLES, &tab4, sizeof(tab4), cudaMemcpyHostToDevice) != cudaSuccess)
+            return MOSS_ENC_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&g_static_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOSS_ENC_ERR_CUDA;
         g_static_ptr[dev] = static_cast<uint8_t *>(p);
     }
@@ -1847,7 +1852,11 @@ extern "C" moss_enc_status moss_enc_logmel_static(const moss_enc_clip *clips, in
     MelClip *d_maxp = reinterpret_cast<MelClip *>(S + ST_MAXP);
     const float *const *d_src = reinterpret_cast<const float *const *>(S + ST_SRC);
     int *d_gmax = reinterpret_cast<int *>(S + ST_GMAX);
-    const MelTables *d_tab = reinterpret_cast<const MelTables *>(S + ST_TABLES);
+    const Mel4Tab *d_tab = reinterpret_cast<const Mel4Tab *>(S + ST_TABLES);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOSS_ENC_ERR_CUDA;
+    const int64_t max_grid = 4 * (int64_t)g_static_sms[dev];
+    auto grid_for = [&](int64_t blocks) { return (int)std::max<int64_t>(1, std::min<int64_t>(blocks, max_grid)); };
     if (cudaMemcpyAsync(S + ST_MAIN, stage.main, sizeof(stage.main), cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(S + ST_MAXP, stage.maxp, sizeof(stage.maxp), cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(S + ST_SRC, stage.src, sizeof(stage.src), cudaMemcpyHostToDevice, st) != cudaSuccess)
@@ -1855,11 +1864,13 @@ extern "C" moss_enc_status moss_enc_logmel_static(const moss_enc_clip *clips, in
     // the maxima start at -inf or at the caller's value
     gmax_init_kernel<<<1, STATIC_MAX_CLIPS, 0, st>>>(d_gmax, d_src, n_clips);
     if (n_max > 0)
-        logmel2_kernel<<<dim3(mel_grid_x(max_clip), n_max), MEL2_THREADS, sizeof(Mel2Smem), st>>>(d_maxp, d_tab, nullptr, d_gmax, 0);
+        logmel4_kernel<<<grid_for(n_max * ((max_clip + MEL4_FRAMES - 1) / MEL4_FRAMES)), MEL4_THREADS, sizeof(Mel4Smem),
+                         st>>>(d_maxp, n_max, d_tab, nullptr, d_gmax, 0);
     for (int i = 0; i < n_clips; i++) {
         const int nf = stage.main[i].f_end - stage.main[i].f_begin;
         if (nf <= 0) continue;
-        logmel2_kernel<<<dim3(mel_grid_x(nf), 1), MEL2_THREADS, sizeof(Mel2Smem), st>>>(d_main + i, d_tab, mel_out[i], d_gmax, 1);
+        logmel4_kernel<<<grid_for((nf + MEL4_FRAMES - 1) / MEL4_FRAMES), MEL4_THREADS, sizeof(Mel4Smem), st>>>(
+            d_main + i, 1, d_tab, mel_out[i], d_gmax, 1);
     }
     for (int i = 0; i < n_clips; i++) {
         const int64_t nf = stage.main[i].f_end - stage.main[i].f_begin;

@@ -281,7 +281,7 @@ moss_enc_status moss_enc_selftest_timeout(moss_enc *h, int limit_ms);
  *
  * It computes the same Whisper log-mel as moss_enc_logmel for up to
  * MOSS_ENC_STATIC_MAX_CLIPS clips.  Its scratch (the filterbank and FFT
- * tables, per-clip range descriptors and per-clip maxima; 20 KiB) is one
+ * tables, per-clip range descriptors and per-clip maxima; 24 KiB) is one
  * statically sized device array inside the library, which every GPU that
  * loads the library keeps until the process exits.
  *  clips        host [n_clips]; same fields and range rules as moss_enc_clip.
