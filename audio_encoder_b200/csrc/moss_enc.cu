@@ -688,6 +688,7 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm2_attr<256, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm2_attr<128, EPI_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_SWIGLU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_F32>()));
@@ -1271,7 +1272,10 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.bqkv;
         a.out = h->qkv;
         a.ldo = DQKV;
-        TRY((gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
+        if (T <= 512)  // two row tiles: 128-wide tiles (30 per row tile) keep more SMs busy than 256-wide (15)
+            TRY((gemm2<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
+        else
+            TRY((gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
         {
             Launch Lk(h, "attention", 4.0 * 64 * 20 * attn_pairs, 2.0 * T * (DQKV + D));
             CUDA_TRY(h, launch_k(h, window_attn_tc_kernel, dim3((unsigned)n_chunks, 20), dim3(128), ATTN_TC_SMEM, tm_qkv,

@@ -138,19 +138,29 @@ def dist_setup(n_gpus):
     return rank, world, dist
 
 
-def oracle_sample(clips, n_layers, windows, blob=None):
+def oracle_sample(clips, n_layers, windows, blob=None, threads=None):
+    """The oracle, as it stands, on the first `windows` 800-frame windows of
+    clip 0 with all host threads (or `threads` of them)."""
     import oracle
     blob = synth.make_weights(n_layers) if blob is None else blob
-    m = oracle.Model(blob, n_layers)
-    pcm = clips[0]
-    gmax = oracle.clip_log_max(pcm)
-    t0 = time.perf_counter()
-    toks = 0
-    for c in range(windows):
-        toks += m.encode_chunks(pcm, c, c + 1, gmax=gmax).shape[0]
-    dt = time.perf_counter() - t0
-    m.close()
-    return dt, toks, oracle.max_threads()
+    all_threads = oracle.max_threads()
+    if threads:
+        oracle.set_threads(threads)
+    try:
+        m = oracle.Model(blob, n_layers)
+        pcm = clips[0]
+        gmax = oracle.clip_log_max(pcm)
+        t0 = time.perf_counter()
+        toks = 0
+        for c in range(windows):
+            toks += m.encode_chunks(pcm, c, c + 1, gmax=gmax).shape[0]
+        dt = time.perf_counter() - t0
+        m.close()
+        used = oracle.max_threads()
+    finally:
+        if threads:
+            oracle.set_threads(all_threads)
+    return dt, toks, used
 
 
 def gemm_source_hash():
@@ -375,6 +385,10 @@ def run_ours(args):
         cpu = {"value": (toks / 12.5) / dt, "unit": "audio-s/s", "cores": cores, "kind": "oracle",
                "sample": f"first {args.cpu_windows} 800-frame windows of clip 0 ({toks} tokens, "
                          f"{toks / 12.5:.0f} s of audio), all {n_layers} layers, {dt:.1f} s"}
+        if args.cpu_one_core:
+            dt1, toks1, _ = oracle_sample(clips, n_layers, windows=1, blob=blob, threads=1)
+            cpu["one_core"] = {"value": (toks1 / 12.5) / dt1, "unit": "audio-s/s", "cores": 1,
+                               "sample": f"first 800-frame window of clip 0 ({toks1} tokens), {dt1:.1f} s"}
 
     line = {
         "metric": "audio-sec encoded/sec", "value": value, "unit": "audio-s/s", "n_gpus": world,
@@ -592,6 +606,8 @@ def main():
     ap.add_argument("--workload", default="batch16_10to30s", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cpu-windows", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-one-core", action="store_true",
+                    help="also time the oracle on one host core (one 800-frame window)")
     ap.add_argument("--shard-clip", action="store_true",
                     help="one long clip (10 or 60 min) split over the ranks by chunk ranges (strong scaling)")
     ap.add_argument("--taps", default="",
