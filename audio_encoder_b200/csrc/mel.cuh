@@ -48,9 +48,14 @@ __device__ __forceinline__ float2 cmul(float2 a, float2 b)
 // 20-point DFT in registers: X[k] = sum_n x[n] exp(-2 pi i n k / 20).
 // n = nb + 5 na, k = 4 kb + ka:  4-point DFTs over na, twiddle
 // exp(-2 pi i nb ka / 20) (compile-time constants), then 5-point DFTs over nb.
-__device__ __forceinline__ void dft20(float2 (&x)[20])
+// Each complex value's real and imaginary parts sit in the two lanes of the
+// paired fp32 instructions: the 4- and 5-point stages' additions and
+// real-constant products take one paired instruction per complex value;
+// (-i) z is the lane swap (z.y, -z.x).
+__device__ __forceinline__ float2 mnegi(float2 z) { return make_float2(z.y, -z.x); }
+__device__ __forceinline__ float2 csub(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ void dft20p(float2 (&x)[20])
 {
-    // cos and sin of 2 pi m / 20, m = 0..12
     constexpr float C20[13] = {1.0f, 9.510565163e-01f, 8.090169944e-01f, 5.877852523e-01f, 3.090169944e-01f, 0.0f,
                                -3.090169944e-01f, -5.877852523e-01f, -8.090169944e-01f, -9.510565163e-01f, -1.0f,
                                -9.510565163e-01f, -8.090169944e-01f};
@@ -60,37 +65,36 @@ __device__ __forceinline__ void dft20(float2 (&x)[20])
     float2 A[5][4];
 #pragma unroll
     for (int nb = 0; nb < 5; nb++) {
-        float2 x0 = x[nb], x1 = x[nb + 5], x2 = x[nb + 10], x3 = x[nb + 15];
-        float2 s02 = make_float2(x0.x + x2.x, x0.y + x2.y), d02 = make_float2(x0.x - x2.x, x0.y - x2.y);
-        float2 s13 = make_float2(x1.x + x3.x, x1.y + x3.y), d13 = make_float2(x1.x - x3.x, x1.y - x3.y);
-        // W4 = -i: (-i) * d13 = (d13.y, -d13.x)
-        A[nb][0] = make_float2(s02.x + s13.x, s02.y + s13.y);
-        A[nb][1] = make_float2(d02.x + d13.y, d02.y - d13.x);
-        A[nb][2] = make_float2(s02.x - s13.x, s02.y - s13.y);
-        A[nb][3] = make_float2(d02.x - d13.y, d02.y + d13.x);
+        const float2 s02 = __fadd2_rn(x[nb], x[nb + 10]), d02 = csub(x[nb], x[nb + 10]);
+        const float2 s13 = __fadd2_rn(x[nb + 5], x[nb + 15]), t = mnegi(csub(x[nb + 5], x[nb + 15]));
+        A[nb][0] = __fadd2_rn(s02, s13);
+        A[nb][1] = __fadd2_rn(d02, t);
+        A[nb][2] = csub(s02, s13);
+        A[nb][3] = csub(d02, t);
     }
 #pragma unroll
     for (int nb = 1; nb < 5; nb++)
 #pragma unroll
         for (int ka = 1; ka < 4; ka++) A[nb][ka] = cmul(A[nb][ka], make_float2(C20[nb * ka], -S20[nb * ka]));
-    // 5-point DFT with c1 = cos(2pi/5), c2 = cos(4pi/5), s1 = sin(2pi/5), s2 = sin(4pi/5)
-    const float c1 = 0.30901699437494742f, c2 = -0.80901699437494742f;
-    const float s1 = 0.95105651629515357f, s2 = 0.58778525229247313f;
+    const float2 c1 = make_float2(0.30901699437494742f, 0.30901699437494742f);
+    const float2 c2 = make_float2(-0.80901699437494742f, -0.80901699437494742f);
+    const float2 s1 = make_float2(0.95105651629515357f, 0.95105651629515357f);
+    const float2 s2 = make_float2(0.58778525229247313f, 0.58778525229247313f);
+    const float2 ms1 = make_float2(-0.95105651629515357f, -0.95105651629515357f);
 #pragma unroll
     for (int ka = 0; ka < 4; ka++) {
-        float2 a0 = A[0][ka], a1 = A[1][ka], a2 = A[2][ka], a3 = A[3][ka], a4 = A[4][ka];
-        float2 t1 = make_float2(a1.x + a4.x, a1.y + a4.y), t2 = make_float2(a2.x + a3.x, a2.y + a3.y);
-        float2 u1 = make_float2(a1.x - a4.x, a1.y - a4.y), u2 = make_float2(a2.x - a3.x, a2.y - a3.y);
-        float2 r1 = make_float2(a0.x + c1 * t1.x + c2 * t2.x, a0.y + c1 * t1.y + c2 * t2.y);
-        float2 r2 = make_float2(a0.x + c2 * t1.x + c1 * t2.x, a0.y + c2 * t1.y + c1 * t2.y);
-        // -i * (s1 u1 + s2 u2) and -i * (s2 u1 - s1 u2)
-        float2 i1 = make_float2(s1 * u1.x + s2 * u2.x, s1 * u1.y + s2 * u2.y);
-        float2 i2 = make_float2(s2 * u1.x - s1 * u2.x, s2 * u1.y - s1 * u2.y);
-        x[ka] = make_float2(a0.x + t1.x + t2.x, a0.y + t1.y + t2.y);
-        x[4 + ka] = make_float2(r1.x + i1.y, r1.y - i1.x);
-        x[16 + ka] = make_float2(r1.x - i1.y, r1.y + i1.x);
-        x[8 + ka] = make_float2(r2.x + i2.y, r2.y - i2.x);
-        x[12 + ka] = make_float2(r2.x - i2.y, r2.y + i2.x);
+        const float2 a0 = A[0][ka], a1 = A[1][ka], a2 = A[2][ka], a3 = A[3][ka], a4 = A[4][ka];
+        const float2 t1 = __fadd2_rn(a1, a4), t2 = __fadd2_rn(a2, a3), u1 = csub(a1, a4), u2 = csub(a2, a3);
+        const float2 r1 = __ffma2_rn(t2, c2, __ffma2_rn(t1, c1, a0));
+        const float2 r2 = __ffma2_rn(t2, c1, __ffma2_rn(t1, c2, a0));
+        // -i (s1 u1 + s2 u2) and -i (s2 u1 - s1 u2)
+        const float2 w1 = mnegi(__ffma2_rn(u2, s2, __fmul2_rn(u1, s1)));
+        const float2 w2 = mnegi(__ffma2_rn(u2, ms1, __fmul2_rn(u1, s2)));
+        x[ka] = __fadd2_rn(a0, __fadd2_rn(t1, t2));
+        x[4 + ka] = __fadd2_rn(r1, w1);
+        x[16 + ka] = csub(r1, w1);
+        x[8 + ka] = __fadd2_rn(r2, w2);
+        x[12 + ka] = csub(r2, w2);
     }
 }
 
@@ -316,7 +320,7 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
                 const float b = has_b ? xb[20 * n2 + (n2 >= 8 ? 20 : 0)] : 0.0f;
                 v[n2] = make_float2(hw[20 * n2] * a, hw[20 * n2] * b);
             }
-            dft20(v);
+            dft20p(v);
             float2 *yr = Y + tj * 20;
             yr[0] = v[0];
 #pragma unroll
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(MEL4_THREADS, 4) logmel4_kernel(const MelClip 
             float2 v[20];
 #pragma unroll
             for (int n1 = 0; n1 < 20; n1++) v[n1] = Y[n1 * 20 + tj];
-            dft20(v);
+            dft20p(v);
 #pragma unroll
             for (int k1 = 0; k1 < 20; k1++) Y[k1 * 20 + tj] = v[k1];
         }
