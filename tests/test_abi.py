@@ -38,6 +38,16 @@ def test_weight_count_matches_generator_and_oracle():
         assert binding.weight_count(n) == total == oracle.weight_count(n)
 
 
+def test_tap_weight_count_is_one_head_and_adapter_set():
+    # a layer tap's weights are laid out like the blob's tail after the layers
+    count = binding.tap_weight_count()
+    assert count == sum(int(np.prod(shape)) for _, shape, _ in synth.head_manifest())
+    names = [name for name, _, _ in synth.weight_manifest(0)]
+    stem = sum(int(np.prod(shape)) for _, shape, _ in synth.weight_manifest(0)[:names.index("ln_post.weight")])
+    assert binding.weight_count(0) == stem + count
+    assert synth.make_tap_weights(2).size == 2 * count
+
+
 @pytest.mark.parametrize("n", [0, 1, 159, 160, 161, 16000, 16159, 127999, 128000, 128160, 480000,
                                9_600_000, 57_600_000, 1_024_000, 160 * 801])
 def test_counts_match_oracle(n):
