@@ -551,6 +551,23 @@ struct Gemm2Cfg {
     static_assert(B_SUB_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
 };
 
+// Tile t of the pair kernel.  Plain GEMMs walk row blocks first (pairs that
+// run together share a column block of the weights).  The implicit convs
+// walk column blocks first: their input (the previous conv's activations) is
+// far larger than L2, and the two 240-wide column blocks of a row block then
+// read its input slab at the same time, once from DRAM.
+template <int AMODE>
+__device__ __forceinline__ void pair_tile(int tile, const GemmArgs &a, int &mt, int &nt)
+{
+    if constexpr (AMODE == A_CONV_S2) {
+        mt = tile / a.n_tiles;
+        nt = tile - mt * a.n_tiles;
+    } else {
+        mt = tile % a.m_tiles;
+        nt = tile / a.m_tiles;
+    }
+}
+
 template <int BN, int EPI, int AMODE = A_PLAIN, int KSUB = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -618,14 +635,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
             for (int kb = 0; kb < npre; kb++) {
                 const uint32_t fb = map_to_rank(smem_u32(&full[kb]), 0);
                 mbar_arrive_expect_tx_remote(fb, C::STAGE_BYTES);
-                load_b(smem + kb * C::STAGE_BYTES, fb, kb, pair / args.m_tiles);
+                int mt0, nt0;
+                pair_tile<AMODE>(pair, args, mt0, nt0);
+                load_b(smem + kb * C::STAGE_BYTES, fb, kb, nt0);
             }
             grid_dep_wait();
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-                const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
+                int mt, nt;
+                pair_tile<AMODE>(tile, args, mt, nt);
                 int chunk = 0, t0 = 0;
                 if constexpr (AMODE == A_CONV_S2) {
                     const int item = args.tile_list[2 * mt + rank];  // padded list: -1 = no rows
@@ -714,7 +734,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
         for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
             const int acc = it % C::ACC;
             const uint32_t aph = (it / C::ACC) & 1;
-            const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
+            int mt, nt;
+            pair_tile<AMODE>(tile, args, mt, nt);
             if constexpr (EPI == EPI_RESID_F32) {
                 // the residual rows this tile adds to go to L2 while the mainloop runs
                 const int row = mt * 256 + (int)rank * 128 + q * 32 + lane;
