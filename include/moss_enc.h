@@ -146,7 +146,9 @@ const char *moss_enc_last_error(const moss_enc *h);
  * sample 160 t with reflect padding at the clip ends, periodic Hann 400,
  * |rFFT|^2 (201 bins), Slaney mel 128 x 201 over 0-8 kHz, log10(max(., 1e-10)),
  * floor at log_max - 8, then (x + 4) / 4.
- *  mel_out      device fp32 [n_frames][128], frame-major.
+ *  mel_out      device fp32 [n_frames][128], frame-major (rows leave by bulk
+ *               copies when mel_out is 16-byte aligned, by plain stores
+ *               otherwise; the values are the same).
  *  n_frames     host, receives the frame count (may be NULL).
  *  log_max_out  device float receiving the clip's log-mel maximum (may be NULL).
  * The range must hold at most cfg.max_samples samples. */
