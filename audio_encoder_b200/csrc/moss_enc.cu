@@ -1832,13 +1832,15 @@ extern "C" moss_enc_status moss_enc_logmel_static(const moss_enc_clip *clips, in
     StaticStage stage;
     std::memset(&stage, 0, sizeof(stage));
     int n_max = 0;
-    int64_t max_range = 0, max_clip = 0;
+    int64_t max_clip = 0;
     for (int i = 0; i < n_clips; i++) {
         const moss_enc_clip &c = clips[i];
+        // a clip with samples is read by the maximum pass even when its range is empty
+        if (c.n_samples > 0 && !c.pcm) return MOSS_ENC_ERR_INVALID_ARG;
         ClipPlan pl;
         if (!plan_clip(c.n_samples, c.begin, c.end, &pl) || pl.F > INT32_MAX) return MOSS_ENC_ERR_INVALID_ARG;
         const int64_t nf = pl.f_end - pl.f_begin;
-        if (nf > 0 && (!c.pcm || !mel_out[i])) return MOSS_ENC_ERR_INVALID_ARG;
+        if (nf > 0 && !mel_out[i]) return MOSS_ENC_ERR_INVALID_ARG;
         const bool whole = pl.f_begin == 0 && pl.f_end == pl.F;
         const bool own = c.log_max == nullptr;
         stage.src[i] = c.log_max;
@@ -1846,9 +1848,13 @@ extern "C" moss_enc_status moss_enc_logmel_static(const moss_enc_clip *clips, in
         // launch below and writes from row 0 of that buffer
         stage.main[i] = MelClip{c.pcm, (long long)pl.n, 0, (int)pl.f_begin, (int)pl.f_end, own && whole ? i : -1, 0};
         if (own && !whole) stage.maxp[n_max++] = MelClip{c.pcm, (long long)pl.n, 0, 0, (int)pl.F, i, 0};
-        max_range = std::max(max_range, nf);
         max_clip = std::max(max_clip, pl.F);
     }
+    // The descriptors are copied from this call's stack frame: a captured copy
+    // would be replayed after the frame is gone, so a capturing stream is refused.
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return MOSS_ENC_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return MOSS_ENC_ERR_INVALID_ARG;
     uint8_t *S = nullptr;
     moss_enc_status s = static_scratch(&S);
     if (s != MOSS_ENC_OK) return s;

@@ -103,7 +103,10 @@ int64_t moss_enc_weight_count(int n_layers);
 int64_t moss_enc_num_frames(int64_t n_samples);
 
 /* Output rows of a whole clip: the sum over 800-frame chunks of
- * ceil(frames_in_chunk / 8) (three stride-2 convs).  Pure. */
+ * ceil(frames_in_chunk / 8) (three stride-2 convs).  Pure.  The rate follows
+ * page "Ossicle-4B", "Model Overview" (12.5 audio tokens per second: 100 mel
+ * frames per second over an 8x time reduction) and the workload's 8 s chunks
+ * (800 frames -> 100 tokens). */
 int64_t moss_enc_num_tokens(int64_t n_samples);
 
 /* Output rows of the sample range [begin, end) of a clip of n_samples
@@ -112,7 +115,10 @@ int64_t moss_enc_range_tokens(int64_t n_samples, int64_t begin, int64_t end);
 
 /* ------------------------------------------------------------- lifetime */
 
-/* Create a handle on the current CUDA device.
+/* Create a handle on the current CUDA device.  The handle holds the encoder
+ * the page "MOSS-Transcribe-preview-2B - GGUF", "Architecture" table,
+ * describes (conv front-end, 32 pre-LN layers, encoder head, SwiGLU adapter);
+ * its weights are the blob's, laid out as moss_enc_weight_count says.
  *  weights        bf16 blob (uint16 bit patterns) of moss_enc_weight_count
  *                 (cfg->n_layers) elements; host or device memory as
  *                 weights_on_device says.  The library copies and repacks
@@ -120,7 +126,10 @@ int64_t moss_enc_range_tokens(int64_t n_samples, int64_t begin, int64_t end);
  *  bytes          size of the blob in bytes (checked).
  *  stream         cudaStream_t to enqueue on (NULL = legacy default stream).
  *  out            receives the handle.
- * Synchronises.  Allocates the weights and a workspace sized from cfg. */
+ * Synchronises.  Allocates the weights and a workspace sized from cfg.
+ * Errors: INVALID_ARG (null pointer, n_layers outside 1..32, max_samples or
+ * max_clips below 1, unknown out_dtype, wrong byte count), OOM, CUDA (also
+ * for a device that is not compute capability 10.x). */
 moss_enc_status moss_enc_create(const moss_enc_config *cfg, const void *weights, size_t bytes,
                                 int weights_on_device, void *stream, moss_enc **out);
 
@@ -131,6 +140,10 @@ moss_enc_status moss_enc_set_stream(moss_enc *h, void *stream);
  * reported a timed-out wait since the last call (and clear the flag). */
 moss_enc_status moss_enc_synchronize(moss_enc *h);
 
+/* Release a handle: synchronises its stream, then frees the weights, the
+ * workspace, the layer taps and any captured forward graph.  NULL is a no-op.
+ * The pages describe no teardown of their own; this is the plain counterpart
+ * of moss_enc_create. */
 void moss_enc_destroy(moss_enc *h);
 
 const char *moss_enc_status_string(moss_enc_status s);
@@ -172,14 +185,21 @@ moss_enc_status moss_enc_log_max(moss_enc *h, const float *pcm, int64_t n_sample
 moss_enc_status moss_enc_range_log_max(moss_enc *h, const float *pcm, int64_t n_samples, int64_t begin,
                                        int64_t end, float *out);
 
-/* Encode n_clips clips (or pieces) into embedding rows.
+/* Encode n_clips clips (or pieces) into embedding rows: audio in, one
+ * 2048-wide embedding row per 80 ms of audio out, the encoder run once per
+ * clip (page "MOSS-Transcribe-preview-2B - GGUF", "Architecture" table, rows
+ * Audio, Conv front-end, Audio encoder, Encoder head, Adapter, and
+ * "Audio injection"; page "Ossicle-4B", "Long Audio" for pieces of a long
+ * clip).
  *  clips        host array [n_clips].
  *  rows_out     device [sum of tokens][2048] of cfg.out_dtype; the rows of
  *               clip i are rows row_offsets[i] .. row_offsets[i+1]-1.
  *  row_offsets  host int64 [n_clips + 1], written before the call returns
  *               (computed on the host, no synchronisation).
  * Each clip is encoded independently: its 800-frame chunks are the conv
- * stem's chunks (zero-padded at the tail) and the attention windows. */
+ * stem's chunks (zero-padded at the tail) and the attention windows.
+ * Errors: INVALID_ARG (null pointer, bad range), CAPACITY (more clips or
+ * samples than cfg allows), CUDA. */
 moss_enc_status moss_enc_forward(moss_enc *h, const moss_enc_clip *clips, int n_clips,
                                  void *rows_out, int64_t *row_offsets);
 
@@ -294,10 +314,14 @@ moss_enc_status moss_enc_selftest_timeout(moss_enc *h, int limit_ms);
  *               or NULL.
  *  stream       cudaStream_t to enqueue on.
  * Returns MOSS_ENC_ERR_CAPACITY when n_clips exceeds MOSS_ENC_STATIC_MAX_CLIPS
- * and MOSS_ENC_ERR_INVALID_ARG for a bad pointer or range.
+ * and MOSS_ENC_ERR_INVALID_ARG for a bad pointer or range (a clip with
+ * n_samples > 0 needs its pcm even when its range is empty, because the
+ * whole-clip maximum reads it) or when the stream is being captured.
  * The first call on a device sets the scratch up (finds the array's device
- * address and fills the tables, synchronously); make that first call before
- * any stream capture.  All calls share the one array, and each call
+ * address and fills the tables, synchronously).  No call may be made while
+ * its stream is being captured into a CUDA graph: each call copies its
+ * per-clip descriptors from host memory that lives only for the call, so the
+ * call refuses a capturing stream (INVALID_ARG) and enqueues nothing.  All calls share the one array, and each call
  * overwrites what the previous call left there: calls whose work overlaps on
  * the GPU (different streams, or several host threads) race and must be
  * serialised by the caller. */

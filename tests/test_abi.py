@@ -79,3 +79,17 @@ def test_create_rejects_bad_arguments_before_touching_a_device():
     st = L.moss_enc_create(ctypes.byref(cfg), blob.ctypes.data_as(ctypes.c_void_p), 8, 0, None, ctypes.byref(h))
     assert st == 1  # blob size does not match 4 layers
     assert L.moss_enc_status_string(2) == b"request exceeds capacity"
+
+
+def test_static_logmel_rejects_a_clip_without_samples_pointer():
+    # A clip with samples but no pcm pointer is refused before anything is
+    # enqueued, even when its encoded range is empty (the whole-clip maximum
+    # would read the samples); no device is touched.
+    import ctypes
+    L = binding.lib()
+    arr = (binding.Clip * 1)()
+    arr[0] = binding.Clip(None, 16000, 0, 0, None)
+    outs = (ctypes.c_void_p * 1)(None)
+    assert L.moss_enc_logmel_static(arr, 1, outs, None, None) == 1
+    arr[0] = binding.Clip(None, 16000, 0, 16000, None)
+    assert L.moss_enc_logmel_static(arr, 1, outs, None, None) == 1

@@ -53,3 +53,26 @@ def test_static_logmel_rejects_too_many_clips():
     with pytest.raises(binding.MossEncError) as e:
         binding.logmel_static([x] * (binding.STATIC_MAX_CLIPS + 1))
     assert e.value.status == 2
+
+
+def test_static_logmel_refuses_a_capturing_stream():
+    # Each call copies its clip descriptors from host memory that lives only
+    # for the call, so it must not be recorded into a CUDA graph: under
+    # capture it returns INVALID_ARG and enqueues nothing.
+    x = torch.from_numpy(synth.pcm_tones(43, 16000)).cuda()
+    binding.logmel_static([x])  # the first call on the device sets up the scratch
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    status = None
+    y = torch.zeros(4, device="cuda")
+    with torch.cuda.graph(g, stream=s):
+        try:
+            binding.logmel_static([x], stream=s)
+        except binding.MossEncError as e:
+            status = e.status
+        y.add_(1.0)  # the graph holds one ordinary kernel
+    assert status == 1
+    g.replay()
+    torch.cuda.synchronize()
+    assert float(y[0].item()) == 1.0
