@@ -253,9 +253,12 @@ template <int BN, int EPI, int NHALF = 2>
 __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensorMap *tmC, uint32_t tbase, int half,
                                                int lane, uint8_t *stage_base, int nbuf, int row0, int col0)
 {
-    static_assert(BN % 64 == 0, "TMA output needs 64-column groups");
-    static_assert(EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 || EPI == EPI_F32, "epilogue");
-    constexpr int NG = BN / 64;
+    constexpr bool F32_OUT = EPI == EPI_RESID_F32 || EPI == EPI_F32;
+    // bf16 boxes are 64 columns wide; fp32 boxes 32, so fp32 tiles may end
+    // in a 32-column group (BN = 160: groups of 64, 64 and 32)
+    static_assert(BN % 64 == 0 || (F32_OUT && BN % 64 == 32), "TMA output needs whole boxes");
+    static_assert(EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || F32_OUT, "epilogue");
+    constexpr int NG = (BN + 63) / 64;
     const bool live = row0 < a.M;  // whole slab outside the output: nothing to write
     // boxes of the previous tile may still be reading the staging buffer
     if (lane == 0) bulk_wait_read();
@@ -272,9 +275,10 @@ __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensor
 #pragma unroll 1
     for (int g = half; g < NG; g += NHALF) {
         const int c0 = g * 64;
+        const int nh = BN - c0 < 64 ? 1 : 2;  // 32-column halves in this group
         uint32_t r[64];
         tmem_ld32(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        if (nh == 2) tmem_ld32(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_ld_wait();
         const float *b = a.bias + col0 + c0;
         if constexpr (EPI == EPI_BF16 || EPI == EPI_GELU_BF16) {
@@ -323,6 +327,7 @@ __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensor
         } else {
 #pragma unroll
             for (int hh = 0; hh < 2; hh++) {
+                if (hh >= nh) break;
                 uint8_t *stage = next_stage();
 #pragma unroll
                 for (int q = 0; q < 8; q++) {
@@ -576,8 +581,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
     using C = Gemm2Cfg<BN, KSUB>;
     // plain row-major outputs leave through TMA boxes (tmC); the conv and
     // conv_out row mappings and SwiGLU keep per-row stores
-    constexpr bool TMA_OUT = AMODE == A_PLAIN && BN % 64 == 0 &&
-                             (EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 || EPI == EPI_F32);
+    constexpr bool TMA_OUT = AMODE == A_PLAIN &&
+                             ((BN % 64 == 0 && (EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 ||
+                                                EPI == EPI_F32)) ||
+                              (BN % 64 == 32 && (EPI == EPI_RESID_F32 || EPI == EPI_F32)));
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES + C::STAGING);

@@ -218,7 +218,7 @@ template <int BN, int EPI>
 static bool tmap_out(CUtensorMap *m, const GemmArgs &a, const CUtensorMap &fallback)
 {
     const bool f32 = EPI == EPI_RESID_F32 || EPI == EPI_F32;
-    const bool tma = BN % 64 == 0 && (f32 || EPI == EPI_BF16 || EPI == EPI_GELU_BF16);
+    const bool tma = (BN % 64 == 0 && (f32 || EPI == EPI_BF16 || EPI == EPI_GELU_BF16)) || (BN % 64 == 32 && f32);
     if (!tma) {
         *m = fallback;
         return true;
@@ -688,6 +688,7 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm2_attr<256, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm2_attr<160, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_SWIGLU_BF16>()));
@@ -1252,14 +1253,36 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
     CUtensorMap tm_qkv;  // Q, K, V slices of one window and head: ATTN_ROWS rows x 64
     if (!tmap_2d(&tm_qkv, h->qkv, (uint64_t)DQKV, (uint64_t)T, (uint64_t)DQKV * 2, 64, ATTN_ROWS))
         return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (qkv)");
-    // The N = 1280 residual GEMMs (out-proj, FC2) on a small batch have few
-    // 320-wide tiles (ceil(T / 256) x 4) for the SMs; 128-wide tiles give them
-    // 2.5 times as many.  The tile width does not change any output element's
-    // arithmetic, so a clip's rows are the same at every batch size.
-    const bool narrow = 4 * ((T + 255) / 256) < h->num_sms / 4;
+    // Tile width of the N = 1280 residual GEMMs (out-proj, FC2): the one whose
+    // busiest SM pair has the fewest output columns to compute (the pair
+    // tiles of one width are spread evenly over the pairs), ties broken
+    // toward 320 for the long K = 5120 mainloop (wider tiles need the least
+    // operand bandwidth per MMA) and toward 160 for K = 1280 (two tiles per
+    // pair let one tile's epilogue run under the other's mainloop).  The tile
+    // width does not change any output element's arithmetic, so a clip's rows
+    // are the same at every batch size.
+    auto resid_width = [&](int K) {
+        static const int long_k[3] = {320, 160, 128}, short_k[3] = {160, 128, 320};
+        const int *order = K > D ? long_k : short_k;
+        const int64_t m = (T + 255) / 256, pairs = std::max(1, h->num_sms / 2);
+        int best = 320;
+        int64_t best_cols = INT64_MAX;
+        for (int i = 0; i < 3; i++) {
+            const int64_t tiles = m * (D / order[i]);
+            const int64_t cols = (tiles + pairs - 1) / pairs * order[i];
+            if (cols < best_cols) {
+                best_cols = cols;
+                best = order[i];
+            }
+        }
+        return best;
+    };
     auto resid_gemm = [&](const char *name, const bf16 *Ain, int K, const bf16 *W, GemmArgs a) -> moss_enc_status {
-        if (narrow) return gemm2<128, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, 2);
-        return gemm2<320, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, K == D ? 2 : 1);
+        switch (resid_width(K)) {
+        case 128: return gemm2<128, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, 2);
+        case 160: return gemm2<160, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, 2);
+        default: return gemm2<320, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, K == D ? 2 : 1);
+        }
     };
     for (size_t l = 0; l < h->layers.size(); l++) {
         const LayerDev &L = h->layers[l];

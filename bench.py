@@ -12,6 +12,11 @@ flush, outside the events); barrier + synchronize on both sides of the K
 steps; multi-GPU runs take the max over ranks, each rank encoding its own
 batch (clips are independent: weak scaling, no collective on the data path).
 
+At N = 1 the line also carries `other_configs`: the 1 s / 4-layer clip, the
+single 30 s clip, the 10-min clip and the 60-min clip streamed in 64 s pieces
+(with the encoder's device memory), each timed the same way; and
+`cpu_baseline` times the oracle on all host cores and on one core.
+
 The reference arm (--impl reference) times the CPU oracle on the host cores
 on one 800-frame window of the same batch per step.
 """
@@ -179,7 +184,7 @@ def profiled_traffic(kernel):
         with open(p) as f:
             d = json.load(f)
         e = d[kernel]
-        if e.get("source_hash") != gemm_source_hash():
+        if e.get("captured_source_hash") != gemm_source_hash():
             return None
         return e["bytes_per_launch_full_size"]
     except Exception:
@@ -362,9 +367,10 @@ def run_ours(args):
     kernel_ms = sum(v["ms"] for v in stats.values())
     if dom["flops"] > 0 and dom_name.startswith("gemm"):
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_sus"],
-                "peak_note": f"{pk['src']} sustained bf16 (kernel timed inside a long step)"}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16"], "frac_of_sustained": achieved / pk["bf16_sus"],
+                "peak_note": f"{pk['src']} burst bf16 (the sustained figure, {pk['bf16_sus']}, gives "
+                             f"frac_of_sustained)"}
     else:
         achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
@@ -385,7 +391,7 @@ def run_ours(args):
         cpu = {"value": (toks / 12.5) / dt, "unit": "audio-s/s", "cores": cores, "kind": "oracle",
                "sample": f"first {args.cpu_windows} 800-frame windows of clip 0 ({toks} tokens, "
                          f"{toks / 12.5:.0f} s of audio), all {n_layers} layers, {dt:.1f} s"}
-        if args.cpu_one_core:
+        if not args.no_cpu_one_core:
             dt1, toks1, _ = oracle_sample(clips, n_layers, windows=1, blob=blob, threads=1)
             cpu["one_core"] = {"value": (toks1 / 12.5) / dt1, "unit": "audio-s/s", "cores": 1,
                                "sample": f"first 800-frame window of clip 0 ({toks1} tokens), {dt1:.1f} s"}
@@ -416,26 +422,25 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "clocks": clk.summary(),
     }
-    print(json.dumps(line), flush=True)
     enc.close()
+    if world == 1 and not args.no_other_configs and not tap_layers:
+        line["other_configs"] = other_configs(args, dev)
+    print(json.dumps(line), flush=True)
     if dist:
         dist.destroy_process_group()
 
 
-def run_streamed(args):
+def measure_streamed(steps, warmup, dev, dist=None, world=1):
     """The 60-min clip encoded as a stream of 64 s pieces (1,024,000 samples,
     the last 256,000): a step is the whole-clip log-mel maximum (one pass)
     and the 57 piece forwards against it, each piece reading its 200-sample
-    halo from the whole clip.  Reports sustained audio-seconds per second and
-    the device memory the encoder holds (weights + workspace for one piece)
-    beside the resident clip and its rows.  Weak scaling: every rank streams
-    its own clip."""
+    halo from the whole clip.  Returns the step time (max over ranks), the
+    launch count, the clock record and the device memory the encoder holds
+    (weights + workspace for one piece)."""
     import torch
 
     from audio_encoder_b200 import binding
 
-    rank, world, dist = dist_setup(args.gpus)
-    dev = torch.device("cuda", torch.cuda.current_device())
     desc, clips, n_layers = workload_clips("clip_60min_streamed")
     pcm = clips[0]
     n = pcm.size
@@ -468,16 +473,16 @@ def run_streamed(args):
             for b, e, o0, o1 in ranges:
                 enc.forward([(x, b, e, lm)], out=out[o0:o1])
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(warmup):
         step()
     enc.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     launches0 = enc.launch_count()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with Clocks(dev.index) as clk:
-        for i in range(args.steps):
+        for i in range(steps):
             with torch.cuda.stream(stream):
                 flush.fill_(float(i))
                 ev[i][0].record(stream)
@@ -489,33 +494,109 @@ def run_streamed(args):
         dist.barrier()
     launches = enc.launch_count() - launches0
     total_ms = reduce_max(float(sum(a.elapsed_time(c) for a, c in ev)), dist, dev)
-    ms = total_ms / args.steps
-    audio_s = n / 16000.0
+    enc.close()
+    return dict(desc=desc, ms=total_ms / steps, audio_s=n / 16000.0, tokens=tokens, n_layers=n_layers,
+                pieces=len(ranges), piece=piece, launches=launches, clocks=clk.summary(),
+                encoder_device_bytes=int(free0 - free1), clip_and_rows_device_bytes=int(4 * n + 2 * tokens * 2048))
+
+
+def run_streamed(args):
+    """bench --workload clip_60min_streamed: sustained audio-seconds per
+    second of the 60-min clip streamed in 64 s pieces, and the device memory
+    the encoder holds.  Weak scaling: every rank streams its own clip."""
+    import torch
+
+    rank, world, dist = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    warmup = max(args.warmup, 3)
+    r = measure_streamed(args.steps, warmup, dev, dist, world)
+    ms = r["ms"]
     pk = peaks()
-    tflops = model_flops(tokens, n_layers) / (ms / 1e3) / 1e12
+    tflops = model_flops(r["tokens"], r["n_layers"]) / (ms / 1e3) / 1e12
     if rank == 0:
         line = {
-            "metric": "audio-sec encoded/sec", "value": weak_scaling_throughput(world, audio_s, ms),
-            "unit": "audio-s/s", "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+            "metric": "audio-sec encoded/sec", "value": weak_scaling_throughput(world, r["audio_s"], ms),
+            "unit": "audio-s/s", "n_gpus": world, "steps": args.steps, "warmup": warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded PCM, random-init bf16 weights)",
-            "tokens_per_s": weak_scaling_throughput(world, tokens, ms),
-            "model_tflops": tflops, "tc_roofline_frac_sustained": tflops / pk["bf16_sus"],
-            "config": {"workload": "clip_60min_streamed", "description": desc, "pieces": len(ranges),
-                       "piece_samples": piece, "audio_s_per_gpu": audio_s, "tokens_per_gpu": tokens,
-                       "layers": n_layers, "out_dtype": "bf16",
-                       "encoder_device_bytes": int(free0 - free1),
-                       "clip_and_rows_device_bytes": int(4 * n + 2 * tokens * 2048),
+            "tokens_per_s": weak_scaling_throughput(world, r["tokens"], ms),
+            "model_tflops": tflops, "tc_roofline_frac": tflops / pk["bf16"],
+            "tc_roofline_frac_sustained": tflops / pk["bf16_sus"],
+            "config": {"workload": "clip_60min_streamed", "description": r["desc"], "pieces": r["pieces"],
+                       "piece_samples": r["piece"], "audio_s_per_gpu": r["audio_s"], "tokens_per_gpu": r["tokens"],
+                       "layers": r["n_layers"], "out_dtype": "bf16",
+                       "encoder_device_bytes": r["encoder_device_bytes"],
+                       "clip_and_rows_device_bytes": r["clip_and_rows_device_bytes"],
                        "l2": "512 MB buffer written between timed steps (outside the events)",
                        "parallelism": f"dp{world}" if world > 1 else "single"},
-            "gpu_launches": launches,
+            "gpu_launches": r["launches"],
             "e2e": None,
-            "clocks": clk.summary(),
+            "clocks": r["clocks"],
         }
         print(json.dumps(line), flush=True)
-    enc.close()
     if dist:
         dist.destroy_process_group()
+
+
+def measure_plain(workload, steps, warmup, dev):
+    """One workload's forward timed as the headline is (device-resident PCM,
+    CUDA events on the encoder's stream, L2 flushed between steps)."""
+    import torch
+
+    from audio_encoder_b200 import binding
+
+    desc, clips, n_layers = workload_clips(workload)
+    stream = torch.cuda.Stream()
+    total = sum(c.size for c in clips)
+    enc = binding.Encoder(synth.make_weights(n_layers), n_layers, max_samples=total, max_clips=len(clips),
+                          out_dtype=binding.OUT_BF16, stream=stream)
+    tokens = sum(binding.num_tokens(c.size) for c in clips)
+    with torch.cuda.stream(stream):
+        xs = [torch.from_numpy(c).to(dev) for c in clips]
+        out = torch.empty((tokens, 2048), dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        enc.forward(xs, out=out)
+    enc.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with Clocks(dev.index) as clk:
+        for i in range(steps):
+            with torch.cuda.stream(stream):
+                flush.fill_(float(i))
+                ev[i][0].record(stream)
+                enc.forward(xs, out=out)
+                ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    enc.synchronize()
+    enc.close()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    return dict(desc=desc, ms=ms, audio_s=total / 16000.0, tokens=tokens, n_layers=n_layers, clocks=clk.summary())
+
+
+def other_configs(args, dev):
+    """Throughput of the other workloads at N = 1, each timed as the headline
+    (the single 30 s clip, the 10-min clip, the 1 s / 4-layer clip, and the
+    60-min clip streamed in 64 s pieces with the encoder's device memory)."""
+    pk = peaks()
+    res = {}
+    steps = max(3, min(args.steps, 20))
+    for w in ("tiny_1s", "single_30s", "clip_10min", "clip_60min_streamed"):
+        if w == "clip_60min_streamed":
+            r = measure_streamed(max(3, min(args.steps, 10)), 3, dev)
+        else:
+            r = measure_plain(w, steps, 3, dev)
+        tf = model_flops(r["tokens"], r["n_layers"]) / (r["ms"] / 1e3) / 1e12
+        e = {"value": r["audio_s"] / (r["ms"] / 1e3), "unit": "audio-s/s", "ms_per_step": r["ms"],
+             "tokens_per_s": r["tokens"] / (r["ms"] / 1e3), "tokens": r["tokens"], "layers": r["n_layers"],
+             "model_tflops": tf, "tc_roofline_frac": tf / pk["bf16"], "tc_roofline_frac_sustained": tf / pk["bf16_sus"],
+             "description": r["desc"], "clocks": r["clocks"]}
+        if w == "clip_60min_streamed":
+            e.update({"pieces": r["pieces"], "piece_samples": r["piece"],
+                      "encoder_device_bytes": r["encoder_device_bytes"],
+                      "clip_and_rows_device_bytes": r["clip_and_rows_device_bytes"]})
+        res[w] = e
+    return res
 
 
 def run_sharded(args):
@@ -606,8 +687,10 @@ def main():
     ap.add_argument("--workload", default="batch16_10to30s", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cpu-windows", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-one-core", action="store_true",
-                    help="also time the oracle on one host core (one 800-frame window)")
+    ap.add_argument("--no-cpu-one-core", action="store_true",
+                    help="skip timing the oracle on one host core (one 800-frame window)")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="report the default workload only (no per-config numbers for the other workloads)")
     ap.add_argument("--shard-clip", action="store_true",
                     help="one long clip (10 or 60 min) split over the ranks by chunk ranges (strong scaling)")
     ap.add_argument("--taps", default="",

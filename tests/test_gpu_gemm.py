@@ -66,10 +66,10 @@ def test_bf16_gemm_does_not_depend_on_tile_width(enc, M, K):
 
 @pytest.mark.parametrize("M,K", [(375, 1280), (800, 5120), (4608, 1280)])
 def test_residual_gemm_does_not_depend_on_tile_width(enc, M, K):
-    # the forward picks 128-wide tiles for the N = 1280 residual GEMMs of small
-    # batches and 320-wide ones for large; every output element's sum over K
-    # runs through the same MMA k-steps either way, so the results agree bit
-    # for bit (which keeps a clip's rows the same alone and in a batch)
+    # the forward picks 128-, 160- or 320-wide tiles for the N = 1280 residual
+    # GEMMs by batch size; every output element's sum over K runs through the
+    # same MMA k-steps whatever the width, so the results agree bit for bit
+    # (which keeps a clip's rows the same alone and in a batch)
     N = 1280
     g = torch.Generator().manual_seed(M + K)
     A = (torch.randn(M, K, generator=g) / K ** 0.25).bfloat16().cuda()
@@ -77,12 +77,12 @@ def test_residual_gemm_does_not_depend_on_tile_width(enc, M, K):
     bias = (torch.randn(N, generator=g) * 0.1).cuda()
     base = torch.randn(M, N, generator=g).cuda()
     outs = []
-    for block_n in (128, 320):
+    for block_n in (128, 160, 320):
         out = base.clone()
         enc.gemm(A, B, bias, out, 2, block_n, True)
         outs.append(out)
     torch.cuda.synchronize()
-    assert torch.equal(outs[0], outs[1])
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
 def test_fast_gelu_matches_erff(enc):
