@@ -689,6 +689,7 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm2_attr<320, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<160, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm2_attr<128, EPI_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_SWIGLU_BF16>()));
@@ -1143,6 +1144,29 @@ static std::vector<uint8_t> request_key(const moss_enc_clip *clips, int n_clips,
     return k;
 }
 
+// Pair-tile width for an M x N x K GEMM among the candidates `order`: the one
+// whose busiest SM pair has the fewest output columns to compute (pair tiles
+// of one width are spread evenly over the pairs), with 128-wide tiles counted
+// 1.5 times for long mainloops (K >= 4096), where an N = 128 MMA's lower rate
+// dominates (measured 2358 against 3707-3811 MACs per clock and SM for N of
+// 256 or 160).  Ties go to the earlier candidate.  The tile width never
+// changes an output element's arithmetic.
+static int pick_width(const moss_enc *h, int64_t M, int N, int K, const int *order, int n)
+{
+    const int64_t m = (M + 255) / 256, pairs = std::max(1, h->num_sms / 2);
+    int best = order[0];
+    double best_cost = 1e300;
+    for (int i = 0; i < n; i++) {
+        const int64_t tiles = m * (N / order[i]);
+        const double cost = (double)((tiles + pairs - 1) / pairs) * order[i] * (order[i] == 128 && K >= 4096 ? 1.5 : 1.0);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = order[i];
+        }
+    }
+    return best;
+}
+
 // ln_post -> proj1 -> GELU -> proj2 -> SwiGLU adapter on the residual stream
 // X [T][1280], with the head set W; stops after proj2 (fp32 rows) when stage
 // is MOSS_ENC_STAGE_HEAD, else writes the adapter rows (cfg.out_dtype).
@@ -1187,8 +1211,13 @@ static moss_enc_status head_launch(moss_enc *h, const HeadDev &W, int64_t T, int
     a.out = out;
     a.ldo = DOUT;
     a.split_off = 0;
-    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32) return gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
-    return gemm2<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
+    static const int down_w[2] = {256, 128};
+    const bool narrow = pick_width(h, T, DOUT, DADP, down_w, 2) == 128;
+    if (h->cfg.out_dtype == MOSS_ENC_OUT_F32)
+        return narrow ? gemm2<128, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a)
+                      : gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
+    return narrow ? gemm2<128, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a)
+                  : gemm2<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
 }
 
 static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt, int stage, void *out,
@@ -1261,24 +1290,9 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
     // pair let one tile's epilogue run under the other's mainloop).  The tile
     // width does not change any output element's arithmetic, so a clip's rows
     // are the same at every batch size.
-    auto resid_width = [&](int K) {
-        static const int long_k[3] = {320, 160, 128}, short_k[3] = {160, 128, 320};
-        const int *order = K > D ? long_k : short_k;
-        const int64_t m = (T + 255) / 256, pairs = std::max(1, h->num_sms / 2);
-        int best = 320;
-        int64_t best_cols = INT64_MAX;
-        for (int i = 0; i < 3; i++) {
-            const int64_t tiles = m * (D / order[i]);
-            const int64_t cols = (tiles + pairs - 1) / pairs * order[i];
-            if (cols < best_cols) {
-                best_cols = cols;
-                best = order[i];
-            }
-        }
-        return best;
-    };
     auto resid_gemm = [&](const char *name, const bf16 *Ain, int K, const bf16 *W, GemmArgs a) -> moss_enc_status {
-        switch (resid_width(K)) {
+        static const int long_k[3] = {320, 160, 128}, short_k[3] = {160, 128, 320};
+        switch (pick_width(h, T, D, K, K > D ? long_k : short_k, 3)) {
         case 128: return gemm2<128, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, 2);
         case 160: return gemm2<160, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, 2);
         default: return gemm2<320, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, K == D ? 2 : 1);

@@ -46,19 +46,20 @@ def test_gemm_epilogues(enc, pair, block_n, epi, M, K):
     assert err <= tol * max(scale, 1.0), (err, scale)
 
 
-@pytest.mark.parametrize("M,K", [(375, 1280), (512, 1280)])
-def test_bf16_gemm_does_not_depend_on_tile_width(enc, M, K):
-    # QKV of a batch of at most 512 tokens runs on 128-wide tiles, larger ones
-    # on 256-wide: same arithmetic per output element, same bits
-    N = 3840
+@pytest.mark.parametrize("M,K,N,epi", [(375, 1280, 3840, 0), (512, 1280, 3840, 0), (375, 8192, 2048, 0),
+                                       (1000, 8192, 2048, 5)])
+def test_gemm_does_not_depend_on_tile_width(enc, M, K, N, epi):
+    # QKV of a batch of at most 512 tokens and the adapter's down-projection
+    # of a small batch run on 128-wide tiles, larger ones on 256-wide: same
+    # arithmetic per output element, same bits
     g = torch.Generator().manual_seed(M + K + 1)
     A = (torch.randn(M, K, generator=g) / K ** 0.25).bfloat16().cuda()
     B = (torch.randn(N, K, generator=g) / K ** 0.25).bfloat16().cuda()
     bias = (torch.randn(N, generator=g) * 0.1).cuda()
     outs = []
     for block_n in (128, 256):
-        out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-        enc.gemm(A, B, bias, out, 0, block_n, True)
+        out = torch.empty(M, N, dtype=torch.bfloat16 if epi == 0 else torch.float32, device="cuda")
+        enc.gemm(A, B, bias, out, epi, block_n, True)
         outs.append(out)
     torch.cuda.synchronize()
     assert torch.equal(outs[0], outs[1])
