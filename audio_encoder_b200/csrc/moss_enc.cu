@@ -86,10 +86,14 @@ struct moss_enc {
     float *pcm_stage = nullptr;
     void *out_stage = nullptr;
 
-    // per-call tables: device copies and one pinned host staging area
+    // per-call tables: device copies and a ring of pinned host staging areas
+    // (a call writes the next area once the copy that last read it has run,
+    // so the host may run several calls ahead of the device)
+    static constexpr int TAB_SLOTS = 4;
     size_t tab_bytes = 0;
-    void *d_tab = nullptr, *h_tab = nullptr;
-    cudaEvent_t tab_event = nullptr;
+    void *d_tab = nullptr, *h_tab = nullptr, *h_tab_ring = nullptr;
+    cudaEvent_t tab_event[TAB_SLOTS] = {};
+    int tab_slot = 0;
 
     // launches may overlap the previous kernel's tail (programmatic dependent
     // launch); MOSS_ENC_PDL=0 in the environment at create turns it off
@@ -586,8 +590,9 @@ extern "C" void moss_enc_destroy(moss_enc *h)
     if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
     if (h->d_tab) cudaFree(h->d_tab);
     if (h->d_tab_graph) cudaFree(h->d_tab_graph);
-    if (h->h_tab) cudaFreeHost(h->h_tab);
-    if (h->tab_event) cudaEventDestroy(h->tab_event);
+    if (h->h_tab_ring) cudaFreeHost(h->h_tab_ring);
+    for (cudaEvent_t e : h->tab_event)
+        if (e) cudaEventDestroy(e);
     for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
     delete h;
 }
@@ -938,8 +943,10 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     h->tab_bytes = tl.total;
     if (cudaMalloc(&h->d_tab, tl.total) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaMalloc(&h->d_tab_graph, tl.total) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
-    if (cudaMallocHost(&h->h_tab, tl.total) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
-    if (cudaEventCreateWithFlags(&h->tab_event, cudaEventDisableTiming) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+    if (cudaMallocHost(&h->h_tab_ring, tl.total * moss_enc::TAB_SLOTS) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
+    h->h_tab = h->h_tab_ring;
+    for (cudaEvent_t &e : h->tab_event)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
     if (cudaDeviceSynchronize() != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
     *out = h;
     return MOSS_ENC_OK;
@@ -967,20 +974,26 @@ extern "C" moss_enc_status moss_enc_synchronize(moss_enc *h)
 
 // --------------------------------------------------------- per-call tables
 
-// The host staging area is reused by every call; wait until the copy that
-// last read it has run (not while a stream is being captured).
+// A call's tables are written into the next host staging area of the ring
+// (h->h_tab), once the copy that last read that area has run (not waited
+// for while a stream is being captured).
 static moss_enc_status tab_begin(moss_enc *h)
 {
+    h->tab_slot = (h->tab_slot + 1) % moss_enc::TAB_SLOTS;
+    h->h_tab = static_cast<uint8_t *>(h->h_tab_ring) + (size_t)h->tab_slot * h->tab_bytes;
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     CUDA_TRY(h, cudaStreamIsCapturing(h->stream, &cs));
-    if (cs == cudaStreamCaptureStatusNone) CUDA_TRY(h, cudaEventSynchronize(h->tab_event));
+    if (cs == cudaStreamCaptureStatusNone) CUDA_TRY(h, cudaEventSynchronize(h->tab_event[h->tab_slot]));
     return MOSS_ENC_OK;
 }
 
-static moss_enc_status tab_upload(moss_enc *h)
+// Copy the current tables to dst (the device tables of launch-by-launch
+// calls, or those a captured forward graph reads), in stream order: the copy
+// runs after every earlier kernel on the stream has finished with them.
+static moss_enc_status tab_upload(moss_enc *h, void *dst = nullptr)
 {
-    CUDA_TRY(h, cudaMemcpyAsync(h->d_tab, h->h_tab, h->tab_bytes, cudaMemcpyHostToDevice, h->stream));
-    CUDA_TRY(h, cudaEventRecord(h->tab_event, h->stream));
+    CUDA_TRY(h, cudaMemcpyAsync(dst ? dst : h->d_tab, h->h_tab, h->tab_bytes, cudaMemcpyHostToDevice, h->stream));
+    CUDA_TRY(h, cudaEventRecord(h->tab_event[h->tab_slot], h->stream));
     return MOSS_ENC_OK;
 }
 
@@ -1123,24 +1136,23 @@ struct FwdPlan {
     std::vector<int> g_off2, g_n2, g_off3, g_n3;
 };
 
-// Identity of a forward request for graph reuse: clips, output and the tap
-// outputs (the tap layers and weights are fixed between set_taps calls, which
-// drop the graph).
-static std::vector<uint8_t> request_key(const moss_enc_clip *clips, int n_clips, const void *out,
-                                        void *const *tap_out, int n_taps)
+// Shape of a forward request for graph reuse: every host-side value the
+// launch sequence depends on (grids, GEMM sizes, the stem groups' tile
+// counts) and the tap outputs.  Two requests of one shape launch the same
+// kernels with the same parameters; what differs between them (the PCM
+// pointers and ranges, the per-chunk tables) is read from the device tables.
+static std::vector<uint8_t> shape_key(const FwdPlan &P, void *const *tap_out, int n_taps)
 {
     const int nt = tap_out ? n_taps : 0;
-    std::vector<uint8_t> k(2 * sizeof(int) + sizeof(void *) * (1 + (size_t)nt) + sizeof(moss_enc_clip) * (size_t)n_clips);
-    uint8_t *q = k.data();
-    std::memcpy(q, &n_clips, sizeof(int));
-    q += sizeof(int);
-    std::memcpy(q, &nt, sizeof(int));
-    q += sizeof(int);
-    std::memcpy(q, &out, sizeof(void *));
-    q += sizeof(void *);
-    if (nt > 0) std::memcpy(q, tap_out, sizeof(void *) * (size_t)nt);
-    q += sizeof(void *) * (size_t)nt;
-    if (n_clips > 0) std::memcpy(q, clips, sizeof(moss_enc_clip) * (size_t)n_clips);
+    std::vector<int64_t> v = {P.n_clips, P.n_chunks, P.T, P.n_max_pass, P.max_clip_frames, P.max_range_frames, nt,
+                              (int64_t)P.g_n2.size()};
+    for (size_t g = 0; g < P.g_n2.size(); g++) {
+        v.push_back(P.g_n2[g]);
+        v.push_back(P.g_n3[g]);
+    }
+    for (int t = 0; t < nt; t++) v.push_back((int64_t)reinterpret_cast<uintptr_t>(tap_out[t]));
+    std::vector<uint8_t> k(v.size() * sizeof(int64_t));
+    std::memcpy(k.data(), v.data(), k.size());
     return k;
 }
 
@@ -1456,22 +1468,32 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     P.g_off3 = std::move(g_off3);
     P.g_n3 = std::move(g_n3);
 
-    // Whole forwards run as one CUDA graph once a request repeats: the second
-    // consecutive call with the same request (clips, ranges, output, taps)
-    // captures it, later ones replay it.  A stream of different requests (the
-    // pieces of a long clip) runs launch by launch and never pays for a
-    // capture.  The graph reads its own copy of the tables.
+    // Whole forwards run as one CUDA graph once a request shape repeats: the
+    // second consecutive call of one shape (clip and chunk structure, taps)
+    // captures it, later calls of that shape replay it with their own tables
+    // (copied, in stream order, into the tables the graph reads).  The graph
+    // writes the rows to the workspace's output area, and one device copy
+    // moves them to the caller's buffer, so pieces of a long clip with
+    // different output ranges share the graph.  A request of a new shape runs
+    // launch by launch and never pays for a capture.
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     CUDA_TRY(h, cudaStreamIsCapturing(h->stream, &cs));
     const int n_taps = (int)h->tap_layers.size();
     const bool graphable = stage == MOSS_ENC_STAGE_ADAPTER && !h->profiling && h->stream != nullptr &&
                            cs == cudaStreamCaptureStatusNone;
+    const size_t out_bytes = (size_t)T * DOUT * (h->cfg.out_dtype == MOSS_ENC_OUT_F32 ? 4 : 2);
+    auto rows_to_caller = [&]() -> moss_enc_status {
+        if (out != h->out_stage)
+            CUDA_TRY(h, cudaMemcpyAsync(out, h->out_stage, out_bytes, cudaMemcpyDeviceToDevice, h->stream));
+        return MOSS_ENC_OK;
+    };
     std::vector<uint8_t> key;
-    if (graphable) key = request_key(clips, n_clips, out, tap_out, n_taps);
+    if (graphable) key = shape_key(P, tap_out, n_taps);
     if (graphable && h->graph_exec && h->graph_key == key) {
+        TRY(tab_upload(h, h->d_tab_graph));
         h->launches += h->graph_launches;
         CUDA_TRY(h, cudaGraphLaunch(h->graph_exec, h->stream));
-        return MOSS_ENC_OK;
+        return rows_to_caller();
     }
     if (!graphable || key != h->last_key) {
         if (graphable) h->last_key = std::move(key);
@@ -1482,11 +1504,10 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
         cudaGraphExecDestroy(h->graph_exec);
         h->graph_exec = nullptr;
     }
-    CUDA_TRY(h, cudaMemcpyAsync(h->d_tab_graph, h->h_tab, h->tab_bytes, cudaMemcpyHostToDevice, h->stream));
-    CUDA_TRY(h, cudaEventRecord(h->tab_event, h->stream));
+    TRY(tab_upload(h, h->d_tab_graph));
     const int64_t launches0 = h->launches;
     CUDA_TRY(h, cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
-    const moss_enc_status st = forward_launch(h, P, static_cast<uint8_t *>(h->d_tab_graph), stage, out, tap_out);
+    const moss_enc_status st = forward_launch(h, P, static_cast<uint8_t *>(h->d_tab_graph), stage, h->out_stage, tap_out);
     cudaGraph_t g = nullptr;
     const cudaError_t ce = cudaStreamEndCapture(h->stream, &g);
     if (st != MOSS_ENC_OK || ce != cudaSuccess) {
@@ -1503,7 +1524,7 @@ static moss_enc_status forward_impl(moss_enc *h, const moss_enc_clip *clips, int
     h->graph_key = std::move(key);
     h->graph_launches = h->launches - launches0;
     CUDA_TRY(h, cudaGraphLaunch(h->graph_exec, h->stream));
-    return MOSS_ENC_OK;
+    return rows_to_caller();
 }
 
 
