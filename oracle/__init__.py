@@ -80,6 +80,9 @@ def lib():
         L.oracle_adapter.argtypes = [vp, vp, i32, vp]
         L.oracle_encode_chunks.restype = i64
         L.oracle_encode_chunks.argtypes = [vp, vp, i64, i64, i64, f32, i32, vp, vp, vp, vp]
+        L.oracle_model_create_bits.restype = vp
+        L.oracle_model_create_bits.argtypes = [vp, i32, i32]
+        L.oracle_quant_rtn4.argtypes = [vp, i32, i32, vp, vp, vp]
         L.oracle_set_threads.argtypes = [i32]
         L.oracle_max_threads.restype = i32
     return _lib
@@ -176,16 +179,32 @@ def weight_count(n_layers: int) -> int:
     return int(lib().oracle_weight_count(n_layers))
 
 
-class Model:
-    """The oracle's copy of a bf16 weight blob (uint16 bit patterns)."""
+def quant_rtn4(w: np.ndarray):
+    """4-bit round-to-nearest quantisation in groups of 128 along the last
+    axis of a bf16 matrix (uint16 bits) [rows][cols]: returns (w' as bf16
+    bits, codes q + 8 as uint8, scales [rows][cols / 128] fp32)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    rows, cols = w.shape
+    if cols % 128:
+        raise ValueError("cols must be a multiple of 128")
+    deq = np.empty_like(w)
+    codes = np.empty((rows, cols), dtype=np.uint8)
+    scales = np.empty((rows, cols // 128), dtype=np.float32)
+    lib().oracle_quant_rtn4(_p(w), rows, cols, _p(deq), _p(codes), _p(scales))
+    return deq, codes, scales
 
-    def __init__(self, blob: np.ndarray, n_layers: int):
+
+class Model:
+    """The oracle's copy of a bf16 weight blob (uint16 bit patterns);
+    weight_bits=4 gives the model with 4-bit quantised linear layers."""
+
+    def __init__(self, blob: np.ndarray, n_layers: int, weight_bits: int = 16):
         blob = np.ascontiguousarray(blob, dtype=np.uint16)
         if blob.size != weight_count(n_layers):
             raise ValueError(f"blob has {blob.size} elements, expected {weight_count(n_layers)}")
         self._blob = blob  # the model points into it
         self.n_layers = n_layers
-        self._h = lib().oracle_model_create(_p(blob), n_layers)
+        self._h = lib().oracle_model_create_bits(_p(blob), n_layers, int(weight_bits))
 
     def close(self):
         if self._h:

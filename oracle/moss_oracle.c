@@ -304,10 +304,80 @@ static uint16_t *transpose_bf16(const uint16_t *w, int out, int in)
     return t;
 }
 
+/* ------------------------------------------------ 4-bit weight quantisation
+ *
+ * Page "Ossicle-4B", "Long Audio", note under the table: the 4-bit variant
+ * keeps "4-bit weights for the language model and the audio encoder, round to
+ * nearest, groups of 128".  Reading (the page gives no more): symmetric
+ * round-to-nearest over groups of 128 consecutive input features of each
+ * output row; the group's scale is its largest magnitude over 7, so codes lie
+ * in [-7, 7] (the 4-bit range [-8, 7] is the clamp); a weight's value in the
+ * quantised model is its code times the scale.  The arithmetic is fixed so
+ * that two implementations agree bit for bit:
+ *   s   = fp32(max |w|) / 7            (fp32 division)
+ *   q   = clamp(rint(w / s), -8, 7)    (fp32 division, ties to even; 0 if s = 0)
+ *   w'  = bf16(fp32(q * s))            (fp32 product, then to bf16, ties to even)
+ * The linear layers of the 32 encoder layers, the encoder head and the adapter
+ * are quantised; the conv stem (conv1..conv3 and conv_out) keeps bf16. */
+
+/* Round an fp32 value to the nearest bf16, ties to even (finite inputs). */
+static uint16_t bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    const uint32_t lsb = (u >> 16) & 1u;
+    return (uint16_t)((u + 0x7FFFu + lsb) >> 16);
+}
+
+/* Quantise w [rows][cols] (bf16 bits, cols % 128 == 0) group by group.
+ * deq receives w' (bf16 bits); codes (optional) q + 8 in [0, 15]; scales
+ * (optional) s per [row][group]. */
+void oracle_quant_rtn4(const uint16_t *w, int rows, int cols, uint16_t *deq, uint8_t *codes, float *scales)
+{
+    const int groups = cols / 128;
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; r++)
+        for (int g = 0; g < groups; g++) {
+            const uint16_t *wg = w + (size_t)r * cols + (size_t)g * 128;
+            float amax = 0.0f;
+            for (int k = 0; k < 128; k++) {
+                const float a = fabsf(bff(wg[k]));
+                if (a > amax) amax = a;
+            }
+            const float s = amax / 7.0f;
+            if (scales) scales[(size_t)r * groups + g] = s;
+            for (int k = 0; k < 128; k++) {
+                float q = 0.0f;
+                if (s > 0.0f) {
+                    q = rintf(bff(wg[k]) / s);
+                    if (q < -8.0f) q = -8.0f;
+                    if (q > 7.0f) q = 7.0f;
+                }
+                const size_t i = (size_t)r * cols + (size_t)g * 128 + k;
+                if (codes) codes[i] = (uint8_t)((int)q + 8);
+                const float v = q * s;
+                deq[i] = bf16_rne(v);
+            }
+        }
+}
+
+/* The blob's [out][in] matrix at p, quantised when bits == 4, transposed. */
+static uint16_t *take_linear(const uint16_t *p, int out, int in, int bits)
+{
+    if (bits != 4) return transpose_bf16(p, out, in);
+    uint16_t *q = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)out * in);
+    oracle_quant_rtn4(p, out, in, q, NULL, NULL);
+    uint16_t *t = transpose_bf16(q, out, in);
+    free(q);
+    return t;
+}
+
 /* Walks the blob in its documented order (conv1, conv2, conv3, conv_out,
  * layers, ln_post, proj1, proj2, adapter gate/up/down; each weight followed
- * by its bias, none for conv_out). */
-oracle_model *oracle_model_create(const uint16_t *blob, int n_layers)
+ * by its bias, none for conv_out).  weight_bits 4 gives the 4-bit model of
+ * the quantisation section above (its linear layers' weights w'); any other
+ * value the bf16 model. */
+oracle_model *oracle_model_create_bits(const uint16_t *blob, int n_layers, int weight_bits)
 {
     oracle_model *m = (oracle_model *)calloc(1, sizeof(oracle_model));
     const uint16_t *p = blob;
@@ -333,34 +403,39 @@ oracle_model *oracle_model_create(const uint16_t *blob, int n_layers)
         layer_w *L = &m->layers[l];
         L->ln1_g = p; p += D;
         L->ln1_b = p; p += D;
-        L->wq_t = transpose_bf16(p, D, D); p += (size_t)D * D;
+        L->wq_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
         L->bq = p; p += D;
-        L->wk_t = transpose_bf16(p, D, D); p += (size_t)D * D;
+        L->wk_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
         L->bk = p; p += D;
-        L->wv_t = transpose_bf16(p, D, D); p += (size_t)D * D;
+        L->wv_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
         L->bv = p; p += D;
-        L->wo_t = transpose_bf16(p, D, D); p += (size_t)D * D;
+        L->wo_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
         L->bo = p; p += D;
         L->ln2_g = p; p += D;
         L->ln2_b = p; p += D;
-        L->w1_t = transpose_bf16(p, D_FFN, D); p += (size_t)D_FFN * D;
+        L->w1_t = take_linear(p, D_FFN, D, weight_bits); p += (size_t)D_FFN * D;
         L->b1 = p; p += D_FFN;
-        L->w2_t = transpose_bf16(p, D, D_FFN); p += (size_t)D * D_FFN;
+        L->w2_t = take_linear(p, D, D_FFN, weight_bits); p += (size_t)D * D_FFN;
         L->b2 = p; p += D;
     }
     m->lnp_g = p; p += D;
     m->lnp_b = p; p += D;
-    m->wp1_t = transpose_bf16(p, D, D); p += (size_t)D * D;
+    m->wp1_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
     m->bp1 = p; p += D;
-    m->wp2_t = transpose_bf16(p, D_OUT, D); p += (size_t)D_OUT * D;
+    m->wp2_t = take_linear(p, D_OUT, D, weight_bits); p += (size_t)D_OUT * D;
     m->bp2 = p; p += D_OUT;
-    m->wg_t = transpose_bf16(p, D_ADP, D_OUT); p += (size_t)D_ADP * D_OUT;
+    m->wg_t = take_linear(p, D_ADP, D_OUT, weight_bits); p += (size_t)D_ADP * D_OUT;
     m->bg = p; p += D_ADP;
-    m->wu_t = transpose_bf16(p, D_ADP, D_OUT); p += (size_t)D_ADP * D_OUT;
+    m->wu_t = take_linear(p, D_ADP, D_OUT, weight_bits); p += (size_t)D_ADP * D_OUT;
     m->bu = p; p += D_ADP;
-    m->wd_t = transpose_bf16(p, D_OUT, D_ADP); p += (size_t)D_OUT * D_ADP;
+    m->wd_t = take_linear(p, D_OUT, D_ADP, weight_bits); p += (size_t)D_OUT * D_ADP;
     m->bd = p; p += D_OUT;
     return m;
+}
+
+oracle_model *oracle_model_create(const uint16_t *blob, int n_layers)
+{
+    return oracle_model_create_bits(blob, n_layers, 16);
 }
 
 /* Number of bf16 elements the blob holds for n_layers layers. */
