@@ -29,8 +29,10 @@ EXPORTED = [
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
     "moss_enc_tap_weight_count", "moss_enc_set_taps", "moss_enc_forward_taps",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
-    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_selftest_gelu", "moss_enc_selftest_timeout",
+    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_gemm_q4", "moss_enc_selftest_gelu",
+    "moss_enc_selftest_timeout",
 ]
+WEIGHTS_4BIT = 4
 STATIC_MAX_CLIPS = 64
 
 
@@ -42,7 +44,7 @@ class MossEncError(RuntimeError):
 
 class Config(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int), ("max_samples", ctypes.c_int64),
-                ("max_clips", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+                ("max_clips", ctypes.c_int), ("out_dtype", ctypes.c_int), ("weight_bits", ctypes.c_int)]
 
 
 class KernelStat(ctypes.Structure):
@@ -118,6 +120,8 @@ def lib():
         L.moss_enc_selftest_gelu.argtypes = [vp, ctypes.POINTER(ctypes.c_float)]
         L.moss_enc_gemm.restype = i32
         L.moss_enc_gemm.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32]
+        L.moss_enc_gemm_q4.restype = i32
+        L.moss_enc_gemm_q4.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32]
         L.moss_enc_logmel_static.restype = i32
         L.moss_enc_logmel_static.argtypes = [ctypes.POINTER(Clip), i32, ctypes.POINTER(vp), vp, vp]
         _lib = L
@@ -156,12 +160,12 @@ class Encoder:
     """
 
     def __init__(self, blob, n_layers: int, max_samples: int, max_clips: int = 1,
-                 out_dtype: int = OUT_F32, stream=None):
+                 out_dtype: int = OUT_F32, stream=None, weight_bits: int = 16):
         import torch
         self.torch = torch
         self.n_layers = n_layers
         self.out_dtype = out_dtype
-        cfg = Config(n_layers, int(max_samples), int(max_clips), int(out_dtype))
+        cfg = Config(n_layers, int(max_samples), int(max_clips), int(out_dtype), int(weight_bits))
         if stream is None:
             stream = torch.cuda.current_stream()
         self.stream = stream
@@ -219,6 +223,15 @@ class Encoder:
         N = B.shape[0]
         self._check(lib().moss_enc_gemm(self.h, _ptr(A), _ptr(B), _ptr(bias), _ptr(out), M, N, K,
                                         int(epilogue), int(block_n), int(bool(cta_pair))))
+        return out
+
+    def gemm_q4(self, A, Bq, Bs, bias, out, epilogue: int, block_n: int):
+        """out = epi(A @ B.T + bias) with B as 4-bit codes Bq [N][K/2] (uint8,
+        even k in the low nibble, code q + 8) and group scales Bs [K/128][N]."""
+        M, K = A.shape
+        N = Bq.shape[0]
+        self._check(lib().moss_enc_gemm_q4(self.h, _ptr(A), _ptr(Bq), _ptr(Bs), _ptr(bias), _ptr(out), M, N, K,
+                                           int(epilogue), int(block_n)))
         return out
 
     def selftest_timeout(self, limit_ms: int = 50):

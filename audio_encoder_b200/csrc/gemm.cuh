@@ -50,6 +50,10 @@ struct GemmArgs {
     // hi = bf16(v) at column c and lo = bf16(v - hi) at column c + split_off,
     // so that a following GEMM over [hi | lo] x [W | W] sees v to ~16 bits.
     int split_off;
+    // 4-bit B only: 64-wide k blocks of the stored matrix; the GEMM's k block
+    // kb reads stored block kb % kq_blocks (a [hi | lo] operand against [W | W]
+    // stores W once)
+    int kq_blocks;
 };
 
 // Each epilogue warp stages 32 rows x 128 B in shared memory (16-byte
@@ -523,7 +527,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 //    commits once to its own and once to the odd CTA's barrier.
 //  - tempty[acc] lives in the even CTA; all 16 epilogue warps of the pair
 //    arrive on it.
-template <int BN, int KSUB = 1>
+template <int BN, int KSUB = 1, int BQ = 0>
 struct Gemm2Cfg {
     // A stage holds KSUB k sub-blocks of 64 (one 128-byte swizzle atom each):
     // larger stages halve the stage hand-offs between the producer, the MMA
@@ -532,7 +536,9 @@ struct Gemm2Cfg {
     // a multiple of 4 (the TMEM lane quarters); 8 measured faster than 4 on
     // the layer GEMMs (FC1 45 vs 48-50 us, out-proj 21.5 vs 24.5-25 us)
     static constexpr int EPI_WARPS = 8;
-    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    // 4-bit B (BQ): four converter warps expand each stage's codes to bf16
+    static constexpr int CONV_WARPS = BQ ? 4 : 0;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * CONV_WARPS;
     // Tiles wider than one MMA (BN = 320) are two MMAs of BN/2 per k-step.
     static constexpr int NSUB = BN > 256 ? 2 : 1;
     static constexpr int NS = BN / NSUB;                        // N of one MMA instruction
@@ -541,7 +547,22 @@ struct Gemm2Cfg {
     static constexpr uint32_t A_BYTES = KSUB * A_SUB;
     static constexpr uint32_t B_KS = NSUB * B_SUB_BYTES;        // B bytes of one k sub-block
     static constexpr uint32_t B_BYTES = KSUB * B_KS;
-    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    // BQ: the codes of this CTA's B rows (32 bytes per row per 64-wide k
+    // block, two per byte, low nibble first) and their group scales (fp32),
+    // after the bf16 B they expand into.  Every TMA destination starts on a
+    // 128-byte boundary (the scale boxes of NS/2 rows are padded to it).
+    static constexpr uint32_t RAW_SUB = (NS / 2) * 32;
+    static constexpr uint32_t SC_BOX = (NS / 2) * 4;                   // bytes one scale box brings
+    static constexpr uint32_t SC_SUB = (SC_BOX + 127) / 128 * 128;     // its slot
+    static constexpr uint32_t RAW_OFF = A_BYTES + B_BYTES;
+    static constexpr uint32_t SC_OFF = RAW_OFF + NSUB * RAW_SUB;
+    static constexpr uint32_t Q_TX = BQ ? NSUB * (RAW_SUB + SC_BOX) : 0;  // bytes completing on rawfull[s]
+    static constexpr uint32_t Q_BYTES = BQ ? NSUB * (RAW_SUB + SC_SUB) : 0;
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + (Q_BYTES + 1023) / 1024 * 1024;
+    static_assert(RAW_OFF % 128 == 0 && SC_OFF % 128 == 0 && RAW_SUB % 128 == 0 && SC_SUB % 128 == 0,
+                  "TMA destinations on 128-byte boundaries");
+    // bytes each CTA's TMA completes on the pair's full barrier per stage
+    static constexpr uint32_t FULL_TX = BQ ? A_BYTES : A_BYTES + B_BYTES;
     static constexpr uint32_t STAGING = EPI_WARPS * EPI_STAGE_BYTES;
     static constexpr int STAGES_RAW = (int)((SMEM_LIMIT - 1024 - 256 - STAGING) / STAGE_BYTES);
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
@@ -554,6 +575,8 @@ struct Gemm2Cfg {
     static_assert(BN % 16 == 0 && BN >= 64 && BN <= 320, "BN must be a multiple of 16 in [64, 320]");
     static_assert(NS % 16 == 0 && NS <= 256, "MMA N");
     static_assert(B_SUB_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+    static_assert(!BQ || KSUB == 1, "4-bit B: one k sub-block per stage");
+    static_assert(3 * STAGES * 8 + 2 * 16 + 4 <= 256, "barriers fit their area");
 };
 
 // Tile t of the pair kernel.  Plain GEMMs walk row blocks first (pairs that
@@ -573,12 +596,53 @@ __device__ __forceinline__ void pair_tile(int tile, const GemmArgs &a, int &mt, 
     }
 }
 
-template <int BN, int EPI, int AMODE = A_PLAIN, int KSUB = 1>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::THREADS, 1)
-    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmC, const GemmArgs args)
+// Expands one stage's 4-bit B codes into the bf16 B tiles the MMA reads
+// (K-major, 128-byte swizzle), for the CTA's NSUB x NS/2 rows.  A value is
+// bf16(fp32(q) * s): the code u = q + 8 becomes q exactly in fp32 as
+// (2^23 + u) - (2^23 + 8) (u placed in the low bits of 2^23's significand),
+// is scaled in fp32 and rounded to bf16 once.  Thread ct of the
+// CONV_WARPS * 32 converters takes 16-byte output chunks ct, ct + 128, ...
+// (a chunk = 8 consecutive k of one row = 4 bytes of codes).
+template <class C>
+__device__ __forceinline__ void expand_q4(uint8_t *stage, int ct)
 {
-    using C = Gemm2Cfg<BN, KSUB>;
+    constexpr int NT = C::CONV_WARPS * 32;
+    constexpr int ROWS = C::NS / 2;
+    const float2 bias = make_float2(-8388616.0f, -8388616.0f);  // -(2^23 + 8)
+#pragma unroll 2
+    for (int i = ct; i < C::NSUB * ROWS * 8; i += NT) {
+        const int j = i / (ROWS * 8), rem = i - j * ROWS * 8, r = rem >> 3, c = rem & 7;
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(stage + C::RAW_OFF + j * C::RAW_SUB + r * 32 + c * 4);
+        const float sc = *reinterpret_cast<const float *>(stage + C::SC_OFF + j * C::SC_SUB + r * 4);
+        const float2 s2 = make_float2(sc, sc);
+        const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+        uint32_t o[4];
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+            // byte b of lo / hi: the codes of k = 8 c + 2 b and 8 c + 2 b + 1
+            const float2 m = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
+                                         __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u + b)));
+            const float2 v = __fmul2_rn(__fadd2_rn(m, bias), s2);
+            o[b] = pack_bf16x2(v.x, v.y);
+        }
+        *reinterpret_cast<uint4 *>(stage + C::A_BYTES + j * C::B_SUB_BYTES + r * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int BN, int EPI, int AMODE = A_PLAIN, int KSUB = 1, int BQ = 0>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, BQ>::THREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
+                    const GemmArgs args)
+{
+    using C = Gemm2Cfg<BN, KSUB, BQ>;
+    static_assert(!BQ || AMODE == A_PLAIN, "4-bit B for plain GEMMs");
     // plain row-major outputs leave through TMA boxes (tmC); the conv and
     // conv_out row mappings and SwiGLU keep per-row stores
     constexpr bool TMA_OUT = AMODE == A_PLAIN &&
@@ -589,7 +653,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES + C::STAGING);
     uint64_t *empty = full + C::STAGES;
-    uint64_t *tfull = empty + C::STAGES;
+    uint64_t *rawfull = empty + C::STAGES;  // BQ: this CTA's codes and scales of stage s have landed
+    uint64_t *tfull = rawfull + C::STAGES;
     uint64_t *tempty = tfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
 
@@ -597,8 +662,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
     const uint32_t rank = cluster_ctarank();
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; s++) {
-            mbar_init(&full[s], 2);
+            // both producers arrive (with their TMA bytes); with 4-bit B also
+            // one converter thread of each CTA once its bf16 B is in place
+            mbar_init(&full[s], BQ ? 4 : 2);
             mbar_init(&empty[s], 1);
+            mbar_init(&rawfull[s], 1);
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(&tfull[i], 1);
@@ -608,6 +676,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
         if constexpr (TMA_OUT) prefetch_tmap(&tmC);
+        if constexpr (BQ) prefetch_tmap(&tmS);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -627,13 +696,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
 
     if (warp == 0) {
         if (lane == 0) {
-            auto load_b = [&](uint8_t *st, uint32_t fb, int kb, int nt) {
+            auto load_b = [&](uint8_t *st, uint32_t fb, int kb, int nt, int s) {
+                if constexpr (BQ) {
+                    // this CTA's codes and scales, completing on its own rawfull[s]
+                    const int kq = kb % args.kq_blocks;
+                    mbar_arrive_expect_tx(&rawfull[s], C::Q_TX);
 #pragma unroll
-                for (int ks = 0; ks < KSUB; ks++)
+                    for (int j = 0; j < C::NSUB; j++) {
+                        const int row0 = nt * BN + j * C::NS + (int)rank * (C::NS / 2);
+                        tma_load_2d(&tmB, &rawfull[s], st + C::RAW_OFF + j * C::RAW_SUB, kq * 32, row0);
+                        tma_load_2d(&tmS, &rawfull[s], st + C::SC_OFF + j * C::SC_SUB, row0, kq >> 1);
+                    }
+                } else {
 #pragma unroll
-                    for (int j = 0; j < C::NSUB; j++)
-                        tma_load_2d_pair(&tmB, fb, st + C::A_BYTES + ks * C::B_KS + j * C::B_SUB_BYTES,
-                                         kb * C::BK + ks * 64, nt * BN + j * C::NS + (int)rank * (C::NS / 2));
+                    for (int ks = 0; ks < KSUB; ks++)
+#pragma unroll
+                        for (int j = 0; j < C::NSUB; j++)
+                            tma_load_2d_pair(&tmB, fb, st + C::A_BYTES + ks * C::B_KS + j * C::B_SUB_BYTES,
+                                             kb * C::BK + ks * 64, nt * BN + j * C::NS + (int)rank * (C::NS / 2));
+                }
             };
             // The weights do not depend on earlier kernels: the first tile's
             // first stages of B are requested before waiting for them (each
@@ -641,10 +722,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
             const int npre = pair < num_tiles ? (num_kb < C::STAGES ? num_kb : C::STAGES) : 0;
             for (int kb = 0; kb < npre; kb++) {
                 const uint32_t fb = map_to_rank(smem_u32(&full[kb]), 0);
-                mbar_arrive_expect_tx_remote(fb, C::STAGE_BYTES);
+                mbar_arrive_expect_tx_remote(fb, C::FULL_TX);
                 int mt0, nt0;
                 pair_tile<AMODE>(pair, args, mt0, nt0);
-                load_b(smem + kb * C::STAGE_BYTES, fb, kb, nt0);
+                load_b(smem + kb * C::STAGE_BYTES, fb, kb, nt0, kb);
             }
             grid_dep_wait();
             int s = 0;
@@ -665,7 +746,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
                     const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
                     if (!pre) {
                         if (!mbar_wait(&empty[s], ph ^ 1, args.err)) { ok = false; break; }
-                        mbar_arrive_expect_tx_remote(fb, C::STAGE_BYTES);
+                        mbar_arrive_expect_tx_remote(fb, C::FULL_TX);
                     }
 #pragma unroll
                     for (int ks = 0; ks < KSUB; ks++) {
@@ -677,7 +758,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
                             tma_load_2d_pair(&tmA, fb, st + ks * C::A_SUB, kb * C::BK + ks * 64, mt * 256 + (int)rank * 128);
                         }
                     }
-                    if (!pre) load_b(st, fb, kb, nt);
+                    if (!pre) load_b(st, fb, kb, nt, s);
                     if (++s == C::STAGES) { s = 0; ph ^= 1; }
                 }
             }
@@ -703,7 +784,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
                 for (int kb = 0; kb < num_kb; kb++) {
-                    if (!mbar_wait(&full[s], ph, args.err)) { ok = false; break; }
+                    // 4-bit B: the phase also publishes both CTAs' converter stores
+                    const bool got = BQ ? mbar_wait_cluster(&full[s], ph, args.err) : mbar_wait(&full[s], ph, args.err);
+                    if (!got) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
                     const uint64_t bd = ad + (C::A_BYTES >> 4);
@@ -732,7 +815,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
                 }
             }
         }
-    } else {
+    } else if (warp < 2 + C::EPI_WARPS) {
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;  // which of the warps on this lane quarter
         uint8_t *stage = smem + C::STAGES * C::STAGE_BYTES + (warp - 2) * EPI_STAGE_BYTES;
@@ -781,6 +864,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB>::
         }
         if constexpr (TMA_OUT) {
             if (lane == 0) bulk_wait_all();  // this warp's output boxes are written before the grid ends
+        }
+    } else if constexpr (BQ) {
+        // converters: stage s's codes -> bf16 B, then one arrive on the pair's
+        // full[s].  The codes are the weights (no earlier kernel writes them),
+        // so there is no wait on earlier grids.  A stage's B is rewritten only
+        // after its next codes land, which the producer requests only once the
+        // MMAs that read the stage have completed.
+        const int ct = threadIdx.x - 32 * (2 + C::EPI_WARPS);
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+            for (int kb = 0; kb < num_kb; kb++) {
+                if (!mbar_wait(&rawfull[s], ph, args.err)) { ok = false; break; }
+                uint8_t *st = smem + s * C::STAGE_BYTES;
+                expand_q4<C>(st, ct);
+                fence_async_smem();  // the generic-proxy stores are seen by the MMA's reads
+                named_bar_sync(1, C::CONV_WARPS * 32);
+                if (ct == 0) mbar_arrive_release_cluster(map_to_rank(smem_u32(&full[s]), 0));
+                if (++s == C::STAGES) { s = 0; ph ^= 1; }
+            }
         }
     }
     tc_fence_before();

@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cmath>
 #include <mutex>
+#include <thread>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -32,17 +33,29 @@ constexpr int CONV_BN = 240;     // conv2/conv3 output channels per pair tile (4
 constexpr int STEM_GROUP_DEFAULT = 32;
 constexpr int C2_TILES = 50, C3_TILES = 13;  // 128-row tiles per chunk of conv2 (4 t x 32 f) / conv3 (8 t x 16 f)
 
+// A weight matrix kept as 4-bit codes: codes [N][Kq/2] bytes (two per byte,
+// low nibble first, code = q + 8) and scales [Kq/128][N] fp32 (group-major).
+struct QW {
+    const uint8_t *codes = nullptr;
+    const float *scales = nullptr;
+    int kq = 0;  // stored K (a [hi | lo] GEMM over [W | W] has K = 2 kq)
+};
+
+// A layer's weights: bf16 matrices, or (4-bit handles) their codes.
 struct LayerDev {
     float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
     bf16 *wqkv, *wo, *w1, *w2;
     float *bqkv, *bo, *b1, *b2;
+    QW qqkv, qo, q1, q2;
 };
 
 // ln_post, proj1, proj2 and the SwiGLU adapter: the encoder's own set, and
-// one per layer tap (the cross-layer taps each have their own projector)
+// one per layer tap (the cross-layer taps each have their own projector).
+// A set with 4-bit matrices has qp1.codes set.
 struct HeadDev {
     float *lnp_g, *lnp_b, *bp1, *bp2, *bgu, *bd;
     bf16 *wp1, *wp2, *wgu, *wd;
+    QW qp1, qp2, qgu, qd;
 };
 
 struct ClipPlan {
@@ -57,8 +70,10 @@ struct moss_enc {
     cudaStream_t stream = nullptr;
     std::string last_error;
 
-    // weights (one allocation)
-    void *wmem = nullptr;
+    // weights (one allocation; 4-bit handles keep the linear layers' codes
+    // and scales in a second one)
+    void *wmem = nullptr, *qmem = nullptr;
+    bool q4 = false;
     float *conv1_w = nullptr, *conv1_b = nullptr, *conv2_b = nullptr, *conv3_b = nullptr;
     bf16 *conv2_w = nullptr, *conv3_w = nullptr, *conv_out_w = nullptr;
     std::vector<LayerDev> layers;
@@ -301,11 +316,74 @@ static moss_enc_status gemm2(moss_enc *h, const char *name, const bf16 *A, int64
     Launch L(h, name, 2.0 * M * N * ka, 2.0 * M * ka + 2.0 * N * ka + epi_out_bytes(EPI) * M * N);
     if (ksub == 2 && K % 128 == 0)
         CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 2>, dim3(grid), dim3(Gemm2Cfg<BN, 2>::THREADS),
-                             Gemm2Cfg<BN, 2>::SMEM, ta, tb, tc, a));
+                             Gemm2Cfg<BN, 2>::SMEM, ta, tb, tc, tb, a));
     else
         CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 1>, dim3(grid), dim3(Gemm2Cfg<BN, 1>::THREADS),
-                             Gemm2Cfg<BN, 1>::SMEM, ta, tb, tc, a));
+                             Gemm2Cfg<BN, 1>::SMEM, ta, tb, tc, tb, a));
     return MOSS_ENC_OK;
+}
+
+// The pair GEMM with a 4-bit B: the codes and scales stream in by TMA and
+// converter warps expand them to bf16 in shared memory for the MMA.
+template <int BN, int EPI>
+static moss_enc_status gemm2q(moss_enc *h, const char *name, const bf16 *A, int64_t M, int K, const QW &B, int N,
+                              GemmArgs a, int k_alg = 0)
+{
+    using C = Gemm2Cfg<BN, 1, 1>;
+    if (M <= 0) return MOSS_ENC_OK;
+    if (K % 64 != 0 || N % BN != 0 || M > INT32_MAX || B.kq % 128 != 0 || K % B.kq != 0)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "gemm shape not supported");
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return fail(h, MOSS_ENC_ERR_CUDA, "no tensor-map encoder");
+    CUtensorMap ta, tq, ts;
+    if (!tmap_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128))
+        return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    {
+        // codes: [N][kq / 2] bytes, boxes of 32 bytes (64 k) x NS/2 rows
+        cuuint64_t dims[2] = {(cuuint64_t)B.kq / 2, (cuuint64_t)N};
+        cuuint64_t strides[1] = {(cuuint64_t)B.kq / 2};
+        cuuint32_t box[2] = {32, (cuuint32_t)(C::NS / 2)};
+        cuuint32_t es[2] = {1, 1};
+        if (fn(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(B.codes), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (codes)");
+    }
+    {
+        // scales: [kq / 128][N] fp32, boxes of NS/2 rows x 1 group
+        cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)B.kq / 128};
+        cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+        cuuint32_t box[2] = {(cuuint32_t)(C::NS / 2), 1};
+        cuuint32_t es[2] = {1, 1};
+        if (fn(&ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(B.scales), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (scales)");
+    }
+    a.M = (int)M;
+    a.N = N;
+    a.K = K;
+    a.m_tiles = (int)((M + 255) / 256);
+    a.n_tiles = N / BN;
+    a.err = h->err;
+    a.kq_blocks = B.kq / 64;
+    CUtensorMap tc;
+    if (!tmap_out<BN, EPI>(&tc, a, tq)) return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (output)");
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int grid = 2 * std::min(tiles, h->num_sms / 2);
+    const double ka = k_alg > 0 ? k_alg : K;
+    Launch L(h, name, 2.0 * M * N * ka, 2.0 * M * ka + 0.5 * N * (double)B.kq + 4.0 * N * (B.kq / 128) +
+                                            epi_out_bytes(EPI) * M * N);
+    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 1, 1>, dim3(grid), dim3(C::THREADS), C::SMEM, ta, tq, tc,
+                         ts, a));
+    return MOSS_ENC_OK;
+}
+
+template <int BN, int EPI>
+static cudaError_t gemm2q_attr()
+{
+    return cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI, A_PLAIN, 1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Gemm2Cfg<BN, 1, 1>::SMEM);
 }
 
 template <int BN, int EPI>
@@ -370,7 +448,7 @@ static moss_enc_status gemm_conv(moss_enc *h, const char *name, const bf16 *in, 
     const int grid = 2 * std::min(a.m_tiles * a.n_tiles, h->num_sms / 2);
     Launch L(h, name, 2.0 * 128.0 * n_items * CST * (9.0 * CST), 2.0 * 128.0 * n_items * (9.0 * CST) * 0.25 + 2.0 * 128.0 * n_items * CST);
     CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<CONV_BN, EPI_GELU_BF16, A_CONV_S2, 2>, dim3(grid),
-                         dim3(Gemm2Cfg<CONV_BN, 2>::THREADS), Gemm2Cfg<CONV_BN, 2>::SMEM, ta, tb, tb, a));
+                         dim3(Gemm2Cfg<CONV_BN, 2>::THREADS), Gemm2Cfg<CONV_BN, 2>::SMEM, ta, tb, tb, tb, a));
     return MOSS_ENC_OK;
 }
 
@@ -585,6 +663,7 @@ extern "C" void moss_enc_destroy(moss_enc *h)
     if (h->stream) cudaStreamSynchronize(h->stream);
     else cudaDeviceSynchronize();
     if (h->wmem) cudaFree(h->wmem);
+    if (h->qmem) cudaFree(h->qmem);
     if (h->tap_wmem) cudaFree(h->tap_wmem);
     if (h->ws) cudaFree(h->ws);
     if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
@@ -605,19 +684,22 @@ struct HeadOff {
     size_t lnp, p1, bp1, p2, bp2, gu, bgu, wd, bd;
 };
 
-template <class Take>
-static HeadOff head_take(Take &take)
+// The small tensors are taken with `small`, the four weight matrices with
+// `big` (the encoder's own set keeps them in the part a 4-bit handle
+// replaces by codes).
+template <class TakeS, class TakeB>
+static HeadOff head_take(TakeS &small, TakeB &big)
 {
     HeadOff o;
-    o.lnp = take(4 * 2 * D);
-    o.p1 = take(2 * (size_t)D * 2 * D);
-    o.bp1 = take(4 * D);
-    o.p2 = take(2 * (size_t)DOUT * 2 * D);
-    o.bp2 = take(4 * DOUT);
-    o.gu = take(2 * (size_t)2 * DADP * DOUT);
-    o.bgu = take(4 * 2 * DADP);
-    o.wd = take(2 * (size_t)DOUT * DADP);
-    o.bd = take(4 * DOUT);
+    o.lnp = small(4 * 2 * D);
+    o.bp1 = small(4 * D);
+    o.bp2 = small(4 * DOUT);
+    o.bgu = small(4 * 2 * DADP);
+    o.bd = small(4 * DOUT);
+    o.p1 = big(2 * (size_t)D * 2 * D);
+    o.p2 = big(2 * (size_t)DOUT * 2 * D);
+    o.gu = big(2 * (size_t)2 * DADP * DOUT);
+    o.wd = big(2 * (size_t)DOUT * DADP);
     return o;
 }
 
@@ -695,6 +777,16 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm2_attr<128, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<160, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_F32>()));
+    CUDA_TRY(h, (gemm2q_attr<128, EPI_BF16>()));
+    CUDA_TRY(h, (gemm2q_attr<256, EPI_BF16>()));
+    CUDA_TRY(h, (gemm2q_attr<128, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm2q_attr<160, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm2q_attr<320, EPI_RESID_F32>()));
+    CUDA_TRY(h, (gemm2q_attr<256, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm2q_attr<320, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm2q_attr<256, EPI_F32>()));
+    CUDA_TRY(h, (gemm2q_attr<256, EPI_SWIGLU_BF16>()));
+    CUDA_TRY(h, (gemm2q_attr<128, EPI_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_BF16>()));
     CUDA_TRY(h, (gemm2_attr<320, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2_attr<256, EPI_SWIGLU_BF16>()));
@@ -719,13 +811,58 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     return MOSS_ENC_OK;
 }
 
+// 4-bit round-to-nearest quantisation of one bf16 matrix [n][kq] (rows
+// `stride` elements apart) in groups of 128 along k: s = fp32(max |w|) / 7,
+// q = clamp(rint(w / s), -8, 7) (0 when s = 0), code q + 8.  Codes [n][kq/2]
+// (even k in the low nibble), scales [kq/128][n].
+static void quantise_rows(const uint16_t *w, int r0, int r1, int n, int kq, int stride, uint8_t *codes, float *scales)
+{
+    const int groups = kq / 128;
+    for (int r = r0; r < r1; r++)
+        for (int g = 0; g < groups; g++) {
+            const uint16_t *x = w + (size_t)r * stride + (size_t)g * 128;
+            float amax = 0.0f;
+            for (int i = 0; i < 128; i++) amax = std::max(amax, std::fabs(bf16_bits_to_float(x[i])));
+            const float s = amax / 7.0f;
+            scales[(size_t)g * n + r] = s;
+            uint8_t *c = codes + (size_t)r * (kq / 2) + (size_t)g * 64;
+            for (int i = 0; i < 128; i += 2) {
+                int u[2];
+                for (int e = 0; e < 2; e++) {
+                    float q = 0.0f;
+                    if (s > 0.0f) q = std::min(7.0f, std::max(-8.0f, std::rint(bf16_bits_to_float(x[i + e]) / s)));
+                    u[e] = (int)q + 8;
+                }
+                c[i / 2] = (uint8_t)(u[0] | (u[1] << 4));
+            }
+        }
+}
+
+template <class QS>
+static void quantise_all(const uint8_t *pk, uint8_t *qk, const QS *qs, size_t nq)
+{
+    const unsigned nt = std::max(1u, std::min(32u, std::thread::hardware_concurrency()));
+    std::vector<std::thread> pool;
+    for (unsigned t = 0; t < nt; t++)
+        pool.emplace_back([&, t]() {
+            for (size_t i = 0; i < nq; i++) {
+                const QS &q = qs[i];
+                const int r0 = (int)((int64_t)q.n * t / nt), r1 = (int)((int64_t)q.n * (t + 1) / nt);
+                quantise_rows(reinterpret_cast<const uint16_t *>(pk + q.bf_off), r0, r1, q.n, q.kq, q.stride, qk + q.q_off,
+                              reinterpret_cast<float *>(qk + q.s_off));
+            }
+        });
+    for (auto &th : pool) th.join();
+}
+
 extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const void *weights, size_t bytes,
                                            int weights_on_device, void *stream, moss_enc **out)
 {
     if (!out) return MOSS_ENC_ERR_INVALID_ARG;
     *out = nullptr;
     if (!cfg || !weights || cfg->n_layers < 1 || cfg->n_layers > 32 || cfg->max_samples < 1 ||
-        cfg->max_clips < 1 || (cfg->out_dtype != MOSS_ENC_OUT_F32 && cfg->out_dtype != MOSS_ENC_OUT_BF16))
+        cfg->max_clips < 1 || (cfg->out_dtype != MOSS_ENC_OUT_F32 && cfg->out_dtype != MOSS_ENC_OUT_BF16) ||
+        (cfg->weight_bits != 0 && cfg->weight_bits != 16 && cfg->weight_bits != 4))
         return MOSS_ENC_ERR_INVALID_ARG;
     const int64_t count = moss_enc_weight_count(cfg->n_layers);
     if ((int64_t)bytes != count * 2) return MOSS_ENC_ERR_INVALID_ARG;
@@ -757,7 +894,9 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         src = host.data();
     }
 
-    // ---- sizes of the packed weights
+    // ---- sizes of the packed weights: the small tensors first, then the
+    // weight matrices of the linear layers (the part a 4-bit handle keeps as
+    // codes and scales only)
     const int L = cfg->n_layers;
     size_t off = 0;
     auto take = [&](size_t b) {
@@ -769,14 +908,37 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     const size_t o_c2w = take(2 * (size_t)CST * CONV_K), o_c2b = take(4 * CST);
     const size_t o_c3w = take(2 * (size_t)CST * CONV_K), o_c3b = take(4 * CST);
     const size_t o_cow = take(2 * (size_t)D * CST * 16);
-    std::vector<size_t> o_layer(L);
-    const size_t layer_bytes = 4 * 4 * D + 2 * ((size_t)DQKV * D + (size_t)D * D + (size_t)DFF * D + (size_t)D * DFF) +
-                               4 * (DQKV + D + DFF + D) + 8 * 256;
-    for (int l = 0; l < L; l++) o_layer[l] = take(layer_bytes);
-    const HeadOff o_head = head_take(take);
+    // per layer: ln1 g/b, ln2 g/b, bqkv, bo, b1, b2 | wqkv, wo, w1, w2
+    std::vector<size_t> lo(L * 12);
+    for (int l = 0; l < L; l++) {
+        size_t *L12 = &lo[l * 12];
+        L12[0] = take(4 * D); L12[1] = take(4 * D); L12[2] = take(4 * D); L12[3] = take(4 * D);
+        L12[5] = take(4 * DQKV); L12[7] = take(4 * D); L12[9] = take(4 * DFF); L12[11] = take(4 * D);
+    }
+    size_t big_off = 0;  // offsets inside the matrix part, rebased below
+    auto take_big = [&](size_t b) {
+        size_t r = big_off;
+        big_off += (b + 255) & ~size_t(255);
+        return r;
+    };
+    for (int l = 0; l < L; l++) {
+        size_t *L12 = &lo[l * 12];
+        L12[4] = take_big(2 * (size_t)DQKV * D);
+        L12[6] = take_big(2 * (size_t)D * D);
+        L12[8] = take_big(2 * (size_t)DFF * D);
+        L12[10] = take_big(2 * (size_t)D * DFF);
+    }
+    HeadOff o_head = head_take(take, take_big);
     const size_t o_pos = take(4 * (size_t)CHUNK_TOKENS * D);
     const size_t o_mel4 = take(sizeof(Mel4Tab));
-    const size_t wtotal = off;
+    const size_t small_total = off;
+    for (int l = 0; l < L; l++)
+        for (int i : {4, 6, 8, 10}) lo[l * 12 + i] += small_total;
+    o_head.p1 += small_total;
+    o_head.p2 += small_total;
+    o_head.gu += small_total;
+    o_head.wd += small_total;
+    const size_t wtotal = small_total + big_off;
 
     std::vector<uint8_t> pk(wtotal, 0);
     auto F32 = [&](size_t o) { return reinterpret_cast<float *>(pk.data() + o); };
@@ -807,23 +969,10 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         p += (size_t)D * 7680;
     }
     h->layers.resize(L);
-    std::vector<size_t> lo(L * 12);
     for (int l = 0; l < L; l++) {
-        size_t b = o_layer[l];
-        size_t q = b;
-        auto sub = [&](size_t n) {
-            size_t r = q;
-            q += (n + 255) & ~size_t(255);
-            return r;
-        };
-        const size_t ln1g = sub(4 * D), ln1b = sub(4 * D), ln2g = sub(4 * D), ln2b = sub(4 * D);
-        const size_t wqkv = sub(2 * (size_t)DQKV * D), bqkv = sub(4 * DQKV);
-        const size_t wo = sub(2 * (size_t)D * D), bo = sub(4 * D);
-        const size_t w1 = sub(2 * (size_t)DFF * D), b1 = sub(4 * DFF);
-        const size_t w2 = sub(2 * (size_t)D * DFF), b2 = sub(4 * D);
-        size_t *L12 = &lo[l * 12];
-        L12[0] = ln1g; L12[1] = ln1b; L12[2] = ln2g; L12[3] = ln2b; L12[4] = wqkv; L12[5] = bqkv;
-        L12[6] = wo; L12[7] = bo; L12[8] = w1; L12[9] = b1; L12[10] = w2; L12[11] = b2;
+        const size_t *L12 = &lo[l * 12];
+        const size_t ln1g = L12[0], ln1b = L12[1], ln2g = L12[2], ln2b = L12[3], wqkv = L12[4], bqkv = L12[5];
+        const size_t wo = L12[6], bo = L12[7], w1 = L12[8], b1 = L12[9], w2 = L12[10], b2 = L12[11];
         for (int i = 0; i < D; i++) F32(ln1g)[i] = bf16_bits_to_float(p[i]);
         p += D;
         for (int i = 0; i < D; i++) F32(ln1b)[i] = bf16_bits_to_float(p[i]);
@@ -867,9 +1016,60 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
             return bail(MOSS_ENC_ERR_INVALID_ARG);
     }
 
-    if (cudaMalloc(&h->wmem, wtotal) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
-    if (cudaMemcpy(h->wmem, pk.data(), wtotal, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+    // ---- 4-bit handles: codes and scales of every linear layer's matrix
+    // (proj1/proj2 are stored [W | W] along K: W is quantised once)
+    h->q4 = cfg->weight_bits == 4;
+    struct QSrc {
+        size_t bf_off;  // bf16 matrix in pk, rows of `stride` elements
+        int n, kq, stride;
+        size_t q_off, s_off;
+    };
+    std::vector<QSrc> qs;
+    std::vector<uint8_t> qk;
+    if (h->q4) {
+        size_t qoff = 0;
+        auto add = [&](size_t bf_off, int n, int kq, int stride) {
+            QSrc q{bf_off, n, kq, stride, 0, 0};
+            q.q_off = qoff;
+            qoff += ((size_t)n * kq / 2 + 255) & ~size_t(255);
+            q.s_off = qoff;
+            qoff += ((size_t)n * (kq / 128) * 4 + 255) & ~size_t(255);
+            qs.push_back(q);
+        };
+        for (int l = 0; l < L; l++) {
+            const size_t *L12 = &lo[l * 12];
+            add(L12[4], DQKV, D, D);
+            add(L12[6], D, D, D);
+            add(L12[8], DFF, D, D);
+            add(L12[10], D, DFF, DFF);
+        }
+        add(o_head.p1, D, D, 2 * D);
+        add(o_head.p2, DOUT, D, 2 * D);
+        add(o_head.gu, 2 * DADP, DOUT, DOUT);
+        add(o_head.wd, DOUT, DADP, DADP);
+        qk.assign(qoff, 0);
+        quantise_all(pk.data(), qk.data(), qs.data(), qs.size());
+    }
+
+    const size_t upload = h->q4 ? small_total : wtotal;
+    if (cudaMalloc(&h->wmem, upload) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
+    if (cudaMemcpy(h->wmem, pk.data(), upload, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+    uint8_t *Q = nullptr;
+    if (h->q4) {
+        if (cudaMalloc(&h->qmem, qk.size()) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
+        if (cudaMemcpy(h->qmem, qk.data(), qk.size(), cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
+        Q = static_cast<uint8_t *>(h->qmem);
+    }
+    auto qw = [&](size_t i) {
+        QW w;
+        w.codes = Q + qs[i].q_off;
+        w.scales = reinterpret_cast<const float *>(Q + qs[i].s_off);
+        w.kq = qs[i].kq;
+        return w;
+    };
     uint8_t *W = static_cast<uint8_t *>(h->wmem);
+    // bf16 matrices exist on the device only for bf16 handles
+    auto big = [&](size_t o) -> bf16 * { return h->q4 ? nullptr : (bf16 *)(W + o); };
     h->conv1_w = (float *)(W + o_c1w);
     h->conv1_b = (float *)(W + o_c1b);
     h->conv2_w = (bf16 *)(W + o_c2w);
@@ -884,16 +1084,29 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         d.ln1_b = (float *)(W + L12[1]);
         d.ln2_g = (float *)(W + L12[2]);
         d.ln2_b = (float *)(W + L12[3]);
-        d.wqkv = (bf16 *)(W + L12[4]);
+        d.wqkv = big(L12[4]);
         d.bqkv = (float *)(W + L12[5]);
-        d.wo = (bf16 *)(W + L12[6]);
+        d.wo = big(L12[6]);
         d.bo = (float *)(W + L12[7]);
-        d.w1 = (bf16 *)(W + L12[8]);
+        d.w1 = big(L12[8]);
         d.b1 = (float *)(W + L12[9]);
-        d.w2 = (bf16 *)(W + L12[10]);
+        d.w2 = big(L12[10]);
         d.b2 = (float *)(W + L12[11]);
+        if (h->q4) {
+            d.qqkv = qw(4 * l);
+            d.qo = qw(4 * l + 1);
+            d.q1 = qw(4 * l + 2);
+            d.q2 = qw(4 * l + 3);
+        }
     }
     h->head = head_bind(o_head, W);
+    if (h->q4) {
+        h->head.wp1 = h->head.wp2 = h->head.wgu = h->head.wd = nullptr;
+        h->head.qp1 = qw(4 * L);
+        h->head.qp2 = qw(4 * L + 1);
+        h->head.qgu = qw(4 * L + 2);
+        h->head.qd = qw(4 * L + 3);
+    }
     h->pos = (float *)(W + o_pos);
     h->mel4_tab = (Mel4Tab *)(W + o_mel4);
 
@@ -1197,34 +1410,47 @@ static moss_enc_status head_launch(moss_enc *h, const HeadDev &W, int64_t T, int
     // rows of the 30 s clip, the 16-clip batch and the 10-min clip the final
     // rows' worst max err/rms is 0.0225 without it and 0.0194 with it, against
     // a bound of 0.03.
+    // a set with 4-bit matrices takes the 4-bit GEMM (same tiles, same epilogues)
+    const bool q = W.qp1.codes != nullptr;
     GemmArgs a{};
     a.bias = W.bp1;
     a.out = h->hb;
     a.ldo = 2 * D;
     a.split_off = D;
-    TRY((gemm2<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, W.wp1, D, a, D)));
+    TRY((q ? gemm2q<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, W.qp1, D, a, D)
+          : gemm2<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, W.wp1, D, a, D)));
     a.bias = W.bp2;
     if (stage == MOSS_ENC_STAGE_HEAD) {
         a.out = out;
         a.ldo = DOUT;
         a.split_off = 0;
-        return gemm2<256, EPI_F32>(h, "gemm_proj2", h->hb, T, 2 * D, W.wp2, DOUT, a, D);
+        return q ? gemm2q<256, EPI_F32>(h, "gemm_proj2", h->hb, T, 2 * D, W.qp2, DOUT, a, D)
+                 : gemm2<256, EPI_F32>(h, "gemm_proj2", h->hb, T, 2 * D, W.wp2, DOUT, a, D);
     }
     a.out = h->h2;
     a.ldo = DOUT;
     a.split_off = 0;
-    TRY((gemm2<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, 2 * D, W.wp2, DOUT, a, D)));
+    TRY((q ? gemm2q<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, 2 * D, W.qp2, DOUT, a, D)
+          : gemm2<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, 2 * D, W.wp2, DOUT, a, D)));
     // ---- SwiGLU adapter
     a.bias = W.bgu;
     a.out = h->gu;
     a.ldo = DADP;
-    TRY((gemm2<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, W.wgu, 2 * DADP, a)));
+    TRY((q ? gemm2q<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, W.qgu, 2 * DADP, a)
+          : gemm2<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, W.wgu, 2 * DADP, a)));
     a.bias = W.bd;
     a.out = out;
     a.ldo = DOUT;
     a.split_off = 0;
     static const int down_w[2] = {256, 128};
     const bool narrow = pick_width(h, T, DOUT, DADP, down_w, 2) == 128;
+    if (q) {
+        if (h->cfg.out_dtype == MOSS_ENC_OUT_F32)
+            return narrow ? gemm2q<128, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.qd, DOUT, a)
+                          : gemm2q<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.qd, DOUT, a);
+        return narrow ? gemm2q<128, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.qd, DOUT, a)
+                      : gemm2q<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.qd, DOUT, a);
+    }
     if (h->cfg.out_dtype == MOSS_ENC_OUT_F32)
         return narrow ? gemm2<128, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a)
                       : gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
@@ -1302,9 +1528,16 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
     // pair let one tile's epilogue run under the other's mainloop).  The tile
     // width does not change any output element's arithmetic, so a clip's rows
     // are the same at every batch size.
-    auto resid_gemm = [&](const char *name, const bf16 *Ain, int K, const bf16 *W, GemmArgs a) -> moss_enc_status {
+    auto resid_gemm = [&](const char *name, const bf16 *Ain, int K, const bf16 *W, const QW &Wq,
+                          GemmArgs a) -> moss_enc_status {
         static const int long_k[3] = {320, 160, 128}, short_k[3] = {160, 128, 320};
-        switch (pick_width(h, T, D, K, K > D ? long_k : short_k, 3)) {
+        const int bn = pick_width(h, T, D, K, K > D ? long_k : short_k, 3);
+        if (h->q4) {
+            if (bn == 128) return gemm2q<128, EPI_RESID_F32>(h, name, Ain, T, K, Wq, D, a);
+            if (bn == 160) return gemm2q<160, EPI_RESID_F32>(h, name, Ain, T, K, Wq, D, a);
+            return gemm2q<320, EPI_RESID_F32>(h, name, Ain, T, K, Wq, D, a);
+        }
+        switch (bn) {
         case 128: return gemm2<128, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, 2);
         case 160: return gemm2<160, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, 2);
         default: return gemm2<320, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, K == D ? 2 : 1);
@@ -1322,9 +1555,11 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.out = h->qkv;
         a.ldo = DQKV;
         if (T <= 512)  // two row tiles: 128-wide tiles (30 per row tile) keep more SMs busy than 256-wide (15)
-            TRY((gemm2<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
+            TRY((h->q4 ? gemm2q<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.qqkv, DQKV, a)
+                      : gemm2<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
         else
-            TRY((gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
+            TRY((h->q4 ? gemm2q<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.qqkv, DQKV, a)
+                      : gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
         {
             Launch Lk(h, "attention", 4.0 * 64 * 20 * attn_pairs, 2.0 * T * (DQKV + D));
             CUDA_TRY(h, launch_k(h, window_attn_tc_kernel, dim3((unsigned)n_chunks, 20), dim3(128), ATTN_TC_SMEM, tm_qkv,
@@ -1333,7 +1568,7 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.bo;
         a.out = h->X;
         a.ldo = D;
-        TRY(resid_gemm("gemm_out", h->attn, D, L.wo, a));
+        TRY(resid_gemm("gemm_out", h->attn, D, L.wo, L.qo, a));
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln2_g, L.ln2_b,
@@ -1342,11 +1577,12 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.b1;
         a.out = h->ffn;
         a.ldo = DFF;
-        TRY((gemm2<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.w1, DFF, a)));
+        TRY((h->q4 ? gemm2q<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.q1, DFF, a)
+                  : gemm2<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.w1, DFF, a)));
         a.bias = L.b2;
         a.out = h->X;
         a.ldo = D;
-        TRY(resid_gemm("gemm_fc2", h->ffn, DFF, L.w2, a));
+        TRY(resid_gemm("gemm_fc2", h->ffn, DFF, L.w2, L.q2, a));
         // layer taps: this layer's hidden states through the tap's own head set
         // (xn, hb, h2 and gu are free between layers)
         if (tap_out)
@@ -1576,7 +1812,7 @@ extern "C" moss_enc_status moss_enc_set_taps(moss_enc *h, const int *layers, int
             return r;
         };
         std::vector<HeadOff> o(n_taps);
-        for (int t = 0; t < n_taps; t++) o[t] = head_take(take);
+        for (int t = 0; t < n_taps; t++) o[t] = head_take(take, take);
         std::vector<uint16_t> host;
         const uint16_t *p = static_cast<const uint16_t *>(weights);
         if (weights_on_device) {
@@ -1760,6 +1996,65 @@ extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void 
         default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "unsupported epilogue");
         }
     default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160, 192, 256 or 320");
+    }
+}
+
+template <int BN>
+static moss_enc_status gemm_q4_one(moss_enc *h, const bf16 *A, const QW &B, const float *bias, void *out, int M,
+                                   int N, int K, int epi)
+{
+    GemmArgs a{};
+    a.bias = bias;
+    a.out = out;
+    a.ldo = N;
+    switch (epi) {
+    case EPI_BF16: return gemm2q<BN, EPI_BF16>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_GELU_BF16: return gemm2q<BN, EPI_GELU_BF16>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_RESID_F32: return gemm2q<BN, EPI_RESID_F32>(h, "gemm_api", A, M, K, B, N, a);
+    case EPI_F32: return gemm2q<BN, EPI_F32>(h, "gemm_api", A, M, K, B, N, a);
+    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "unsupported epilogue");
+    }
+}
+
+template <int BN>
+static cudaError_t gemm_q4_api_attrs()
+{
+    cudaError_t e;
+    if ((e = gemm2q_attr<BN, EPI_BF16>()) != cudaSuccess) return e;
+    if ((e = gemm2q_attr<BN, EPI_GELU_BF16>()) != cudaSuccess) return e;
+    if ((e = gemm2q_attr<BN, EPI_RESID_F32>()) != cudaSuccess) return e;
+    return gemm2q_attr<BN, EPI_F32>();
+}
+
+extern "C" moss_enc_status moss_enc_gemm_q4(moss_enc *h, const void *A, const void *Bq, const float *Bs,
+                                            const float *bias, void *out, int M, int N, int K, int epilogue,
+                                            int block_n)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (!A || !Bq || !Bs || !bias || !out || M < 0 || N <= 0 || K <= 0 || K % 128 != 0)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad gemm arguments");
+    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(Bq) | reinterpret_cast<uintptr_t>(Bs)) & 15)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A, Bq and Bs must be 16-byte aligned");
+    if (N % block_n != 0 || N % 4 != 0) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n != 0");
+    static bool attrs_done = false;
+    if (!attrs_done) {
+        CUDA_TRY(h, gemm_q4_api_attrs<128>());
+        CUDA_TRY(h, gemm_q4_api_attrs<160>());
+        CUDA_TRY(h, gemm_q4_api_attrs<256>());
+        CUDA_TRY(h, gemm_q4_api_attrs<320>());
+        attrs_done = true;
+    }
+    QW q;
+    q.codes = static_cast<const uint8_t *>(Bq);
+    q.scales = Bs;
+    q.kq = K;
+    const bf16 *a = static_cast<const bf16 *>(A);
+    switch (block_n) {
+    case 128: return gemm_q4_one<128>(h, a, q, bias, out, M, N, K, epilogue);
+    case 160: return gemm_q4_one<160>(h, a, q, bias, out, M, N, K, epilogue);
+    case 256: return gemm_q4_one<256>(h, a, q, bias, out, M, N, K, epilogue);
+    case 320: return gemm_q4_one<320>(h, a, q, bias, out, M, N, K, epilogue);
+    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160, 256 or 320");
     }
 }
 

@@ -61,7 +61,25 @@ typedef struct {
     int64_t max_samples;   /* capacity: sum over clips of encoded samples per call */
     int max_clips;         /* capacity: clips per call */
     int out_dtype;         /* MOSS_ENC_OUT_F32 or MOSS_ENC_OUT_BF16 */
+    int weight_bits;       /* 16 (or 0): bf16 weights; 4: the linear layers of the
+                              encoder layers, head and adapter are kept as 4-bit
+                              codes (see MOSS_ENC_WEIGHTS_4BIT) */
 } moss_enc_config;
+
+/* 4-bit weights (page "Ossicle-4B", "Long Audio", the note under the table:
+ * "4-bit weights for ... the audio encoder, round to nearest, groups of 128").
+ * With cfg.weight_bits = 4, moss_enc_create quantises the weight matrix of
+ * every linear layer of the 32 encoder layers (q, k, v, o, fc1, fc2), of the
+ * encoder head (proj1, proj2) and of the adapter (gate, up, down) in groups of
+ * 128 consecutive input features of each output row:
+ *   s = fp32(max |w|) / 7,  q = clamp(rint(w / s), -8, 7) (0 if s = 0),
+ *   w' = bf16(fp32(q * s))   (fp32 arithmetic, ties to even)
+ * and keeps only the codes (4 bits) and the scales (fp32 per group); the GEMMs
+ * expand them to w' on the fly.  The conv stem (conv1..conv3, conv_out), the
+ * biases and the LayerNorm parameters keep their bf16/fp32 values.  Weight
+ * memory falls from about 1.4 GB to about 0.4 GB for 32 layers.  Layer taps
+ * (moss_enc_set_taps) keep bf16 weights. */
+#define MOSS_ENC_WEIGHTS_4BIT 4
 
 /* One clip (or one piece of a clip) to encode.
  *  pcm        device, 16 kHz mono fp32, the WHOLE clip [n_samples].
@@ -277,6 +295,16 @@ moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host,
  *  K % 64 == 0.  Enqueued on the handle's stream. */
 moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const float *bias, void *out,
                               int M, int N, int K, int epilogue, int block_n, int cta_pair);
+
+/* The same GEMM with a 4-bit B (the form the linear layers take with
+ * cfg.weight_bits = 4): B is given as
+ *  Bq         device uint8 [N][K/2]: codes q + 8 of B[n][k], two per byte, the
+ *             even k in the low nibble;
+ *  Bs         device fp32 [K/128][N]: the scale of each group of 128 k;
+ * and the product uses B[n][k] = bf16(fp32(q * s)).  block_n 128, 160, 256
+ * or 320, CTA pairs only; K % 128 == 0; epilogues as moss_enc_gemm. */
+moss_enc_status moss_enc_gemm_q4(moss_enc *h, const void *A, const void *Bq, const float *Bs, const float *bias,
+                                 void *out, int M, int N, int K, int epilogue, int block_n);
 
 /* The GEMM epilogues and conv1 evaluate GELU's erf with a short rational
  * approximation (Abramowitz & Stegun 7.1.28, error <= 3e-7), one value at a

@@ -78,6 +78,10 @@ def test_create_rejects_bad_arguments_before_touching_a_device():
     cfg = binding.Config(4, 1000, 1, 0)
     st = L.moss_enc_create(ctypes.byref(cfg), blob.ctypes.data_as(ctypes.c_void_p), 8, 0, None, ctypes.byref(h))
     assert st == 1  # blob size does not match 4 layers
+    # weight_bits must be 16 (or 0) or 4: refused before the blob is read
+    cfg = binding.Config(1, 1000, 1, 0, 8)
+    assert L.moss_enc_create(ctypes.byref(cfg), blob.ctypes.data_as(ctypes.c_void_p), 2 * binding.weight_count(1), 0,
+                             None, ctypes.byref(h)) == 1
     assert L.moss_enc_status_string(2) == b"request exceeds capacity"
 
 
