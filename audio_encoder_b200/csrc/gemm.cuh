@@ -536,8 +536,9 @@ struct Gemm2Cfg {
     // a multiple of 4 (the TMEM lane quarters); 8 measured faster than 4 on
     // the layer GEMMs (FC1 45 vs 48-50 us, out-proj 21.5 vs 24.5-25 us)
     static constexpr int EPI_WARPS = 8;
-    // 4-bit B (BQ): four converter warps expand each stage's codes to bf16
-    static constexpr int CONV_WARPS = BQ ? 4 : 0;
+    // 4-bit B (BQ): two converter warps expand each stage's codes to bf16
+    // (384 threads leave the epilogue its registers: with four, it spilled)
+    static constexpr int CONV_WARPS = BQ ? 2 : 0;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * CONV_WARPS;
     // Tiles wider than one MMA (BN = 320) are two MMAs of BN/2 per k-step.
     static constexpr int NSUB = BN > 256 ? 2 : 1;
@@ -600,33 +601,98 @@ __device__ __forceinline__ void pair_tile(int tile, const GemmArgs &a, int &mt, 
 // (K-major, 128-byte swizzle), for the CTA's NSUB x NS/2 rows.  A value is
 // bf16(fp32(q) * s): the code u = q + 8 becomes q exactly in fp32 as
 // (2^23 + u) - (2^23 + 8) (u placed in the low bits of 2^23's significand),
-// is scaled in fp32 and rounded to bf16 once.  Thread ct of the
-// CONV_WARPS * 32 converters takes 16-byte output chunks ct, ct + 128, ...
-// (a chunk = 8 consecutive k of one row = 4 bytes of codes).
+// is scaled in fp32 and rounded to bf16 once.  Converter thread ct takes whole
+// rows ct, ct + 64, ...: two 16-byte loads of codes, one scale, eight 16-byte
+// stores (the 8 threads of a store wavefront write 8 consecutive rows, whose
+// swizzled chunk positions differ).
 template <class C>
 __device__ __forceinline__ void expand_q4(uint8_t *stage, int ct)
 {
     constexpr int NT = C::CONV_WARPS * 32;
     constexpr int ROWS = C::NS / 2;
     const float2 bias = make_float2(-8388616.0f, -8388616.0f);  // -(2^23 + 8)
-#pragma unroll 2
-    for (int i = ct; i < C::NSUB * ROWS * 8; i += NT) {
-        const int j = i / (ROWS * 8), rem = i - j * ROWS * 8, r = rem >> 3, c = rem & 7;
-        const uint32_t w = *reinterpret_cast<const uint32_t *>(stage + C::RAW_OFF + j * C::RAW_SUB + r * 32 + c * 4);
+#pragma unroll 1
+    for (int rr = ct; rr < C::NSUB * ROWS; rr += NT) {
+        const int j = rr / ROWS, r = rr - j * ROWS;
+        const uint4 *src = reinterpret_cast<const uint4 *>(stage + C::RAW_OFF + j * C::RAW_SUB + r * 32);
+        const uint4 c0 = src[0], c1 = src[1];
         const float sc = *reinterpret_cast<const float *>(stage + C::SC_OFF + j * C::SC_SUB + r * 4);
         const float2 s2 = make_float2(sc, sc);
-        const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-        uint32_t o[4];
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        uint8_t *row = stage + C::A_BYTES + j * C::B_SUB_BYTES + r * 128;
 #pragma unroll
-        for (int b = 0; b < 4; b++) {
-            // byte b of lo / hi: the codes of k = 8 c + 2 b and 8 c + 2 b + 1
-            const float2 m = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
-                                         __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u + b)));
-            const float2 v = __fmul2_rn(__fadd2_rn(m, bias), s2);
-            o[b] = pack_bf16x2(v.x, v.y);
+        for (int c = 0; c < 8; c++) {
+            // chunk c: k = 8 c .. 8 c + 7; byte b holds k = 8 c + 2 b (low nibble), 8 c + 2 b + 1
+            const uint32_t lo = words[c] & 0x0F0F0F0Fu, hi = (words[c] >> 4) & 0x0F0F0F0Fu;
+            uint32_t o[4];
+#pragma unroll
+            for (int b = 0; b < 4; b++) {
+                const float2 m = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
+                                             __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u + b)));
+                const float2 v = __fmul2_rn(__fadd2_rn(m, bias), s2);
+                o[b] = pack_bf16x2(v.x, v.y);
+            }
+            *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        *reinterpret_cast<uint4 *>(stage + C::A_BYTES + j * C::B_SUB_BYTES + r * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// Up to four 4-bit matrices to expand in one launch: codes [n][kq/2], scales
+// [kq/128][n] -> bf16 rows out [n][reps * kq] (the row's kq values repeated
+// reps times along k).
+struct Q4Job {
+    const uint8_t *codes;
+    const float *scales;
+    bf16 *out;
+    int n, kq, reps;
+    long long first;  // first item of this job (items: 32 values of one row)
+};
+struct Q4Jobs {
+    Q4Job j[4];
+    int count;
+    long long items;
+};
+
+// Expands the jobs' matrices with the arithmetic of expand_q4.  Thread i
+// takes 32 consecutive k of one row (16 bytes of codes, one scale) and writes
+// 64 bytes per repeat.  The outputs are scratch that earlier kernels may
+// still read: the writes wait for them.
+__global__ void __launch_bounds__(256) q4_expand_kernel(const __grid_constant__ Q4Jobs jobs)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    const float2 bias = make_float2(-8388616.0f, -8388616.0f);  // -(2^23 + 8)
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < jobs.items;
+         i += (long long)gridDim.x * blockDim.x) {
+        int jb = 0;
+        while (jb + 1 < jobs.count && i >= jobs.j[jb + 1].first) jb++;
+        const Q4Job &J = jobs.j[jb];
+        const long long li = i - J.first;
+        const int per_row = J.kq / 32;
+        const int r = (int)(li / per_row), k0 = (int)(li - (long long)r * per_row) * 32;
+        const uint4 c = *reinterpret_cast<const uint4 *>(J.codes + (size_t)r * (J.kq / 2) + k0 / 2);
+        const float sc = J.scales[(size_t)(k0 / 128) * J.n + r];
+        const float2 s2 = make_float2(sc, sc);
+        const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+        uint4 o[4];
+#pragma unroll
+        for (int w = 0; w < 4; w++) {
+            const uint32_t lo = words[w] & 0x0F0F0F0Fu, hi = (words[w] >> 4) & 0x0F0F0F0Fu;
+            uint32_t v[4];
+#pragma unroll
+            for (int b = 0; b < 4; b++) {
+                const float2 m = make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u + b)),
+                                             __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u + b)));
+                const float2 x = __fmul2_rn(__fadd2_rn(m, bias), s2);
+                v[b] = pack_bf16x2(x.x, x.y);
+            }
+            o[w] = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+        for (int rep = 0; rep < J.reps; rep++) {
+            uint4 *dst = reinterpret_cast<uint4 *>(J.out + (size_t)r * J.reps * J.kq + (size_t)rep * J.kq + k0);
+#pragma unroll
+            for (int w = 0; w < 4; w++) dst[w] = o[w];
+        }
     }
 }
 

@@ -100,6 +100,7 @@ struct moss_enc {
     int *err = nullptr;
     float *pcm_stage = nullptr;
     void *out_stage = nullptr;
+    bf16 *qscratch = nullptr;  // 4-bit handles: one expanded weight matrix
 
     // per-call tables: device copies and a ring of pinned host staging areas
     // (a call writes the next area once the copy that last read it has run,
@@ -111,8 +112,11 @@ struct moss_enc {
     int tab_slot = 0;
 
     // launches may overlap the previous kernel's tail (programmatic dependent
-    // launch); MOSS_ENC_PDL=0 in the environment at create turns it off
-    bool pdl = true;
+    // launch); MOSS_ENC_PDL=0 in the environment at create turns it off.
+    // pdl_skip_once: the next launch waits for the previous kernel in full (a
+    // GEMM whose B operand the previous kernel writes, since GEMMs request
+    // their first B stages before waiting on earlier kernels).
+    bool pdl = true, pdl_skip_once = false;
 
     // measurement: launch counter and optional per-launch CUDA events
     int64_t launches = 0;
@@ -175,7 +179,8 @@ static cudaError_t launch_k(moss_enc *h, void (*kern)(KArgs...), dim3 grid, dim3
     cfg.stream = h->stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = h->pdl ? 1 : 0;
+    attr[0].val.programmaticStreamSerializationAllowed = h->pdl && !h->pdl_skip_once ? 1 : 0;
+    h->pdl_skip_once = false;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, args...);
@@ -1113,7 +1118,10 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     // ---- workspace
     h->max_tokens = cfg->max_samples / 1280 + cfg->max_clips + 1;
     h->max_chunks = cfg->max_samples / CHUNK_SAMPLES + cfg->max_clips + 1;
-    h->stem_group = (int)std::min<int64_t>(STEM_GROUP_DEFAULT, h->max_chunks);
+    // A 4-bit handle is the memory-saving configuration: it also runs the conv
+    // stem in groups of 4 chunks (a group's conv1 activations, 24.6 MB per
+    // chunk, dominate the workspace of a small handle).
+    h->stem_group = (int)std::min<int64_t>(h->q4 ? 4 : STEM_GROUP_DEFAULT, h->max_chunks);
     const int64_t T = h->max_tokens, G = h->stem_group;
     off = 0;
     const size_t w_mel = take(4 * (size_t)h->max_chunks * CHUNK_FRAMES * 128);
@@ -1132,6 +1140,9 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     const size_t w_err = take(256);
     const size_t w_pcm = take(4 * (size_t)cfg->max_samples);
     const size_t w_out = take(4 * (size_t)T * DOUT);
+    // 4-bit handles: one linear layer's matrix expanded to bf16 (the largest is
+    // the adapter's interleaved gate/up, 16384 x 2048)
+    const size_t w_qs = h->q4 ? take(2 * (size_t)2 * DADP * DOUT) : 0;
     if (cudaMalloc(&h->ws, off) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     uint8_t *S = static_cast<uint8_t *>(h->ws);
     h->mel_raw = (float *)(S + w_mel);
@@ -1150,6 +1161,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     h->err = (int *)(S + w_err);
     h->pcm_stage = (float *)(S + w_pcm);
     h->out_stage = (void *)(S + w_out);
+    h->qscratch = h->q4 ? (bf16 *)(S + w_qs) : nullptr;
     if (cudaMemset(h->err, 0, 256) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
 
     const TabLayout tl = tab_layout(cfg->max_clips, h->max_chunks);
@@ -1369,6 +1381,43 @@ static std::vector<uint8_t> shape_key(const FwdPlan &P, void *const *tap_out, in
     return k;
 }
 
+// 4-bit handles.  A GEMM of one 256-row tile expands the codes in shared
+// memory as it goes (gemm2q); a larger one would expand the same matrix once
+// per 256-row tile, so the matrices are expanded once per forward, into the
+// workspace's scratch, by a bandwidth-bound kernel, and the bf16 GEMMs run on
+// them (same values, same arithmetic).  q4_expand launches one expansion of
+// up to four matrices (mats[i] -> outs[i], rows repeated reps[i] times along
+// k).  A GEMM that starts its weight loads before waiting on earlier kernels
+// is safe behind it as long as one kernel that waits before letting its
+// dependents start (LayerNorm) lies between them; right after it, the GEMM is
+// launched without overlap (after_expand).
+static moss_enc_status q4_expand(moss_enc *h, const QW *const *mats, const int *n, const int *reps, bf16 *const *outs,
+                                 int count, bool after_expand)
+{
+    Q4Jobs J{};
+    J.count = count;
+    double bytes = 0.0;
+    for (int i = 0; i < count; i++) {
+        J.j[i] = Q4Job{mats[i]->codes, mats[i]->scales, outs[i], n[i], mats[i]->kq, reps[i], J.items};
+        J.items += (long long)n[i] * (mats[i]->kq / 32);
+        bytes += 0.5 * n[i] * (double)mats[i]->kq + 4.0 * n[i] * (mats[i]->kq / 128) + 2.0 * n[i] * reps[i] * (double)mats[i]->kq;
+    }
+    const int grid = (int)std::min<long long>((J.items + 255) / 256, 8LL * h->num_sms);
+    Launch L(h, "q4_expand", 0.0, bytes);
+    CUDA_TRY(h, launch_k(h, q4_expand_kernel, dim3(grid), dim3(256), 0, J));
+    if (after_expand) h->pdl_skip_once = true;
+    return MOSS_ENC_OK;
+}
+
+// One matrix into the scratch, for the GEMM launched next.
+static const bf16 *q4_expand_one(moss_enc *h, const QW &q, int n, int reps, moss_enc_status *st)
+{
+    const QW *m = &q;
+    bf16 *o = h->qscratch;
+    *st = q4_expand(h, &m, &n, &reps, &o, 1, true);
+    return h->qscratch;
+}
+
 // Pair-tile width for an M x N x K GEMM among the candidates `order`: the one
 // whose busiest SM pair has the fewest output columns to compute (pair tiles
 // of one width are spread evenly over the pairs), with 128-wide tiles counted
@@ -1410,40 +1459,63 @@ static moss_enc_status head_launch(moss_enc *h, const HeadDev &W, int64_t T, int
     // rows of the 30 s clip, the 16-clip batch and the 10-min clip the final
     // rows' worst max err/rms is 0.0225 without it and 0.0194 with it, against
     // a bound of 0.03.
-    // a set with 4-bit matrices takes the 4-bit GEMM (same tiles, same epilogues)
-    const bool q = W.qp1.codes != nullptr;
+    // a set with 4-bit matrices: one 256-row tile takes the 4-bit GEMM (same
+    // tiles, same epilogues), a larger batch expands each matrix once
+    const bool q = W.qp1.codes != nullptr && T <= 256;
+    const bool qx = W.qp1.codes != nullptr && T > 256;
+    moss_enc_status qst = MOSS_ENC_OK;
     GemmArgs a{};
     a.bias = W.bp1;
     a.out = h->hb;
     a.ldo = 2 * D;
     a.split_off = D;
-    TRY((q ? gemm2q<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, W.qp1, D, a, D)
-          : gemm2<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, W.wp1, D, a, D)));
+    if (q) {
+        TRY((gemm2q<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, W.qp1, D, a, D)));
+    } else {
+        const bf16 *B = qx ? q4_expand_one(h, W.qp1, D, 2, &qst) : W.wp1;
+        TRY(qst);
+        TRY((gemm2<320, EPI_GELU_BF16>(h, "gemm_proj1", h->xn, T, 2 * D, B, D, a, D)));
+    }
     a.bias = W.bp2;
+    const bf16 *B2 = W.wp2;
+    if (qx) {
+        B2 = q4_expand_one(h, W.qp2, DOUT, 2, &qst);
+        TRY(qst);
+    }
     if (stage == MOSS_ENC_STAGE_HEAD) {
         a.out = out;
         a.ldo = DOUT;
         a.split_off = 0;
         return q ? gemm2q<256, EPI_F32>(h, "gemm_proj2", h->hb, T, 2 * D, W.qp2, DOUT, a, D)
-                 : gemm2<256, EPI_F32>(h, "gemm_proj2", h->hb, T, 2 * D, W.wp2, DOUT, a, D);
+                 : gemm2<256, EPI_F32>(h, "gemm_proj2", h->hb, T, 2 * D, B2, DOUT, a, D);
     }
     a.out = h->h2;
     a.ldo = DOUT;
     a.split_off = 0;
     TRY((q ? gemm2q<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, 2 * D, W.qp2, DOUT, a, D)
-          : gemm2<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, 2 * D, W.wp2, DOUT, a, D)));
+          : gemm2<256, EPI_BF16>(h, "gemm_proj2", h->hb, T, 2 * D, B2, DOUT, a, D)));
     // ---- SwiGLU adapter
     a.bias = W.bgu;
     a.out = h->gu;
     a.ldo = DADP;
+    const bf16 *Bgu = W.wgu;
+    if (qx) {
+        Bgu = q4_expand_one(h, W.qgu, 2 * DADP, 1, &qst);
+        TRY(qst);
+    }
     TRY((q ? gemm2q<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, W.qgu, 2 * DADP, a)
-          : gemm2<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, W.wgu, 2 * DADP, a)));
+          : gemm2<256, EPI_SWIGLU_BF16>(h, "gemm_gate_up", h->h2, T, DOUT, Bgu, 2 * DADP, a)));
     a.bias = W.bd;
     a.out = out;
     a.ldo = DOUT;
     a.split_off = 0;
     static const int down_w[2] = {256, 128};
     const bool narrow = pick_width(h, T, DOUT, DADP, down_w, 2) == 128;
+    const bf16 *Bd = W.wd;
+    if (qx) {
+        Bd = q4_expand_one(h, W.qd, DOUT, 1, &qst);
+        TRY(qst);
+    }
     if (q) {
         if (h->cfg.out_dtype == MOSS_ENC_OUT_F32)
             return narrow ? gemm2q<128, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.qd, DOUT, a)
@@ -1452,10 +1524,10 @@ static moss_enc_status head_launch(moss_enc *h, const HeadDev &W, int64_t T, int
                       : gemm2q<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.qd, DOUT, a);
     }
     if (h->cfg.out_dtype == MOSS_ENC_OUT_F32)
-        return narrow ? gemm2<128, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a)
-                      : gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
-    return narrow ? gemm2<128, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a)
-                  : gemm2<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, W.wd, DOUT, a);
+        return narrow ? gemm2<128, EPI_F32>(h, "gemm_down", h->gu, T, DADP, Bd, DOUT, a)
+                      : gemm2<256, EPI_F32>(h, "gemm_down", h->gu, T, DADP, Bd, DOUT, a);
+    return narrow ? gemm2<128, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, Bd, DOUT, a)
+                  : gemm2<256, EPI_BF16>(h, "gemm_down", h->gu, T, DADP, Bd, DOUT, a);
 }
 
 static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt, int stage, void *out,
@@ -1528,11 +1600,14 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
     // pair let one tile's epilogue run under the other's mainloop).  The tile
     // width does not change any output element's arithmetic, so a clip's rows
     // are the same at every batch size.
+    // 4-bit handles: a batch of one 256-row tile takes the 4-bit GEMM, a
+    // larger one expands each matrix once into the scratch (q4_expand)
+    const bool qf = h->q4 && T <= 256, qx = h->q4 && T > 256;
     auto resid_gemm = [&](const char *name, const bf16 *Ain, int K, const bf16 *W, const QW &Wq,
                           GemmArgs a) -> moss_enc_status {
         static const int long_k[3] = {320, 160, 128}, short_k[3] = {160, 128, 320};
         const int bn = pick_width(h, T, D, K, K > D ? long_k : short_k, 3);
-        if (h->q4) {
+        if (qf) {
             if (bn == 128) return gemm2q<128, EPI_RESID_F32>(h, name, Ain, T, K, Wq, D, a);
             if (bn == 160) return gemm2q<160, EPI_RESID_F32>(h, name, Ain, T, K, Wq, D, a);
             return gemm2q<320, EPI_RESID_F32>(h, name, Ain, T, K, Wq, D, a);
@@ -1543,8 +1618,24 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         default: return gemm2<320, EPI_RESID_F32>(h, name, Ain, T, K, W, D, a, 0, K == D ? 2 : 1);
         }
     };
+    // 4-bit handles, larger batches: the layer's four matrices in the scratch
+    bf16 *xs_qkv = h->qscratch, *xs_o = xs_qkv + (size_t)DQKV * D, *xs_1 = xs_o + (size_t)D * D,
+         *xs_2 = xs_1 + (size_t)DFF * D;
     for (size_t l = 0; l < h->layers.size(); l++) {
         const LayerDev &L = h->layers[l];
+        const bf16 *Wqkv = L.wqkv, *Wo = L.wo, *W1 = L.w1, *W2 = L.w2;
+        if (qx) {
+            // expanded before LN1, which waits on it before letting the QKV
+            // GEMM start (that GEMM requests its weights before waiting)
+            const QW *m[4] = {&L.qqkv, &L.qo, &L.q1, &L.q2};
+            const int n[4] = {DQKV, D, DFF, D}, r[4] = {1, 1, 1, 1};
+            bf16 *const o[4] = {xs_qkv, xs_o, xs_1, xs_2};
+            TRY(q4_expand(h, m, n, r, o, 4, false));
+            Wqkv = xs_qkv;
+            Wo = xs_o;
+            W1 = xs_1;
+            W2 = xs_2;
+        }
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln1_g, L.ln1_b,
@@ -1554,12 +1645,12 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.bqkv;
         a.out = h->qkv;
         a.ldo = DQKV;
-        if (T <= 512)  // two row tiles: 128-wide tiles (30 per row tile) keep more SMs busy than 256-wide (15)
-            TRY((h->q4 ? gemm2q<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.qqkv, DQKV, a)
-                      : gemm2<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
+        if (qf)
+            TRY((gemm2q<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.qqkv, DQKV, a)));
+        else if (T <= 512)  // two row tiles: 128-wide tiles (30 per row tile) keep more SMs busy than 256-wide (15)
+            TRY((gemm2<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, Wqkv, DQKV, a)));
         else
-            TRY((h->q4 ? gemm2q<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.qqkv, DQKV, a)
-                      : gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.wqkv, DQKV, a)));
+            TRY((gemm2<256, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, Wqkv, DQKV, a)));
         {
             Launch Lk(h, "attention", 4.0 * 64 * 20 * attn_pairs, 2.0 * T * (DQKV + D));
             CUDA_TRY(h, launch_k(h, window_attn_tc_kernel, dim3((unsigned)n_chunks, 20), dim3(128), ATTN_TC_SMEM, tm_qkv,
@@ -1568,7 +1659,7 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.bo;
         a.out = h->X;
         a.ldo = D;
-        TRY(resid_gemm("gemm_out", h->attn, D, L.wo, L.qo, a));
+        TRY(resid_gemm("gemm_out", h->attn, D, Wo, L.qo, a));
         {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln2_g, L.ln2_b,
@@ -1577,12 +1668,12 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.b1;
         a.out = h->ffn;
         a.ldo = DFF;
-        TRY((h->q4 ? gemm2q<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.q1, DFF, a)
-                  : gemm2<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.w1, DFF, a)));
+        TRY((qf ? gemm2q<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.q1, DFF, a)
+                : gemm2<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, W1, DFF, a)));
         a.bias = L.b2;
         a.out = h->X;
         a.ldo = D;
-        TRY(resid_gemm("gemm_fc2", h->ffn, DFF, L.w2, L.q2, a));
+        TRY(resid_gemm("gemm_fc2", h->ffn, DFF, W2, L.q2, a));
         // layer taps: this layer's hidden states through the tap's own head set
         // (xn, hb, h2 and gu are free between layers)
         if (tap_out)

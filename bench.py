@@ -14,7 +14,8 @@ batch (clips are independent: weak scaling, no collective on the data path).
 
 At N = 1 the line also carries `other_configs`: the 1 s / 4-layer clip, the
 single 30 s clip, the 10-min clip and the 60-min clip streamed in 64 s pieces
-(with the encoder's device memory), each timed the same way; and
+(with the encoder's device memory), each timed the same way, and the batch
+and the streamed clip again with 4-bit weights (`_w4`); and
 `cpu_baseline` times the oracle on all host cores and on one core.
 
 The reference arm (--impl reference) times the CPU oracle on the host cores
@@ -430,7 +431,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def measure_streamed(steps, warmup, dev, dist=None, world=1):
+def measure_streamed(steps, warmup, dev, dist=None, world=1, weight_bits=16):
     """The 60-min clip encoded as a stream of 64 s pieces (1,024,000 samples,
     the last 256,000): a step is the whole-clip log-mel maximum (one pass)
     and the 57 piece forwards against it, each piece reading its 200-sample
@@ -449,7 +450,7 @@ def measure_streamed(steps, warmup, dev, dist=None, world=1):
     free0, _ = torch.cuda.mem_get_info()
     stream = torch.cuda.Stream()
     enc = binding.Encoder(synth.make_weights(n_layers), n_layers, max_samples=piece, max_clips=1,
-                          out_dtype=binding.OUT_BF16, stream=stream)
+                          out_dtype=binding.OUT_BF16, stream=stream, weight_bits=weight_bits)
     torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info()
     tokens = binding.num_tokens(n)
@@ -538,7 +539,7 @@ def run_streamed(args):
         dist.destroy_process_group()
 
 
-def measure_plain(workload, steps, warmup, dev):
+def measure_plain(workload, steps, warmup, dev, weight_bits=16):
     """One workload's forward timed as the headline is (device-resident PCM,
     CUDA events on the encoder's stream, L2 flushed between steps)."""
     import torch
@@ -549,7 +550,7 @@ def measure_plain(workload, steps, warmup, dev):
     stream = torch.cuda.Stream()
     total = sum(c.size for c in clips)
     enc = binding.Encoder(synth.make_weights(n_layers), n_layers, max_samples=total, max_clips=len(clips),
-                          out_dtype=binding.OUT_BF16, stream=stream)
+                          out_dtype=binding.OUT_BF16, stream=stream, weight_bits=weight_bits)
     tokens = sum(binding.num_tokens(c.size) for c in clips)
     with torch.cuda.stream(stream):
         xs = [torch.from_numpy(c).to(dev) for c in clips]
@@ -581,11 +582,13 @@ def other_configs(args, dev):
     pk = peaks()
     res = {}
     steps = max(3, min(args.steps, 20))
-    for w in ("tiny_1s", "single_30s", "clip_10min", "clip_60min_streamed"):
+    # the last two: the 4-bit-weight encoder (round to nearest, groups of 128)
+    for w, bits in (("tiny_1s", 16), ("single_30s", 16), ("clip_10min", 16), ("clip_60min_streamed", 16),
+                    ("batch16_10to30s", 4), ("clip_60min_streamed", 4)):
         if w == "clip_60min_streamed":
-            r = measure_streamed(max(3, min(args.steps, 10)), 3, dev)
+            r = measure_streamed(max(3, min(args.steps, 10)), 3, dev, weight_bits=bits)
         else:
-            r = measure_plain(w, steps, 3, dev)
+            r = measure_plain(w, steps, 3, dev, weight_bits=bits)
         tf = model_flops(r["tokens"], r["n_layers"]) / (r["ms"] / 1e3) / 1e12
         e = {"value": r["audio_s"] / (r["ms"] / 1e3), "unit": "audio-s/s", "ms_per_step": r["ms"],
              "tokens_per_s": r["tokens"] / (r["ms"] / 1e3), "tokens": r["tokens"], "layers": r["n_layers"],
@@ -595,7 +598,8 @@ def other_configs(args, dev):
             e.update({"pieces": r["pieces"], "piece_samples": r["piece"],
                       "encoder_device_bytes": r["encoder_device_bytes"],
                       "clip_and_rows_device_bytes": r["clip_and_rows_device_bytes"]})
-        res[w] = e
+        e["weight_bits"] = bits
+        res[w if bits == 16 else w + "_w4"] = e
     return res
 
 

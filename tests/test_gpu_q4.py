@@ -111,3 +111,19 @@ def test_q4_single_30s_clip_matches_oracle_and_saves_memory():
     assert used4 < 0.5 * used16, (used4, used16)
     e4.close()
     e16.close()
+
+
+def test_q4_fused_and_expanded_paths_agree_bit_for_bit(tiny_q4):
+    # a batch of one 256-row tile expands the codes inside the GEMM; a larger
+    # batch expands each matrix once into a scratch and runs the bf16 GEMM:
+    # the same weight values and arithmetic, so a clip's rows are the same
+    blob, pcm, _ = tiny_q4
+    e = binding.Encoder(blob, 4, 600_000, 2, weight_bits=4)
+    x = torch.from_numpy(pcm).cuda()
+    alone, _ = e.forward([x])
+    other = torch.from_numpy(synth.pcm_tones(9, 480000)).cuda()
+    both, offs = e.forward([x, other])
+    e.synchronize()
+    assert offs[-1] > 256
+    assert torch.equal(both[:13], alone)
+    e.close()
