@@ -83,6 +83,9 @@ def lib():
         L.oracle_model_create_bits.restype = vp
         L.oracle_model_create_bits.argtypes = [vp, i32, i32]
         L.oracle_quant_rtn4.argtypes = [vp, i32, i32, vp, vp, vp]
+        L.oracle_e4m3.restype = f32
+        L.oracle_e4m3.argtypes = [f32]
+        L.oracle_quant_e4m3_rows.argtypes = [vp, i32, i32, vp, vp]
         L.oracle_set_threads.argtypes = [i32]
         L.oracle_max_threads.restype = i32
     return _lib
@@ -194,9 +197,26 @@ def quant_rtn4(w: np.ndarray):
     return deq, codes, scales
 
 
+def e4m3(x: float) -> float:
+    """The nearest e4m3 value (ties to even, saturating at +-448)."""
+    return float(lib().oracle_e4m3(float(x)))
+
+
+def quant_e4m3_rows(w: np.ndarray):
+    """Per-row e4m3 quantisation of a bf16 matrix (uint16 bits) [rows][cols]:
+    returns (e4m3 values as bf16 bits, scales [rows] fp32), row max -> 448."""
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    rows, cols = w.shape
+    q = np.empty_like(w)
+    s = np.empty(rows, dtype=np.float32)
+    lib().oracle_quant_e4m3_rows(_p(w), rows, cols, _p(q), _p(s))
+    return q, s
+
+
 class Model:
     """The oracle's copy of a bf16 weight blob (uint16 bit patterns);
-    weight_bits=4 gives the model with 4-bit quantised linear layers."""
+    weight_bits=4 gives the model with 4-bit quantised linear layers, 8 the
+    model whose q, k, v and fc1 GEMMs take e4m3 operands."""
 
     def __init__(self, blob: np.ndarray, n_layers: int, weight_bits: int = 16):
         blob = np.ascontiguousarray(blob, dtype=np.uint16)

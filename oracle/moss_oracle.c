@@ -281,10 +281,12 @@ typedef struct {
     const uint16_t *ln1_g, *ln1_b, *ln2_g, *ln2_b;
     const uint16_t *bq, *bk, *bv, *bo, *b1, *b2;
     uint16_t *wq_t, *wk_t, *wv_t, *wo_t, *w1_t, *w2_t; /* [in][out] */
+    float *sq, *sk, *sv, *s1; /* FP8 models: per-channel scales of q, k, v, fc1 */
 } layer_w;
 
 typedef struct oracle_model {
     int n_layers;
+    int fp8;            /* q, k, v and fc1 on e4m3 operands */
     float *conv_w_t[3]; /* [in][3][3][out] */
     const uint16_t *conv_b[3];
     int conv_in[3];
@@ -361,6 +363,78 @@ void oracle_quant_rtn4(const uint16_t *w, int rows, int cols, uint16_t *deq, uin
         }
 }
 
+/* ------------------------------------------------ FP8 (e4m3) GEMM operands
+ *
+ * Page "Ossicle-4B", "Quantized: NVFP4 and INT4 in vLLM": the low-precision
+ * builds quantise weights and activations of the audio encoder and run on
+ * Blackwell's low-precision tensor cores.  Reading for an FP8 encoder (the
+ * page fixes no format): the two GEMMs fed by a LayerNorm in every layer (q,
+ * k, v and fc1) take e4m3 operands, scaled per weight output channel and per
+ * activation row so that each row's largest magnitude maps to 448:
+ *   s_w[n] = fp32(max_k |w[n][k]|) / 448,  w8 = e4m3(w / s_w[n])
+ *   s_a[m] = fp32(max_k |y[m][k]|) / 448,  a8 = e4m3(y / s_a[m])
+ *   out[m][n] = (sum_k a8 w8) * s_a[m] * s_w[n] + b[n]
+ * e4m3: 1 sign, 4 exponent (bias 7) and 3 mantissa bits, largest finite
+ * 448, smallest step 2^-9; conversion rounds to nearest, ties to even, and
+ * saturates at +-448 (fp32 arithmetic for the scales and the divisions; a
+ * zero row or channel has scale 0 and operands 0). */
+
+/* fp32 -> the nearest e4m3 value (ties to even), saturating at +-448. */
+float oracle_e4m3(float x)
+{
+    if (x != x) return x;
+    const float a = fabsf(x);
+    float r;
+    if (a >= 448.0f) {
+        r = 448.0f;
+    } else {
+        int e;
+        frexpf(a, &e);  /* a = f * 2^e, f in [0.5, 1): the leading bit is 2^(e-1) */
+        int lead = e - 1;
+        if (lead < -6) lead = -6;  /* below the normal range the step stays 2^-9 */
+        const float step = ldexpf(1.0f, lead - 3);
+        r = rintf(a / step) * step;  /* exact: a / step and the product are powers-of-two scalings */
+        if (r > 448.0f) r = 448.0f;
+    }
+    return x < 0.0f ? -r : r;
+}
+
+/* Quantise w [rows][cols] (bf16 bits) per row: q receives e4m3 values as
+ * bf16 bits (every e4m3 value is a bf16 value), scales s[row]. */
+void oracle_quant_e4m3_rows(const uint16_t *w, int rows, int cols, uint16_t *q, float *scales)
+{
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; r++) {
+        const uint16_t *x = w + (size_t)r * cols;
+        float amax = 0.0f;
+        for (int k = 0; k < cols; k++) {
+            const float a = fabsf(bff(x[k]));
+            if (a > amax) amax = a;
+        }
+        const float s = amax / 448.0f;
+        scales[r] = s;
+        for (int k = 0; k < cols; k++)
+            q[(size_t)r * cols + k] = s > 0.0f ? bf16_rne(oracle_e4m3(bff(x[k]) / s)) : 0;
+    }
+}
+
+/* Quantise activation rows y [M][K] in place to e4m3 values, scales s[M]. */
+static void quant_e4m3_act(float *y, int64_t M, int K, float *s)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        float *r = y + m * K;
+        float amax = 0.0f;
+        for (int k = 0; k < K; k++) {
+            const float a = fabsf(r[k]);
+            if (a > amax) amax = a;
+        }
+        const float sc = amax / 448.0f;
+        s[m] = sc;
+        for (int k = 0; k < K; k++) r[k] = sc > 0.0f ? oracle_e4m3(r[k] / sc) : 0.0f;
+    }
+}
+
 /* The blob's [out][in] matrix at p, quantised when bits == 4, transposed. */
 static uint16_t *take_linear(const uint16_t *p, int out, int in, int bits)
 {
@@ -372,16 +446,29 @@ static uint16_t *take_linear(const uint16_t *p, int out, int in, int bits)
     return t;
 }
 
+/* The blob's [out][in] matrix at p as e4m3 values per output channel,
+ * transposed; *scales receives s_w [out] (malloc'd). */
+static uint16_t *take_linear_e4m3(const uint16_t *p, int out, int in, float **scales)
+{
+    uint16_t *q = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)out * in);
+    *scales = (float *)malloc(sizeof(float) * out);
+    oracle_quant_e4m3_rows(p, out, in, q, *scales);
+    uint16_t *t = transpose_bf16(q, out, in);
+    free(q);
+    return t;
+}
+
 /* Walks the blob in its documented order (conv1, conv2, conv3, conv_out,
  * layers, ln_post, proj1, proj2, adapter gate/up/down; each weight followed
  * by its bias, none for conv_out).  weight_bits 4 gives the 4-bit model of
- * the quantisation section above (its linear layers' weights w'); any other
- * value the bf16 model. */
+ * the quantisation section above (its linear layers' weights w'), 8 the FP8
+ * model (q, k, v and fc1 on e4m3 operands), any other value the bf16 model. */
 oracle_model *oracle_model_create_bits(const uint16_t *blob, int n_layers, int weight_bits)
 {
     oracle_model *m = (oracle_model *)calloc(1, sizeof(oracle_model));
     const uint16_t *p = blob;
     m->n_layers = n_layers;
+    m->fp8 = weight_bits == 8;
     int cin[3] = {1, C_STEM, C_STEM};
     for (int c = 0; c < 3; c++) {
         m->conv_in[c] = cin[c];
@@ -403,17 +490,25 @@ oracle_model *oracle_model_create_bits(const uint16_t *blob, int n_layers, int w
         layer_w *L = &m->layers[l];
         L->ln1_g = p; p += D;
         L->ln1_b = p; p += D;
-        L->wq_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
+        if (weight_bits == 8) L->wq_t = take_linear_e4m3(p, D, D, &L->sq);
+        else L->wq_t = take_linear(p, D, D, weight_bits);
+        p += (size_t)D * D;
         L->bq = p; p += D;
-        L->wk_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
+        if (weight_bits == 8) L->wk_t = take_linear_e4m3(p, D, D, &L->sk);
+        else L->wk_t = take_linear(p, D, D, weight_bits);
+        p += (size_t)D * D;
         L->bk = p; p += D;
-        L->wv_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
+        if (weight_bits == 8) L->wv_t = take_linear_e4m3(p, D, D, &L->sv);
+        else L->wv_t = take_linear(p, D, D, weight_bits);
+        p += (size_t)D * D;
         L->bv = p; p += D;
         L->wo_t = take_linear(p, D, D, weight_bits); p += (size_t)D * D;
         L->bo = p; p += D;
         L->ln2_g = p; p += D;
         L->ln2_b = p; p += D;
-        L->w1_t = take_linear(p, D_FFN, D, weight_bits); p += (size_t)D_FFN * D;
+        if (weight_bits == 8) L->w1_t = take_linear_e4m3(p, D_FFN, D, &L->s1);
+        else L->w1_t = take_linear(p, D_FFN, D, weight_bits);
+        p += (size_t)D_FFN * D;
         L->b1 = p; p += D_FFN;
         L->w2_t = take_linear(p, D, D_FFN, weight_bits); p += (size_t)D * D_FFN;
         L->b2 = p; p += D;
@@ -462,6 +557,7 @@ void oracle_model_destroy(oracle_model *m)
         layer_w *L = &m->layers[l];
         free(L->wq_t); free(L->wk_t); free(L->wv_t); free(L->wo_t);
         free(L->w1_t); free(L->w2_t);
+        free(L->sq); free(L->sk); free(L->sv); free(L->s1);
     }
     free(m->layers);
     free(m->wp1_t); free(m->wp2_t); free(m->wg_t); free(m->wu_t); free(m->wd_t);
@@ -492,6 +588,30 @@ static void linear(const float *x, int64_t M, int K, const uint16_t *wt, const u
             }
             for (int n = 0; n < N; n++)
                 y[m * N + n] = (float)(acc[n] + (bias ? bf(bias[n]) : 0.0));
+        }
+        free(acc);
+    }
+}
+
+/* The FP8 GEMM: y[m][n] = (sum_k x8[m][k] w8[n][k]) * sa[m] * sw[n] + b[n],
+ * x8 and w8 e4m3 values (w8 given transposed [K][N] as bf16 bits), the sum
+ * in fp64 over k in order. */
+static void linear_e4m3(const float *x8, int64_t M, int K, const uint16_t *w8t, const float *sa, const float *sw,
+                        const uint16_t *bias, int N, float *y)
+{
+#pragma omp parallel
+    {
+        double *acc = (double *)malloc(sizeof(double) * N);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t m = 0; m < M; m++) {
+            for (int n = 0; n < N; n++) acc[n] = 0.0;
+            const float *xr = x8 + m * K;
+            for (int k = 0; k < K; k++) {
+                double a = xr[k];
+                const uint16_t *w = w8t + (size_t)k * N;
+                for (int n = 0; n < N; n++) acc[n] += a * (double)bff(w[n]);
+            }
+            for (int n = 0; n < N; n++) y[m * N + n] = (float)(acc[n] * sa[m] * sw[n] + bf(bias[n]));
         }
         free(acc);
     }
@@ -671,12 +791,20 @@ int oracle_layers(const oracle_model *m, float *x, int T, const int *win, int n_
     float *v = (float *)malloc(sizeof(float) * td);
     float *a = (float *)malloc(sizeof(float) * td);
     float *f = (float *)malloc(sizeof(float) * (size_t)T * D_FFN);
+    float *sa = (float *)malloc(sizeof(float) * (size_t)T);
     for (int l = l0; l < l1; l++) {
         const layer_w *L = &m->layers[l];
         layernorm(x, T, D, L->ln1_g, L->ln1_b, h);
-        linear(h, T, D, L->wq_t, L->bq, D, q);
-        linear(h, T, D, L->wk_t, L->bk, D, k);
-        linear(h, T, D, L->wv_t, L->bv, D, v);
+        if (m->fp8) {
+            quant_e4m3_act(h, T, D, sa);
+            linear_e4m3(h, T, D, L->wq_t, sa, L->sq, L->bq, D, q);
+            linear_e4m3(h, T, D, L->wk_t, sa, L->sk, L->bk, D, k);
+            linear_e4m3(h, T, D, L->wv_t, sa, L->sv, L->bv, D, v);
+        } else {
+            linear(h, T, D, L->wq_t, L->bq, D, q);
+            linear(h, T, D, L->wk_t, L->bk, D, k);
+            linear(h, T, D, L->wv_t, L->bv, D, v);
+        }
         if (attn_full)
             attention_full_masked(q, k, v, win, n_win, T, a);
         else
@@ -684,12 +812,17 @@ int oracle_layers(const oracle_model *m, float *x, int T, const int *win, int n_
         linear(a, T, D, L->wo_t, L->bo, D, h);
         for (size_t i = 0; i < td; i++) x[i] = (float)((double)x[i] + h[i]);
         layernorm(x, T, D, L->ln2_g, L->ln2_b, h);
-        linear(h, T, D, L->w1_t, L->b1, D_FFN, f);
+        if (m->fp8) {
+            quant_e4m3_act(h, T, D, sa);
+            linear_e4m3(h, T, D, L->w1_t, sa, L->s1, L->b1, D_FFN, f);
+        } else {
+            linear(h, T, D, L->w1_t, L->b1, D_FFN, f);
+        }
         for (size_t i = 0; i < (size_t)T * D_FFN; i++) f[i] = (float)gelu(f[i]);
         linear(f, T, D_FFN, L->w2_t, L->b2, D, h);
         for (size_t i = 0; i < td; i++) x[i] = (float)((double)x[i] + h[i]);
     }
-    free(h); free(q); free(k); free(v); free(a); free(f);
+    free(h); free(q); free(k); free(v); free(a); free(f); free(sa);
     return 0;
 }
 

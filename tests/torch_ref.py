@@ -45,8 +45,25 @@ class TorchRef:
         y = F.linear(x[:tc], W["conv_out.weight"])
         return y + self.positions(tc)
 
-    def layers(self, x: torch.Tensor, windows, l0=0, l1=None) -> torch.Tensor:
+    @staticmethod
+    def e4m3_rows(x64: torch.Tensor):
+        """Per-row e4m3 operands of x (fp32 values): scale = row max / 448 in
+        fp32, values rounded by torch's float8_e4m3fn conversion."""
+        x = x64.to(torch.float32)
+        s = x.abs().amax(dim=1) / 448.0
+        safe = torch.where(s > 0, s, torch.ones_like(s))
+        q = (x / safe[:, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).to(torch.float64)
+        q = torch.where(s[:, None] > 0, q, torch.zeros_like(q))
+        return q, s.to(torch.float64)
+
+    def linear_e4m3(self, h: torch.Tensor, w: torch.Tensor, b: torch.Tensor) -> torch.Tensor:
+        a8, sa = self.e4m3_rows(h)
+        w8, sw = self.e4m3_rows(w)
+        return (a8 @ w8.T) * sa[:, None] * sw[None, :] + b
+
+    def layers(self, x: torch.Tensor, windows, l0=0, l1=None, fp8=False) -> torch.Tensor:
         W = self.w
+        lin = self.linear_e4m3 if fp8 else (lambda h, w, b: F.linear(h, w, b))
         T = x.shape[0]
         wid = torch.empty(T, dtype=torch.long)
         for i in range(len(windows) - 1):
@@ -56,14 +73,14 @@ class TorchRef:
         for l in range(l0, l1):
             p = f"layers.{l}."
             h = F.layer_norm(x, (1280,), W[p + "ln1.weight"], W[p + "ln1.bias"], eps=1e-5)
-            q = F.linear(h, W[p + "q.weight"], W[p + "q.bias"]).view(T, 20, 64).transpose(0, 1)
-            k = F.linear(h, W[p + "k.weight"], W[p + "k.bias"]).view(T, 20, 64).transpose(0, 1)
-            v = F.linear(h, W[p + "v.weight"], W[p + "v.bias"]).view(T, 20, 64).transpose(0, 1)
+            q = lin(h, W[p + "q.weight"], W[p + "q.bias"]).view(T, 20, 64).transpose(0, 1)
+            k = lin(h, W[p + "k.weight"], W[p + "k.bias"]).view(T, 20, 64).transpose(0, 1)
+            v = lin(h, W[p + "v.weight"], W[p + "v.bias"]).view(T, 20, 64).transpose(0, 1)
             a = F.scaled_dot_product_attention(q, k, v, attn_mask=mask)
             a = a.transpose(0, 1).reshape(T, 1280)
             x = x + F.linear(a, W[p + "o.weight"], W[p + "o.bias"])
             h = F.layer_norm(x, (1280,), W[p + "ln2.weight"], W[p + "ln2.bias"], eps=1e-5)
-            f = F.gelu(F.linear(h, W[p + "fc1.weight"], W[p + "fc1.bias"]))
+            f = F.gelu(lin(h, W[p + "fc1.weight"], W[p + "fc1.bias"]))
             x = x + F.linear(f, W[p + "fc2.weight"], W[p + "fc2.bias"])
         return x
 
