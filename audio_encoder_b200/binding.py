@@ -29,7 +29,7 @@ EXPORTED = [
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
     "moss_enc_tap_weight_count", "moss_enc_set_taps", "moss_enc_forward_taps",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
-    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_gemm_q4", "moss_enc_selftest_gelu",
+    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_gemm_q4", "moss_enc_gemm_f8", "moss_enc_selftest_gelu",
     "moss_enc_selftest_timeout",
 ]
 WEIGHTS_4BIT = 4
@@ -44,7 +44,8 @@ class MossEncError(RuntimeError):
 
 class Config(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int), ("max_samples", ctypes.c_int64),
-                ("max_clips", ctypes.c_int), ("out_dtype", ctypes.c_int), ("weight_bits", ctypes.c_int)]
+                ("max_clips", ctypes.c_int), ("out_dtype", ctypes.c_int), ("weight_bits", ctypes.c_int),
+                ("fp8", ctypes.c_int)]
 
 
 class KernelStat(ctypes.Structure):
@@ -122,6 +123,8 @@ def lib():
         L.moss_enc_gemm.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32]
         L.moss_enc_gemm_q4.restype = i32
         L.moss_enc_gemm_q4.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32]
+        L.moss_enc_gemm_f8.restype = i32
+        L.moss_enc_gemm_f8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32]
         L.moss_enc_logmel_static.restype = i32
         L.moss_enc_logmel_static.argtypes = [ctypes.POINTER(Clip), i32, ctypes.POINTER(vp), vp, vp]
         _lib = L
@@ -160,12 +163,12 @@ class Encoder:
     """
 
     def __init__(self, blob, n_layers: int, max_samples: int, max_clips: int = 1,
-                 out_dtype: int = OUT_F32, stream=None, weight_bits: int = 16):
+                 out_dtype: int = OUT_F32, stream=None, weight_bits: int = 16, fp8: bool = False):
         import torch
         self.torch = torch
         self.n_layers = n_layers
         self.out_dtype = out_dtype
-        cfg = Config(n_layers, int(max_samples), int(max_clips), int(out_dtype), int(weight_bits))
+        cfg = Config(n_layers, int(max_samples), int(max_clips), int(out_dtype), int(weight_bits), int(bool(fp8)))
         if stream is None:
             stream = torch.cuda.current_stream()
         self.stream = stream
@@ -232,6 +235,15 @@ class Encoder:
         N = Bq.shape[0]
         self._check(lib().moss_enc_gemm_q4(self.h, _ptr(A), _ptr(Bq), _ptr(Bs), _ptr(bias), _ptr(out), M, N, K,
                                            int(epilogue), int(block_n)))
+        return out
+
+    def gemm_f8(self, A8, B8, sa, sb, bias, out, epilogue: int, block_n: int):
+        """out = epi((A8 @ B8.T) * sa[:, None] * sb[None, :] + bias) on e4m3
+        operands (uint8 bits) A8 [M][K], B8 [N][K]."""
+        M, K = A8.shape
+        N = B8.shape[0]
+        self._check(lib().moss_enc_gemm_f8(self.h, _ptr(A8), _ptr(B8), _ptr(sa), _ptr(sb), _ptr(bias), _ptr(out),
+                                           M, N, K, int(epilogue), int(block_n)))
         return out
 
     def selftest_timeout(self, limit_ms: int = 50):

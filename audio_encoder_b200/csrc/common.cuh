@@ -466,6 +466,27 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, 
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
+// The same pair MMA on e4m3 operands (kind::f8f6f4, K = 32 per instruction:
+// one 32-byte step of the 128-byte swizzled rows, like kind::f16's K = 16).
+__device__ __forceinline__ void mma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// Instruction descriptor: kind::f8f6f4, e4m3 A and B (format 0, K-major), fp32
+// D, M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N)
+{
+    return (1u << 4)                      // D format f32
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
 // Arrive once on the barrier at cluster address `bar` when the pair's prior
 // MMAs have completed.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar)

@@ -54,6 +54,8 @@ struct GemmArgs {
     // kb reads stored block kb % kq_blocks (a [hi | lo] operand against [W | W]
     // stores W once)
     int kq_blocks;
+    // e4m3 operands only: out = acc * row_scale[m] * col_scale[n] + bias ...
+    const float *row_scale, *col_scale;
 };
 
 // Each epilogue warp stages 32 rows x 128 B in shared memory (16-byte
@@ -253,10 +255,13 @@ __device__ __forceinline__ void drain_tile(const GemmArgs &a, uint32_t tbase, in
 // Boxes are staged in `nbuf` 4 KB buffers used in turn (1024-byte aligned,
 // EPI_STAGE_BYTES apart); a buffer is rewritten only after the boxes in
 // flight have been read out of shared memory.
-template <int BN, int EPI, int NHALF = 2>
+template <int BN, int EPI, int NHALF = 2, bool SCALED = false>
 __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensorMap *tmC, uint32_t tbase, int half,
                                                int lane, uint8_t *stage_base, int nbuf, int row0, int col0)
 {
+    static_assert(!SCALED || EPI == EPI_BF16 || EPI == EPI_GELU_BF16, "scaled operands: bf16 outputs");
+    // e4m3 operands: this lane's row scale (its row of the slab)
+    const float rs = SCALED && row0 + lane < a.M ? a.row_scale[row0 + lane] : 0.0f;
     constexpr bool F32_OUT = EPI == EPI_RESID_F32 || EPI == EPI_F32;
     // bf16 boxes are 64 columns wide; fp32 boxes 32, so fp32 tiles may end
     // in a 32-column group (BN = 160: groups of 64, 64 and 32)
@@ -291,8 +296,15 @@ __device__ __forceinline__ void drain_tile_tma(const GemmArgs &a, const CUtensor
                 const float4 bb = ld_f4(b + 4 * q);
                 float2 v0 = make_float2(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]));
                 float2 v1 = make_float2(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-                v0 = __fadd2_rn(v0, make_float2(bb.x, bb.y));
-                v1 = __fadd2_rn(v1, make_float2(bb.z, bb.w));
+                if constexpr (SCALED) {
+                    // (acc * row scale) * column scale + bias
+                    const float4 cs = ld_f4(a.col_scale + col0 + c0 + 4 * q);
+                    v0 = __ffma2_rn(__fmul2_rn(v0, make_float2(rs, rs)), make_float2(cs.x, cs.y), make_float2(bb.x, bb.y));
+                    v1 = __ffma2_rn(__fmul2_rn(v1, make_float2(rs, rs)), make_float2(cs.z, cs.w), make_float2(bb.z, bb.w));
+                } else {
+                    v0 = __fadd2_rn(v0, make_float2(bb.x, bb.y));
+                    v1 = __fadd2_rn(v1, make_float2(bb.z, bb.w));
+                }
                 if constexpr (EPI == EPI_GELU_BF16) {
                     v0 = gelu2(v0);
                     v1 = gelu2(v1);
@@ -701,7 +713,10 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-template <int BN, int EPI, int AMODE = A_PLAIN, int KSUB = 1, int BQ = 0>
+// F8: A and B are e4m3 (one byte per element, so a 128-byte swizzled row holds
+// 128 k, and the stages' byte sizes are the bf16 ones), multiplied with
+// kind::f8f6f4; the epilogue scales by the row and column scales.
+template <int BN, int EPI, int AMODE = A_PLAIN, int KSUB = 1, int BQ = 0, int F8 = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, BQ>::THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
@@ -709,6 +724,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
 {
     using C = Gemm2Cfg<BN, KSUB, BQ>;
     static_assert(!BQ || AMODE == A_PLAIN, "4-bit B for plain GEMMs");
+    static_assert(!F8 || (AMODE == A_PLAIN && !BQ), "e4m3 operands for plain GEMMs");
+    constexpr int EK = F8 ? 128 : 64;  // k elements per 128-byte row
     // plain row-major outputs leave through TMA boxes (tmC); the conv and
     // conv_out row mappings and SwiGLU keep per-row stores
     constexpr bool TMA_OUT = AMODE == A_PLAIN &&
@@ -755,7 +772,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
     const uint32_t tmem_base = *tmem_slot;
 
     const int num_tiles = args.m_tiles * args.n_tiles;  // m_tiles counts 256-row pair tiles
-    const int num_kb = args.K / C::BK;
+    const int num_kb = args.K / (EK * KSUB);
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     // TMEM is held by every started CTA of this grid: the next kernel may start
     if (threadIdx.x == 0) grid_dep_launch();
@@ -779,7 +796,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
 #pragma unroll
                         for (int j = 0; j < C::NSUB; j++)
                             tma_load_2d_pair(&tmB, fb, st + C::A_BYTES + ks * C::B_KS + j * C::B_SUB_BYTES,
-                                             kb * C::BK + ks * 64, nt * BN + j * C::NS + (int)rank * (C::NS / 2));
+                                             (kb * KSUB + ks) * EK, nt * BN + j * C::NS + (int)rank * (C::NS / 2));
                 }
             };
             // The weights do not depend on earlier kernels: the first tile's
@@ -821,7 +838,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
                             const int b = kb * KSUB + ks, tap = b >> 3, kf = tap / 3, kt = tap - 3 * kf;
                             tma_load_4d_pair(&tmA, fb, st + ks * C::A_SUB, (b & 7) * 64, kf - 1, 2 * t0 + kt - 1, chunk);
                         } else {
-                            tma_load_2d_pair(&tmA, fb, st + ks * C::A_SUB, kb * C::BK + ks * 64, mt * 256 + (int)rank * 128);
+                            tma_load_2d_pair(&tmA, fb, st + ks * C::A_SUB, (kb * KSUB + ks) * EK, mt * 256 + (int)rank * 128);
                         }
                     }
                     if (!pre) load_b(st, fb, kb, nt, s);
@@ -831,7 +848,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = idesc_bf16(256, C::NS);
+            constexpr uint32_t idesc = F8 ? idesc_e4m3(256, C::NS) : idesc_bf16(256, C::NS);
             // Descriptors and barrier addresses are formed once: the issue loop
             // shares its SM sub-partition with epilogue warps, and every
             // instruction it saves brings the next MMA to the tensor pipe sooner.
@@ -865,10 +882,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
                         for (int k = 0; k < 4; k++)
 #pragma unroll
                             for (int j = 0; j < C::NSUB; j++)
-                                if (k < nk)
-                                    mma_bf16_pair(d + j * C::NS, ad + ks * (C::A_SUB >> 4) + 2 * k,
-                                                  bd + ks * (C::B_KS >> 4) + j * (C::B_SUB_BYTES >> 4) + 2 * k, idesc,
-                                                  (kb | ks | k) != 0);
+                                if (k < nk) {
+                                    const uint64_t da = ad + ks * (C::A_SUB >> 4) + 2 * k;
+                                    const uint64_t db = bd + ks * (C::B_KS >> 4) + j * (C::B_SUB_BYTES >> 4) + 2 * k;
+                                    if constexpr (F8)
+                                        mma_e4m3_pair(d + j * C::NS, da, db, idesc, (kb | ks | k) != 0);
+                                    else
+                                        mma_bf16_pair(d + j * C::NS, da, db, idesc, (kb | ks | k) != 0);
+                                }
                     }
                     mma_commit_pair(emp0 + 8 * s);
                     mma_commit_pair(emp1 + 8 * s);
@@ -920,8 +941,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
                 constexpr int RING_BUFS = (int)(C::STAGES * C::STAGE_BYTES / C::EPI_WARPS / EPI_STAGE_BYTES);
                 const bool last = tile + npairs >= num_tiles;
                 uint8_t *stg = last ? smem + (warp - 2) * RING_BUFS * EPI_STAGE_BYTES : stage;
-                drain_tile_tma<BN, EPI, C::EPI_WARPS / 4>(args, &tmC, tbase, half, lane, stg, last ? RING_BUFS : 1,
-                                        mt * 256 + (int)rank * 128 + q * 32, nt * BN);
+                drain_tile_tma<BN, EPI, C::EPI_WARPS / 4, F8 != 0>(args, &tmC, tbase, half, lane, stg,
+                                                                     last ? RING_BUFS : 1,
+                                                                     mt * 256 + (int)rank * 128 + q * 32, nt * BN);
             } else
                 drain_tile<BN, EPI, C::EPI_WARPS / 4>(args, tbase, half, lane, stage, grow, ok, aux, nt * BN);
             tc_fence_before();

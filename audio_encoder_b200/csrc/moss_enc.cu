@@ -14,6 +14,8 @@
 #include <string>
 #include <vector>
 
+#include <cuda_fp8.h>
+
 #include "../../include/moss_enc.h"
 #include "attn.cuh"
 #include "common.cuh"
@@ -47,6 +49,9 @@ struct LayerDev {
     bf16 *wqkv, *wo, *w1, *w2;
     float *bqkv, *bo, *b1, *b2;
     QW qqkv, qo, q1, q2;
+    // FP8 handles: q/k/v and fc1 as e4m3 [N][K] with per-channel scales [N]
+    const uint8_t *wqkv8 = nullptr, *w18 = nullptr;
+    const float *sqkv = nullptr, *s1 = nullptr;
 };
 
 // ln_post, proj1, proj2 and the SwiGLU adapter: the encoder's own set, and
@@ -73,7 +78,7 @@ struct moss_enc {
     // weights (one allocation; 4-bit handles keep the linear layers' codes
     // and scales in a second one)
     void *wmem = nullptr, *qmem = nullptr;
-    bool q4 = false;
+    bool q4 = false, fp8 = false;
     float *conv1_w = nullptr, *conv1_b = nullptr, *conv2_b = nullptr, *conv3_b = nullptr;
     bf16 *conv2_w = nullptr, *conv3_w = nullptr, *conv_out_w = nullptr;
     std::vector<LayerDev> layers;
@@ -101,6 +106,7 @@ struct moss_enc {
     float *pcm_stage = nullptr;
     void *out_stage = nullptr;
     bf16 *qscratch = nullptr;  // 4-bit handles: one expanded weight matrix
+    float *row_scale = nullptr;  // FP8 handles: the e4m3 LayerNorm rows' scales [T]
 
     // per-call tables: device copies and a ring of pinned host staging areas
     // (a call writes the next area once the copy that last read it has run,
@@ -382,6 +388,54 @@ static moss_enc_status gemm2q(moss_enc *h, const char *name, const bf16 *A, int6
     CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 1, 1>, dim3(grid), dim3(C::THREADS), C::SMEM, ta, tq, tc,
                          ts, a));
     return MOSS_ENC_OK;
+}
+
+// The pair GEMM on e4m3 operands: A8 [M][K] and B8 [N][K] bytes, row scales
+// a.row_scale [M] and column scales a.col_scale [N] applied in the epilogue
+// (bf16 outputs).  Two 128-wide k rows per stage.
+template <int BN, int EPI>
+static moss_enc_status gemm2f8(moss_enc *h, const char *name, const uint8_t *A8, int64_t M, int K, const uint8_t *B8,
+                               int N, GemmArgs a)
+{
+    using C = Gemm2Cfg<BN, 2>;
+    if (M <= 0) return MOSS_ENC_OK;
+    if (K % 256 != 0 || N % BN != 0 || M > INT32_MAX || !a.row_scale || !a.col_scale)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "gemm shape not supported");
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return fail(h, MOSS_ENC_ERR_CUDA, "no tensor-map encoder");
+    CUtensorMap ta, tb;
+    auto map8 = [&](CUtensorMap *m, const uint8_t *p, uint64_t rows, uint32_t box_rows) {
+        cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+        cuuint64_t strides[1] = {(cuuint64_t)K};
+        cuuint32_t box[2] = {128, box_rows};
+        cuuint32_t es[2] = {1, 1};
+        return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(p), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    if (!map8(&ta, A8, (uint64_t)M, 128) || !map8(&tb, B8, (uint64_t)N, C::NS / 2))
+        return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (e4m3)");
+    a.M = (int)M;
+    a.N = N;
+    a.K = K;
+    a.m_tiles = (int)((M + 255) / 256);
+    a.n_tiles = N / BN;
+    a.err = h->err;
+    CUtensorMap tc;
+    if (!tmap_out<BN, EPI>(&tc, a, tb)) return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (output)");
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int grid = 2 * std::min(tiles, h->num_sms / 2);
+    Launch L(h, name, 2.0 * M * N * K, 1.0 * M * K + 1.0 * N * K + epi_out_bytes(EPI) * M * N);
+    CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 2, 0, 1>, dim3(grid), dim3(C::THREADS), C::SMEM, ta, tb, tc,
+                         tb, a));
+    return MOSS_ENC_OK;
+}
+
+template <int BN, int EPI>
+static cudaError_t gemm2f8_attr()
+{
+    return cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI, A_PLAIN, 2, 0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Gemm2Cfg<BN, 2>::SMEM);
 }
 
 template <int BN, int EPI>
@@ -782,6 +836,10 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm2_attr<128, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<160, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_F32>()));
+    CUDA_TRY(h, (gemm2f8_attr<128, EPI_BF16>()));
+    CUDA_TRY(h, (gemm2f8_attr<256, EPI_BF16>()));
+    CUDA_TRY(h, (gemm2f8_attr<128, EPI_GELU_BF16>()));
+    CUDA_TRY(h, (gemm2f8_attr<256, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2q_attr<128, EPI_BF16>()));
     CUDA_TRY(h, (gemm2q_attr<256, EPI_BF16>()));
     CUDA_TRY(h, (gemm2q_attr<128, EPI_RESID_F32>()));
@@ -814,6 +872,32 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, cudaFuncSetAttribute(logmel4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel4Smem)));
     CUDA_TRY(h, cudaFuncSetAttribute(logmel4_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     return MOSS_ENC_OK;
+}
+
+// e4m3 quantisation of a bf16 matrix [n][k] in place, per row: s = fp32(max
+// |w|) / 448, codes e4m3(w / s) (round to nearest even, saturating) as bytes
+// [n][k] from the matrix's start, then the scales [n] at f8_scale_off.  A
+// zero row has scale 0 and zero codes.
+static size_t f8_scale_off(int n, int k) { return ((size_t)n * k + 255) & ~size_t(255); }
+
+static void quantise_e4m3_rows(uint8_t *mat, int n, int k)
+{
+    std::vector<uint8_t> codes((size_t)n * k);
+    std::vector<float> sc(n);
+    const uint16_t *w = reinterpret_cast<const uint16_t *>(mat);
+    for (int r = 0; r < n; r++) {
+        float amax = 0.0f;
+        for (int i = 0; i < k; i++) amax = std::max(amax, std::fabs(bf16_bits_to_float(w[(size_t)r * k + i])));
+        const float s = amax / 448.0f;
+        sc[r] = s;
+        for (int i = 0; i < k; i++)
+            codes[(size_t)r * k + i] =
+                s > 0.0f ? (uint8_t)__nv_cvt_float_to_fp8(bf16_bits_to_float(w[(size_t)r * k + i]) / s, __NV_SATFINITE,
+                                                          __NV_E4M3)
+                         : 0;
+    }
+    std::memcpy(mat, codes.data(), codes.size());
+    std::memcpy(mat + f8_scale_off(n, k), sc.data(), sizeof(float) * n);
 }
 
 // 4-bit round-to-nearest quantisation of one bf16 matrix [n][kq] (rows
@@ -867,7 +951,8 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     *out = nullptr;
     if (!cfg || !weights || cfg->n_layers < 1 || cfg->n_layers > 32 || cfg->max_samples < 1 ||
         cfg->max_clips < 1 || (cfg->out_dtype != MOSS_ENC_OUT_F32 && cfg->out_dtype != MOSS_ENC_OUT_BF16) ||
-        (cfg->weight_bits != 0 && cfg->weight_bits != 16 && cfg->weight_bits != 4))
+        (cfg->weight_bits != 0 && cfg->weight_bits != 16 && cfg->weight_bits != 4) ||
+        (cfg->fp8 != 0 && cfg->fp8 != 1) || (cfg->fp8 && cfg->weight_bits == 4))
         return MOSS_ENC_ERR_INVALID_ARG;
     const int64_t count = moss_enc_weight_count(cfg->n_layers);
     if ((int64_t)bytes != count * 2) return MOSS_ENC_ERR_INVALID_ARG;
@@ -1056,6 +1141,19 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         quantise_all(pk.data(), qk.data(), qs.data(), qs.size());
     }
 
+    // ---- FP8 handles: q/k/v and fc1 as e4m3 per output channel, written over
+    // their bf16 slots (codes [N][K], then the scales [N] at the next 256 bytes)
+    h->fp8 = cfg->fp8 == 1;
+    if (h->fp8) {
+        std::vector<std::thread> pool;
+        for (int l = 0; l < L; l++)
+            for (int which = 0; which < 2; which++) {
+                const size_t o = lo[l * 12 + (which == 0 ? 4 : 8)];
+                const int n = which == 0 ? DQKV : DFF;
+                pool.emplace_back([&pk, o, n]() { quantise_e4m3_rows(pk.data() + o, n, D); });
+            }
+        for (auto &th : pool) th.join();
+    }
     const size_t upload = h->q4 ? small_total : wtotal;
     if (cudaMalloc(&h->wmem, upload) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaMemcpy(h->wmem, pk.data(), upload, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
@@ -1097,6 +1195,13 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         d.b1 = (float *)(W + L12[9]);
         d.w2 = big(L12[10]);
         d.b2 = (float *)(W + L12[11]);
+        if (h->fp8) {
+            d.wqkv = d.w1 = nullptr;
+            d.wqkv8 = W + L12[4];
+            d.sqkv = (const float *)(W + L12[4] + f8_scale_off(DQKV, D));
+            d.w18 = W + L12[8];
+            d.s1 = (const float *)(W + L12[8] + f8_scale_off(DFF, D));
+        }
         if (h->q4) {
             d.qqkv = qw(4 * l);
             d.qo = qw(4 * l + 1);
@@ -1143,6 +1248,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     // 4-bit handles: one linear layer's matrix expanded to bf16 (the largest is
     // the adapter's interleaved gate/up, 16384 x 2048)
     const size_t w_qs = h->q4 ? take(2 * (size_t)2 * DADP * DOUT) : 0;
+    const size_t w_rs = take(4 * (size_t)T);
     if (cudaMalloc(&h->ws, off) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     uint8_t *S = static_cast<uint8_t *>(h->ws);
     h->mel_raw = (float *)(S + w_mel);
@@ -1162,6 +1268,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     h->pcm_stage = (float *)(S + w_pcm);
     h->out_stage = (void *)(S + w_out);
     h->qscratch = h->q4 ? (bf16 *)(S + w_qs) : nullptr;
+    h->row_scale = (float *)(S + w_rs);
     if (cudaMemset(h->err, 0, 256) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
 
     const TabLayout tl = tab_layout(cfg->max_clips, h->max_chunks);
@@ -1636,7 +1743,12 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
             W1 = xs_1;
             W2 = xs_2;
         }
-        {
+        uint8_t *xn8 = reinterpret_cast<uint8_t *>(h->xn);  // FP8 handles: e4m3 LayerNorm rows
+        if (h->fp8) {
+            Launch Lk(h, "layernorm", 8.0 * T * D, 5.0 * T * D);
+            CUDA_TRY(h, launch_k(h, layernorm1280_e4m3_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln1_g,
+                                 L.ln1_b, xn8, h->row_scale, (int)T));
+        } else {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln1_g, L.ln1_b,
                                  h->xn, (int)T, D, 0));
@@ -1645,7 +1757,15 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.bqkv;
         a.out = h->qkv;
         a.ldo = DQKV;
-        if (qf)
+        if (h->fp8) {
+            a.row_scale = h->row_scale;
+            a.col_scale = L.sqkv;
+            if (T <= 512)
+                TRY((gemm2f8<128, EPI_BF16>(h, "gemm_qkv", xn8, T, D, L.wqkv8, DQKV, a)));
+            else
+                TRY((gemm2f8<256, EPI_BF16>(h, "gemm_qkv", xn8, T, D, L.wqkv8, DQKV, a)));
+            a.row_scale = a.col_scale = nullptr;
+        } else if (qf)
             TRY((gemm2q<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, L.qqkv, DQKV, a)));
         else if (T <= 512)  // two row tiles: 128-wide tiles (30 per row tile) keep more SMs busy than 256-wide (15)
             TRY((gemm2<128, EPI_BF16>(h, "gemm_qkv", h->xn, T, D, Wqkv, DQKV, a)));
@@ -1660,7 +1780,11 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.out = h->X;
         a.ldo = D;
         TRY(resid_gemm("gemm_out", h->attn, D, Wo, L.qo, a));
-        {
+        if (h->fp8) {
+            Launch Lk(h, "layernorm", 8.0 * T * D, 5.0 * T * D);
+            CUDA_TRY(h, launch_k(h, layernorm1280_e4m3_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln2_g,
+                                 L.ln2_b, xn8, h->row_scale, (int)T));
+        } else {
             Launch Lk(h, "layernorm", 8.0 * T * D, 6.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln2_g, L.ln2_b,
                                  h->xn, (int)T, D, 0));
@@ -1668,6 +1792,12 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.b1;
         a.out = h->ffn;
         a.ldo = DFF;
+        if (h->fp8) {
+            a.row_scale = h->row_scale;
+            a.col_scale = L.s1;
+            TRY((gemm2f8<256, EPI_GELU_BF16>(h, "gemm_fc1", xn8, T, D, L.w18, DFF, a)));
+            a.row_scale = a.col_scale = nullptr;
+        } else
         TRY((qf ? gemm2q<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, L.q1, DFF, a)
                 : gemm2<256, EPI_GELU_BF16>(h, "gemm_fc1", h->xn, T, D, W1, DFF, a)));
         a.bias = L.b2;
@@ -2146,6 +2276,33 @@ extern "C" moss_enc_status moss_enc_gemm_q4(moss_enc *h, const void *A, const vo
     case 256: return gemm_q4_one<256>(h, a, q, bias, out, M, N, K, epilogue);
     case 320: return gemm_q4_one<320>(h, a, q, bias, out, M, N, K, epilogue);
     default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160, 256 or 320");
+    }
+}
+
+extern "C" moss_enc_status moss_enc_gemm_f8(moss_enc *h, const void *A8, const void *B8, const float *sa,
+                                            const float *sb, const float *bias, void *out, int M, int N, int K,
+                                            int epilogue, int block_n)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (!A8 || !B8 || !sa || !sb || !bias || !out || M < 0 || N <= 0 || K <= 0 || K % 256 != 0)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad gemm arguments");
+    if ((reinterpret_cast<uintptr_t>(A8) | reinterpret_cast<uintptr_t>(B8)) & 15)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A8 and B8 must be 16-byte aligned");
+    if (block_n != 128 && block_n != 256) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128 or 256");
+    if (N % block_n != 0) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n != 0");
+    GemmArgs a{};
+    a.bias = bias;
+    a.out = out;
+    a.ldo = N;
+    a.row_scale = sa;
+    a.col_scale = sb;
+    const uint8_t *a8 = static_cast<const uint8_t *>(A8), *b8 = static_cast<const uint8_t *>(B8);
+    switch (epilogue * 2 + (block_n == 256 ? 1 : 0)) {
+    case EPI_BF16 * 2: return gemm2f8<128, EPI_BF16>(h, "gemm_api", a8, M, K, b8, N, a);
+    case EPI_BF16 * 2 + 1: return gemm2f8<256, EPI_BF16>(h, "gemm_api", a8, M, K, b8, N, a);
+    case EPI_GELU_BF16 * 2: return gemm2f8<128, EPI_GELU_BF16>(h, "gemm_api", a8, M, K, b8, N, a);
+    case EPI_GELU_BF16 * 2 + 1: return gemm2f8<256, EPI_GELU_BF16>(h, "gemm_api", a8, M, K, b8, N, a);
+    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "epilogue must be 0 or 1");
     }
 }
 

@@ -14,8 +14,9 @@ batch (clips are independent: weak scaling, no collective on the data path).
 
 At N = 1 the line also carries `other_configs`: the 1 s / 4-layer clip, the
 single 30 s clip, the 10-min clip and the 60-min clip streamed in 64 s pieces
-(with the encoder's device memory), each timed the same way, and the batch
-and the streamed clip again with 4-bit weights (`_w4`); and
+(with the encoder's device memory), each timed the same way, the batch and
+the streamed clip again with 4-bit weights (`_w4`), and the batch with FP8
+q/k/v and fc1 GEMMs (`_fp8`); and
 `cpu_baseline` times the oracle on all host cores and on one core.
 
 The reference arm (--impl reference) times the CPU oracle on the host cores
@@ -539,7 +540,7 @@ def run_streamed(args):
         dist.destroy_process_group()
 
 
-def measure_plain(workload, steps, warmup, dev, weight_bits=16):
+def measure_plain(workload, steps, warmup, dev, weight_bits=16, fp8=False):
     """One workload's forward timed as the headline is (device-resident PCM,
     CUDA events on the encoder's stream, L2 flushed between steps)."""
     import torch
@@ -550,7 +551,7 @@ def measure_plain(workload, steps, warmup, dev, weight_bits=16):
     stream = torch.cuda.Stream()
     total = sum(c.size for c in clips)
     enc = binding.Encoder(synth.make_weights(n_layers), n_layers, max_samples=total, max_clips=len(clips),
-                          out_dtype=binding.OUT_BF16, stream=stream, weight_bits=weight_bits)
+                          out_dtype=binding.OUT_BF16, stream=stream, weight_bits=weight_bits, fp8=fp8)
     tokens = sum(binding.num_tokens(c.size) for c in clips)
     with torch.cuda.stream(stream):
         xs = [torch.from_numpy(c).to(dev) for c in clips]
@@ -582,13 +583,14 @@ def other_configs(args, dev):
     pk = peaks()
     res = {}
     steps = max(3, min(args.steps, 20))
-    # the last two: the 4-bit-weight encoder (round to nearest, groups of 128)
+    # then the 4-bit-weight encoder (round to nearest, groups of 128) and the
+    # FP8 encoder (q/k/v and fc1 on e4m3 operands)
     for w, bits in (("tiny_1s", 16), ("single_30s", 16), ("clip_10min", 16), ("clip_60min_streamed", 16),
-                    ("batch16_10to30s", 4), ("clip_60min_streamed", 4)):
+                    ("batch16_10to30s", 4), ("clip_60min_streamed", 4), ("batch16_10to30s", 8)):
         if w == "clip_60min_streamed":
             r = measure_streamed(max(3, min(args.steps, 10)), 3, dev, weight_bits=bits)
         else:
-            r = measure_plain(w, steps, 3, dev, weight_bits=bits)
+            r = measure_plain(w, steps, 3, dev, weight_bits=4 if bits == 4 else 16, fp8=bits == 8)
         tf = model_flops(r["tokens"], r["n_layers"]) / (r["ms"] / 1e3) / 1e12
         e = {"value": r["audio_s"] / (r["ms"] / 1e3), "unit": "audio-s/s", "ms_per_step": r["ms"],
              "tokens_per_s": r["tokens"] / (r["ms"] / 1e3), "tokens": r["tokens"], "layers": r["n_layers"],
@@ -598,8 +600,9 @@ def other_configs(args, dev):
             e.update({"pieces": r["pieces"], "piece_samples": r["piece"],
                       "encoder_device_bytes": r["encoder_device_bytes"],
                       "clip_and_rows_device_bytes": r["clip_and_rows_device_bytes"]})
-        e["weight_bits"] = bits
-        res[w if bits == 16 else w + "_w4"] = e
+        e["weight_bits"] = 4 if bits == 4 else 16
+        e["fp8_qkv_fc1"] = bits == 8
+        res[w if bits == 16 else w + ("_w4" if bits == 4 else "_fp8")] = e
     return res
 
 

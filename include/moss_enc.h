@@ -64,7 +64,26 @@ typedef struct {
     int weight_bits;       /* 16 (or 0): bf16 weights; 4: the linear layers of the
                               encoder layers, head and adapter are kept as 4-bit
                               codes (see MOSS_ENC_WEIGHTS_4BIT) */
+    int fp8;               /* 1: the q/k/v and fc1 GEMMs of every layer take e4m3
+                              operands (see MOSS_ENC_FP8); 0: bf16.  Not with
+                              weight_bits = 4. */
 } moss_enc_config;
+
+/* FP8 GEMMs (page "Ossicle-4B", "Quantized: NVFP4 and INT4 in vLLM": the
+ * low-precision builds quantise the audio encoder's weights and activations
+ * for Blackwell's low-precision tensor cores).  With cfg.fp8 = 1 the two
+ * GEMMs of every layer that a LayerNorm feeds (q/k/v and fc1) multiply e4m3
+ * operands on the tensor cores (kind::f8f6f4, fp32 accumulation):
+ *   weights, per output channel n:  s_w[n] = max_k |w[n][k]| / 448,
+ *                                   w8 = e4m3(w / s_w[n])   (at create)
+ *   LayerNorm rows, per row m:      s_a[m] = max_k |y[m][k]| / 448,
+ *                                   a8 = e4m3(y / s_a[m])   (the LayerNorm
+ *                                   kernel writes a8 and s_a)
+ *   out[m][n] = (sum_k a8 w8) * s_a[m] * s_w[n] + b[n]      (then GELU for fc1)
+ * e4m3 rounds to nearest (ties to even) and saturates at +-448; scales and
+ * divisions in fp32.  The other GEMMs keep bf16 operands.  The rows then
+ * match the FP8 model of the same definition (not the bf16 model). */
+#define MOSS_ENC_FP8 1
 
 /* 4-bit weights (page "Ossicle-4B", "Long Audio", the note under the table:
  * "4-bit weights for ... the audio encoder, round to nearest, groups of 128").
@@ -305,6 +324,15 @@ moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const f
  * or 320, CTA pairs only; K % 128 == 0; epilogues as moss_enc_gemm. */
 moss_enc_status moss_enc_gemm_q4(moss_enc *h, const void *A, const void *Bq, const float *Bs, const float *bias,
                                  void *out, int M, int N, int K, int epilogue, int block_n);
+
+/* The same GEMM on e4m3 operands (the form the q/k/v and fc1 GEMMs take with
+ * cfg.fp8 = 1): A8 device uint8 [M][K] and B8 device uint8 [N][K] (e4m3
+ * bits), sa device fp32 [M], sb device fp32 [N];
+ *   out[m][n] = epi((sum_k A8 B8) * sa[m] * sb[n] + bias[n]),
+ * epilogue 0 (bf16 out) or 1 (GELU, bf16 out); block_n 128 or 256 (CTA
+ * pairs); K % 256 == 0. */
+moss_enc_status moss_enc_gemm_f8(moss_enc *h, const void *A8, const void *B8, const float *sa, const float *sb,
+                                 const float *bias, void *out, int M, int N, int K, int epilogue, int block_n);
 
 /* The GEMM epilogues and conv1 evaluate GELU's erf with a short rational
  * approximation (Abramowitz & Stegun 7.1.28, error <= 3e-7), one value at a

@@ -6,6 +6,15 @@ import numpy as np
 MEL_ATOL = 1e-4
 ROW_COS = 0.999
 ROW_MAXERR_RMS = 3e-2
+# The FP8 variant (q/k/v and fc1 on e4m3 operands) against the oracle's FP8
+# model: an e4m3 step is up to 2^-3 of its value (bf16's is 2^-8), and the
+# GPU's fp32 LayerNorm rows and the oracle's differ by ~1e-6 relative, so the
+# few operands within that distance of a rounding midpoint round to
+# neighbouring e4m3 values in the two implementations.  Measured: min cosine
+# 0.99956 and max |err| 0.138 rms on the single 30 s clip (0.43 rms against
+# the bf16 model); the bound keeps the cosine and allows 0.25 rms.
+FP8_ROW_COS = 0.999
+FP8_ROW_MAXERR_RMS = 0.25
 
 
 def row_metrics(got, ref):
@@ -19,12 +28,12 @@ def row_metrics(got, ref):
     return cos, maxerr / (rms + 1e-30)
 
 
-def assert_rows_close(got, ref, what=""):
+def assert_rows_close(got, ref, what="", cos_min=ROW_COS, maxerr_rms=ROW_MAXERR_RMS):
     if np.asarray(ref).shape[0] == 0:
         assert np.asarray(got).shape == np.asarray(ref).shape
         return
     cos, rel = row_metrics(got, ref)
-    bad = (cos < ROW_COS) | (rel > ROW_MAXERR_RMS)
+    bad = (cos < cos_min) | (rel > maxerr_rms)
     assert not bad.any(), (f"{what}: {bad.sum()} of {len(cos)} rows out of tolerance; "
                            f"min cos {cos.min():.6f}, max err/rms {rel.max():.4f} (row {int(rel.argmax())})")
     return cos.min(), rel.max()
