@@ -539,7 +539,11 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 //    commits once to its own and once to the odd CTA's barrier.
 //  - tempty[acc] lives in the even CTA; all 16 epilogue warps of the pair
 //    arrive on it.
-template <int BN, int KSUB = 1, int BQ = 0>
+// RING: every CTA pair computes at most one tile (the launch has no more
+// tiles than pairs), so the epilogue always stages its output boxes in the
+// idle stage ring and the separate staging area is left out: the room goes
+// to the pipeline (320-wide tiles get three stages of two k sub-blocks).
+template <int BN, int KSUB = 1, int BQ = 0, int RING = 0>
 struct Gemm2Cfg {
     // A stage holds KSUB k sub-blocks of 64 (one 128-byte swizzle atom each):
     // larger stages halve the stage hand-offs between the producer, the MMA
@@ -576,7 +580,7 @@ struct Gemm2Cfg {
                   "TMA destinations on 128-byte boundaries");
     // bytes each CTA's TMA completes on the pair's full barrier per stage
     static constexpr uint32_t FULL_TX = BQ ? A_BYTES : A_BYTES + B_BYTES;
-    static constexpr uint32_t STAGING = EPI_WARPS * EPI_STAGE_BYTES;
+    static constexpr uint32_t STAGING = RING ? 0 : EPI_WARPS * EPI_STAGE_BYTES;
     static constexpr int STAGES_RAW = (int)((SMEM_LIMIT - 1024 - 256 - STAGING) / STAGE_BYTES);
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr int ACC = 2 * BN <= 512 ? 2 : 1;  // TMEM accumulators (double buffer when they fit)
@@ -716,13 +720,13 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads)
 // F8: A and B are e4m3 (one byte per element, so a 128-byte swizzled row holds
 // 128 k, and the stages' byte sizes are the bf16 ones), multiplied with
 // kind::f8f6f4; the epilogue scales by the row and column scales.
-template <int BN, int EPI, int AMODE = A_PLAIN, int KSUB = 1, int BQ = 0, int F8 = 0>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, BQ>::THREADS, 1)
+template <int BN, int EPI, int AMODE = A_PLAIN, int KSUB = 1, int BQ = 0, int F8 = 0, int RING = 0>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, BQ, RING>::THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
                     const GemmArgs args)
 {
-    using C = Gemm2Cfg<BN, KSUB, BQ>;
+    using C = Gemm2Cfg<BN, KSUB, BQ, RING>;
     static_assert(!BQ || AMODE == A_PLAIN, "4-bit B for plain GEMMs");
     static_assert(!F8 || (AMODE == A_PLAIN && !BQ), "e4m3 operands for plain GEMMs");
     constexpr int EK = F8 ? 128 : 64;  // k elements per 128-byte row
@@ -732,6 +736,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
                              ((BN % 64 == 0 && (EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 ||
                                                 EPI == EPI_F32)) ||
                               (BN % 64 == 32 && (EPI == EPI_RESID_F32 || EPI == EPI_F32)));
+    static_assert(!RING || TMA_OUT, "only the TMA epilogue stages in the ring");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES + C::STAGING);
@@ -939,7 +944,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, KSUB, B
                 // so each epilogue warp stages through its eighth of the ring and
                 // keeps several boxes in flight; otherwise one 4 KB buffer.
                 constexpr int RING_BUFS = (int)(C::STAGES * C::STAGE_BYTES / C::EPI_WARPS / EPI_STAGE_BYTES);
-                const bool last = tile + npairs >= num_tiles;
+                const bool last = RING || tile + npairs >= num_tiles;
                 uint8_t *stg = last ? smem + (warp - 2) * RING_BUFS * EPI_STAGE_BYTES : stage;
                 drain_tile_tma<BN, EPI, C::EPI_WARPS / 4, F8 != 0>(args, &tmC, tbase, half, lane, stg,
                                                                      last ? RING_BUFS : 1,

@@ -325,7 +325,13 @@ static moss_enc_status gemm2(moss_enc *h, const char *name, const bf16 *A, int64
     const int grid = 2 * std::min(tiles, h->num_sms / 2);
     const double ka = k_alg > 0 ? k_alg : K;
     Launch L(h, name, 2.0 * M * N * ka, 2.0 * M * ka + 2.0 * N * ka + epi_out_bytes(EPI) * M * N);
-    if (ksub == 2 && K % 128 == 0)
+    // 320-wide tiles of a launch with no more tiles than SM pairs: two k
+    // sub-blocks per stage, three stages, output staged in the idle ring
+    constexpr bool ring_ok = BN == 320 && (EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 || EPI == EPI_F32);
+    if (ring_ok && tiles <= h->num_sms / 2 && K % 128 == 0)
+        CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 2, 0, 0, ring_ok ? 1 : 0>, dim3(grid),
+                             dim3(Gemm2Cfg<BN, 2, 0, 1>::THREADS), Gemm2Cfg<BN, 2, 0, 1>::SMEM, ta, tb, tc, tb, a));
+    else if (ksub == 2 && K % 128 == 0)
         CUDA_TRY(h, launch_k(h, gemm_tc2_kernel<BN, EPI, A_PLAIN, 2>, dim3(grid), dim3(Gemm2Cfg<BN, 2>::THREADS),
                              Gemm2Cfg<BN, 2>::SMEM, ta, tb, tc, tb, a));
     else
@@ -451,6 +457,12 @@ static cudaError_t gemm2_attr()
     cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI, A_PLAIN, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Gemm2Cfg<BN, 1>::SMEM);
     if (e != cudaSuccess) return e;
+    constexpr bool ring_ok = BN == 320 && (EPI == EPI_BF16 || EPI == EPI_GELU_BF16 || EPI == EPI_RESID_F32 || EPI == EPI_F32);
+    if (ring_ok) {
+        e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI, A_PLAIN, 2, 0, 0, ring_ok ? 1 : 0>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Gemm2Cfg<BN, 2, 0, 1>::SMEM);
+        if (e != cudaSuccess) return e;
+    }
     return cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI, A_PLAIN, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)Gemm2Cfg<BN, 2>::SMEM);
 }
