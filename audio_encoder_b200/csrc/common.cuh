@@ -85,6 +85,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     }
 }
 
+// Barrier `id` (1..15) over the first `threads` threads' warps that reach it.
+__device__ __forceinline__ void named_bar_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// After a wait gave up: wait, at most WAIT_LIMIT_NS and whatever *err says,
+// for the phase with the given parity (copies or MMAs this CTA started), so
+// that nothing still writes shared memory or TMEM once they are released.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((i & 255u) == 0 && globaltimer_ns() - t0 > WAIT_LIMIT_NS) return;
+    }
+}
+
 // ------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,

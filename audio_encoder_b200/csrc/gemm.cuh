@@ -712,10 +712,6 @@ __global__ void __launch_bounds__(256) q4_expand_kernel(const __grid_constant__ 
     }
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int threads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
 
 // F8: A and B are e4m3 (one byte per element, so a 128-byte swizzled row holds
 // 128 k, and the stages' byte sizes are the bf16 ones), multiplied with

@@ -79,7 +79,8 @@ struct moss_enc {
     // and scales in a second one)
     void *wmem = nullptr, *qmem = nullptr;
     bool q4 = false, fp8 = false;
-    float *conv1_w = nullptr, *conv1_b = nullptr, *conv2_b = nullptr, *conv3_b = nullptr;
+    const uint4 *conv1_wt = nullptr;  // conv1 as the B operand of its GEMM (see conv1_tc_kernel)
+    float *conv2_b = nullptr, *conv3_b = nullptr;
     bf16 *conv2_w = nullptr, *conv3_w = nullptr, *conv_out_w = nullptr;
     std::vector<LayerDev> layers;
     HeadDev head{};
@@ -226,7 +227,7 @@ static PFN_encodeTiled_t encode_fn()
 // 2-D bf16 tensor map: rows of `inner` elements, `row_bytes` apart; box of
 // box_inner x box_rows with 128-byte swizzle (box_inner = 64).
 static bool tmap_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, uint64_t row_bytes,
-                    uint32_t box_inner, uint32_t box_rows)
+                    uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     PFN_encodeTiled_t fn = encode_fn();
     if (!fn) return false;
@@ -235,7 +236,7 @@ static bool tmap_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t ro
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -881,6 +882,7 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm_attr<128, EPI_F32>()));
     CUDA_TRY(h, (gemm_attr<128, EPI_BF16>()));
     CUDA_TRY(h, cudaFuncSetAttribute(window_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATTN_TC_SMEM));
+    CUDA_TRY(h, cudaFuncSetAttribute(conv1_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C1_SMEM));
     CUDA_TRY(h, cudaFuncSetAttribute(logmel4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Mel4Smem)));
     CUDA_TRY(h, cudaFuncSetAttribute(logmel4_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     return MOSS_ENC_OK;
@@ -1006,7 +1008,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         off += (b + 255) & ~size_t(255);
         return r;
     };
-    const size_t o_c1w = take(4 * CST * 9), o_c1b = take(4 * CST);
+    const size_t o_c1t = take(C1_B_BYTES);
     const size_t o_c2w = take(2 * (size_t)CST * CONV_K), o_c2b = take(4 * CST);
     const size_t o_c3w = take(2 * (size_t)CST * CONV_K), o_c3b = take(4 * CST);
     const size_t o_cow = take(2 * (size_t)D * CST * 16);
@@ -1046,11 +1048,19 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     auto F32 = [&](size_t o) { return reinterpret_cast<float *>(pk.data() + o); };
     auto U16 = [&](size_t o) { return reinterpret_cast<uint16_t *>(pk.data() + o); };
     const uint16_t *p = src;
-    // conv1 [480][1][3][3] -> fp32 [480][9]
-    for (int i = 0; i < CST * 9; i++) F32(o_c1w)[i] = bf16_bits_to_float(p[i]);
-    p += CST * 9;
-    for (int i = 0; i < CST; i++) F32(o_c1b)[i] = bf16_bits_to_float(p[i]);
-    p += CST;
+    // conv1 [480][1][3][3] and its bias -> the K-major B operand of conv1_tc_kernel:
+    // row c = [w(c, tap 0..8), w(c, tap 0..8), b(c), 0 ...] (64 bf16, tap = 3 kf + kt),
+    // its 16-byte chunks swizzled by the row's position in its 8-row group
+    {
+        uint16_t *dst = U16(o_c1t);
+        for (int c = 0; c < CST; c++) {
+            uint16_t row[64] = {};
+            for (int tap = 0; tap < 9; tap++) row[tap] = row[9 + tap] = p[c * 9 + tap];
+            row[18] = p[CST * 9 + c];
+            for (int k = 0; k < 64; k++) dst[c * 64 + (((k >> 3) ^ (c & 7)) << 3) + (k & 7)] = row[k];
+        }
+    }
+    p += CST * 9 + CST;
     // conv2/conv3 [o][c][kf][kt] -> [o][(kf*3+kt)*512 + c]
     for (int which = 0; which < 2; which++) {
         uint16_t *dst = U16(which == 0 ? o_c2w : o_c3w);
@@ -1185,8 +1195,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     uint8_t *W = static_cast<uint8_t *>(h->wmem);
     // bf16 matrices exist on the device only for bf16 handles
     auto big = [&](size_t o) -> bf16 * { return h->q4 ? nullptr : (bf16 *)(W + o); };
-    h->conv1_w = (float *)(W + o_c1w);
-    h->conv1_b = (float *)(W + o_c1b);
+    h->conv1_wt = (const uint4 *)(W + o_c1t);
     h->conv2_w = (bf16 *)(W + o_c2w);
     h->conv2_b = (float *)(W + o_c2b);
     h->conv3_w = (bf16 *)(W + o_c3w);
@@ -1683,9 +1692,15 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         {
             double px = 0.0;
             for (int j = 0; j < gc; j++) px += 64.0 * sc[g0 + j].t1_lim;
+            int tiles = 0;  // 128-pixel tiles (two time steps) inside the receptive fields
+            for (int j = 0; j < gc; j++) tiles += (sc[g0 + j].t1_lim + 1) / 2;
             Launch L1(h, "conv1", 2.0 * 9 * CST * px, 2.0 * CST * px + 4.0 * 128 * 2 * px / 64.0);
-            CUDA_TRY(h, launch_k(h, conv1_kernel, dim3(200, gc), dim3(240), 0, (const float *)h->mel_raw, d_chunks + g0,
-                                 (const int *)h->gmax_ord, (const float *)h->conv1_w, (const float *)h->conv1_b, h->c1out));
+            CUtensorMap tm_c1;  // conv1 output rows [chunk][t][f] x 480 channels: boxes of 80 x 32
+            if (!tmap_2d(&tm_c1, h->c1out, CST, (uint64_t)gc * 400 * 64, 2 * CST, 80, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+                return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (conv1 output)");
+            CUDA_TRY(h, launch_k(h, conv1_tc_kernel, dim3(std::max(1, std::min(tiles, h->num_sms))), dim3(C1_THREADS),
+                                 C1_SMEM, (const float *)h->mel_raw, d_chunks + g0, gc, (const int *)h->gmax_ord,
+                                 h->conv1_wt, tm_c1, h->err));
         }
         TRY(gemm_conv(h, "gemm_conv2", h->c1out, gc, 400, 64, d_t2 + g_off2[gi], g_n2[gi], h->conv2_w, h->conv2_b,
                       h->c2out));
