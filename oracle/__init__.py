@@ -86,6 +86,11 @@ def lib():
         L.oracle_e4m3.restype = f32
         L.oracle_e4m3.argtypes = [f32]
         L.oracle_quant_e4m3_rows.argtypes = [vp, i32, i32, vp, vp]
+        L.oracle_e2m1.restype = f32
+        L.oracle_e2m1.argtypes = [f32]
+        L.oracle_quant_nvfp4.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
+        L.oracle_model_create_nvfp4.restype = vp
+        L.oracle_model_create_nvfp4.argtypes = [vp, i32]
         L.oracle_set_threads.argtypes = [i32]
         L.oracle_max_threads.restype = i32
     return _lib
@@ -213,18 +218,43 @@ def quant_e4m3_rows(w: np.ndarray):
     return q, s
 
 
+def e2m1(x: float) -> float:
+    """The nearest E2M1 value (ties to even, saturating at +-6)."""
+    return float(lib().oracle_e2m1(float(x)))
+
+
+def quant_nvfp4(x: np.ndarray, per_row: bool):
+    """NVFP4 quantisation of x [rows][cols] (cols a multiple of 16): returns
+    (units q * s_b [rows][cols] fp32, g [rows] or [1] fp32, E2M1 codes
+    [rows][cols] uint8 (sign bit 3), block scales [rows][cols / 16] fp32)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    if cols % 16:
+        raise ValueError("cols must be a multiple of 16")
+    unit = np.empty_like(x)
+    g = np.empty(rows if per_row else 1, dtype=np.float32)
+    codes = np.empty((rows, cols), dtype=np.uint8)
+    bs = np.empty((rows, cols // 16), dtype=np.float32)
+    lib().oracle_quant_nvfp4(_p(x), rows, cols, int(per_row), _p(unit), _p(g), _p(codes), _p(bs))
+    return unit, g, codes, bs
+
+
 class Model:
     """The oracle's copy of a bf16 weight blob (uint16 bit patterns);
     weight_bits=4 gives the model with 4-bit quantised linear layers, 8 the
-    model whose q, k, v and fc1 GEMMs take e4m3 operands."""
+    model whose q, k, v and fc1 GEMMs take e4m3 operands; nvfp4=True the model
+    whose q, k, v and fc1 GEMMs take NVFP4 operands."""
 
-    def __init__(self, blob: np.ndarray, n_layers: int, weight_bits: int = 16):
+    def __init__(self, blob: np.ndarray, n_layers: int, weight_bits: int = 16, nvfp4: bool = False):
         blob = np.ascontiguousarray(blob, dtype=np.uint16)
         if blob.size != weight_count(n_layers):
             raise ValueError(f"blob has {blob.size} elements, expected {weight_count(n_layers)}")
         self._blob = blob  # the model points into it
         self.n_layers = n_layers
-        self._h = lib().oracle_model_create_bits(_p(blob), n_layers, int(weight_bits))
+        if nvfp4:
+            self._h = lib().oracle_model_create_nvfp4(_p(blob), n_layers)
+        else:
+            self._h = lib().oracle_model_create_bits(_p(blob), n_layers, int(weight_bits))
 
     def close(self):
         if self._h:

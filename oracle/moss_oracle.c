@@ -287,6 +287,7 @@ typedef struct {
 typedef struct oracle_model {
     int n_layers;
     int fp8;            /* q, k, v and fc1 on e4m3 operands */
+    int nvfp4;          /* q, k, v and fc1 on NVFP4 operands (sq.. hold the weight tensors' g) */
     float *conv_w_t[3]; /* [in][3][3][out] */
     const uint16_t *conv_b[3];
     int conv_in[3];
@@ -458,6 +459,133 @@ static uint16_t *take_linear_e4m3(const uint16_t *p, int out, int in, float **sc
     return t;
 }
 
+/* ------------------------------------------------ NVFP4 GEMM operands
+ *
+ * Page "Ossicle-4B", "Quantized: NVFP4 and INT4 in vLLM": the nvfp4 build
+ * quantises the weights and the activations of the audio encoder to NVFP4
+ * with NVIDIA ModelOpt and runs on Blackwell's native FP4 kernels.  Reading
+ * (the page names the format, no more): NVFP4 as ModelOpt defines it.
+ * Elements are E2M1 (1 sign, 2 exponent and 1 mantissa bit: 0, 0.5, 1, 1.5,
+ * 2, 3, 4, 6 and their negatives); each block of 16 consecutive elements
+ * along the contraction shares a positive E4M3 scale; one fp32 scale g
+ * covers a whole tensor, so that the block scales use E4M3's range:
+ *   g = fp32(amax) / 2688          (2688 = 6 x 448)
+ *   s_b = e4m3(fp32(amax_b) / (g * 6))
+ *   q = e2m1(x / (s_b * g))        (0 when s_b = 0; ties to even, +-6 saturates)
+ *   x' = q * s_b * g
+ * all in fp32.  Weights: one g per weight matrix.  Activations (the
+ * LayerNorm rows that feed q, k, v and fc1, the GEMMs the FP8 reading also
+ * takes): one g per row, so that a row's operands never depend on the other
+ * rows of a batch.  A GEMM is then
+ *   out[m][n] = (sum_k (q_a s_a)[m][k] (q_w s_w)[n][k]) * g_a[m] * g_w + b[n]
+ * where every product q s (at most 7 significant bits) is exact in bf16. */
+
+/* fp32 -> the nearest E2M1 value (ties to even), saturating at +-6. */
+float oracle_e2m1(float x)
+{
+    if (x != x) return x;
+    static const float grid[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    const float a = fabsf(x);
+    float r = 6.0f;
+    for (int i = 0; i < 7; i++) {
+        const float mid = 0.5f * (grid[i] + grid[i + 1]);  /* exact */
+        if (a < mid || (a == mid && (i % 2) == 0)) {  /* grid[i] has an even code when i is even */
+            r = grid[i];
+            break;
+        }
+        if (a == mid) {  /* the tie goes up to the even code */
+            r = grid[i + 1];
+            break;
+        }
+    }
+    return x < 0.0f ? -r : r;
+}
+
+/* NVFP4 quantisation of x [rows][cols] (cols a multiple of 16).  With
+ * per_row, one g per row (g[rows]), else one g for the whole matrix (g[0]).
+ * unit[r][k] receives q * s_b (the operand the tensor cores multiply, before
+ * g), codes[r][k] the E2M1 code (sign bit 3, magnitude index 0..7),
+ * bscale[r][k / 16] the block scales; codes and bscale may be NULL. */
+void oracle_quant_nvfp4(const float *x, int64_t rows, int cols, int per_row, float *unit, float *g,
+                        uint8_t *codes, float *bscale)
+{
+    float gt = 0.0f;
+    if (!per_row) {
+        float amax = 0.0f;
+        for (int64_t i = 0; i < rows * (int64_t)cols; i++) {
+            const float a = fabsf(x[i]);
+            if (a > amax) amax = a;
+        }
+        gt = amax / 2688.0f;
+        g[0] = gt;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        const float *xr = x + r * cols;
+        float gr = gt;
+        if (per_row) {
+            float amax = 0.0f;
+            for (int k = 0; k < cols; k++) {
+                const float a = fabsf(xr[k]);
+                if (a > amax) amax = a;
+            }
+            gr = amax / 2688.0f;
+            g[r] = gr;
+        }
+        for (int b0 = 0; b0 < cols; b0 += 16) {
+            float bmax = 0.0f;
+            for (int k = b0; k < b0 + 16; k++) {
+                const float a = fabsf(xr[k]);
+                if (a > bmax) bmax = a;
+            }
+            const float sb = gr > 0.0f ? oracle_e4m3(bmax / (gr * 6.0f)) : 0.0f;
+            if (bscale) bscale[r * (cols / 16) + b0 / 16] = sb;
+            const float sg = sb * gr;
+            for (int k = b0; k < b0 + 16; k++) {
+                const float q = sb > 0.0f ? oracle_e2m1(xr[k] / sg) : 0.0f;
+                unit[r * cols + k] = q * sb;
+                if (codes) {
+                    static const float grid[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+                    int idx = 0;
+                    while (grid[idx] != fabsf(q)) idx++;
+                    codes[r * cols + k] = (uint8_t)(idx | (q < 0.0f || (q == 0.0f && signbit(q)) ? 8 : 0));
+                }
+            }
+        }
+    }
+}
+
+/* The blob's [out][in] matrix at p as NVFP4 units q * s_b (bf16 bits, exact),
+ * transposed; *g receives the matrix's g repeated out times (malloc'd), the
+ * per-column factor of linear_e4m3. */
+static uint16_t *take_linear_nvfp4(const uint16_t *p, int out, int in, float **g)
+{
+    float *x = (float *)malloc(sizeof(float) * (size_t)out * in);
+    float *u = (float *)malloc(sizeof(float) * (size_t)out * in);
+    for (size_t i = 0; i < (size_t)out * in; i++) x[i] = bff(p[i]);
+    float gw = 0.0f;
+    oracle_quant_nvfp4(x, out, in, 0, u, &gw, NULL, NULL);
+    uint16_t *q = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)out * in);
+    for (size_t i = 0; i < (size_t)out * in; i++) q[i] = bf16_rne(u[i]);
+    uint16_t *t = transpose_bf16(q, out, in);
+    *g = (float *)malloc(sizeof(float) * out);
+    for (int n = 0; n < out; n++) (*g)[n] = gw;
+    free(x); free(u); free(q);
+    return t;
+}
+
+/* Activation rows y [M][K] in place -> NVFP4 units q * s_b, g[M] per row. */
+static void quant_nvfp4_act(float *y, int64_t M, int K, float *g)
+{
+    float *u = (float *)malloc(sizeof(float) * (size_t)M * K);
+    oracle_quant_nvfp4(y, M, K, 1, u, g, NULL, NULL);
+    memcpy(y, u, sizeof(float) * (size_t)M * K);
+    free(u);
+}
+
+/* weight_bits value of the NVFP4 model (oracle_model_create_nvfp4) */
+#define NVFP4_BITS 0x4f4
+
 /* Walks the blob in its documented order (conv1, conv2, conv3, conv_out,
  * layers, ln_post, proj1, proj2, adapter gate/up/down; each weight followed
  * by its bias, none for conv_out).  weight_bits 4 gives the 4-bit model of
@@ -469,6 +597,7 @@ oracle_model *oracle_model_create_bits(const uint16_t *blob, int n_layers, int w
     const uint16_t *p = blob;
     m->n_layers = n_layers;
     m->fp8 = weight_bits == 8;
+    m->nvfp4 = weight_bits == NVFP4_BITS;
     int cin[3] = {1, C_STEM, C_STEM};
     for (int c = 0; c < 3; c++) {
         m->conv_in[c] = cin[c];
@@ -491,14 +620,17 @@ oracle_model *oracle_model_create_bits(const uint16_t *blob, int n_layers, int w
         L->ln1_g = p; p += D;
         L->ln1_b = p; p += D;
         if (weight_bits == 8) L->wq_t = take_linear_e4m3(p, D, D, &L->sq);
+        else if (weight_bits == NVFP4_BITS) L->wq_t = take_linear_nvfp4(p, D, D, &L->sq);
         else L->wq_t = take_linear(p, D, D, weight_bits);
         p += (size_t)D * D;
         L->bq = p; p += D;
         if (weight_bits == 8) L->wk_t = take_linear_e4m3(p, D, D, &L->sk);
+        else if (weight_bits == NVFP4_BITS) L->wk_t = take_linear_nvfp4(p, D, D, &L->sk);
         else L->wk_t = take_linear(p, D, D, weight_bits);
         p += (size_t)D * D;
         L->bk = p; p += D;
         if (weight_bits == 8) L->wv_t = take_linear_e4m3(p, D, D, &L->sv);
+        else if (weight_bits == NVFP4_BITS) L->wv_t = take_linear_nvfp4(p, D, D, &L->sv);
         else L->wv_t = take_linear(p, D, D, weight_bits);
         p += (size_t)D * D;
         L->bv = p; p += D;
@@ -507,6 +639,7 @@ oracle_model *oracle_model_create_bits(const uint16_t *blob, int n_layers, int w
         L->ln2_g = p; p += D;
         L->ln2_b = p; p += D;
         if (weight_bits == 8) L->w1_t = take_linear_e4m3(p, D_FFN, D, &L->s1);
+        else if (weight_bits == NVFP4_BITS) L->w1_t = take_linear_nvfp4(p, D_FFN, D, &L->s1);
         else L->w1_t = take_linear(p, D_FFN, D, weight_bits);
         p += (size_t)D_FFN * D;
         L->b1 = p; p += D_FFN;
@@ -526,6 +659,11 @@ oracle_model *oracle_model_create_bits(const uint16_t *blob, int n_layers, int w
     m->wd_t = take_linear(p, D_OUT, D_ADP, weight_bits); p += (size_t)D_OUT * D_ADP;
     m->bd = p; p += D_OUT;
     return m;
+}
+
+oracle_model *oracle_model_create_nvfp4(const uint16_t *blob, int n_layers)
+{
+    return oracle_model_create_bits(blob, n_layers, NVFP4_BITS);
 }
 
 oracle_model *oracle_model_create(const uint16_t *blob, int n_layers)
@@ -795,7 +933,12 @@ int oracle_layers(const oracle_model *m, float *x, int T, const int *win, int n_
     for (int l = l0; l < l1; l++) {
         const layer_w *L = &m->layers[l];
         layernorm(x, T, D, L->ln1_g, L->ln1_b, h);
-        if (m->fp8) {
+        if (m->nvfp4) {
+            quant_nvfp4_act(h, T, D, sa);
+            linear_e4m3(h, T, D, L->wq_t, sa, L->sq, L->bq, D, q);
+            linear_e4m3(h, T, D, L->wk_t, sa, L->sk, L->bk, D, k);
+            linear_e4m3(h, T, D, L->wv_t, sa, L->sv, L->bv, D, v);
+        } else if (m->fp8) {
             quant_e4m3_act(h, T, D, sa);
             linear_e4m3(h, T, D, L->wq_t, sa, L->sq, L->bq, D, q);
             linear_e4m3(h, T, D, L->wk_t, sa, L->sk, L->bk, D, k);
@@ -812,7 +955,10 @@ int oracle_layers(const oracle_model *m, float *x, int T, const int *win, int n_
         linear(a, T, D, L->wo_t, L->bo, D, h);
         for (size_t i = 0; i < td; i++) x[i] = (float)((double)x[i] + h[i]);
         layernorm(x, T, D, L->ln2_g, L->ln2_b, h);
-        if (m->fp8) {
+        if (m->nvfp4) {
+            quant_nvfp4_act(h, T, D, sa);
+            linear_e4m3(h, T, D, L->w1_t, sa, L->s1, L->b1, D_FFN, f);
+        } else if (m->fp8) {
             quant_e4m3_act(h, T, D, sa);
             linear_e4m3(h, T, D, L->w1_t, sa, L->s1, L->b1, D_FFN, f);
         } else {

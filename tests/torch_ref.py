@@ -61,9 +61,42 @@ class TorchRef:
         w8, sw = self.e4m3_rows(w)
         return (a8 @ w8.T) * sa[:, None] * sw[None, :] + b
 
-    def layers(self, x: torch.Tensor, windows, l0=0, l1=None, fp8=False) -> torch.Tensor:
+    # E2M1 values with the even codes first, so that argmin settles a tie on
+    # the even neighbour
+    E2M1_EVEN_FIRST = torch.tensor([0.0, 1.0, 2.0, 4.0, 0.5, 1.5, 3.0, 6.0], dtype=torch.float32)
+
+    @classmethod
+    def nvfp4_rows(cls, x64: torch.Tensor, per_row: bool):
+        """NVFP4 operands of x (fp32 values): g = amax / 2688 per row or per
+        tensor, block scales of 16 by torch's float8_e4m3fn conversion, E2M1
+        values by nearest-on-the-grid (ties to the even code, +-6 saturates).
+        Returns (q * s_b as fp64, g as fp64 [rows] or scalar)."""
+        x = x64.to(torch.float32)
+        rows, cols = x.shape
+        amax = x.abs().amax(dim=1) if per_row else x.abs().amax().expand(rows)
+        g = amax / 2688.0
+        xb = x.view(rows, cols // 16, 16)
+        bmax = xb.abs().amax(dim=2)
+        safe_g = torch.where(g > 0, g, torch.ones_like(g))
+        sb = (bmax / (safe_g[:, None] * 6.0)).clamp(max=448.0).to(torch.float8_e4m3fn).to(torch.float32)
+        sb = torch.where(g[:, None] > 0, sb, torch.zeros_like(sb))
+        sg = sb * g[:, None]
+        y = xb / torch.where(sg > 0, sg, torch.ones_like(sg))[:, :, None]
+        d = (y.abs()[..., None] - cls.E2M1_EVEN_FIRST).abs()
+        q = cls.E2M1_EVEN_FIRST[d.argmin(dim=-1)] * torch.sign(y)
+        q = torch.where(sg[:, :, None] > 0, q, torch.zeros_like(q))
+        unit = (q * sb[:, :, None]).view(rows, cols)
+        return unit.to(torch.float64), g.to(torch.float64)
+
+    def linear_nvfp4(self, h: torch.Tensor, w: torch.Tensor, b: torch.Tensor) -> torch.Tensor:
+        ua, ga = self.nvfp4_rows(h, per_row=True)
+        uw, gw = self.nvfp4_rows(w, per_row=False)
+        return (ua @ uw.T) * ga[:, None] * gw[0] + b
+
+    def layers(self, x: torch.Tensor, windows, l0=0, l1=None, fp8=False, nvfp4=False) -> torch.Tensor:
         W = self.w
-        lin = self.linear_e4m3 if fp8 else (lambda h, w, b: F.linear(h, w, b))
+        lin = (self.linear_nvfp4 if nvfp4 else self.linear_e4m3 if fp8
+               else (lambda h, w, b: F.linear(h, w, b)))
         T = x.shape[0]
         wid = torch.empty(T, dtype=torch.long)
         for i in range(len(windows) - 1):
