@@ -29,7 +29,8 @@ EXPORTED = [
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
     "moss_enc_tap_weight_count", "moss_enc_set_taps", "moss_enc_forward_taps",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
-    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_gemm_q4", "moss_enc_gemm_f8", "moss_enc_selftest_gelu",
+    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_gemm_q4", "moss_enc_gemm_f8", "moss_enc_gemm_nvf4",
+    "moss_enc_selftest_gelu",
     "moss_enc_selftest_timeout",
 ]
 WEIGHTS_4BIT = 4
@@ -125,6 +126,8 @@ def lib():
         L.moss_enc_gemm_q4.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32]
         L.moss_enc_gemm_f8.restype = i32
         L.moss_enc_gemm_f8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32]
+        L.moss_enc_gemm_nvf4.restype = i32
+        L.moss_enc_gemm_nvf4.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32]
         L.moss_enc_logmel_static.restype = i32
         L.moss_enc_logmel_static.argtypes = [ctypes.POINTER(Clip), i32, ctypes.POINTER(vp), vp, vp]
         _lib = L
@@ -244,6 +247,16 @@ class Encoder:
         N = B8.shape[0]
         self._check(lib().moss_enc_gemm_f8(self.h, _ptr(A8), _ptr(B8), _ptr(sa), _ptr(sb), _ptr(bias), _ptr(out),
                                            M, N, K, int(epilogue), int(block_n)))
+        return out
+
+    def gemm_nvf4(self, A4, sfa, ga, B4, sfb, gb, bias, out, epilogue: int):
+        """out = epi((a @ b.T) * ga[:, None] * gb[None, :] + bias) on NVFP4
+        operands: A4 [M][K/2], B4 [N][K/2] packed E2M1 codes (uint8), sfa, sfb
+        their E4M3 block-scale atoms (uint8), ga [M], gb [N] fp32."""
+        M, K2 = A4.shape
+        N = B4.shape[0]
+        self._check(lib().moss_enc_gemm_nvf4(self.h, _ptr(A4), _ptr(sfa), _ptr(ga), _ptr(B4), _ptr(sfb), _ptr(gb),
+                                             _ptr(bias), _ptr(out), M, N, 2 * K2, int(epilogue)))
         return out
 
     def selftest_timeout(self, limit_ms: int = 50):

@@ -56,6 +56,8 @@ struct GemmArgs {
     int kq_blocks;
     // e4m3 operands only: out = acc * row_scale[m] * col_scale[n] + bias ...
     const float *row_scale, *col_scale;
+    // NVFP4 operands only (fp4.cuh): the block-scale atoms of A and B
+    const uint8_t *sfa, *sfb;
 };
 
 // Each epilogue warp stages 32 rows x 128 B in shared memory (16-byte

@@ -23,6 +23,7 @@
 #include "mel.cuh"
 #include "norm.cuh"
 #include "stem.cuh"
+#include "fp4.cuh"
 
 using namespace moss;
 
@@ -438,6 +439,47 @@ static moss_enc_status gemm2f8(moss_enc *h, const char *name, const uint8_t *A8,
     return MOSS_ENC_OK;
 }
 
+// The NVFP4 GEMM (fp4.cuh): A4 [M][K/2] and B4 [N][K/2] E2M1 bytes, their
+// block-scale atoms a.sfa and a.sfb, row factors a.row_scale [M] (g of each
+// activation row) and column factors a.col_scale [N] (the weight's g);
+// bf16 outputs.  128 x 128 tiles, 256 k per stage.
+template <int EPI>
+static moss_enc_status gemm_nvf4(moss_enc *h, const char *name, const uint8_t *A4, int64_t M, int K, const uint8_t *B4,
+                                 int N, GemmArgs a)
+{
+    using C = Fp4Cfg<128>;
+    if (M <= 0) return MOSS_ENC_OK;
+    if (K % 256 != 0 || N % 128 != 0 || M > INT32_MAX || !a.row_scale || !a.col_scale || !a.sfa || !a.sfb)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "gemm shape not supported");
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return fail(h, MOSS_ENC_ERR_CUDA, "no tensor-map encoder");
+    CUtensorMap ta, tb;
+    auto map4 = [&](CUtensorMap *m, const uint8_t *p, uint64_t rows) {
+        cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)rows};
+        cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+        cuuint32_t box[2] = {128, 128};
+        cuuint32_t es[2] = {1, 1};
+        return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(p), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    if (!map4(&ta, A4, (uint64_t)M) || !map4(&tb, B4, (uint64_t)N))
+        return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (fp4)");
+    a.M = (int)M;
+    a.N = N;
+    a.K = K;
+    a.m_tiles = (int)((M + 127) / 128);
+    a.n_tiles = N / 128;
+    a.err = h->err;
+    CUtensorMap tc;
+    if (!tmap_out<128, EPI>(&tc, a, tb)) return fail(h, MOSS_ENC_ERR_CUDA, "cuTensorMapEncodeTiled failed (output)");
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int grid = std::min(tiles, h->num_sms);
+    Launch L(h, name, 2.0 * M * N * K, 0.5 * M * K + 0.5 * N * K + (M + N) * K / 16.0 + epi_out_bytes(EPI) * M * N);
+    CUDA_TRY(h, launch_k(h, gemm_nvf4_kernel<128, EPI>, dim3(grid), dim3(C::THREADS), C::SMEM, ta, tb, tc, a));
+    return MOSS_ENC_OK;
+}
+
 template <int BN, int EPI>
 static cudaError_t gemm2f8_attr()
 {
@@ -850,6 +892,10 @@ static moss_enc_status set_kernel_attrs(moss_enc *h)
     CUDA_TRY(h, (gemm2_attr<160, EPI_RESID_F32>()));
     CUDA_TRY(h, (gemm2_attr<128, EPI_F32>()));
     CUDA_TRY(h, (gemm2f8_attr<128, EPI_BF16>()));
+    CUDA_TRY(h, cudaFuncSetAttribute(gemm_nvf4_kernel<128, EPI_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)Fp4Cfg<128>::SMEM));
+    CUDA_TRY(h, cudaFuncSetAttribute(gemm_nvf4_kernel<128, EPI_GELU_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)Fp4Cfg<128>::SMEM));
     CUDA_TRY(h, (gemm2f8_attr<256, EPI_BF16>()));
     CUDA_TRY(h, (gemm2f8_attr<128, EPI_GELU_BF16>()));
     CUDA_TRY(h, (gemm2f8_attr<256, EPI_GELU_BF16>()));
@@ -2329,6 +2375,33 @@ extern "C" moss_enc_status moss_enc_gemm_f8(moss_enc *h, const void *A8, const v
     case EPI_BF16 * 2 + 1: return gemm2f8<256, EPI_BF16>(h, "gemm_api", a8, M, K, b8, N, a);
     case EPI_GELU_BF16 * 2: return gemm2f8<128, EPI_GELU_BF16>(h, "gemm_api", a8, M, K, b8, N, a);
     case EPI_GELU_BF16 * 2 + 1: return gemm2f8<256, EPI_GELU_BF16>(h, "gemm_api", a8, M, K, b8, N, a);
+    default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "epilogue must be 0 or 1");
+    }
+}
+
+extern "C" moss_enc_status moss_enc_gemm_nvf4(moss_enc *h, const void *A4, const void *sfa, const float *ga,
+                                              const void *B4, const void *sfb, const float *gb, const float *bias,
+                                              void *out, int M, int N, int K, int epilogue)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (!A4 || !sfa || !ga || !B4 || !sfb || !gb || !bias || !out || M < 0 || N <= 0 || K <= 0 || K % 256 != 0 ||
+        N % 128 != 0)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad gemm arguments");
+    if ((reinterpret_cast<uintptr_t>(A4) | reinterpret_cast<uintptr_t>(B4) | reinterpret_cast<uintptr_t>(sfa) |
+         reinterpret_cast<uintptr_t>(sfb)) & 15)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A4, B4 and the scale atoms must be 16-byte aligned");
+    GemmArgs a{};
+    a.bias = bias;
+    a.out = out;
+    a.ldo = N;
+    a.row_scale = ga;
+    a.col_scale = gb;
+    a.sfa = static_cast<const uint8_t *>(sfa);
+    a.sfb = static_cast<const uint8_t *>(sfb);
+    const uint8_t *a4 = static_cast<const uint8_t *>(A4), *b4 = static_cast<const uint8_t *>(B4);
+    switch (epilogue) {
+    case EPI_BF16: return gemm_nvf4<EPI_BF16>(h, "gemm_api", a4, M, K, b4, N, a);
+    case EPI_GELU_BF16: return gemm_nvf4<EPI_GELU_BF16>(h, "gemm_api", a4, M, K, b4, N, a);
     default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "epilogue must be 0 or 1");
     }
 }

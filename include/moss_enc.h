@@ -334,6 +334,24 @@ moss_enc_status moss_enc_gemm_q4(moss_enc *h, const void *A, const void *Bq, con
 moss_enc_status moss_enc_gemm_f8(moss_enc *h, const void *A8, const void *B8, const float *sa, const float *sb,
                                  const float *bias, void *out, int M, int N, int K, int epilogue, int block_n);
 
+/* The same GEMM on NVFP4 operands (page "Ossicle-4B", section "Quantized:
+ * NVFP4 and INT4 in vLLM"):
+ *  A4, B4     device uint8 [M][K/2], [N][K/2]: E2M1 codes (sign bit 3,
+ *             magnitude index 0..7 of 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per
+ *             byte, the even k in the low nibble;
+ *  sfa, sfb   device uint8: the E4M3 scale of every 16 k of every row, in
+ *             512-byte atoms of 128 rows x 64 k ordered [rows/128][K/64]
+ *             (rows padded to a multiple of 128), row r of an atom at byte
+ *             (r % 32) * 16 + (r / 32) * 4 + (k % 64) / 16;
+ *  ga [M], gb [N] device fp32 factors (a row's and the weight's g);
+ *   out[m][n] = epi((sum_k a[m][k] b[n][k]) * ga[m] * gb[n] + bias[n]),
+ * a and b the E2M1 values times their block scales.  epilogue 0 (bf16 out)
+ * or 1 (GELU, bf16 out); 128 x 128 tiles on one CTA each; K % 256 == 0,
+ * N % 128 == 0; all four operand pointers 16-byte aligned. */
+moss_enc_status moss_enc_gemm_nvf4(moss_enc *h, const void *A4, const void *sfa, const float *ga, const void *B4,
+                                   const void *sfb, const float *gb, const float *bias, void *out, int M, int N,
+                                   int K, int epilogue);
+
 /* The GEMM epilogues and conv1 evaluate GELU's erf with a short rational
  * approximation (Abramowitz & Stegun 7.1.28, error <= 3e-7), one value at a
  * time and in pairs (paired fp32 instructions).  This runs both forms
