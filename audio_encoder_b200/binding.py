@@ -29,7 +29,7 @@ EXPORTED = [
     "moss_enc_forward", "moss_enc_forward_stage", "moss_enc_forward_host",
     "moss_enc_tap_weight_count", "moss_enc_set_taps", "moss_enc_forward_taps",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
-    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_gemm_q4", "moss_enc_gemm_f8", "moss_enc_gemm_nvf4",
+    "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_gemm_q4", "moss_enc_gemm_f8", "moss_enc_gemm_nvf4", "moss_enc_nvf4_quant_rows",
     "moss_enc_selftest_gelu",
     "moss_enc_selftest_timeout",
 ]
@@ -46,7 +46,7 @@ class MossEncError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int), ("max_samples", ctypes.c_int64),
                 ("max_clips", ctypes.c_int), ("out_dtype", ctypes.c_int), ("weight_bits", ctypes.c_int),
-                ("fp8", ctypes.c_int)]
+                ("fp8", ctypes.c_int), ("nvfp4", ctypes.c_int)]
 
 
 class KernelStat(ctypes.Structure):
@@ -128,6 +128,8 @@ def lib():
         L.moss_enc_gemm_f8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32]
         L.moss_enc_gemm_nvf4.restype = i32
         L.moss_enc_gemm_nvf4.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32]
+        L.moss_enc_nvf4_quant_rows.restype = i32
+        L.moss_enc_nvf4_quant_rows.argtypes = [vp, vp, vp, vp, vp, i32]
         L.moss_enc_logmel_static.restype = i32
         L.moss_enc_logmel_static.argtypes = [ctypes.POINTER(Clip), i32, ctypes.POINTER(vp), vp, vp]
         _lib = L
@@ -166,12 +168,14 @@ class Encoder:
     """
 
     def __init__(self, blob, n_layers: int, max_samples: int, max_clips: int = 1,
-                 out_dtype: int = OUT_F32, stream=None, weight_bits: int = 16, fp8: bool = False):
+                 out_dtype: int = OUT_F32, stream=None, weight_bits: int = 16, fp8: bool = False,
+                 nvfp4: bool = False):
         import torch
         self.torch = torch
         self.n_layers = n_layers
         self.out_dtype = out_dtype
-        cfg = Config(n_layers, int(max_samples), int(max_clips), int(out_dtype), int(weight_bits), int(bool(fp8)))
+        cfg = Config(n_layers, int(max_samples), int(max_clips), int(out_dtype), int(weight_bits), int(bool(fp8)),
+                     int(bool(nvfp4)))
         if stream is None:
             stream = torch.cuda.current_stream()
         self.stream = stream
@@ -258,6 +262,10 @@ class Encoder:
         self._check(lib().moss_enc_gemm_nvf4(self.h, _ptr(A4), _ptr(sfa), _ptr(ga), _ptr(B4), _ptr(sfb), _ptr(gb),
                                              _ptr(bias), _ptr(out), M, N, 2 * K2, int(epilogue)))
         return out
+
+    def nvf4_quant_rows(self, x, codes, sfa, g):
+        """NVFP4 codes, scale atoms and per-row g of fp32 rows x [M][1280]."""
+        self._check(lib().moss_enc_nvf4_quant_rows(self.h, _ptr(x), _ptr(codes), _ptr(sfa), _ptr(g), x.shape[0]))
 
     def selftest_timeout(self, limit_ms: int = 50):
         self._check(lib().moss_enc_selftest_timeout(self.h, int(limit_ms)))

@@ -249,3 +249,98 @@ __global__ void __launch_bounds__(Fp4Cfg<BN>::THREADS, 1)
 }
 
 }  // namespace moss
+
+namespace moss {
+
+// fp32 pair -> two E2M1 codes in one byte, round to nearest even with
+// saturation at +-6 (the value of `lo` in the low nibble).
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+// NVFP4 activation rows of 1280 (the operands of the q/k/v and fc1 GEMMs):
+// with LN, the LayerNorm of the residual-stream row first (the same
+// arithmetic as layernorm1280_kernel), else the row as given.  Then, per row,
+// g = amax / 2688, per block of 16 s_b = e4m3(amax_b / (g * 6)) and the
+// codes e2m1(x / (s_b * g)) (0 when s_b = 0), all in fp32: codes [rows][640]
+// bytes, scale atoms [rows / 128][20][512] bytes (the GEMM's layout), g
+// [rows].  One warp per row; lane l holds columns 128 i + 4 l .. + 3, so a
+// block of 16 is four neighbouring lanes.
+template <bool LN>
+__global__ void __launch_bounds__(256) nvf4_rows1280_kernel(const float *__restrict__ x, const float *__restrict__ gamma,
+                                                           const float *__restrict__ beta, uint8_t *__restrict__ codes,
+                                                           uint8_t *__restrict__ atoms, float *__restrict__ g_out,
+                                                           int rows)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)row * 1280);
+    float4 v[10];
+#pragma unroll
+    for (int i = 0; i < 10; i++) v[i] = xr[lane + 32 * i];
+    if (LN) {
+        float s = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 10; i++) s += v[i].x + v[i].y + v[i].z + v[i].w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        const float mean = s * (1.0f / 1280.0f);
+        float q = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 10; i++) {
+            const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+            q += a * a + b * b + c * c + d * d;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+        const float rstd = rsqrtf(q * (1.0f / 1280.0f) + 1e-5f);
+        const float4 *g4 = reinterpret_cast<const float4 *>(gamma);
+        const float4 *b4 = reinterpret_cast<const float4 *>(beta);
+#pragma unroll
+        for (int i = 0; i < 10; i++) {
+            const float4 g = g4[lane + 32 * i], b = b4[lane + 32 * i];
+            v[i].x = (v[i].x - mean) * rstd * g.x + b.x;
+            v[i].y = (v[i].y - mean) * rstd * g.y + b.y;
+            v[i].z = (v[i].z - mean) * rstd * g.z + b.z;
+            v[i].w = (v[i].w - mean) * rstd * g.w + b.w;
+        }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 10; i++)
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float g = amax / 2688.0f;
+    if (lane == 0) g_out[row] = g;
+    uint16_t *crow = reinterpret_cast<uint16_t *>(codes + (size_t)row * 640);
+    uint8_t *arow = atoms + (size_t)(row >> 7) * 20 * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4;
+#pragma unroll
+    for (int i = 0; i < 10; i++) {
+        float bmax = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
+        const __nv_fp8_storage_t sc = g > 0.0f ? __nv_cvt_float_to_fp8(bmax / (g * 6.0f), __NV_SATFINITE, __NV_E4M3)
+                                               : (__nv_fp8_storage_t)0;
+        const float sb = __half2float(__half(__nv_cvt_fp8_to_halfraw(sc, __NV_E4M3)));
+        const float sg = sb * g;
+        uint32_t c = 0;
+        if (sb > 0.0f)
+            c = e2m1x2(v[i].x / sg, v[i].y / sg) | (e2m1x2(v[i].z / sg, v[i].w / sg) << 8);
+        crow[64 * i / 2 + lane] = (uint16_t)c;  // columns 128 i + 4 l .. + 3: bytes 64 i + 2 l, + 1
+        const int b = 8 * i + (lane >> 2);       // block of 16 along the row
+        if ((lane & 3) == 0) arow[(b >> 2) * 512 + (b & 3)] = (uint8_t)sc;
+    }
+}
+
+}  // namespace moss

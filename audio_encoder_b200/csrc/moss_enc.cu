@@ -53,6 +53,9 @@ struct LayerDev {
     // FP8 handles: q/k/v and fc1 as e4m3 [N][K] with per-channel scales [N]
     const uint8_t *wqkv8 = nullptr, *w18 = nullptr;
     const float *sqkv = nullptr, *s1 = nullptr;
+    // NVFP4 handles: q/k/v and fc1 codes, scale atoms and per-column g
+    const uint8_t *wqkv4 = nullptr, *sqkv4 = nullptr, *w14 = nullptr, *s14 = nullptr;
+    const float *gqkv4 = nullptr, *g14 = nullptr;
 };
 
 // ln_post, proj1, proj2 and the SwiGLU adapter: the encoder's own set, and
@@ -79,7 +82,8 @@ struct moss_enc {
     // weights (one allocation; 4-bit handles keep the linear layers' codes
     // and scales in a second one)
     void *wmem = nullptr, *qmem = nullptr;
-    bool q4 = false, fp8 = false;
+    bool q4 = false, fp8 = false, nvfp4 = false;
+    uint8_t *sfa4 = nullptr;  // NVFP4 handles: the activation rows' scale atoms
     const uint4 *conv1_wt = nullptr;  // conv1 as the B operand of its GEMM (see conv1_tc_kernel)
     float *conv2_b = nullptr, *conv3_b = nullptr;
     bf16 *conv2_w = nullptr, *conv3_w = nullptr, *conv_out_w = nullptr;
@@ -960,6 +964,62 @@ static void quantise_e4m3_rows(uint8_t *mat, int n, int k)
     std::memcpy(mat + f8_scale_off(n, k), sc.data(), sizeof(float) * n);
 }
 
+// NVFP4 quantisation of a bf16 matrix [n][k] in place (n a multiple of 128,
+// k of 64), in `parts` equal row ranges with a g each (the q, k and v
+// weights of the fused QKV matrix keep their own): g = fp32(amax) / 2688,
+// s_b = e4m3(fp32(amax_b) / (g * 6)) per 16 k, code = e2m1(w / (s_b * g))
+// (0 when s_b = 0; fp32 arithmetic, ties to even).  Written over the
+// matrix: codes [n][k/2] (even k in the low nibble) from its start, the
+// scale atoms [n/128][k/64][512] at nvf4_sf_off, g per row at nvf4_g_off.
+static size_t nvf4_sf_off(int n, int k) { return ((size_t)n * k / 2 + 255) & ~size_t(255); }
+static size_t nvf4_g_off(int n, int k) { return (nvf4_sf_off(n, k) + (size_t)n * k / 16 + 255) & ~size_t(255); }
+
+// E2M1 code (sign bit 3, magnitude index 0..7 of 0, .5, 1, 1.5, 2, 3, 4, 6)
+// of the value nearest to x; a tie goes to the even index; |x| > 6 -> 6.
+static uint8_t host_e2m1(float x)
+{
+    static const float mid[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+    const float a = std::fabs(x);
+    int i = 0;
+    while (i < 7 && (a > mid[i] || (a == mid[i] && (i & 1)))) i++;
+    return (uint8_t)(i | (std::signbit(x) ? 8 : 0));
+}
+
+static void quantise_nvfp4(uint8_t *mat, int n, int k, int parts)
+{
+    const uint16_t *w = reinterpret_cast<const uint16_t *>(mat);
+    std::vector<uint8_t> codes((size_t)n * k / 2), atoms((size_t)n * k / 16);
+    std::vector<float> gr(n);
+    const int rows = n / parts;
+    for (int p = 0; p < parts; p++) {
+        float amax = 0.0f;
+        for (size_t i = (size_t)p * rows * k; i < (size_t)(p + 1) * rows * k; i++)
+            amax = std::max(amax, std::fabs(bf16_bits_to_float(w[i])));
+        const float g = amax / 2688.0f;
+        for (int r = p * rows; r < (p + 1) * rows; r++) {
+            gr[r] = g;
+            for (int b = 0; b < k / 16; b++) {
+                float bmax = 0.0f;
+                for (int i = 0; i < 16; i++) bmax = std::max(bmax, std::fabs(bf16_bits_to_float(w[(size_t)r * k + 16 * b + i])));
+                const __nv_fp8_storage_t sc = g > 0.0f ? __nv_cvt_float_to_fp8(bmax / (g * 6.0f), __NV_SATFINITE, __NV_E4M3)
+                                                       : (__nv_fp8_storage_t)0;
+                const float sb = __half2float(__half(__nv_cvt_fp8_to_halfraw(sc, __NV_E4M3)));
+                const float sg = sb * g;
+                atoms[((size_t)(r / 128) * (k / 64) + b / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + b % 4] = sc;
+                for (int i = 0; i < 16; i += 2) {
+                    const size_t e = (size_t)r * k + 16 * b + i;
+                    const uint8_t c0 = sb > 0.0f ? host_e2m1(bf16_bits_to_float(w[e]) / sg) : 0;
+                    const uint8_t c1 = sb > 0.0f ? host_e2m1(bf16_bits_to_float(w[e + 1]) / sg) : 0;
+                    codes[e / 2] = (uint8_t)(c0 | (c1 << 4));
+                }
+            }
+        }
+    }
+    std::memcpy(mat, codes.data(), codes.size());
+    std::memcpy(mat + nvf4_sf_off(n, k), atoms.data(), atoms.size());
+    std::memcpy(mat + nvf4_g_off(n, k), gr.data(), sizeof(float) * n);
+}
+
 // 4-bit round-to-nearest quantisation of one bf16 matrix [n][kq] (rows
 // `stride` elements apart) in groups of 128 along k: s = fp32(max |w|) / 7,
 // q = clamp(rint(w / s), -8, 7) (0 when s = 0), code q + 8.  Codes [n][kq/2]
@@ -1012,7 +1072,8 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     if (!cfg || !weights || cfg->n_layers < 1 || cfg->n_layers > 32 || cfg->max_samples < 1 ||
         cfg->max_clips < 1 || (cfg->out_dtype != MOSS_ENC_OUT_F32 && cfg->out_dtype != MOSS_ENC_OUT_BF16) ||
         (cfg->weight_bits != 0 && cfg->weight_bits != 16 && cfg->weight_bits != 4) ||
-        (cfg->fp8 != 0 && cfg->fp8 != 1) || (cfg->fp8 && cfg->weight_bits == 4))
+        (cfg->fp8 != 0 && cfg->fp8 != 1) || (cfg->fp8 && cfg->weight_bits == 4) ||
+        (cfg->nvfp4 != 0 && cfg->nvfp4 != 1) || (cfg->nvfp4 && (cfg->fp8 || cfg->weight_bits == 4)))
         return MOSS_ENC_ERR_INVALID_ARG;
     const int64_t count = moss_enc_weight_count(cfg->n_layers);
     if ((int64_t)bytes != count * 2) return MOSS_ENC_ERR_INVALID_ARG;
@@ -1222,6 +1283,18 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
             }
         for (auto &th : pool) th.join();
     }
+    // ---- NVFP4 handles: q/k/v (a g each) and fc1 as NVFP4 over their bf16 slots
+    h->nvfp4 = cfg->nvfp4 == 1;
+    if (h->nvfp4) {
+        std::vector<std::thread> pool;
+        for (int l = 0; l < L; l++)
+            for (int which = 0; which < 2; which++) {
+                const size_t o = lo[l * 12 + (which == 0 ? 4 : 8)];
+                const int n = which == 0 ? DQKV : DFF, parts = which == 0 ? 3 : 1;
+                pool.emplace_back([&pk, o, n, parts]() { quantise_nvfp4(pk.data() + o, n, D, parts); });
+            }
+        for (auto &th : pool) th.join();
+    }
     const size_t upload = h->q4 ? small_total : wtotal;
     if (cudaMalloc(&h->wmem, upload) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     if (cudaMemcpy(h->wmem, pk.data(), upload, cudaMemcpyHostToDevice) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
@@ -1262,6 +1335,15 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
         d.b1 = (float *)(W + L12[9]);
         d.w2 = big(L12[10]);
         d.b2 = (float *)(W + L12[11]);
+        if (h->nvfp4) {
+            d.wqkv = d.w1 = nullptr;
+            d.wqkv4 = W + L12[4];
+            d.sqkv4 = W + L12[4] + nvf4_sf_off(DQKV, D);
+            d.gqkv4 = (const float *)(W + L12[4] + nvf4_g_off(DQKV, D));
+            d.w14 = W + L12[8];
+            d.s14 = W + L12[8] + nvf4_sf_off(DFF, D);
+            d.g14 = (const float *)(W + L12[8] + nvf4_g_off(DFF, D));
+        }
         if (h->fp8) {
             d.wqkv = d.w1 = nullptr;
             d.wqkv8 = W + L12[4];
@@ -1316,6 +1398,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     // the adapter's interleaved gate/up, 16384 x 2048)
     const size_t w_qs = h->q4 ? take(2 * (size_t)2 * DADP * DOUT) : 0;
     const size_t w_rs = take(4 * (size_t)T);
+    const size_t w_sf4 = h->nvfp4 ? take((size_t)(T / 128 + 1) * 20 * 512) : 0;  // NVFP4 activation scale atoms
     if (cudaMalloc(&h->ws, off) != cudaSuccess) return bail(MOSS_ENC_ERR_OOM);
     uint8_t *S = static_cast<uint8_t *>(h->ws);
     h->mel_raw = (float *)(S + w_mel);
@@ -1336,6 +1419,7 @@ extern "C" moss_enc_status moss_enc_create(const moss_enc_config *cfg, const voi
     h->out_stage = (void *)(S + w_out);
     h->qscratch = h->q4 ? (bf16 *)(S + w_qs) : nullptr;
     h->row_scale = (float *)(S + w_rs);
+    h->sfa4 = h->nvfp4 ? S + w_sf4 : nullptr;
     if (cudaMemset(h->err, 0, 256) != cudaSuccess) return bail(MOSS_ENC_ERR_CUDA);
 
     const TabLayout tl = tab_layout(cfg->max_clips, h->max_chunks);
@@ -1816,8 +1900,12 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
             W1 = xs_1;
             W2 = xs_2;
         }
-        uint8_t *xn8 = reinterpret_cast<uint8_t *>(h->xn);  // FP8 handles: e4m3 LayerNorm rows
-        if (h->fp8) {
+        uint8_t *xn8 = reinterpret_cast<uint8_t *>(h->xn);  // FP8 / NVFP4 handles: the LayerNorm rows' codes
+        if (h->nvfp4) {
+            Launch Lk(h, "layernorm", 8.0 * T * D, 4.0 * T * D + 0.5 * T * D + T * D / 16.0);
+            CUDA_TRY(h, launch_k(h, nvf4_rows1280_kernel<true>, dim3(ln_grid), dim3(256), 0, (const float *)h->X,
+                                 L.ln1_g, L.ln1_b, xn8, h->sfa4, h->row_scale, (int)T));
+        } else if (h->fp8) {
             Launch Lk(h, "layernorm", 8.0 * T * D, 5.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_e4m3_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln1_g,
                                  L.ln1_b, xn8, h->row_scale, (int)T));
@@ -1830,7 +1918,15 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.bqkv;
         a.out = h->qkv;
         a.ldo = DQKV;
-        if (h->fp8) {
+        if (h->nvfp4) {
+            a.row_scale = h->row_scale;
+            a.col_scale = L.gqkv4;
+            a.sfa = h->sfa4;
+            a.sfb = L.sqkv4;
+            TRY((gemm_nvf4<EPI_BF16>(h, "gemm_qkv", xn8, T, D, L.wqkv4, DQKV, a)));
+            a.row_scale = a.col_scale = nullptr;
+            a.sfa = a.sfb = nullptr;
+        } else if (h->fp8) {
             a.row_scale = h->row_scale;
             a.col_scale = L.sqkv;
             if (T <= 512)
@@ -1853,7 +1949,11 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.out = h->X;
         a.ldo = D;
         TRY(resid_gemm("gemm_out", h->attn, D, Wo, L.qo, a));
-        if (h->fp8) {
+        if (h->nvfp4) {
+            Launch Lk(h, "layernorm", 8.0 * T * D, 4.0 * T * D + 0.5 * T * D + T * D / 16.0);
+            CUDA_TRY(h, launch_k(h, nvf4_rows1280_kernel<true>, dim3(ln_grid), dim3(256), 0, (const float *)h->X,
+                                 L.ln2_g, L.ln2_b, xn8, h->sfa4, h->row_scale, (int)T));
+        } else if (h->fp8) {
             Launch Lk(h, "layernorm", 8.0 * T * D, 5.0 * T * D);
             CUDA_TRY(h, launch_k(h, layernorm1280_e4m3_kernel, dim3(ln_grid), dim3(256), 0, (const float *)h->X, L.ln2_g,
                                  L.ln2_b, xn8, h->row_scale, (int)T));
@@ -1865,7 +1965,15 @@ static moss_enc_status forward_launch(moss_enc *h, const FwdPlan &P, uint8_t *Dt
         a.bias = L.b1;
         a.out = h->ffn;
         a.ldo = DFF;
-        if (h->fp8) {
+        if (h->nvfp4) {
+            a.row_scale = h->row_scale;
+            a.col_scale = L.g14;
+            a.sfa = h->sfa4;
+            a.sfb = L.s14;
+            TRY((gemm_nvf4<EPI_GELU_BF16>(h, "gemm_fc1", xn8, T, D, L.w14, DFF, a)));
+            a.row_scale = a.col_scale = nullptr;
+            a.sfa = a.sfb = nullptr;
+        } else if (h->fp8) {
             a.row_scale = h->row_scale;
             a.col_scale = L.s1;
             TRY((gemm2f8<256, EPI_GELU_BF16>(h, "gemm_fc1", xn8, T, D, L.w18, DFF, a)));
@@ -2404,6 +2512,20 @@ extern "C" moss_enc_status moss_enc_gemm_nvf4(moss_enc *h, const void *A4, const
     case EPI_GELU_BF16: return gemm_nvf4<EPI_GELU_BF16>(h, "gemm_api", a4, M, K, b4, N, a);
     default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "epilogue must be 0 or 1");
     }
+}
+
+extern "C" moss_enc_status moss_enc_nvf4_quant_rows(moss_enc *h, const float *x, void *codes, void *sfa, float *g,
+                                                    int M)
+{
+    if (!h) return MOSS_ENC_ERR_INVALID_ARG;
+    if (M < 0 || (M > 0 && (!x || !codes || !sfa || !g)))
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad quantisation arguments");
+    if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(codes) & 1))
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "x must be 16-byte and codes 2-byte aligned");
+    if (M == 0) return MOSS_ENC_OK;
+    CUDA_TRY(h, launch_k(h, nvf4_rows1280_kernel<false>, dim3((M + 7) / 8), dim3(256), 0, x, (const float *)nullptr,
+                         (const float *)nullptr, static_cast<uint8_t *>(codes), static_cast<uint8_t *>(sfa), g, M));
+    return MOSS_ENC_OK;
 }
 
 // --------------------------------------------------------- GELU self-test

@@ -540,7 +540,7 @@ def run_streamed(args):
         dist.destroy_process_group()
 
 
-def measure_plain(workload, steps, warmup, dev, weight_bits=16, fp8=False):
+def measure_plain(workload, steps, warmup, dev, weight_bits=16, fp8=False, nvfp4=False):
     """One workload's forward timed as the headline is (device-resident PCM,
     CUDA events on the encoder's stream, L2 flushed between steps)."""
     import torch
@@ -551,7 +551,7 @@ def measure_plain(workload, steps, warmup, dev, weight_bits=16, fp8=False):
     stream = torch.cuda.Stream()
     total = sum(c.size for c in clips)
     enc = binding.Encoder(synth.make_weights(n_layers), n_layers, max_samples=total, max_clips=len(clips),
-                          out_dtype=binding.OUT_BF16, stream=stream, weight_bits=weight_bits, fp8=fp8)
+                          out_dtype=binding.OUT_BF16, stream=stream, weight_bits=weight_bits, fp8=fp8, nvfp4=nvfp4)
     tokens = sum(binding.num_tokens(c.size) for c in clips)
     with torch.cuda.stream(stream):
         xs = [torch.from_numpy(c).to(dev) for c in clips]
@@ -583,14 +583,17 @@ def other_configs(args, dev):
     pk = peaks()
     res = {}
     steps = max(3, min(args.steps, 20))
-    # then the 4-bit-weight encoder (round to nearest, groups of 128) and the
-    # FP8 encoder (q/k/v and fc1 on e4m3 operands)
+    # then the 4-bit-weight encoder (round to nearest, groups of 128), the FP8
+    # encoder (q/k/v and fc1 on e4m3 operands) and the NVFP4 encoder (q/k/v
+    # and fc1 on NVFP4 operands; "bits" 44 below)
     for w, bits in (("tiny_1s", 16), ("single_30s", 16), ("clip_10min", 16), ("clip_60min_streamed", 16),
-                    ("batch16_10to30s", 4), ("clip_60min_streamed", 4), ("batch16_10to30s", 8)):
+                    ("batch16_10to30s", 4), ("clip_60min_streamed", 4), ("batch16_10to30s", 8),
+                    ("batch16_10to30s", 44)):
         if w == "clip_60min_streamed":
             r = measure_streamed(max(3, min(args.steps, 10)), 3, dev, weight_bits=bits)
         else:
-            r = measure_plain(w, steps, 3, dev, weight_bits=4 if bits == 4 else 16, fp8=bits == 8)
+            r = measure_plain(w, steps, 3, dev, weight_bits=4 if bits == 4 else 16, fp8=bits == 8,
+                              nvfp4=bits == 44)
         tf = model_flops(r["tokens"], r["n_layers"]) / (r["ms"] / 1e3) / 1e12
         e = {"value": r["audio_s"] / (r["ms"] / 1e3), "unit": "audio-s/s", "ms_per_step": r["ms"],
              "tokens_per_s": r["tokens"] / (r["ms"] / 1e3), "tokens": r["tokens"], "layers": r["n_layers"],
@@ -602,7 +605,8 @@ def other_configs(args, dev):
                       "clip_and_rows_device_bytes": r["clip_and_rows_device_bytes"]})
         e["weight_bits"] = 4 if bits == 4 else 16
         e["fp8_qkv_fc1"] = bits == 8
-        res[w if bits == 16 else w + ("_w4" if bits == 4 else "_fp8")] = e
+        e["nvfp4_qkv_fc1"] = bits == 44
+        res[w if bits == 16 else w + {4: "_w4", 8: "_fp8", 44: "_nvfp4"}[bits]] = e
     return res
 
 

@@ -67,6 +67,9 @@ typedef struct {
     int fp8;               /* 1: the q/k/v and fc1 GEMMs of every layer take e4m3
                               operands (see MOSS_ENC_FP8); 0: bf16.  Not with
                               weight_bits = 4. */
+    int nvfp4;             /* 1: the q/k/v and fc1 GEMMs of every layer take NVFP4
+                              operands (see MOSS_ENC_NVFP4); 0: bf16.  Not with
+                              fp8 = 1 or weight_bits = 4. */
 } moss_enc_config;
 
 /* FP8 GEMMs (page "Ossicle-4B", "Quantized: NVFP4 and INT4 in vLLM": the
@@ -84,6 +87,24 @@ typedef struct {
  * divisions in fp32.  The other GEMMs keep bf16 operands.  The rows then
  * match the FP8 model of the same definition (not the bf16 model). */
 #define MOSS_ENC_FP8 1
+
+/* NVFP4 GEMMs (page "Ossicle-4B", section "Quantized: NVFP4 and INT4 in
+ * vLLM": an NVFP4 build quantises the audio encoder's weights and
+ * activations with NVIDIA ModelOpt and needs Blackwell's native FP4 kernels).
+ * With cfg.nvfp4 = 1 the q/k/v and fc1 GEMMs of every layer multiply NVFP4
+ * operands on the block-scaled FP4 tensor cores (kind::mxf4nvf4, fp32
+ * accumulation).  NVFP4 as ModelOpt defines it: E2M1 elements (0, 0.5, 1,
+ * 1.5, 2, 3, 4, 6 and negatives), an E4M3 scale per 16 consecutive k, and one
+ * fp32 factor g per tensor:
+ *   g = amax / 2688,  s_b = e4m3(amax_b / (g * 6)),  q = e2m1(x / (s_b * g))
+ * (fp32 arithmetic, ties to even, saturating; q = 0 when s_b = 0), with one g
+ * per weight matrix (q, k, v and fc1 each; at create) and one g per LayerNorm
+ * row (the LayerNorm kernel writes the codes, the scales and g, so a row's
+ * operands do not depend on the rest of the batch);
+ *   out[m][n] = (sum_k q_a s_a q_w s_w) * g_a[m] * g_w + b[n]   (GELU for fc1).
+ * The other GEMMs keep bf16 operands.  The rows then match the NVFP4 model of
+ * the same definition. */
+#define MOSS_ENC_NVFP4 1
 
 /* 4-bit weights (page "Ossicle-4B", "Long Audio", the note under the table:
  * "4-bit weights for ... the audio encoder, round to nearest, groups of 128").
@@ -351,6 +372,14 @@ moss_enc_status moss_enc_gemm_f8(moss_enc *h, const void *A8, const void *B8, co
 moss_enc_status moss_enc_gemm_nvf4(moss_enc *h, const void *A4, const void *sfa, const float *ga, const void *B4,
                                    const void *sfb, const float *gb, const float *bias, void *out, int M, int N,
                                    int K, int epilogue);
+
+/* The NVFP4 quantisation of activation rows of 1280 (what the LayerNorm
+ * kernel of an NVFP4 handle applies after the norm), on rows given as they
+ * are: x device fp32 [M][1280]; codes device uint8 [M][640], sfa device
+ * uint8 [ceil(M/128)][20][512] (layout of moss_enc_gemm_nvf4; the bytes of
+ * rows >= M in the last block are left as they are), g device fp32 [M].
+ * Enqueued on the handle's stream. */
+moss_enc_status moss_enc_nvf4_quant_rows(moss_enc *h, const float *x, void *codes, void *sfa, float *g, int M);
 
 /* The GEMM epilogues and conv1 evaluate GELU's erf with a short rational
  * approximation (Abramowitz & Stegun 7.1.28, error <= 3e-7), one value at a

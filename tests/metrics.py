@@ -15,6 +15,19 @@ ROW_MAXERR_RMS = 3e-2
 # the bf16 model); the bound keeps the cosine and allows 0.25 rms.
 FP8_ROW_COS = 0.999
 FP8_ROW_MAXERR_RMS = 0.25
+# The NVFP4 variant (q/k/v and fc1 on NVFP4 operands) against the oracle's
+# NVFP4 model.  E2M1 steps are up to a third of an operand's value, so the
+# model is discontinuous in the rows it quantises, and the GPU's bf16
+# activations between GEMMs (q/k/v, attention, the FFN hidden rows: ~2^-9
+# relative, the bf16 path's own tolerance) move about 1 % of the fc1 operands
+# across an E2M1 midpoint.  Measured, one layer from the same stem rows:
+# err/rms mean 0.040 (0.40 from the bf16 model); it grows with depth (0.10,
+# 0.16, 0.21 after 2, 4, 8 layers); 32 layers, 30 s clip: min cosine 0.9919,
+# max err/rms 0.558, mean 0.398 (1.06 from the bf16 model).  The bound keeps a
+# cosine of 0.985 and allows 0.8 rms; the tests also require the rows to sit
+# at most half as far from the NVFP4 model as from the bf16 one.
+NVFP4_ROW_COS = 0.985
+NVFP4_ROW_MAXERR_RMS = 0.8
 
 
 def row_metrics(got, ref):

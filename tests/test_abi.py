@@ -79,8 +79,10 @@ def test_create_rejects_bad_arguments_before_touching_a_device():
     st = L.moss_enc_create(ctypes.byref(cfg), blob.ctypes.data_as(ctypes.c_void_p), 8, 0, None, ctypes.byref(h))
     assert st == 1  # blob size does not match 4 layers
     # weight_bits must be 16 (or 0) or 4: refused before the blob is read
-    for bits, fp8 in [(8, 0), (4, 1), (16, 2)]:  # weight_bits 16/0/4; fp8 0/1, not with 4-bit weights
-        cfg = binding.Config(1, 1000, 1, 0, bits, fp8)
+    # weight_bits 16/0/4; fp8 0/1, not with 4-bit weights; nvfp4 0/1, with
+    # neither fp8 nor 4-bit weights
+    for bits, fp8, nvfp4 in [(8, 0, 0), (4, 1, 0), (16, 2, 0), (16, 0, 2), (16, 1, 1), (4, 0, 1)]:
+        cfg = binding.Config(1, 1000, 1, 0, bits, fp8, nvfp4)
         assert L.moss_enc_create(ctypes.byref(cfg), blob.ctypes.data_as(ctypes.c_void_p), 2 * binding.weight_count(1),
                                  0, None, ctypes.byref(h)) == 1
     assert L.moss_enc_status_string(2) == b"request exceeds capacity"
