@@ -246,7 +246,8 @@ def run_ours(args):
     stream = torch.cuda.Stream()
     mel_samples = 9_600_000  # the 10-min clip, for the log-mel roofline
     enc = binding.Encoder(blob, n_layers, max_samples=max(total_samples + 4 * len(clips), mel_samples),
-                          max_clips=len(clips), out_dtype=binding.OUT_BF16, stream=stream)
+                          max_clips=len(clips), out_dtype=binding.OUT_BF16, stream=stream,
+                          fp8=args.gemm_dtype == "fp8", nvfp4=args.gemm_dtype == "nvfp4")
     tap_layers = [int(v) for v in args.taps.split(",")] if args.taps else []
     with torch.cuda.stream(stream):
         xs = [torch.from_numpy(c).to(dev) for c in clips]
@@ -401,7 +402,8 @@ def run_ours(args):
     line = {
         "metric": "audio-sec encoded/sec", "value": value, "unit": "audio-s/s", "n_gpus": world,
         "steps": args.steps, "warmup": warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if args.gemm_dtype == "bf16" else f"bf16 ({args.gemm_dtype} q/k/v and fc1 GEMMs)",
         "data": "synthetic (seeded PCM, random-init bf16 weights)",
         "tokens_per_s": weak_scaling_throughput(world, tokens, ms_per_step),
         "model_tflops": tflops,
@@ -411,6 +413,7 @@ def run_ours(args):
                    "audio_s_per_gpu": audio_s, "tokens_per_gpu": tokens, "layers": n_layers,
                    "out_dtype": "bf16", "l2": "512 MB buffer written between timed steps (outside the events)",
                    "parallelism": f"dp{world}" if world > 1 else "single",
+                   **({"gemm_dtype": args.gemm_dtype} if args.gemm_dtype != "bf16" else {}),
                    **({"tap_layers": tap_layers} if tap_layers else {})},
         "roofline": roof,
         "mel_roofline": mel_roof,
@@ -707,6 +710,9 @@ def main():
     ap.add_argument("--taps", default="",
                     help="comma-separated encoder layers (0-based) whose hidden states also go through a "
                          "head + adapter set of their own (layer taps); the step is forward_taps")
+    ap.add_argument("--gemm-dtype", default="bf16", choices=["bf16", "fp8", "nvfp4"],
+                    help="operands of every layer's q/k/v and fc1 GEMMs (the other GEMMs stay bf16); the "
+                         "roofline stays the bf16 one")
     ap.add_argument("--ncu", action="store_true",
                     help="capture run for ncu: warm-up as given (may be 0), the timed steps only, no report")
     args = ap.parse_args()
