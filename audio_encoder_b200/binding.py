@@ -30,6 +30,7 @@ EXPORTED = [
     "moss_enc_tap_weight_count", "moss_enc_set_taps", "moss_enc_forward_taps",
     "moss_enc_profile_enable", "moss_enc_profile_read", "moss_enc_launch_count",
     "moss_enc_logmel_static", "moss_enc_gemm", "moss_enc_gemm_q4", "moss_enc_gemm_f8", "moss_enc_gemm_nvf4", "moss_enc_nvf4_quant_rows",
+    "moss_enc_nvf4_quant_weights",
     "moss_enc_selftest_gelu",
     "moss_enc_selftest_timeout",
 ]
@@ -130,6 +131,8 @@ def lib():
         L.moss_enc_gemm_nvf4.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32]
         L.moss_enc_nvf4_quant_rows.restype = i32
         L.moss_enc_nvf4_quant_rows.argtypes = [vp, vp, vp, vp, vp, i32]
+        L.moss_enc_nvf4_quant_weights.restype = i32
+        L.moss_enc_nvf4_quant_weights.argtypes = [vp, i32, i32, i32, vp, vp, vp]
         L.moss_enc_logmel_static.restype = i32
         L.moss_enc_logmel_static.argtypes = [ctypes.POINTER(Clip), i32, ctypes.POINTER(vp), vp, vp]
         _lib = L
@@ -150,6 +153,23 @@ def num_tokens(n: int) -> int:
 
 def range_tokens(n: int, begin: int, end: int) -> int:
     return int(lib().moss_enc_range_tokens(n, begin, end))
+
+
+def nvf4_quant_weights(w: np.ndarray, parts: int = 1):
+    """The create-time NVFP4 quantisation of a bf16 matrix (uint16 bits)
+    [n][k] in `parts` row ranges (host only): (codes [n][k/2] uint8, scale
+    atoms uint8, g [n] fp32)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    n, k = w.shape
+    codes = np.empty((n, k // 2), dtype=np.uint8)
+    sfa = np.empty(n * k // 16, dtype=np.uint8)
+    g = np.empty(n, dtype=np.float32)
+    st = lib().moss_enc_nvf4_quant_weights(w.ctypes.data_as(ctypes.c_void_p), n, k, parts,
+                                           codes.ctypes.data_as(ctypes.c_void_p), sfa.ctypes.data_as(ctypes.c_void_p),
+                                           g.ctypes.data_as(ctypes.c_void_p))
+    if st != OK:
+        raise MossEncError(st, "nvf4_quant_weights")
+    return codes, sfa, g
 
 
 def tap_weight_count() -> int:

@@ -985,11 +985,8 @@ static uint8_t host_e2m1(float x)
     return (uint8_t)(i | (std::signbit(x) ? 8 : 0));
 }
 
-static void quantise_nvfp4(uint8_t *mat, int n, int k, int parts)
+static void quantise_nvfp4_to(const uint16_t *w, int n, int k, int parts, uint8_t *codes, uint8_t *atoms, float *gr)
 {
-    const uint16_t *w = reinterpret_cast<const uint16_t *>(mat);
-    std::vector<uint8_t> codes((size_t)n * k / 2), atoms((size_t)n * k / 16);
-    std::vector<float> gr(n);
     const int rows = n / parts;
     for (int p = 0; p < parts; p++) {
         float amax = 0.0f;
@@ -1015,6 +1012,13 @@ static void quantise_nvfp4(uint8_t *mat, int n, int k, int parts)
             }
         }
     }
+}
+
+static void quantise_nvfp4(uint8_t *mat, int n, int k, int parts)
+{
+    std::vector<uint8_t> codes((size_t)n * k / 2), atoms((size_t)n * k / 16);
+    std::vector<float> gr(n);
+    quantise_nvfp4_to(reinterpret_cast<const uint16_t *>(mat), n, k, parts, codes.data(), atoms.data(), gr.data());
     std::memcpy(mat, codes.data(), codes.size());
     std::memcpy(mat + nvf4_sf_off(n, k), atoms.data(), atoms.size());
     std::memcpy(mat + nvf4_g_off(n, k), gr.data(), sizeof(float) * n);
@@ -2512,6 +2516,17 @@ extern "C" moss_enc_status moss_enc_gemm_nvf4(moss_enc *h, const void *A4, const
     case EPI_GELU_BF16: return gemm_nvf4<EPI_GELU_BF16>(h, "gemm_api", a4, M, K, b4, N, a);
     default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "epilogue must be 0 or 1");
     }
+}
+
+extern "C" moss_enc_status moss_enc_nvf4_quant_weights(const void *w, int n, int k, int parts, void *codes, void *sfa,
+                                                       float *g)
+{
+    if (!w || !codes || !sfa || !g || n <= 0 || k <= 0 || parts <= 0 || n % parts != 0 || (n / parts) % 128 != 0 ||
+        k % 64 != 0)
+        return MOSS_ENC_ERR_INVALID_ARG;
+    quantise_nvfp4_to(static_cast<const uint16_t *>(w), n, k, parts, static_cast<uint8_t *>(codes),
+                      static_cast<uint8_t *>(sfa), g);
+    return MOSS_ENC_OK;
 }
 
 extern "C" moss_enc_status moss_enc_nvf4_quant_rows(moss_enc *h, const float *x, void *codes, void *sfa, float *g,

@@ -381,6 +381,15 @@ moss_enc_status moss_enc_gemm_nvf4(moss_enc *h, const void *A4, const void *sfa,
  * Enqueued on the handle's stream. */
 moss_enc_status moss_enc_nvf4_quant_rows(moss_enc *h, const float *x, void *codes, void *sfa, float *g, int M);
 
+/* The NVFP4 quantisation moss_enc_create applies to the q/k/v and fc1
+ * weights of an NVFP4 handle, on the host (no device, no handle): w host
+ * bf16 bits [n][k], in `parts` equal row ranges with one g each (3 for the
+ * fused q/k/v matrix, 1 for fc1); codes host uint8 [n][k/2], sfa host uint8
+ * [n/128][k/64][512] (the layout of moss_enc_gemm_nvf4), g host fp32 [n]
+ * (each row's part's g).  n/parts % 128 == 0, k % 64 == 0; INVALID_ARG
+ * otherwise. */
+moss_enc_status moss_enc_nvf4_quant_weights(const void *w, int n, int k, int parts, void *codes, void *sfa, float *g);
+
 /* The GEMM epilogues and conv1 evaluate GELU's erf with a short rational
  * approximation (Abramowitz & Stegun 7.1.28, error <= 3e-7), one value at a
  * time and in pairs (paired fp32 instructions).  This runs both forms

@@ -100,3 +100,38 @@ def test_static_logmel_rejects_a_clip_without_samples_pointer():
     assert L.moss_enc_logmel_static(arr, 1, outs, None, None) == 1
     arr[0] = binding.Clip(None, 16000, 0, 16000, None)
     assert L.moss_enc_logmel_static(arr, 1, outs, None, None) == 1
+
+
+def test_nvf4_weight_quantiser_matches_oracle():
+    # the create-time NVFP4 quantisation of a weight matrix (host code of the
+    # library) against the oracle's, part by part: g, block scales and codes
+    # bit for bit (a zero may carry either sign); no device is touched
+    import oracle
+    import torch
+    from audio_encoder_b200 import synth
+    rng = np.random.default_rng(11)
+    n, k, parts = 384, 256, 3
+    w = (rng.standard_normal((n, k)) * np.repeat([0.02, 0.3, 5.0], n // parts)[:, None]).astype(np.float32)
+    w[5, :32] = 0.0
+    wb = synth.f32_to_bf16_bits(w)
+    codes, sfa, g = binding.nvf4_quant_weights(wb, parts)
+    got = np.empty((n, k), dtype=np.uint8)
+    got[:, 0::2] = codes & 15
+    got[:, 1::2] = codes >> 4
+    atoms = sfa.reshape(n // 128, k // 64, 512)
+    r = np.arange(n)[:, None]
+    b = np.arange(k // 16)[None, :]
+    e4 = atoms[r // 128, b // 4, (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4]
+    bs = torch.from_numpy(np.ascontiguousarray(e4)).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    wf = synth.bf16_bits_to_f32(wb)
+    rows = n // parts
+    for p in range(parts):
+        sl = slice(p * rows, (p + 1) * rows)
+        _, g_ref, c_ref, bs_ref = oracle.quant_nvfp4(wf[sl], per_row=False)
+        assert np.all(g[sl] == g_ref[0])
+        np.testing.assert_array_equal(bs[sl], bs_ref)
+        np.testing.assert_array_equal(got[sl] & 7, c_ref & 7)
+        nz = (c_ref & 7) != 0
+        np.testing.assert_array_equal((got[sl] & 8)[nz], (c_ref & 8)[nz])
+    with pytest.raises(binding.MossEncError):
+        binding.nvf4_quant_weights(wb[:, :100], 1)  # k not a multiple of 64
