@@ -133,5 +133,25 @@ def test_nvf4_weight_quantiser_matches_oracle():
         np.testing.assert_array_equal(got[sl] & 7, c_ref & 7)
         nz = (c_ref & 7) != 0
         np.testing.assert_array_equal((got[sl] & 8)[nz], (c_ref & 8)[nz])
+    # exact ties: with the part's maximum 2688 (g = 1) and a block maximum of
+    # 2688 (scale 448), x = m * 448 lands exactly on every E2M1 midpoint m;
+    # each tie must go to the even code, as in the oracle
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], dtype=np.float32)
+    t = np.zeros((128, 64), dtype=np.float32)
+    t[0, 0] = 2688.0
+    t[0, 1:8] = mids * 448.0
+    t[0, 8:15] = -mids * 448.0
+    tb = synth.f32_to_bf16_bits(t)
+    assert np.array_equal(synth.bf16_bits_to_f32(tb), t)  # every value is exact in bf16
+    c, _, gt = binding.nvf4_quant_weights(tb, 1)
+    mag = np.empty(64, dtype=np.uint8)
+    mag[0::2] = c[0] & 15
+    mag[1::2] = c[0] >> 4
+    assert gt[0] == 1.0 and mag[0] == 7  # 2688 / 448 = 6
+    np.testing.assert_array_equal(mag[1:8] & 7, [0, 2, 2, 4, 4, 6, 6])  # 0, 1, 1, 2, 2, 4, 4
+    np.testing.assert_array_equal(mag[9:15] & 7, [2, 2, 4, 4, 6, 6])
+    assert np.all(mag[9:15] & 8)  # negative
+    _, _, c_ref, _ = oracle.quant_nvfp4(t, per_row=False)
+    np.testing.assert_array_equal(mag[:15] & 7, c_ref[0, :15] & 7)
     with pytest.raises(binding.MossEncError):
         binding.nvf4_quant_weights(wb[:, :100], 1)  # k not a multiple of 64
