@@ -191,6 +191,23 @@ def test_positions_special_cases():
         assert oracle.position(0, 640 + c) == 1.0
 
 
+def test_positions_pair_channels_and_geometric_frequencies():
+    # every channel c < 640 and its partner 640 + c are the sine and cosine of
+    # one angle (sin^2 + cos^2 = 1, and the angle grows linearly with the
+    # position), and the angle rates fall geometrically from 1 to 1/10000
+    # over the 640 channels (log-rate linear in c with step ln(10^4)/639)
+    rates = np.empty(640)
+    for c in range(640):
+        s1, c1 = oracle.position(1, c), oracle.position(1, 640 + c)
+        assert s1 * s1 + c1 * c1 == pytest.approx(1.0, abs=1e-12)
+        rates[c] = np.arctan2(s1, c1)  # angle at p = 1 (below pi: rates <= 1)
+        s3, c3 = oracle.position(3, c), oracle.position(3, 640 + c)
+        assert np.arctan2(s3, c3) == pytest.approx(np.angle(np.exp(3j * rates[c])), abs=1e-12)
+    steps = np.diff(np.log(rates))
+    np.testing.assert_allclose(steps, -np.log(10000.0) / 639.0, rtol=1e-9)
+    assert rates[0] == pytest.approx(1.0, abs=1e-15) and rates[639] == pytest.approx(1e-4, rel=1e-12)
+
+
 # ----------------------------------------------------- model vs library
 
 def _tref(n_layers):
