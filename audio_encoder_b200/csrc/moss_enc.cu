@@ -2392,15 +2392,20 @@ extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void 
     case 160: return gemm_one<160>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
     case 192: return gemm_one<192>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
     case 256: return gemm_one<256>(h, a, b, bias, out, M, N, K, epilogue, cta_pair);
-    case 320:
+    case 320: {
         if (!cta_pair) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n 320 needs cta_pair");
+        GemmArgs g{};
+        g.bias = bias;
+        g.out = out;
+        g.ldo = N;
         switch (epilogue) {
-        case EPI_BF16: return gemm2<320, EPI_BF16>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
-        case EPI_GELU_BF16: return gemm2<320, EPI_GELU_BF16>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
-        case EPI_RESID_F32: return gemm2<320, EPI_RESID_F32>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
-        case EPI_F32: return gemm2<320, EPI_F32>(h, "gemm_api", a, M, K, b, N, GemmArgs{0, 0, 0, 0, 0, nullptr, bias, out, N});
+        case EPI_BF16: return gemm2<320, EPI_BF16>(h, "gemm_api", a, M, K, b, N, g);
+        case EPI_GELU_BF16: return gemm2<320, EPI_GELU_BF16>(h, "gemm_api", a, M, K, b, N, g);
+        case EPI_RESID_F32: return gemm2<320, EPI_RESID_F32>(h, "gemm_api", a, M, K, b, N, g);
+        case EPI_F32: return gemm2<320, EPI_F32>(h, "gemm_api", a, M, K, b, N, g);
         default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "unsupported epilogue");
         }
+    }
     default: return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128, 160, 192, 256 or 320");
     }
 }
