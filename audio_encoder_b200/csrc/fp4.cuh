@@ -274,7 +274,7 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
 // [rows].  One warp per row; lane l holds columns 128 i + 4 l .. + 3, so a
 // block of 16 is four neighbouring lanes.
 template <bool LN>
-__global__ void __launch_bounds__(256) nvf4_rows1280_kernel(const float *__restrict__ x, const float *__restrict__ gamma,
+__global__ void __launch_bounds__(256, 4) nvf4_rows1280_kernel(const float *__restrict__ x, const float *__restrict__ gamma,
                                                            const float *__restrict__ beta, uint8_t *__restrict__ codes,
                                                            uint8_t *__restrict__ atoms, float *__restrict__ g_out,
                                                            int rows)
