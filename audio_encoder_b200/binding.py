@@ -279,13 +279,20 @@ class Encoder:
         their E4M3 block-scale atoms (uint8), ga [M], gb [N] fp32."""
         M, K2 = A4.shape
         N = B4.shape[0]
+        if B4.shape[1] != K2 or sfa.numel() < (M + 127) // 128 * (2 * K2 // 64) * 512 or \
+                sfb.numel() < (N + 127) // 128 * (2 * K2 // 64) * 512 or ga.numel() < M or gb.numel() < N:
+            raise ValueError("A4 [M][K/2], B4 [N][K/2], their scale atoms, ga [M], gb [N]")
         self._check(lib().moss_enc_gemm_nvf4(self.h, _ptr(A4), _ptr(sfa), _ptr(ga), _ptr(B4), _ptr(sfb), _ptr(gb),
                                              _ptr(bias), _ptr(out), M, N, 2 * K2, int(epilogue)))
         return out
 
     def nvf4_quant_rows(self, x, codes, sfa, g):
         """NVFP4 codes, scale atoms and per-row g of fp32 rows x [M][1280]."""
-        self._check(lib().moss_enc_nvf4_quant_rows(self.h, _ptr(x), _ptr(codes), _ptr(sfa), _ptr(g), x.shape[0]))
+        M = x.shape[0]
+        if (x.dim() != 2 or x.shape[1] != D_MODEL or not x.is_contiguous() or tuple(codes.shape) != (M, D_MODEL // 2)
+                or sfa.numel() < (M + 127) // 128 * 20 * 512 or g.numel() < M):
+            raise ValueError("x [M][1280] fp32, codes [M][640], sfa ceil(M/128)*20*512 bytes, g [M]")
+        self._check(lib().moss_enc_nvf4_quant_rows(self.h, _ptr(x), _ptr(codes), _ptr(sfa), _ptr(g), M))
 
     def selftest_timeout(self, limit_ms: int = 50):
         self._check(lib().moss_enc_selftest_timeout(self.h, int(limit_ms)))
