@@ -2371,8 +2371,8 @@ extern "C" moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void 
     if (!h) return MOSS_ENC_ERR_INVALID_ARG;
     if (!A || !B || !bias || !out || M < 0 || N <= 0 || K <= 0 || K % 64 != 0)
         return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad gemm arguments");
-    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15)
-        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A and B must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(bias)) & 15)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A, B and bias must be 16-byte aligned");
     static bool attrs_done = false;
     if (!attrs_done) {
         CUDA_TRY(h, gemm_api_attrs<128>());
@@ -2444,8 +2444,9 @@ extern "C" moss_enc_status moss_enc_gemm_q4(moss_enc *h, const void *A, const vo
     if (!h) return MOSS_ENC_ERR_INVALID_ARG;
     if (!A || !Bq || !Bs || !bias || !out || M < 0 || N <= 0 || K <= 0 || K % 128 != 0)
         return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad gemm arguments");
-    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(Bq) | reinterpret_cast<uintptr_t>(Bs)) & 15)
-        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A, Bq and Bs must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(Bq) | reinterpret_cast<uintptr_t>(Bs) |
+         reinterpret_cast<uintptr_t>(bias)) & 15)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A, Bq, Bs and bias must be 16-byte aligned");
     if (N % block_n != 0 || N % 4 != 0) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n != 0");
     static bool attrs_done = false;
     if (!attrs_done) {
@@ -2476,8 +2477,9 @@ extern "C" moss_enc_status moss_enc_gemm_f8(moss_enc *h, const void *A8, const v
     if (!h) return MOSS_ENC_ERR_INVALID_ARG;
     if (!A8 || !B8 || !sa || !sb || !bias || !out || M < 0 || N <= 0 || K <= 0 || K % 256 != 0)
         return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad gemm arguments");
-    if ((reinterpret_cast<uintptr_t>(A8) | reinterpret_cast<uintptr_t>(B8)) & 15)
-        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A8 and B8 must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(A8) | reinterpret_cast<uintptr_t>(B8) | reinterpret_cast<uintptr_t>(bias) |
+         reinterpret_cast<uintptr_t>(sb)) & 15)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A8, B8, sb and bias must be 16-byte aligned");
     if (block_n != 128 && block_n != 256) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "block_n must be 128 or 256");
     if (N % block_n != 0) return fail(h, MOSS_ENC_ERR_INVALID_ARG, "N % block_n != 0");
     GemmArgs a{};
@@ -2505,8 +2507,8 @@ extern "C" moss_enc_status moss_enc_gemm_nvf4(moss_enc *h, const void *A4, const
         N % 128 != 0)
         return fail(h, MOSS_ENC_ERR_INVALID_ARG, "bad gemm arguments");
     if ((reinterpret_cast<uintptr_t>(A4) | reinterpret_cast<uintptr_t>(B4) | reinterpret_cast<uintptr_t>(sfa) |
-         reinterpret_cast<uintptr_t>(sfb)) & 15)
-        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A4, B4 and the scale atoms must be 16-byte aligned");
+         reinterpret_cast<uintptr_t>(sfb) | reinterpret_cast<uintptr_t>(gb) | reinterpret_cast<uintptr_t>(bias)) & 15)
+        return fail(h, MOSS_ENC_ERR_INVALID_ARG, "A4, B4, the scale atoms, gb and bias must be 16-byte aligned");
     GemmArgs a{};
     a.bias = bias;
     a.out = out;

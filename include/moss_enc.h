@@ -332,7 +332,9 @@ moss_enc_status moss_enc_forward_host(moss_enc *h, const float *const *pcm_host,
  *             N % block_n == 0.
  *  cta_pair   0: one CTA per 128 x block_n tile; 1: CTA pairs (cluster of
  *             2) on 256 x block_n tiles, as the forward uses.
- *  K % 64 == 0.  Enqueued on the handle's stream. */
+ *  K % 64 == 0; A, B and bias 16-byte aligned (INVALID_ARG otherwise: the
+ *  epilogue reads bias four floats at a time).  Enqueued on the handle's
+ *  stream. */
 moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const float *bias, void *out,
                               int M, int N, int K, int epilogue, int block_n, int cta_pair);
 
@@ -342,7 +344,8 @@ moss_enc_status moss_enc_gemm(moss_enc *h, const void *A, const void *B, const f
  *             even k in the low nibble;
  *  Bs         device fp32 [K/128][N]: the scale of each group of 128 k;
  * and the product uses B[n][k] = bf16(fp32(q * s)).  block_n 128, 160, 256
- * or 320, CTA pairs only; K % 128 == 0; epilogues as moss_enc_gemm. */
+ * or 320, CTA pairs only; K % 128 == 0; epilogues as moss_enc_gemm; A, Bq,
+ * Bs and bias 16-byte aligned. */
 moss_enc_status moss_enc_gemm_q4(moss_enc *h, const void *A, const void *Bq, const float *Bs, const float *bias,
                                  void *out, int M, int N, int K, int epilogue, int block_n);
 
@@ -351,7 +354,7 @@ moss_enc_status moss_enc_gemm_q4(moss_enc *h, const void *A, const void *Bq, con
  * bits), sa device fp32 [M], sb device fp32 [N];
  *   out[m][n] = epi((sum_k A8 B8) * sa[m] * sb[n] + bias[n]),
  * epilogue 0 (bf16 out) or 1 (GELU, bf16 out); block_n 128 or 256 (CTA
- * pairs); K % 256 == 0. */
+ * pairs); K % 256 == 0; A8, B8, sb and bias 16-byte aligned. */
 moss_enc_status moss_enc_gemm_f8(moss_enc *h, const void *A8, const void *B8, const float *sa, const float *sb,
                                  const float *bias, void *out, int M, int N, int K, int epilogue, int block_n);
 
@@ -368,7 +371,7 @@ moss_enc_status moss_enc_gemm_f8(moss_enc *h, const void *A8, const void *B8, co
  *   out[m][n] = epi((sum_k a[m][k] b[n][k]) * ga[m] * gb[n] + bias[n]),
  * a and b the E2M1 values times their block scales.  epilogue 0 (bf16 out)
  * or 1 (GELU, bf16 out); 128 x 128 tiles on one CTA each; K % 256 == 0,
- * N % 128 == 0; all four operand pointers 16-byte aligned. */
+ * N % 128 == 0; A4, B4, sfa, sfb, gb and bias 16-byte aligned. */
 moss_enc_status moss_enc_gemm_nvf4(moss_enc *h, const void *A4, const void *sfa, const float *ga, const void *B4,
                                    const void *sfb, const float *gb, const float *bias, void *out, int M, int N,
                                    int K, int epilogue);
